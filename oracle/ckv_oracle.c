@@ -1,0 +1,486 @@
+/*
+ * ClusterKV CPU oracle: TEST INFRASTRUCTURE ONLY.
+ *
+ * This is a plain, slow and direct restatement of what the ClusterKV hot path computes.
+ * The tests, the smoke check and the bench's CPU-baseline leg use it to check the CUDA
+ * library. The product path never calls it. It shares no code, header, table or
+ * constant generator with the CUDA sources.
+ *
+ * Sources, cited by page title and section:
+ *   [EXPL] "大模型KV Cache压缩技术：ClusterKV的语义空间优化" (ClusterKV explainer),
+ *          section 3.1 (attention formula, centroid mean, cluster-importance relation),
+ *          section 3.2 (16 sinks, cosine K-means at prefill, incremental clustering
+ *          every 320 tokens), section 3.3 (select_clusters listing), section 4.1
+ *          (half-precision distance matmul, cluster-contiguous KV layout).
+ *   [ABS]  "ClusterKV: Manipulating LLM KV Cache in Semantic Space for Recallable
+ *          Compression" (arXiv 2412.03213 listing), abstract.
+ *
+ * Precision: every sum is in double. The bf16 rounding of the normalised centroid
+ * follows [EXPL] 4.1 ("half-precision matmul" for the cosine distances). Inputs (keys,
+ * values, queries) are bf16 bit patterns (uint16).
+ *
+ * Parity status: every function here is pinned by a CPU test (brute force, closed form,
+ * invariant or published test vector). The end-to-end attention quality on real models
+ * is not pinned (the pages print no numbers for it).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_D 128
+
+/* ---------------------------------------------------------------- bf16 ---------- */
+
+double orc_bf16_to_double(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* Round a double to the nearest bf16 value, ties to even (IEEE 754 roundTiesToEven on a
+ * format with 8 significand bits and float32's exponent range). */
+uint16_t orc_bf16_from_double(double x) {
+    if (isnan(x)) return 0x7FC0;
+    uint16_t sign = signbit(x) ? 0x8000 : 0;
+    double ax = fabs(x);
+    if (ax == 0.0) return sign;
+    if (isinf(ax)) return sign | 0x7F80;
+    int e;
+    frexp(ax, &e);              /* ax = f * 2^e, f in [0.5, 1) */
+    int ex = e - 1;             /* ax in [2^ex, 2^(ex+1)) */
+    if (ex < -126) ex = -126;   /* subnormal range keeps the fixed quantum 2^-133 */
+    double quantum = ldexp(1.0, ex - 7);
+    double r = nearbyint(ax / quantum) * quantum; /* default mode: nearest, ties to even */
+    if (r >= ldexp(1.0, 128)) return sign | 0x7F80;
+    float f = (float)r;         /* exact: r has at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return sign | (uint16_t)(u >> 16);
+}
+
+void orc_bf16_from_double_array(const double* x, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < n; i++) out[i] = orc_bf16_from_double(x[i]);
+}
+
+/* -------------------------------------------------------- seeded init ---------- */
+/* The pages only say the K-means is seeded. The reading used here: the initial centroids
+ * are the first C entries of a Fisher-Yates shuffle (Durstenfeld's form) of the candidate
+ * token indices. The shuffle is driven by SplitMix64 (Steele, Lea & Flood, OOPSLA 2014),
+ * and each draw is mapped into [0, r) by Lemire's multiply-shift (ACM TOMACS 2019,
+ * without the rejection step). */
+
+uint64_t orc_splitmix64_next(uint64_t* state) {
+    uint64_t z = (*state += 0x9E3779B97F4A7C15ULL);
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+    return z ^ (z >> 31);
+}
+
+uint32_t orc_bounded(uint64_t x, uint32_t r) {
+    return (uint32_t)(((x >> 32) * (uint64_t)r) >> 32);
+}
+
+/* Stream key of one unit's clustering run: window 0 is the prefill, window w >= 1 is the
+ * w-th incremental re-clustering of that unit. */
+uint64_t orc_stream_key(uint64_t seed, int64_t unit, uint64_t window) {
+    return seed ^ ((uint64_t)unit << 32) ^ window;
+}
+
+/* out[0..C) = first C entries of the shuffled sequence 0..m-1. Requires 1 <= C <= m. */
+void orc_init_indices(int64_t m, int32_t C, uint64_t key, int32_t* out) {
+    int32_t* a = (int32_t*)malloc(sizeof(int32_t) * (size_t)m);
+    for (int64_t j = 0; j < m; j++) a[j] = (int32_t)j;
+    uint64_t state = key;
+    for (int32_t i = 0; i < C; i++) {
+        uint64_t x = orc_splitmix64_next(&state);
+        int64_t j = i + (int64_t)orc_bounded(x, (uint32_t)(m - i));
+        int32_t t = a[i];
+        a[i] = a[j];
+        a[j] = t;
+        out[i] = a[i];
+    }
+    free(a);
+}
+
+/* ---------------------------------------------------------- K-means ---------- */
+
+static double dot_bf16_bf16(const uint16_t* a, const uint16_t* b) {
+    double s = 0.0;
+    for (int d = 0; d < ORC_D; d++) s += orc_bf16_to_double(a[d]) * orc_bf16_to_double(b[d]);
+    return s;
+}
+
+/* Assignment operand: mu_hat_c = bf16(mu_c / ||mu_c||). A zero centroid maps to zero.
+ * Cosine similarity of k with mu_c is (k . mu_hat_c) / ||k||, and ||k|| does not depend
+ * on c, so the argmax over c of k . mu_hat_c is the argmax of the cosine ([EXPL] 3.2,
+ * "cosine distance"). The bf16 rounding follows [EXPL] 4.1. */
+void orc_normalize(const double* mu, int32_t C, uint16_t* mu_hat) {
+    for (int32_t c = 0; c < C; c++) {
+        const double* m = mu + (int64_t)c * ORC_D;
+        double ss = 0.0;
+        for (int d = 0; d < ORC_D; d++) ss += m[d] * m[d];
+        double nrm = sqrt(ss);
+        for (int d = 0; d < ORC_D; d++)
+            mu_hat[(int64_t)c * ORC_D + d] = nrm > 0.0 ? orc_bf16_from_double(m[d] / nrm) : 0;
+    }
+}
+
+/* a_i = argmax_c k_i . mu_hat_c, ties to the lower c. */
+void orc_assign(const uint16_t* keys, int64_t m, const uint16_t* mu_hat, int32_t C,
+                int32_t* assign) {
+    for (int64_t i = 0; i < m; i++) {
+        double best = -INFINITY;
+        int32_t arg = 0;
+        for (int32_t c = 0; c < C; c++) {
+            double s = dot_bf16_bf16(keys + i * ORC_D, mu_hat + (int64_t)c * ORC_D);
+            if (s > best) { best = s; arg = c; }
+        }
+        assign[i] = arg;
+    }
+}
+
+/* Cosine gap between the oracle's best cluster and another assignment of the same key:
+ * gap_i = (k_i . mu_hat_best - k_i . mu_hat_other_i) / ||k_i||. A zero gap means
+ * other_i is also a correct answer. Tests use it to accept near-tie disagreements. */
+void orc_assign_gap(const uint16_t* keys, int64_t m, const uint16_t* mu_hat, int32_t C,
+                    const int32_t* other, double* gap) {
+    for (int64_t i = 0; i < m; i++) {
+        const uint16_t* k = keys + i * ORC_D;
+        double best = -INFINITY, nk = 0.0;
+        for (int32_t c = 0; c < C; c++) {
+            double s = dot_bf16_bf16(k, mu_hat + (int64_t)c * ORC_D);
+            if (s > best) best = s;
+        }
+        for (int d = 0; d < ORC_D; d++) {
+            double x = orc_bf16_to_double(k[d]);
+            nk += x * x;
+        }
+        int32_t o = other[i];
+        double so = (o >= 0 && o < C) ? dot_bf16_bf16(k, mu_hat + (int64_t)o * ORC_D) : -INFINITY;
+        gap[i] = (best - so) / (nk > 0.0 ? sqrt(nk) : 1.0);
+    }
+}
+
+/* Update: counting sort of the keys by cluster, then mu_c = (1/|c|) sum of its members
+ * (the raw mean of [EXPL] 3.1). sizes/offsets/perm describe the cluster-contiguous
+ * layout of [EXPL] 4.1: perm[offsets[c] .. offsets[c+1]) lists the members of cluster c
+ * in ascending key index. An empty cluster keeps its previous centroid. */
+void orc_update(const uint16_t* keys, int64_t m, const int32_t* assign, int32_t C,
+                double* mu, int32_t* offsets, int32_t* perm) {
+    int64_t* fill = (int64_t*)calloc((size_t)C + 1, sizeof(int64_t));
+    for (int32_t c = 0; c <= C; c++) offsets[c] = 0;
+    for (int64_t i = 0; i < m; i++) offsets[assign[i] + 1]++;
+    for (int32_t c = 0; c < C; c++) offsets[c + 1] += offsets[c];
+    for (int64_t i = 0; i < m; i++) {
+        int32_t c = assign[i];
+        perm[offsets[c] + fill[c]++] = (int32_t)i;
+    }
+    for (int32_t c = 0; c < C; c++) {
+        int32_t lo = offsets[c], hi = offsets[c + 1];
+        if (hi == lo) continue;
+        double acc[ORC_D] = {0};
+        for (int32_t j = lo; j < hi; j++)
+            for (int d = 0; d < ORC_D; d++) acc[d] += orc_bf16_to_double(keys[(int64_t)perm[j] * ORC_D + d]);
+        for (int d = 0; d < ORC_D; d++) mu[(int64_t)c * ORC_D + d] = acc[d] / (double)(hi - lo);
+    }
+    free(fill);
+}
+
+/* Lloyd's K-means with cosine assignment ([EXPL] 3.2) from the given initial members.
+ * Every iteration normalises, assigns, then updates. After the last iteration, mu holds
+ * the means of the final assignment, and offsets/perm hold its layout. */
+void orc_kmeans(const uint16_t* keys, int64_t m, int32_t C, int32_t iters,
+                const int32_t* init, double* mu, int32_t* offsets, int32_t* perm,
+                int32_t* assign) {
+    uint16_t* mu_hat = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)C * ORC_D);
+    for (int32_t c = 0; c < C; c++)
+        for (int d = 0; d < ORC_D; d++)
+            mu[(int64_t)c * ORC_D + d] = orc_bf16_to_double(keys[(int64_t)init[c] * ORC_D + d]);
+    for (int32_t t = 0; t < iters; t++) {
+        orc_normalize(mu, C, mu_hat);
+        orc_assign(keys, m, mu_hat, C, assign);
+        orc_update(keys, m, assign, C, mu, offsets, perm);
+    }
+    free(mu_hat);
+}
+
+/* --------------------------------------------------------- cluster store ---------- */
+/* One unit = one (layer, sequence, KV head). Its store is the cluster-contiguous KV
+ * layout of [EXPL] 4.1 plus the uncompressed rows:
+ *   sp_k/sp_v   [n_sink + pending, 128]: sink rows (token ids 0..n_sink-1), then the
+ *               pending rows appended since the last clustering (ids n_sink + m + j);
+ *   kp/vp       [m, 128]: clustered rows, cluster-major;
+ *   ids         [m]: original token id of each clustered row;
+ *   offsets     [C + 1]: cluster c owns rows offsets[c] .. offsets[c+1];
+ *   mu          [C, 128]: centroids (raw means). */
+typedef struct {
+    int32_t n_sink, pending, C;
+    int64_t m;
+    const uint16_t* sp_k;
+    const uint16_t* sp_v;
+    const uint16_t* kp;
+    const uint16_t* vp;
+    const int32_t* ids;
+    const int32_t* offsets;
+    const double* mu;
+} orc_store;
+
+/* Prefill of one unit ([EXPL] 3.2): the first n_sink tokens are kept as sinks. Cosine
+ * K-means runs on the rest, and K and V are permuted into the cluster-major store.
+ * K, V: [n, 128]. Outputs are sized by the caller: kp/vp [n - n_sink, 128],
+ * ids [n - n_sink], offsets [C + 1], mu [C, 128], assign [n - n_sink]. */
+void orc_prefill_unit(const uint16_t* K, const uint16_t* V, int64_t n, int32_t n_sink,
+                      int32_t C, int32_t iters, uint64_t key, uint16_t* kp, uint16_t* vp,
+                      int32_t* ids, int32_t* offsets, double* mu, int32_t* assign) {
+    int64_t m = n - n_sink;
+    const uint16_t* keys = K + (int64_t)n_sink * ORC_D;
+    int32_t* init = (int32_t*)malloc(sizeof(int32_t) * (size_t)C);
+    int32_t* perm = (int32_t*)malloc(sizeof(int32_t) * (size_t)m);
+    orc_init_indices(m, C, key, init);
+    orc_kmeans(keys, m, C, iters, init, mu, offsets, perm, assign);
+    for (int64_t j = 0; j < m; j++) {
+        int64_t src = (int64_t)n_sink + perm[j];
+        memcpy(kp + j * ORC_D, K + src * ORC_D, sizeof(uint16_t) * ORC_D);
+        memcpy(vp + j * ORC_D, V + src * ORC_D, sizeof(uint16_t) * ORC_D);
+        ids[j] = (int32_t)src;
+    }
+    free(init);
+    free(perm);
+}
+
+/* Incremental clustering of one full window ([EXPL] 3.2, "every 320 new tokens"). Cosine
+ * K-means with C_new clusters runs on the window's rows alone, with the same init rule
+ * and the given stream key. It writes the window's cluster-major rows, their token ids
+ * (first_id + local index), the C_new + 1 offsets relative to the window start, and the
+ * C_new centroids. Existing clusters are left unchanged. */
+void orc_recluster_window(const uint16_t* wk, const uint16_t* wv, int64_t w, int32_t C_new,
+                          int32_t iters, uint64_t key, int64_t first_id, uint16_t* kp,
+                          uint16_t* vp, int32_t* ids, int32_t* offsets, double* mu,
+                          int32_t* assign) {
+    int32_t* init = (int32_t*)malloc(sizeof(int32_t) * (size_t)C_new);
+    int32_t* perm = (int32_t*)malloc(sizeof(int32_t) * (size_t)w);
+    orc_init_indices(w, C_new, key, init);
+    orc_kmeans(wk, w, C_new, iters, init, mu, offsets, perm, assign);
+    for (int64_t j = 0; j < w; j++) {
+        memcpy(kp + j * ORC_D, wk + (int64_t)perm[j] * ORC_D, sizeof(uint16_t) * ORC_D);
+        memcpy(vp + j * ORC_D, wv + (int64_t)perm[j] * ORC_D, sizeof(uint16_t) * ORC_D);
+        ids[j] = (int32_t)(first_id + perm[j]);
+    }
+    free(init);
+    free(perm);
+}
+
+/* ------------------------------------------------------------- selection ---------- */
+
+typedef struct { double score; int32_t idx; int32_t id; } orc_ranked;
+
+/* Descending score, ties to the lower index. */
+static int cmp_cluster(const void* a, const void* b) {
+    const orc_ranked* x = (const orc_ranked*)a;
+    const orc_ranked* y = (const orc_ranked*)b;
+    if (x->score > y->score) return -1;
+    if (x->score < y->score) return 1;
+    return (x->idx > y->idx) - (x->idx < y->idx);
+}
+
+/* Descending score, ties to the lower original token id. */
+static int cmp_token(const void* a, const void* b) {
+    const orc_ranked* x = (const orc_ranked*)a;
+    const orc_ranked* y = (const orc_ranked*)b;
+    if (x->score > y->score) return -1;
+    if (x->score < y->score) return 1;
+    return (x->id > y->id) - (x->id < y->id);
+}
+
+/* Group query of one KV head: qbar = sum of its G query heads. One selection per KV head
+ * is shared by the G query heads. Scoring one query against a centroid ([EXPL] 3.3) with
+ * this sum gives the sum of the heads' own scores. q: [G, 128] bf16. */
+void orc_group_query(const uint16_t* q, int32_t G, double* qbar) {
+    for (int d = 0; d < ORC_D; d++) {
+        double s = 0.0;
+        for (int32_t g = 0; g < G; g++) s += orc_bf16_to_double(q[(int64_t)g * ORC_D + d]);
+        qbar[d] = s;
+    }
+}
+
+/* select_clusters of [EXPL] 3.3, for one KV head.
+ * 1. score every cluster by qbar . mu_c;
+ * 2. visit clusters by descending score (ties: lower cluster index);
+ * 3. take a whole cluster while its size fits the remaining budget;
+ * 4. the first cluster that does not fit gives its top-`remaining` tokens by qbar . k
+ *    (descending; ties: lower token id), then the walk stops.
+ * Two readings of the listing: the partial fill takes the highest-scoring tokens (the
+ * printed ascending sort would take the lowest), and the sinks and pending rows are
+ * always kept and counted against the budget: remaining = budget - n_sink - pending.
+ *
+ * Output: sel_ids[0..count) = original ids (sinks, pending, whole clusters in visit order,
+ * then partial tokens in rank order). sel_rows encodes where each row sits:
+ * r >= 0 is clustered row r of kp/vp, and r < 0 is row (-r - 1) of sp_k/sp_v.
+ * info[0..4) = { number of whole clusters, cut cluster (-1 if none), partial count r,
+ * selected count }. Returns the selected count, or -1 if budget < n_sink + pending. */
+int32_t orc_select(const orc_store* s, const double* qbar, int32_t budget, int32_t* sel_ids,
+                   int32_t* sel_rows, int32_t* info, double* scores_out) {
+    int64_t remaining = (int64_t)budget - s->n_sink - s->pending;
+    if (remaining < 0) return -1;
+    int32_t count = 0;
+    for (int32_t i = 0; i < s->n_sink + s->pending; i++) {
+        sel_ids[count] = i < s->n_sink ? i : (int32_t)(s->n_sink + s->m + (i - s->n_sink));
+        sel_rows[count] = -i - 1;
+        count++;
+    }
+    orc_ranked* cl = (orc_ranked*)malloc(sizeof(orc_ranked) * (size_t)(s->C > 0 ? s->C : 1));
+    for (int32_t c = 0; c < s->C; c++) {
+        double sc = 0.0;
+        for (int d = 0; d < ORC_D; d++) sc += qbar[d] * s->mu[(int64_t)c * ORC_D + d];
+        cl[c].score = sc;
+        cl[c].idx = c;
+        cl[c].id = c;
+        if (scores_out) scores_out[c] = sc;
+    }
+    qsort(cl, (size_t)s->C, sizeof(orc_ranked), cmp_cluster);
+    int32_t n_whole = 0, cut = -1, r = 0;
+    for (int32_t k = 0; k < s->C; k++) {
+        int32_t c = cl[k].idx;
+        int32_t lo = s->offsets[c], hi = s->offsets[c + 1];
+        int64_t size = hi - lo;
+        if (size <= remaining) {
+            for (int32_t j = lo; j < hi; j++) {
+                sel_ids[count] = s->ids[j];
+                sel_rows[count] = j;
+                count++;
+            }
+            remaining -= size;
+            n_whole++;
+        } else {
+            orc_ranked* tk = (orc_ranked*)malloc(sizeof(orc_ranked) * (size_t)size);
+            for (int32_t j = lo; j < hi; j++) {
+                double t = 0.0;
+                for (int d = 0; d < ORC_D; d++)
+                    t += qbar[d] * orc_bf16_to_double(s->kp[(int64_t)j * ORC_D + d]);
+                tk[j - lo].score = t;
+                tk[j - lo].idx = j;
+                tk[j - lo].id = s->ids[j];
+            }
+            qsort(tk, (size_t)size, sizeof(orc_ranked), cmp_token);
+            for (int64_t j = 0; j < remaining; j++) {
+                sel_ids[count] = tk[j].id;
+                sel_rows[count] = tk[j].idx;
+                count++;
+            }
+            cut = c;
+            r = (int32_t)remaining;
+            free(tk);
+            break;
+        }
+    }
+    free(cl);
+    if (info) {
+        info[0] = n_whole;
+        info[1] = cut;
+        info[2] = r;
+        info[3] = count;
+    }
+    return count;
+}
+
+/* Attention over the selected rows ([EXPL] 3.1): o_g = softmax(q_g K_sel^T / sqrt(128)) V_sel
+ * for each of the G query heads, all in double. */
+void orc_attend(const orc_store* s, const uint16_t* q, int32_t G, const int32_t* sel_rows,
+                int32_t count, double* out) {
+    double* z = (double*)malloc(sizeof(double) * (size_t)(count > 0 ? count : 1));
+    const double scale = 1.0 / sqrt((double)ORC_D);
+    for (int32_t g = 0; g < G; g++) {
+        const uint16_t* qg = q + (int64_t)g * ORC_D;
+        double zmax = -INFINITY;
+        for (int32_t i = 0; i < count; i++) {
+            int32_t r = sel_rows[i];
+            const uint16_t* k = r >= 0 ? s->kp + (int64_t)r * ORC_D : s->sp_k + (int64_t)(-r - 1) * ORC_D;
+            z[i] = dot_bf16_bf16(qg, k) * scale;
+            if (z[i] > zmax) zmax = z[i];
+        }
+        double den = 0.0;
+        double acc[ORC_D] = {0};
+        for (int32_t i = 0; i < count; i++) {
+            int32_t r = sel_rows[i];
+            const uint16_t* v = r >= 0 ? s->vp + (int64_t)r * ORC_D : s->sp_v + (int64_t)(-r - 1) * ORC_D;
+            double p = exp(z[i] - zmax);
+            den += p;
+            for (int d = 0; d < ORC_D; d++) acc[d] += p * orc_bf16_to_double(v[d]);
+        }
+        for (int d = 0; d < ORC_D; d++) out[(int64_t)g * ORC_D + d] = acc[d] / den;
+    }
+    free(z);
+}
+
+/* Dense attention over all n rows of K, V ([EXPL] 3.1), the full-KV reference. */
+void orc_dense_attention(const uint16_t* K, const uint16_t* V, int64_t n, const uint16_t* q,
+                         int32_t G, double* out) {
+    double* z = (double*)malloc(sizeof(double) * (size_t)n);
+    const double scale = 1.0 / sqrt((double)ORC_D);
+    for (int32_t g = 0; g < G; g++) {
+        double zmax = -INFINITY, den = 0.0;
+        double acc[ORC_D] = {0};
+        for (int64_t i = 0; i < n; i++) {
+            z[i] = dot_bf16_bf16(q + (int64_t)g * ORC_D, K + i * ORC_D) * scale;
+            if (z[i] > zmax) zmax = z[i];
+        }
+        for (int64_t i = 0; i < n; i++) {
+            double p = exp(z[i] - zmax);
+            den += p;
+            for (int d = 0; d < ORC_D; d++) acc[d] += p * orc_bf16_to_double(V[i * ORC_D + d]);
+        }
+        for (int d = 0; d < ORC_D; d++) out[(int64_t)g * ORC_D + d] = acc[d] / den;
+    }
+    free(z);
+}
+
+/* ---------------------------------------------------- batched (timing) ---------- */
+/* Independent units run in parallel (OpenMP, when compiled with it). Each unit's
+ * arithmetic is exactly the single-unit function above. */
+
+void orc_prefill_batch(int32_t U, const uint16_t* K, const uint16_t* V, int64_t n,
+                       int32_t n_sink, int32_t C, int32_t iters, const uint64_t* keys,
+                       uint16_t* kp, uint16_t* vp, int32_t* ids, int32_t* offsets,
+                       double* mu, int32_t* assign) {
+    int64_t m = n - n_sink;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int32_t u = 0; u < U; u++)
+        orc_prefill_unit(K + (int64_t)u * n * ORC_D, V + (int64_t)u * n * ORC_D, n, n_sink, C,
+                         iters, keys[u], kp + (int64_t)u * m * ORC_D, vp + (int64_t)u * m * ORC_D,
+                         ids + (int64_t)u * m, offsets + (int64_t)u * (C + 1),
+                         mu + (int64_t)u * C * ORC_D, assign + (int64_t)u * m);
+}
+
+/* select + attend for U units that share C, m, pending and budget (stores laid out back
+ * to back). q: [U, G, 128]; out: [U, G, 128]; sel_ids: [U, budget]; counts: [U]. */
+void orc_select_attend_batch(int32_t U, int32_t n_sink, int32_t pending, int64_t m, int32_t C,
+                             const uint16_t* sp_k, const uint16_t* sp_v, const uint16_t* kp,
+                             const uint16_t* vp, const int32_t* ids, const int32_t* offsets,
+                             const double* mu, const uint16_t* q, int32_t G, int32_t budget,
+                             double* out, int32_t* sel_ids, int32_t* counts) {
+    int64_t sp = (int64_t)n_sink + pending;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int32_t u = 0; u < U; u++) {
+        orc_store s;
+        s.n_sink = n_sink;
+        s.pending = pending;
+        s.C = C;
+        s.m = m;
+        s.sp_k = sp_k + (int64_t)u * sp * ORC_D;
+        s.sp_v = sp_v + (int64_t)u * sp * ORC_D;
+        s.kp = kp + (int64_t)u * m * ORC_D;
+        s.vp = vp + (int64_t)u * m * ORC_D;
+        s.ids = ids + (int64_t)u * m;
+        s.offsets = offsets + (int64_t)u * (C + 1);
+        s.mu = mu + (int64_t)u * C * ORC_D;
+        double qbar[ORC_D];
+        orc_group_query(q + (int64_t)u * G * ORC_D, G, qbar);
+        int32_t* rows = (int32_t*)malloc(sizeof(int32_t) * (size_t)budget);
+        int32_t cnt = orc_select(&s, qbar, budget, sel_ids + (int64_t)u * budget, rows, NULL, NULL);
+        counts[u] = cnt;
+        if (cnt > 0) orc_attend(&s, q + (int64_t)u * G * ORC_D, G, rows, cnt, out + (int64_t)u * G * ORC_D);
+        free(rows);
+    }
+}
