@@ -1,0 +1,213 @@
+/*
+ * ckv.h: C-ABI of the ClusterKV hot path on B200 (sm_100a).
+ *
+ * ClusterKV recalls KV-cache tokens at the granularity of semantic clusters. Sources:
+ *   [EXPL] the ClusterKV explainer page "大模型KV Cache压缩技术：ClusterKV的语义空间优化",
+ *          sections 3.1 (attention, centroid = mean of member keys), 3.2 (16 sink tokens,
+ *          cosine K-means at prefill, incremental clustering every 320 new tokens),
+ *          3.3 (select_clusters), 4.1 (half-precision distance matmul; each cluster's KV
+ *          stored contiguously);
+ *   [ABS]  "ClusterKV: Manipulating LLM KV Cache in Semantic Space for Recallable
+ *          Compression" (arXiv 2412.03213), abstract.
+ *
+ * Conventions for every call:
+ *   - Pointers named "device" are caller-owned CUDA device memory. The library never
+ *     frees caller memory and never keeps a caller pointer past the call.
+ *   - bf16 tensors are passed as `const void*` (IEEE bfloat16, row-major, rows of 128
+ *     elements, 16-byte aligned base). fp32 and int32 tensors are 16-byte aligned too.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Work is enqueued
+ *     asynchronously on it. No call synchronises the host, except ckv_create,
+ *     ckv_destroy, ckv_check_device_error, ckv_export_unit and ckv_import_unit.
+ *   - Return 0 (CKV_OK) on success or a negative CKV_E* code. All arguments are checked on
+ *     the host before anything is enqueued. A call that fails its checks leaves the
+ *     cluster store unchanged. ckv_last_error() gives a one-line reason (per thread).
+ *   - A "unit" is one (layer, sequence b, KV head). All units of a layer share the same
+ *     token counts. Unit u = b * n_kv_heads + h inside a layer.
+ */
+#ifndef CKV_H
+#define CKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define CKV_API __attribute__((visibility("default")))
+#else
+#define CKV_API
+#endif
+
+#define CKV_OK 0
+#define CKV_EINVAL (-1)     /* bad argument (null/misaligned pointer, size out of range) */
+#define CKV_ENOMEM (-2)     /* device allocation failed (ckv_create only) */
+#define CKV_ECUDA (-3)      /* a CUDA runtime call or kernel launch failed */
+#define CKV_ECAPACITY (-4)  /* the cluster store is full (tokens or clusters) */
+#define CKV_ETIMEOUT (-5)   /* a kernel's bounded wait gave up (see ckv_check_device_error) */
+#define CKV_ESTATE (-6)     /* call out of order (e.g. select before prefill) */
+
+#define CKV_HEAD_DIM 128
+#define CKV_MAX_CLUSTERS 4096 /* upper bound of ckv_config.max_clusters */
+#define CKV_MAX_GROUP 8       /* upper bound of n_q_heads / n_kv_heads */
+
+typedef struct ckv_ctx ckv_ctx;
+
+typedef struct ckv_config {
+    int32_t n_layers;      /* layer stores held by the context */
+    int32_t batch;         /* sequences per layer */
+    int32_t n_kv_heads;    /* KV heads per layer */
+    int32_t n_q_heads;     /* query heads; a multiple of n_kv_heads, group <= CKV_MAX_GROUP */
+    int32_t head_dim;      /* must be 128 */
+    int32_t n_sink;        /* uncompressed leading tokens, 16 in [EXPL] 3.2 */
+    int32_t window;        /* tokens per incremental clustering, 320 in [EXPL] 3.2; <= 768 */
+    int32_t new_clusters;  /* clusters made from each window (4) */
+    int32_t iters;         /* Lloyd iterations per clustering run (10) */
+    int32_t max_clusters;  /* capacity in clusters per unit, prefill + incremental */
+    int64_t capacity;      /* capacity in tokens per unit (sinks + clustered + pending) */
+    uint64_t seed;         /* K-means init seed */
+} ckv_config;
+
+/* Fills the defaults above: n_sink 16, window 320, new_clusters 4, iters 10, head_dim
+ * 128, seed 0. Shape fields are zeroed and must be set by the caller. */
+CKV_API int ckv_config_default(ckv_config* cfg);
+
+/* Allocates the cluster stores of all layers (the cluster-contiguous layout of [EXPL]
+ * 4.1) plus one layer's clustering workspace. Synchronous. CKV_ENOMEM if the device
+ * allocation fails. *out receives the context. */
+CKV_API int ckv_create(const ckv_config* cfg, ckv_ctx** out);
+
+/* Frees everything ckv_create allocated. Waits for the device to go idle first. */
+CKV_API int ckv_destroy(ckv_ctx* ctx);
+
+CKV_API const char* ckv_strerror(int code);
+CKV_API const char* ckv_last_error(void);
+
+/* Device bytes held by the context (stores + workspace). */
+CKV_API int64_t ckv_device_bytes(const ckv_ctx* ctx);
+
+/* Prefill clustering of one layer ([EXPL] 3.2; steps: sinks, seeded init, `iters` Lloyd
+ * iterations of cosine assignment on tensor cores and mean update, then the relayout of
+ * K and V into cluster-major order, [EXPL] 4.1).
+ *   K, V : device bf16 [batch, n_kv_heads, n, 128].
+ *   n    : tokens per sequence, n_sink + C <= n <= capacity.
+ *   C    : clusters per unit, 1 <= C <= max_clusters.
+ * Replaces whatever the layer held. Afterwards the layer has m = n - n_sink clustered
+ * tokens and no pending tokens. Uses the context's workspace, so prefill calls on
+ * different streams must not overlap in time. */
+CKV_API int cluster_prefill(ckv_ctx* ctx, int32_t layer, const void* K, const void* V, int64_t n,
+                    int32_t C, void* stream);
+
+/* One decode step of one layer ([EXPL] 3.3 then 3.1), fused in one kernel launch:
+ * qbar = sum of the group's query heads; score every cluster by qbar . mu_c; walk the
+ * clusters by descending score (ties: lower index) taking whole clusters while they fit in
+ * remaining = budget - n_sink - pending; fill the first cluster that does not fit with
+ * its top-`remaining` tokens by qbar . k (ties: lower token id); then attend every query
+ * head of the group over sinks + pending + selected rows: o = softmax(q K^T / sqrt(128)) V.
+ *   q         : device bf16 [batch, n_q_heads, 128]; query head j uses KV head j / group.
+ *   budget    : tokens attended per unit (sinks and pending included), >= n_sink + pending.
+ *   out       : device fp32 [batch, n_q_heads, 128].
+ *   sel_idx   : optional device int32 [batch, n_kv_heads, budget]. Original token ids of
+ *               the selected rows in selection order: sinks, pending, whole clusters by
+ *               descending score (each in store order), then the partial tokens (in store
+ *               order). Entries past the count are -1.
+ *   sel_count : optional device int32 [batch, n_kv_heads] = min(budget, n_total).
+ * Reads the store only, so it can be captured in a CUDA graph. The token counts are read
+ * at call time and baked into a captured launch. */
+CKV_API int select_and_attend(ckv_ctx* ctx, int32_t layer, const void* q, int32_t budget, float* out,
+                      int32_t* sel_idx, int32_t* sel_count, void* stream);
+
+/* Appends one generated token's K/V per unit to the layer's pending rows (the tokens a
+ * later recluster_increment will cluster).
+ *   k, v : device bf16 [batch, n_kv_heads, 128].
+ * CKV_ECAPACITY if the layer already holds `window` pending tokens (call
+ * recluster_increment first) or if the unit capacity would be exceeded. */
+CKV_API int ckv_append_kv(ckv_ctx* ctx, int32_t layer, const void* k, const void* v, void* stream);
+
+/* Incremental clustering of one layer ([EXPL] 3.2, every 320 new tokens): cosine K-means
+ * with `new_clusters` clusters and `iters` iterations on the `window` pending rows of each
+ * unit. The init stream is keyed by (seed, unit, window number). The new clusters, their
+ * centroids and their permuted K/V rows are appended to the store. Existing clusters are
+ * unchanged and the pending rows are emptied.
+ * CKV_ESTATE unless exactly `window` tokens are pending. CKV_ECAPACITY if the store is full.
+ *   mu_trace     : optional device fp32 [units, iters + 1, new_clusters, 128], the centroids
+ *                  before each iteration and after the last (for stage-wise checks).
+ *   assign_trace : optional device int32 [units, iters, window], each iteration's assignment. */
+CKV_API int recluster_increment(ckv_ctx* ctx, int32_t layer, void* stream);
+CKV_API int recluster_increment_traced(ckv_ctx* ctx, int32_t layer, float* mu_trace,
+                               int32_t* assign_trace, void* stream);
+
+typedef struct ckv_layer_info {
+    int64_t n_total;   /* tokens per unit: n_sink + m + pending */
+    int64_t m;         /* clustered tokens per unit */
+    int32_t C;         /* clusters per unit */
+    int32_t pending;   /* tokens appended since the last clustering */
+    int32_t windows;   /* incremental clusterings done since prefill */
+    int32_t prefilled; /* 1 once cluster_prefill (or ckv_import_unit) set the layer */
+} ckv_layer_info;
+
+CKV_API int ckv_get_layer_info(const ckv_ctx* ctx, int32_t layer, ckv_layer_info* out);
+
+/* Copy of one unit's store. Any NULL pointer is skipped. Buffers may be host or device
+ * memory (cudaMemcpyDefault). The call synchronises `stream` before it returns.
+ *   mu      fp32 [C, 128]          offsets int32 [C + 1]        ids int32 [m]
+ *   kp, vp  bf16 [m, 128]          sp_k, sp_v bf16 [n_sink + pending, 128] */
+typedef struct ckv_unit_buffers {
+    float* mu;
+    int32_t* offsets;
+    int32_t* ids;
+    void* kp;
+    void* vp;
+    void* sp_k;
+    void* sp_v;
+} ckv_unit_buffers;
+
+CKV_API int ckv_export_unit(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h,
+                    const ckv_unit_buffers* dst, void* stream);
+
+/* Loads one unit's store from caller buffers (all seven non-NULL; layouts as above),
+ * for decoding over stores built elsewhere. Synchronous, like ckv_export_unit. Sets the layer's counts to (m, C, pending),
+ * which must then agree across the layer's units. Offsets must be non-decreasing from 0
+ * to m, ids must lie in [n_sink, n_total) and ascend inside each cluster (the decode's
+ * lower-id tie rule relies on store order). */
+CKV_API int ckv_import_unit(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h, int64_t m, int32_t C,
+                    int32_t pending, const ckv_unit_buffers* src, void* stream);
+
+/* Reads and clears the device error word. Synchronises `stream`. Returns CKV_OK,
+ * CKV_ETIMEOUT if a kernel's bounded wait gave up, or CKV_EINVAL if a kernel skipped an
+ * out-of-range input (a caller-supplied assignment outside [0, C)). */
+CKV_API int ckv_check_device_error(ckv_ctx* ctx, void* stream);
+
+/* ---- Stage-level K-means calls: the same kernels cluster_prefill runs, exposed so that
+ * each stage can be checked on its own. They run on U units whose keys are rows
+ * [row0, row0 + m) of `keys`, a device bf16 [U, n_rows, 128] tensor. They use the context's
+ * workspace (U <= batch * n_kv_heads, m <= capacity, C <= max_clusters). ---- */
+
+/* Seeded init ([EXPL] 3.2 "K-means", init reading: first C entries of a Fisher-Yates
+ * shuffle of 0..m-1 driven by SplitMix64 with key seed ^ (unit << 32) ^ window,
+ * unit = unit_base + u). Writes init_idx int32 [U, C] (optional), mu fp32 [U, C, 128]
+ * (the chosen keys) and mu_hat bf16 [U, C, 128] = bf16(mu / |mu|). */
+CKV_API int ckv_kmeans_init(ckv_ctx* ctx, const void* keys, int64_t n_rows, int64_t row0, int64_t m,
+                    int32_t U, int32_t C, uint64_t seed, int64_t unit_base, uint64_t window,
+                    int32_t* init_idx, float* mu, void* mu_hat, void* stream);
+
+/* Cosine assignment ([EXPL] 3.2 and 4.1): assign[u, i] = argmax_c keys[u, row0+i] . mu_hat[u, c]
+ * (ties: lower c), as a bf16 tcgen05 contraction with fp32 accumulation in tensor memory.
+ * mu_hat: bf16 [U, C, 128]. assign: int32 [U, m]. */
+CKV_API int ckv_kmeans_assign(ckv_ctx* ctx, const void* keys, int64_t n_rows, int64_t row0, int64_t m,
+                      int32_t U, const void* mu_hat, int32_t C, int32_t* assign, void* stream);
+
+/* Centroid update ([EXPL] 3.1 mean, 4.1 contiguous layout): stable counting sort by
+ * cluster (offsets int32 [U, C + 1], perm int32 [U, m] = member indices in ascending
+ * order per cluster), then mu[u, c] = mean of its members (fp32, summed in perm order),
+ * empty clusters keep mu, and mu_hat = bf16(mu / |mu|). mu: fp32 [U, C, 128], in/out. */
+CKV_API int ckv_kmeans_update(ckv_ctx* ctx, const void* keys, int64_t n_rows, int64_t row0, int64_t m,
+                      int32_t U, const int32_t* assign, int32_t C, float* mu, void* mu_hat,
+                      int32_t* offsets, int32_t* perm, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CKV_H */

@@ -1,0 +1,600 @@
+// C-ABI of the ClusterKV hot path: context, argument checks and orchestration of the
+// kernels. The ABI is declared and documented in include/ckv.h.
+#include <cudaTypedefs.h>
+#include <stdio.h>
+
+#include <mutex>
+#include <string>
+
+#include "ckv_common.cuh"
+#include "ckv_internal.h"
+
+namespace ckv {
+
+static thread_local std::string g_err;
+
+void set_error(const std::string& msg) { g_err = msg; }
+
+int cuda_fail(cudaError_t e, const char* what) {
+    set_error(std::string(what) + ": " + cudaGetErrorString(e));
+    return CKV_ECUDA;
+}
+
+int num_sms_of_current_device() {
+    static int cache[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int v = 0;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        cache[dev] = v > 0 ? v : 148;
+    }
+    return cache[dev];
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+    });
+    return fn;
+}
+
+int encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                   uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1) {
+    auto fn = encode_fn();
+    if (!fn) {
+        set_error("cuTensorMapEncodeTiled is not available from the driver");
+        return CKV_ECUDA;
+    }
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+    cuuint32_t box[3] = {box0, box1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("cuTensorMapEncodeTiled failed (code " + std::to_string((int)r) + ")");
+        return CKV_ECUDA;
+    }
+    return CKV_OK;
+}
+
+}  // namespace ckv
+
+using namespace ckv;
+
+namespace {
+
+bool aligned16(const void* p) { return p != nullptr && ((uintptr_t)p & 15u) == 0; }
+
+int einval(const std::string& m) {
+    set_error(m);
+    return CKV_EINVAL;
+}
+
+int check_ctx(const ckv_ctx* c) {
+    if (!c) return einval("null context");
+    int dev = -1;
+    cudaGetDevice(&dev);
+    if (dev != reinterpret_cast<const Ctx*>(c)->device)
+        return einval("the context's device is not the current device");
+    return CKV_OK;
+}
+
+Ctx* C_(ckv_ctx* c) { return reinterpret_cast<Ctx*>(c); }
+const Ctx* C_(const ckv_ctx* c) { return reinterpret_cast<const Ctx*>(c); }
+
+int check_layer(const Ctx* c, int32_t layer) {
+    if (layer < 0 || layer >= c->cfg.n_layers) return einval("layer out of range");
+    return CKV_OK;
+}
+
+template <class T>
+int dev_alloc(T** p, size_t count, Ctx* c) {
+    const size_t bytes = count * sizeof(T);
+    if (bytes == 0) {
+        *p = nullptr;
+        return CKV_OK;
+    }
+    cudaError_t e = cudaMalloc((void**)p, bytes);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        set_error("cudaMalloc of " + std::to_string(bytes) + " bytes failed");
+        return CKV_ENOMEM;
+    }
+    c->bytes += (int64_t)bytes;
+    return CKV_OK;
+}
+
+void free_all(Ctx* c) {
+    void* ptrs[] = {c->kp, c->vp, c->spk, c->spv, c->ids, c->offsets, c->mu, c->ws.mu_hat,
+                    c->ws.assign, c->ws.best, c->ws.perm, c->ws.chunk, c->ws.part, c->err};
+    for (void* p : ptrs)
+        if (p) cudaFree(p);
+}
+
+}  // namespace
+
+extern "C" {
+
+int ckv_config_default(ckv_config* cfg) {
+    if (!cfg) return einval("null config");
+    *cfg = ckv_config{};
+    cfg->head_dim = CKV_HEAD_DIM;
+    cfg->n_sink = 16;
+    cfg->window = 320;
+    cfg->new_clusters = 4;
+    cfg->iters = 10;
+    cfg->seed = 0;
+    return CKV_OK;
+}
+
+const char* ckv_strerror(int code) {
+    switch (code) {
+        case CKV_OK: return "ok";
+        case CKV_EINVAL: return "invalid argument";
+        case CKV_ENOMEM: return "out of device memory";
+        case CKV_ECUDA: return "CUDA error";
+        case CKV_ECAPACITY: return "cluster store capacity exceeded";
+        case CKV_ETIMEOUT: return "device wait timed out";
+        case CKV_ESTATE: return "call out of order";
+        default: return "unknown error";
+    }
+}
+
+const char* ckv_last_error(void) { return g_err.c_str(); }
+
+int ckv_create(const ckv_config* cfg, ckv_ctx** out) {
+    if (!cfg || !out) return einval("null argument");
+    *out = nullptr;
+    const ckv_config& f = *cfg;
+    if (f.head_dim != CKV_HEAD_DIM) return einval("head_dim must be 128");
+    if (f.n_layers <= 0 || f.batch <= 0 || f.n_kv_heads <= 0 || f.n_q_heads <= 0)
+        return einval("n_layers, batch, n_kv_heads and n_q_heads must be positive");
+    if (f.n_q_heads % f.n_kv_heads != 0) return einval("n_q_heads must be a multiple of n_kv_heads");
+    const int group = f.n_q_heads / f.n_kv_heads;
+    if (group > CKV_MAX_GROUP) return einval("group size above 8");
+    if (f.n_sink < 0 || f.window <= 0 || f.window > 768 || f.new_clusters <= 0 ||
+        f.new_clusters > f.window || f.iters <= 0 || f.iters > 1000)
+        return einval("bad n_sink/window/new_clusters/iters");
+    if (f.max_clusters <= 0 || f.max_clusters > CKV_MAX_CLUSTERS)
+        return einval("max_clusters must be in 1..4096");
+    if (f.capacity <= f.n_sink || f.capacity - f.n_sink > (int64_t)INT32_MAX / 2)
+        return einval("capacity out of range");
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail(cudaGetLastError(), "cudaGetDevice");
+    int major = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (major != 10) return einval("this library targets sm_100a (B200); current device differs");
+
+    Ctx* c = new Ctx();
+    c->cfg = f;
+    c->units = f.batch * f.n_kv_heads;
+    c->group = group;
+    c->cap_c = f.capacity - f.n_sink;
+    c->sp_rows = f.n_sink + f.window;
+    c->device = dev;
+    c->num_sms = num_sms_of_current_device();
+    c->layers.assign((size_t)f.n_layers, LayerState{});
+    const int64_t LU = (int64_t)f.n_layers * c->units;
+    const int64_t U = c->units;
+    const int64_t cmax = f.max_clusters;
+    int rc = CKV_OK;
+    rc = rc ? rc : dev_alloc(&c->kp, (size_t)(LU * c->cap_c * kD), c);
+    rc = rc ? rc : dev_alloc(&c->vp, (size_t)(LU * c->cap_c * kD), c);
+    rc = rc ? rc : dev_alloc(&c->spk, (size_t)(LU * c->sp_rows * kD), c);
+    rc = rc ? rc : dev_alloc(&c->spv, (size_t)(LU * c->sp_rows * kD), c);
+    rc = rc ? rc : dev_alloc(&c->ids, (size_t)(LU * c->cap_c), c);
+    rc = rc ? rc : dev_alloc(&c->offsets, (size_t)(LU * (cmax + 1)), c);
+    rc = rc ? rc : dev_alloc(&c->mu, (size_t)(LU * cmax * kD), c);
+    rc = rc ? rc : dev_alloc(&c->ws.mu_hat, (size_t)(U * cmax * kD), c);
+    rc = rc ? rc : dev_alloc(&c->ws.assign, (size_t)(U * c->cap_c), c);
+    rc = rc ? rc : dev_alloc(&c->ws.best, (size_t)(U * c->cap_c), c);
+    rc = rc ? rc : dev_alloc(&c->ws.perm, (size_t)(U * c->cap_c), c);
+    rc = rc ? rc : dev_alloc(&c->ws.chunk, (size_t)(U * n_chunks(c->cap_c) * cmax), c);
+    rc = rc ? rc : dev_alloc(&c->ws.part, (size_t)(U * c->cap_c), c);
+    rc = rc ? rc : dev_alloc(&c->err, 4, c);
+    if (rc == CKV_OK) {
+        cudaError_t e = cudaMemset(c->err, 0, 16);
+        if (e == cudaSuccess) e = cudaMemset(c->offsets, 0, sizeof(int32_t) * LU * (cmax + 1));
+        if (e == cudaSuccess) e = cudaDeviceSynchronize();
+        if (e != cudaSuccess) rc = cuda_fail(e, "create: memset");
+    }
+    if (rc != CKV_OK) {
+        free_all(c);
+        delete c;
+        return rc;
+    }
+    c->ws.U = c->units;
+    c->ws.cap = c->cap_c;
+    c->ws.cmax = f.max_clusters;
+    *out = reinterpret_cast<ckv_ctx*>(c);
+    return CKV_OK;
+}
+
+int ckv_destroy(ckv_ctx* ctx) {
+    if (!ctx) return CKV_OK;
+    Ctx* c = C_(ctx);
+    int cur = 0;
+    cudaGetDevice(&cur);
+    cudaSetDevice(c->device);
+    cudaDeviceSynchronize();
+    free_all(c);
+    cudaSetDevice(cur);
+    delete c;
+    return CKV_OK;
+}
+
+int64_t ckv_device_bytes(const ckv_ctx* ctx) { return ctx ? C_(ctx)->bytes : 0; }
+
+int cluster_prefill(ckv_ctx* ctx, int32_t layer, const void* K, const void* V, int64_t n,
+                    int32_t C, void* stream) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    Ctx* c = C_(ctx);
+    if ((rc = check_layer(c, layer))) return rc;
+    if (!aligned16(K) || !aligned16(V)) return einval("K and V must be non-null and 16-byte aligned");
+    const int32_t ns = c->cfg.n_sink;
+    if (n > c->cfg.capacity) {
+        set_error("n exceeds the context capacity");
+        return CKV_ECAPACITY;
+    }
+    if (C < 1 || C > c->cfg.max_clusters) return einval("C must be in 1..max_clusters");
+    if (n - ns < C) return einval("need n - n_sink >= C");
+    cudaStream_t s = (cudaStream_t)stream;
+    const int32_t U = c->units;
+    const int64_t cmax = c->cfg.max_clusters;
+    KeysView kv{(const uint16_t*)K, n, ns, n - ns, U};
+    float* mu = c->mu + c->mu_rows(layer, 0) * kD;
+    int32_t* offs = c->offsets + c->off_base(layer, 0);
+    rc = launch_kmeans_init(kv, C, c->cfg.seed, (int64_t)layer * U, 0, nullptr, mu, cmax,
+                            c->ws.mu_hat, cmax, c->err, s);
+    if (rc) return rc;
+    Relayout rl;
+    rl.V = (const uint16_t*)V;
+    rl.kp = c->kp + c->rows_kp(layer, 0) * kD;
+    rl.vp = c->vp + c->rows_kp(layer, 0) * kD;
+    rl.ids = c->ids + c->rows_kp(layer, 0);
+    rl.ustride_rows = c->cap_c;
+    rl.id_base = ns;
+    for (int it = 0; it < c->cfg.iters; ++it) {
+        rc = launch_kmeans_assign(kv, c->ws.mu_hat, cmax, C, c->ws.assign, c->cap_c, c->ws.best,
+                                  c->cap_c, c->err, s);
+        if (rc) return rc;
+        const bool last = it + 1 == c->cfg.iters;
+        rc = launch_kmeans_update(kv, c->ws.assign, c->cap_c, C, mu, cmax, c->ws.mu_hat, cmax,
+                                  offs, cmax + 1, c->ws.perm, c->cap_c, c->ws.chunk,
+                                  last ? &rl : nullptr, c->err, s);
+        if (rc) return rc;
+    }
+    if (ns > 0) {
+        rc = launch_copy_sinks((const uint16_t*)K, (const uint16_t*)V, n, U, ns,
+                               c->spk + c->rows_sp(layer, 0) * kD,
+                               c->spv + c->rows_sp(layer, 0) * kD, c->sp_rows, s);
+        if (rc) return rc;
+    }
+    LayerState& L = c->layers[(size_t)layer];
+    L.prefilled = 1;
+    L.m = n - ns;
+    L.C = C;
+    L.pending = 0;
+    L.windows = 0;
+    return CKV_OK;
+}
+
+int select_and_attend(ckv_ctx* ctx, int32_t layer, const void* q, int32_t budget, float* out,
+                      int32_t* sel_idx, int32_t* sel_count, void* stream) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    Ctx* c = C_(ctx);
+    if ((rc = check_layer(c, layer))) return rc;
+    const LayerState& L = c->layers[(size_t)layer];
+    if (!L.prefilled) {
+        set_error("select_and_attend before cluster_prefill for this layer");
+        return CKV_ESTATE;
+    }
+    if (!aligned16(q) || !aligned16(out)) return einval("q and out must be non-null and 16-byte aligned");
+    if ((sel_idx && ((uintptr_t)sel_idx & 3u)) || (sel_count && ((uintptr_t)sel_count & 3u)))
+        return einval("sel_idx / sel_count must be 4-byte aligned");
+    if (budget < 1 || (int64_t)budget < (int64_t)c->cfg.n_sink + L.pending)
+        return einval("budget must be >= n_sink + pending and >= 1");
+    DecodeArgs a{};
+    a.q = (const uint16_t*)q;
+    a.out = out;
+    a.sel_idx = sel_idx;
+    a.sel_count = sel_count;
+    a.budget = budget;
+    a.B = c->cfg.batch;
+    a.Hkv = c->cfg.n_kv_heads;
+    a.G = c->group;
+    a.n_sink = c->cfg.n_sink;
+    a.pending = L.pending;
+    a.C = L.C;
+    a.m = L.m;
+    a.kp = c->kp + c->rows_kp(layer, 0) * kD;
+    a.vp = c->vp + c->rows_kp(layer, 0) * kD;
+    a.spk = c->spk + c->rows_sp(layer, 0) * kD;
+    a.spv = c->spv + c->rows_sp(layer, 0) * kD;
+    a.ids = c->ids + c->rows_kp(layer, 0);
+    a.offsets = c->offsets + c->off_base(layer, 0);
+    a.mu = c->mu + c->mu_rows(layer, 0) * kD;
+    a.kp_ustride = c->cap_c;
+    a.sp_ustride = c->sp_rows;
+    a.off_ustride = c->cfg.max_clusters + 1;
+    a.mu_ustride = c->cfg.max_clusters;
+    a.part_scratch = c->ws.part;
+    a.part_ustride = c->cap_c;
+    a.err = c->err;
+    return launch_select_attend(a, c->num_sms, (cudaStream_t)stream);
+}
+
+int ckv_append_kv(ckv_ctx* ctx, int32_t layer, const void* k, const void* v, void* stream) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    Ctx* c = C_(ctx);
+    if ((rc = check_layer(c, layer))) return rc;
+    LayerState& L = c->layers[(size_t)layer];
+    if (!L.prefilled) {
+        set_error("append before cluster_prefill for this layer");
+        return CKV_ESTATE;
+    }
+    if (!aligned16(k) || !aligned16(v)) return einval("k and v must be non-null and 16-byte aligned");
+    if (L.pending >= c->cfg.window) {
+        set_error("pending window is full; call recluster_increment first");
+        return CKV_ECAPACITY;
+    }
+    if ((int64_t)c->cfg.n_sink + L.m + L.pending + 1 > c->cfg.capacity) {
+        set_error("unit capacity exceeded");
+        return CKV_ECAPACITY;
+    }
+    rc = launch_append((const uint16_t*)k, (const uint16_t*)v, c->units,
+                       c->spk + c->rows_sp(layer, 0) * kD, c->spv + c->rows_sp(layer, 0) * kD,
+                       c->sp_rows, c->cfg.n_sink + L.pending, (cudaStream_t)stream);
+    if (rc) return rc;
+    L.pending += 1;
+    return CKV_OK;
+}
+
+int recluster_increment_traced(ckv_ctx* ctx, int32_t layer, float* mu_trace,
+                               int32_t* assign_trace, void* stream) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    Ctx* c = C_(ctx);
+    if ((rc = check_layer(c, layer))) return rc;
+    LayerState& L = c->layers[(size_t)layer];
+    if (!L.prefilled || L.pending != c->cfg.window) {
+        set_error("recluster_increment needs exactly `window` pending tokens");
+        return CKV_ESTATE;
+    }
+    if (L.m + c->cfg.window > c->cap_c || L.C + c->cfg.new_clusters > c->cfg.max_clusters) {
+        set_error("cluster store full (tokens or clusters)");
+        return CKV_ECAPACITY;
+    }
+    if ((mu_trace && ((uintptr_t)mu_trace & 15u)) || (assign_trace && ((uintptr_t)assign_trace & 3u)))
+        return einval("misaligned trace buffer");
+    ReclusterArgs a{};
+    a.U = c->units;
+    a.n_sink = c->cfg.n_sink;
+    a.window = c->cfg.window;
+    a.C_new = c->cfg.new_clusters;
+    a.iters = c->cfg.iters;
+    a.C_old = L.C;
+    a.m_old = L.m;
+    a.seed = c->cfg.seed;
+    a.unit_base = (int64_t)layer * c->units;
+    a.window_no = (uint64_t)L.windows + 1;
+    a.spk = c->spk + c->rows_sp(layer, 0) * kD;
+    a.spv = c->spv + c->rows_sp(layer, 0) * kD;
+    a.sp_ustride = c->sp_rows;
+    a.kp = c->kp + c->rows_kp(layer, 0) * kD;
+    a.vp = c->vp + c->rows_kp(layer, 0) * kD;
+    a.ids = c->ids + c->rows_kp(layer, 0);
+    a.kp_ustride = c->cap_c;
+    a.offsets = c->offsets + c->off_base(layer, 0);
+    a.off_ustride = c->cfg.max_clusters + 1;
+    a.mu = c->mu + c->mu_rows(layer, 0) * kD;
+    a.mu_ustride = c->cfg.max_clusters;
+    a.mu_trace = mu_trace;
+    a.assign_trace = assign_trace;
+    rc = launch_recluster(a, (cudaStream_t)stream);
+    if (rc) return rc;
+    L.m += c->cfg.window;
+    L.C += c->cfg.new_clusters;
+    L.pending = 0;
+    L.windows += 1;
+    return CKV_OK;
+}
+
+int recluster_increment(ckv_ctx* ctx, int32_t layer, void* stream) {
+    return recluster_increment_traced(ctx, layer, nullptr, nullptr, stream);
+}
+
+int ckv_get_layer_info(const ckv_ctx* ctx, int32_t layer, ckv_layer_info* out) {
+    if (!ctx || !out) return einval("null argument");
+    const Ctx* c = C_(ctx);
+    int rc = check_layer(c, layer);
+    if (rc) return rc;
+    const LayerState& L = c->layers[(size_t)layer];
+    out->m = L.m;
+    out->C = L.C;
+    out->pending = L.pending;
+    out->windows = L.windows;
+    out->prefilled = L.prefilled;
+    out->n_total = L.prefilled ? c->cfg.n_sink + L.m + L.pending : 0;
+    return CKV_OK;
+}
+
+int ckv_export_unit(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h,
+                    const ckv_unit_buffers* dst, void* stream) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    Ctx* c = C_(ctx);
+    if ((rc = check_layer(c, layer))) return rc;
+    if (!dst) return einval("null buffers");
+    if (b < 0 || b >= c->cfg.batch || h < 0 || h >= c->cfg.n_kv_heads) return einval("unit out of range");
+    const LayerState& L = c->layers[(size_t)layer];
+    if (!L.prefilled) {
+        set_error("layer not prefilled");
+        return CKV_ESTATE;
+    }
+    const int u = b * c->cfg.n_kv_heads + h;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t sp = c->cfg.n_sink + L.pending;
+    struct Item { void* d; const void* s; size_t n; } items[] = {
+        {dst->mu, c->mu + c->mu_rows(layer, u) * kD, sizeof(float) * L.C * kD},
+        {dst->offsets, c->offsets + c->off_base(layer, u), sizeof(int32_t) * (L.C + 1)},
+        {dst->ids, c->ids + c->rows_kp(layer, u), sizeof(int32_t) * L.m},
+        {dst->kp, c->kp + c->rows_kp(layer, u) * kD, 2 * L.m * kD},
+        {dst->vp, c->vp + c->rows_kp(layer, u) * kD, 2 * L.m * kD},
+        {dst->sp_k, c->spk + c->rows_sp(layer, u) * kD, (size_t)(2 * sp * kD)},
+        {dst->sp_v, c->spv + c->rows_sp(layer, u) * kD, (size_t)(2 * sp * kD)},
+    };
+    for (auto& it : items) {
+        if (!it.d || it.n == 0) continue;
+        cudaError_t e = cudaMemcpyAsync(it.d, it.s, it.n, cudaMemcpyDefault, s);
+        if (e != cudaSuccess) return cuda_fail(e, "export: copy");
+    }
+    cudaError_t e = cudaStreamSynchronize(s);
+    return e == cudaSuccess ? CKV_OK : cuda_fail(e, "export: sync");
+}
+
+int ckv_import_unit(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h, int64_t m, int32_t C,
+                    int32_t pending, const ckv_unit_buffers* src, void* stream) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    Ctx* c = C_(ctx);
+    if ((rc = check_layer(c, layer))) return rc;
+    if (!src || !src->mu || !src->offsets || !src->ids || !src->kp || !src->vp || !src->sp_k || !src->sp_v)
+        return einval("all seven buffers are required");
+    if (b < 0 || b >= c->cfg.batch || h < 0 || h >= c->cfg.n_kv_heads) return einval("unit out of range");
+    if (m < 0 || m > c->cap_c || C < 1 || C > c->cfg.max_clusters || pending < 0 ||
+        pending > c->cfg.window || c->cfg.n_sink + m + pending > c->cfg.capacity)
+        return einval("import sizes out of range");
+    LayerState& L = c->layers[(size_t)layer];
+    const bool first = !L.prefilled || (L.m != m || L.C != C || L.pending != pending);
+    cudaStream_t s = (cudaStream_t)stream;
+    // content checks on a host copy of offsets and ids
+    std::vector<int32_t> off((size_t)C + 1), ids((size_t)m);
+    cudaError_t e = cudaMemcpy(off.data(), src->offsets, sizeof(int32_t) * (C + 1), cudaMemcpyDefault);
+    if (e == cudaSuccess && m > 0) e = cudaMemcpy(ids.data(), src->ids, sizeof(int32_t) * m, cudaMemcpyDefault);
+    if (e != cudaSuccess) return cuda_fail(e, "import: read offsets/ids");
+    if (off[0] != 0 || off[(size_t)C] != m) return einval("offsets must run from 0 to m");
+    for (int32_t i = 0; i < C; ++i) {
+        if (off[(size_t)i + 1] < off[(size_t)i]) return einval("offsets must be non-decreasing");
+        for (int32_t j = off[(size_t)i] + 1; j < off[(size_t)i + 1]; ++j)
+            if (ids[(size_t)j] <= ids[(size_t)j - 1])
+                return einval("ids must ascend inside each cluster (the lower-id tie rule)");
+    }
+    const int64_t n_total = c->cfg.n_sink + m + pending;
+    for (int64_t i = 0; i < m; ++i)
+        if (ids[(size_t)i] < c->cfg.n_sink || ids[(size_t)i] >= n_total) return einval("id out of range");
+    const int u = b * c->cfg.n_kv_heads + h;
+    const int64_t sp = c->cfg.n_sink + pending;
+    struct Item { void* d; const void* s; size_t n; } items[] = {
+        {c->mu + c->mu_rows(layer, u) * kD, src->mu, sizeof(float) * C * kD},
+        {c->offsets + c->off_base(layer, u), src->offsets, sizeof(int32_t) * (C + 1)},
+        {c->ids + c->rows_kp(layer, u), src->ids, sizeof(int32_t) * m},
+        {c->kp + c->rows_kp(layer, u) * kD, src->kp, (size_t)(2 * m * kD)},
+        {c->vp + c->rows_kp(layer, u) * kD, src->vp, (size_t)(2 * m * kD)},
+        {c->spk + c->rows_sp(layer, u) * kD, src->sp_k, (size_t)(2 * sp * kD)},
+        {c->spv + c->rows_sp(layer, u) * kD, src->sp_v, (size_t)(2 * sp * kD)},
+    };
+    for (auto& it : items) {
+        if (it.n == 0) continue;
+        e = cudaMemcpyAsync(it.d, it.s, it.n, cudaMemcpyDefault, s);
+        if (e != cudaSuccess) return cuda_fail(e, "import: copy");
+    }
+    e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "import: sync");
+    if (first) {
+        L.prefilled = 1;
+        L.m = m;
+        L.C = C;
+        L.pending = pending;
+        L.windows = 0;
+    }
+    return CKV_OK;
+}
+
+int ckv_check_device_error(ckv_ctx* ctx, void* stream) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    Ctx* c = C_(ctx);
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "check: sync");
+    uint32_t w = 0;
+    e = cudaMemcpy(&w, c->err, 4, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemset(c->err, 0, 4);
+    if (e != cudaSuccess) return cuda_fail(e, "check: read error word");
+    if (w & kErrTimeout) {
+        set_error("a kernel wait timed out on the device (error word " + std::to_string(w) + ")");
+        return CKV_ETIMEOUT;
+    }
+    if (w) {
+        set_error("a kernel saw an out-of-range input and skipped it (error word " +
+                  std::to_string(w) + ")");
+        return CKV_EINVAL;
+    }
+    return CKV_OK;
+}
+
+static int check_stage(const Ctx* c, const void* keys, int64_t n_rows, int64_t row0, int64_t m,
+                       int32_t U, int32_t C) {
+    if (!aligned16(keys)) return einval("keys must be non-null and 16-byte aligned");
+    if (U < 1 || U > c->units) return einval("U must be in 1..batch*n_kv_heads");
+    if (m < 1 || m > c->cap_c) return einval("m out of range");
+    if (row0 < 0 || row0 + m > n_rows) return einval("rows [row0, row0+m) exceed n_rows");
+    if (C < 1 || C > c->cfg.max_clusters || C > m) return einval("C must be in 1..min(max_clusters, m)");
+    return CKV_OK;
+}
+
+int ckv_kmeans_init(ckv_ctx* ctx, const void* keys, int64_t n_rows, int64_t row0, int64_t m,
+                    int32_t U, int32_t C, uint64_t seed, int64_t unit_base, uint64_t window,
+                    int32_t* init_idx, float* mu, void* mu_hat, void* stream) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    Ctx* c = C_(ctx);
+    if ((rc = check_stage(c, keys, n_rows, row0, m, U, C))) return rc;
+    if (!aligned16(mu) || !aligned16(mu_hat)) return einval("mu and mu_hat must be 16-byte aligned");
+    KeysView kv{(const uint16_t*)keys, n_rows, row0, m, U};
+    return launch_kmeans_init(kv, C, seed, unit_base, window, init_idx, mu, C, (uint16_t*)mu_hat, C,
+                              c->err, (cudaStream_t)stream);
+}
+
+int ckv_kmeans_assign(ckv_ctx* ctx, const void* keys, int64_t n_rows, int64_t row0, int64_t m,
+                      int32_t U, const void* mu_hat, int32_t C, int32_t* assign, void* stream) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    Ctx* c = C_(ctx);
+    if ((rc = check_stage(c, keys, n_rows, row0, m, U, C))) return rc;
+    if (!aligned16(mu_hat) || !assign) return einval("mu_hat must be 16-byte aligned; assign non-null");
+    KeysView kv{(const uint16_t*)keys, n_rows, row0, m, U};
+    return launch_kmeans_assign(kv, (const uint16_t*)mu_hat, C, C, assign, m, c->ws.best, c->cap_c,
+                                c->err, (cudaStream_t)stream);
+}
+
+int ckv_kmeans_update(ckv_ctx* ctx, const void* keys, int64_t n_rows, int64_t row0, int64_t m,
+                      int32_t U, const int32_t* assign, int32_t C, float* mu, void* mu_hat,
+                      int32_t* offsets, int32_t* perm, void* stream) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    Ctx* c = C_(ctx);
+    if ((rc = check_stage(c, keys, n_rows, row0, m, U, C))) return rc;
+    if (!assign || !aligned16(mu) || !aligned16(mu_hat) || !offsets || !perm)
+        return einval("null or misaligned output");
+    KeysView kv{(const uint16_t*)keys, n_rows, row0, m, U};
+    return launch_kmeans_update(kv, assign, m, C, mu, C, (uint16_t*)mu_hat, C, offsets, C + 1, perm,
+                                m, c->ws.chunk, nullptr, c->err, (cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,169 @@
+// Host-side internals shared by the library's translation units: the context object and
+// the kernel launchers. Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "ckv.h"
+
+namespace ckv {
+
+struct LayerState {
+    int prefilled = 0;
+    int64_t m = 0;
+    int32_t C = 0;
+    int32_t pending = 0;
+    int32_t windows = 0;
+};
+
+// Keys of U units: rows [row0, row0 + m) of a [U, n_rows, 128] bf16 tensor.
+struct KeysView {
+    const uint16_t* base;
+    int64_t n_rows;
+    int64_t row0;
+    int64_t m;
+    int32_t U;
+};
+
+struct Workspace {
+    uint16_t* mu_hat = nullptr;  // [U][Cmax][128]
+    int32_t* assign = nullptr;   // [U][cap_c]
+    float* best = nullptr;       // [U][cap_c]
+    int32_t* perm = nullptr;     // [U][cap_c]
+    int32_t* chunk = nullptr;    // [U][n_chunks(cap_c)][Cmax]
+    float* part = nullptr;       // decode partial-cut scratch [U][cap_c] (keys of the cut cluster)
+    int32_t U = 0;
+    int64_t cap = 0;
+    int32_t cmax = 0;
+};
+
+struct Ctx {
+    ckv_config cfg{};
+    int32_t units = 0;   // batch * n_kv_heads
+    int32_t group = 0;   // n_q_heads / n_kv_heads
+    int64_t cap_c = 0;   // clustered-row capacity per unit
+    int32_t sp_rows = 0; // n_sink + window
+    int device = 0;
+    int num_sms = 0;
+    // Stores of all layers, [L][U][...].
+    uint16_t* kp = nullptr;
+    uint16_t* vp = nullptr;
+    uint16_t* spk = nullptr;
+    uint16_t* spv = nullptr;
+    int32_t* ids = nullptr;
+    int32_t* offsets = nullptr;
+    float* mu = nullptr;
+    Workspace ws;
+    uint32_t* err = nullptr;  // device error word
+    std::vector<LayerState> layers;
+    int64_t bytes = 0;
+
+    int64_t rows_kp(int layer, int u) const { return ((int64_t)layer * units + u) * cap_c; }
+    int64_t rows_sp(int layer, int u) const { return ((int64_t)layer * units + u) * sp_rows; }
+    int64_t off_base(int layer, int u) const {
+        return ((int64_t)layer * units + u) * (cfg.max_clusters + 1);
+    }
+    int64_t mu_rows(int layer, int u) const {
+        return ((int64_t)layer * units + u) * cfg.max_clusters;
+    }
+};
+
+void set_error(const std::string& msg);
+int cuda_fail(cudaError_t e, const char* what);
+
+constexpr int kD = 128;       // head dim
+constexpr int kChunk = 1024;  // keys per counting-sort chunk
+inline int64_t n_chunks(int64_t m) { return (m + kChunk - 1) / kChunk; }
+
+// Tensor-map encoder from the driver, fetched through the runtime (no libcuda link).
+int encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                   uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1);
+
+int num_sms_of_current_device();
+
+// ---- launchers (each returns CKV_OK or an error code; all asynchronous on `stream`)
+int launch_kmeans_init(const KeysView& k, int32_t C, uint64_t seed, int64_t unit_base,
+                       uint64_t window, int32_t* init_idx, float* mu, int64_t mu_ustride,
+                       uint16_t* mu_hat, int64_t muhat_ustride, uint32_t* err, cudaStream_t s);
+
+int launch_kmeans_assign(const KeysView& k, const uint16_t* mu_hat, int64_t muhat_ustride,
+                         int32_t C, int32_t* assign, int64_t assign_ustride, float* best,
+                         int64_t best_ustride, uint32_t* err, cudaStream_t s);
+
+struct Relayout {  // final-iteration relayout of K and V into the cluster-major store
+    const uint16_t* V = nullptr;  // same shape as the keys tensor
+    uint16_t* kp = nullptr;
+    uint16_t* vp = nullptr;
+    int32_t* ids = nullptr;
+    int64_t ustride_rows = 0;  // rows between units in kp/vp/ids
+    int32_t id_base = 0;       // original id of local key 0
+};
+
+int launch_kmeans_update(const KeysView& k, const int32_t* assign, int64_t assign_ustride,
+                         int32_t C, float* mu, int64_t mu_ustride, uint16_t* mu_hat,
+                         int64_t muhat_ustride, int32_t* offsets, int64_t off_ustride,
+                         int32_t* perm, int64_t perm_ustride, int32_t* chunk_ws,
+                         const Relayout* relayout, uint32_t* err, cudaStream_t s);
+
+int launch_copy_sinks(const uint16_t* K, const uint16_t* V, int64_t n, int32_t U, int32_t n_sink,
+                      uint16_t* spk, uint16_t* spv, int64_t sp_ustride_rows, cudaStream_t s);
+
+struct DecodeArgs {
+    const uint16_t* q;
+    float* out;
+    int32_t* sel_idx;
+    int32_t* sel_count;
+    int32_t budget;
+    int32_t B, Hkv, G;
+    int32_t n_sink, pending, C;
+    int64_t m;
+    const uint16_t* kp;
+    const uint16_t* vp;
+    const uint16_t* spk;
+    const uint16_t* spv;
+    const int32_t* ids;
+    const int32_t* offsets;
+    const float* mu;
+    int64_t kp_ustride;   // rows
+    int64_t sp_ustride;   // rows
+    int64_t off_ustride;  // ints
+    int64_t mu_ustride;   // rows of 128
+    float* part_scratch;  // [U][cap]
+    int64_t part_ustride;
+    uint32_t* err;
+};
+int launch_select_attend(const DecodeArgs& a, int num_sms, cudaStream_t s);
+
+int launch_append(const uint16_t* k, const uint16_t* v, int32_t U, uint16_t* spk, uint16_t* spv,
+                  int64_t sp_ustride_rows, int32_t row, cudaStream_t s);
+
+struct ReclusterArgs {
+    int32_t U;
+    int32_t n_sink, window, C_new, iters;
+    int32_t C_old;
+    int64_t m_old;
+    uint64_t seed;
+    int64_t unit_base;
+    uint64_t window_no;
+    uint16_t* spk;
+    uint16_t* spv;
+    int64_t sp_ustride;
+    uint16_t* kp;
+    uint16_t* vp;
+    int32_t* ids;
+    int64_t kp_ustride;
+    int32_t* offsets;
+    int64_t off_ustride;
+    float* mu;
+    int64_t mu_ustride;
+    float* mu_trace;
+    int32_t* assign_trace;
+};
+int launch_recluster(const ReclusterArgs& a, cudaStream_t s);
+
+}  // namespace ckv

@@ -1,0 +1,363 @@
+// K-means init and centroid update for ClusterKV prefill clustering (sm_100a, CUDA cores).
+//
+// Page: "大模型KV Cache压缩技术：ClusterKV的语义空间优化" (ClusterKV explainer).
+//  - section 3.1: a cluster's centroid is the mean of its member keys, mu = (1/n) sum k_i;
+//  - section 3.2: K-means over the non-sink keys (seeded; init reading below);
+//  - section 4.1: each cluster's KV is stored contiguously. The update therefore builds
+//    the cluster-major layout with a stable counting sort (histogram -> exclusive scan ->
+//    scatter), and the mean is a segmented reduction that reads the keys in that order.
+//    The last iteration also writes the permuted K and V rows into the cluster store.
+//
+// Determinism: integer counts only (no float atomics). Each centroid is summed by one
+// warp in a fixed order (ascending key index within the cluster), so runs are
+// bit-reproducible.
+#include "ckv_common.cuh"
+#include "ckv_internal.h"
+
+namespace ckv {
+namespace {
+
+// Writes mu (fp32) and mu_hat = bf16_rn(mu / |mu|) for one centroid. The calling warp holds
+// dims 4*lane .. 4*lane+3 in `v`. A zero centroid gives mu_hat = 0.
+CKV_DEV void store_centroid(float4 v, float* mu_row, uint16_t* muhat_row) {
+    const int lane = lane_id();
+    float ss = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float nrm = __fsqrt_rn(ss);
+    reinterpret_cast<float4*>(mu_row)[lane] = v;
+    uint2 h = make_uint2(0u, 0u);
+    if (nrm > 0.f) {
+        const __nv_bfloat16 a = __float2bfloat16_rn(__fdiv_rn(v.x, nrm));
+        const __nv_bfloat16 b = __float2bfloat16_rn(__fdiv_rn(v.y, nrm));
+        const __nv_bfloat16 c = __float2bfloat16_rn(__fdiv_rn(v.z, nrm));
+        const __nv_bfloat16 d = __float2bfloat16_rn(__fdiv_rn(v.w, nrm));
+        h.x = (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
+        h.y = (uint32_t)__bfloat16_as_ushort(c) | ((uint32_t)__bfloat16_as_ushort(d) << 16);
+    }
+    reinterpret_cast<uint2*>(muhat_row)[lane] = h;
+}
+
+CKV_DEV float4 load_row4_bf16(const uint16_t* row) {
+    const uint2 w = reinterpret_cast<const uint2*>(row)[lane_id()];
+    return make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
+}
+
+// ---------------------------------------------------------------------- init
+// Seeded init: the first C entries of a Fisher-Yates shuffle of 0..m-1, driven by SplitMix64
+// with key seed ^ (unit << 32) ^ window, each draw mapped into [0, m-i) by Lemire's
+// multiply-shift. Only the <= C displaced positions of the virtual array are stored, in a
+// shared-memory open-addressing table.
+__global__ void __launch_bounds__(256) kmeans_init_kernel(KeysView k, int32_t C, uint64_t seed,
+                                                          int64_t unit_base, uint64_t window,
+                                                          int32_t* init_idx, float* mu,
+                                                          int64_t mu_ustride, uint16_t* mu_hat,
+                                                          int64_t muhat_ustride, int32_t tbits) {
+    extern __shared__ int32_t sm[];
+    const int32_t tsize = 1 << tbits;
+    int32_t* tkey = sm;
+    int32_t* tval = sm + tsize;
+    int32_t* chosen = sm + 2 * tsize;
+    const int u = blockIdx.x;
+    for (int i = threadIdx.x; i < tsize; i += blockDim.x) tkey[i] = -1;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint64_t state = seed ^ ((uint64_t)(unit_base + u) << 32) ^ window;
+        auto slot = [&](int32_t pos) -> int32_t {
+            uint32_t hsh = ((uint32_t)pos * 2654435761u) >> (32 - tbits);
+            while (tkey[hsh] != -1 && tkey[hsh] != pos) hsh = (hsh + 1) & (uint32_t)(tsize - 1);
+            return (int32_t)hsh;
+        };
+        for (int32_t i = 0; i < C; ++i) {
+            const uint64_t x = splitmix64_next(state);
+            const int32_t j = i + (int32_t)bounded_draw(x, (uint32_t)(k.m - i));
+            const int32_t si = slot(i);
+            const int32_t vi = tkey[si] == i ? tval[si] : i;
+            const int32_t sj = slot(j);
+            const int32_t vj = tkey[sj] == j ? tval[sj] : j;
+            // a[i] <- a[j] (position i is never read again), a[j] <- old a[i]
+            tkey[sj] = j;
+            tval[sj] = vi;
+            chosen[i] = vj;
+        }
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const uint16_t* keys = k.base + ((int64_t)u * k.n_rows + k.row0) * kD;
+    for (int c = warp; c < C; c += nw) {
+        const int32_t idx = chosen[c];
+        const float4 v = load_row4_bf16(keys + (int64_t)idx * kD);
+        store_centroid(v, mu + ((int64_t)u * mu_ustride + c) * kD,
+                       mu_hat + ((int64_t)u * muhat_ustride + c) * kD);
+        if (init_idx && lane_id() == 0) init_idx[(int64_t)u * C + c] = idx;
+    }
+}
+
+// ---------------------------------------------------------------------- count
+// chunk[u][ch][c] = number of keys of chunk ch (kChunk keys) assigned to c.
+__global__ void __launch_bounds__(256) kmeans_count_kernel(const int32_t* assign, int64_t a_ustride,
+                                                           int64_t m, int32_t C, int32_t nch,
+                                                           int32_t* chunk, uint32_t* err) {
+    extern __shared__ int32_t hist[];
+    const int ch = blockIdx.x, u = blockIdx.y;
+    for (int c = threadIdx.x; c < C; c += blockDim.x) hist[c] = 0;
+    __syncthreads();
+    const int64_t lo = (int64_t)ch * kChunk;
+    const int64_t hi = lo + kChunk < m ? lo + kChunk : m;
+    const int32_t* a = assign + (int64_t)u * a_ustride;
+    for (int64_t i = lo + threadIdx.x; i < hi; i += blockDim.x) {
+        const int32_t c = a[i];
+        if ((uint32_t)c < (uint32_t)C) {
+            atomicAdd(&hist[c], 1);
+        } else if (err) {
+            atomicOr(err, kErrBadState);  // caller-supplied assignment out of range: skipped
+        }
+    }
+    __syncthreads();
+    int32_t* out = chunk + ((int64_t)u * nch + ch) * C;
+    for (int c = threadIdx.x; c < C; c += blockDim.x) out[c] = hist[c];
+}
+
+// ---------------------------------------------------------------------- scan
+// Per unit: sizes[c] = sum over chunks; offsets = exclusive scan of sizes (offsets[C] = m);
+// chunk[u][ch][c] becomes the number of keys of cluster c in chunks before ch.
+__global__ void __launch_bounds__(1024) kmeans_scan_kernel(int32_t* chunk, int32_t nch, int32_t C,
+                                                           int64_t m, int32_t* offsets,
+                                                           int64_t off_ustride) {
+    extern __shared__ int32_t sz[];  // [C] then [32] warp totals
+    int32_t* wsum = sz + C;
+    const int u = blockIdx.x;
+    int32_t* ck = chunk + (int64_t)u * nch * C;
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+        int32_t run = 0;
+        for (int ch = 0; ch < nch; ++ch) {
+            const int32_t h = ck[(int64_t)ch * C + c];
+            ck[(int64_t)ch * C + c] = run;
+            run += h;
+        }
+        sz[c] = run;
+    }
+    __syncthreads();
+    // exclusive scan of sz[0..C) with a contiguous run per thread
+    const int per = (C + blockDim.x - 1) / blockDim.x;
+    const int c0 = threadIdx.x * per;
+    int32_t local = 0;
+    for (int j = 0; j < per; ++j)
+        if (c0 + j < C) local += sz[c0 + j];
+    int32_t incl = local;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int32_t w = lane < (int)(blockDim.x >> 5) ? wsum[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        wsum[lane] = w;  // inclusive over warps
+    }
+    __syncthreads();
+    int32_t run = incl - local + (warp > 0 ? wsum[warp - 1] : 0);
+    int32_t* off = offsets + (int64_t)u * off_ustride;
+    for (int j = 0; j < per; ++j)
+        if (c0 + j < C) {
+            off[c0 + j] = run;
+            run += sz[c0 + j];
+        }
+    if (threadIdx.x == 0) off[C] = (int32_t)m;
+}
+
+// ---------------------------------------------------------------------- scatter
+// One warp per chunk, keys in index order, 32 at a time: lanes with equal clusters are
+// grouped with match.any and ranked by lane. This gives a stable counting sort.
+__global__ void __launch_bounds__(32) kmeans_scatter_kernel(const int32_t* assign, int64_t a_ustride,
+                                                            int64_t m, int32_t C, int32_t nch,
+                                                            const int32_t* chunk,
+                                                            const int32_t* offsets,
+                                                            int64_t off_ustride, int32_t* perm,
+                                                            int64_t perm_ustride) {
+    extern __shared__ int32_t cnt[];
+    const int ch = blockIdx.x, u = blockIdx.y;
+    const int lane = threadIdx.x;
+    const int32_t* base = chunk + ((int64_t)u * nch + ch) * C;
+    const int32_t* off = offsets + (int64_t)u * off_ustride;
+    for (int c = lane; c < C; c += 32) cnt[c] = off[c] + base[c];
+    __syncwarp();
+    const int32_t* a = assign + (int64_t)u * a_ustride;
+    int32_t* pm = perm + (int64_t)u * perm_ustride;
+    const int64_t lo = (int64_t)ch * kChunk;
+    const int64_t hi = lo + kChunk < m ? lo + kChunk : m;
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int64_t i0 = lo; i0 < hi; i0 += 32) {
+        const int64_t i = i0 + lane;
+        int32_t c = i < hi ? a[i] : -1;
+        if ((uint32_t)c >= (uint32_t)C) c = -1;  // out of range (flagged by the count kernel)
+        const uint32_t same = __match_any_sync(0xffffffffu, c);
+        const int32_t pos = c >= 0 ? cnt[c] + __popc(same & lt) : 0;
+        __syncwarp();
+        if (c >= 0 && (same & lt) == 0) cnt[c] += __popc(same);
+        __syncwarp();
+        if (c >= 0) pm[pos] = (int32_t)i;
+    }
+}
+
+// ---------------------------------------------------------------------- mean
+// One warp per cluster: mu_c = (1/|c|) sum of member keys (fp32, ascending member order),
+// empty clusters keep mu_c; then mu_hat. With a relayout, the same pass copies the member K
+// rows and their V rows into the cluster-major store and records the original token ids.
+__global__ void __launch_bounds__(256) kmeans_mean_kernel(KeysView k, const int32_t* perm,
+                                                          int64_t perm_ustride,
+                                                          const int32_t* offsets,
+                                                          int64_t off_ustride, int32_t C,
+                                                          float* mu, int64_t mu_ustride,
+                                                          uint16_t* mu_hat, int64_t muhat_ustride,
+                                                          Relayout rl) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x * (blockDim.x >> 5) + warp;
+    const int u = blockIdx.y;
+    if (c >= C) return;
+    const int32_t* off = offsets + (int64_t)u * off_ustride;
+    const int32_t lo = off[c], hi = off[c + 1];
+    const int32_t* pm = perm + (int64_t)u * perm_ustride;
+    const int64_t ubase = (int64_t)u * k.n_rows + k.row0;
+    const uint16_t* keys = k.base + ubase * kD;
+    const bool relay = rl.kp != nullptr;
+    const uint16_t* vals = relay ? rl.V + ubase * kD : nullptr;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int32_t j = lo;
+    for (; j + 4 <= hi; j += 4) {
+        int32_t idx[4];
+        uint2 w[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) idx[t] = pm[j + t];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+            w[t] = reinterpret_cast<const uint2*>(keys + (int64_t)idx[t] * kD)[lane];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            acc.x += bf16_lo(w[t].x);
+            acc.y += bf16_hi(w[t].x);
+            acc.z += bf16_lo(w[t].y);
+            acc.w += bf16_hi(w[t].y);
+        }
+        if (relay) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const int64_t dst = (int64_t)u * rl.ustride_rows + j + t;
+                reinterpret_cast<uint2*>(rl.kp + dst * kD)[lane] = w[t];
+                reinterpret_cast<uint2*>(rl.vp + dst * kD)[lane] =
+                    reinterpret_cast<const uint2*>(vals + (int64_t)idx[t] * kD)[lane];
+                if (lane == 0) rl.ids[dst] = rl.id_base + idx[t];
+            }
+        }
+    }
+    for (; j < hi; ++j) {
+        const int32_t idx = pm[j];
+        const uint2 w = reinterpret_cast<const uint2*>(keys + (int64_t)idx * kD)[lane];
+        acc.x += bf16_lo(w.x);
+        acc.y += bf16_hi(w.x);
+        acc.z += bf16_lo(w.y);
+        acc.w += bf16_hi(w.y);
+        if (relay) {
+            const int64_t dst = (int64_t)u * rl.ustride_rows + j;
+            reinterpret_cast<uint2*>(rl.kp + dst * kD)[lane] = w;
+            reinterpret_cast<uint2*>(rl.vp + dst * kD)[lane] =
+                reinterpret_cast<const uint2*>(vals + (int64_t)idx * kD)[lane];
+            if (lane == 0) rl.ids[dst] = rl.id_base + idx;
+        }
+    }
+    float* mrow = mu + ((int64_t)u * mu_ustride + c) * kD;
+    float4 v;
+    if (hi > lo) {
+        const float n = (float)(hi - lo);
+        v = make_float4(__fdiv_rn(acc.x, n), __fdiv_rn(acc.y, n), __fdiv_rn(acc.z, n),
+                        __fdiv_rn(acc.w, n));
+    } else {
+        v = reinterpret_cast<const float4*>(mrow)[lane];
+    }
+    store_centroid(v, mrow, mu_hat + ((int64_t)u * muhat_ustride + c) * kD);
+}
+
+__global__ void copy_sinks_kernel(const uint16_t* K, const uint16_t* V, int64_t n, int32_t n_sink,
+                                  uint16_t* spk, uint16_t* spv, int64_t sp_ustride) {
+    const int u = blockIdx.x;
+    const int64_t words = (int64_t)n_sink * kD / 8;  // 16-byte words
+    const uint4* ks = reinterpret_cast<const uint4*>(K + (int64_t)u * n * kD);
+    const uint4* vs = reinterpret_cast<const uint4*>(V + (int64_t)u * n * kD);
+    uint4* kd = reinterpret_cast<uint4*>(spk + (int64_t)u * sp_ustride * kD);
+    uint4* vd = reinterpret_cast<uint4*>(spv + (int64_t)u * sp_ustride * kD);
+    for (int64_t i = threadIdx.x; i < words; i += blockDim.x) {
+        kd[i] = ks[i];
+        vd[i] = vs[i];
+    }
+}
+
+}  // namespace
+
+int launch_kmeans_init(const KeysView& k, int32_t C, uint64_t seed, int64_t unit_base,
+                       uint64_t window, int32_t* init_idx, float* mu, int64_t mu_ustride,
+                       uint16_t* mu_hat, int64_t muhat_ustride, uint32_t* err, cudaStream_t s) {
+    (void)err;
+    int tbits = 6;
+    while ((1 << tbits) < 2 * C) ++tbits;
+    const size_t smem = (size_t)(2 * (1 << tbits) + C) * sizeof(int32_t);
+    cudaError_t e = cudaFuncSetAttribute(kmeans_init_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "init: set smem");
+    kmeans_init_kernel<<<k.U, 256, smem, s>>>(k, C, seed, unit_base, window, init_idx, mu,
+                                              mu_ustride, mu_hat, muhat_ustride, tbits);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? CKV_OK : cuda_fail(e, "init: launch");
+}
+
+int launch_kmeans_update(const KeysView& k, const int32_t* assign, int64_t assign_ustride,
+                         int32_t C, float* mu, int64_t mu_ustride, uint16_t* mu_hat,
+                         int64_t muhat_ustride, int32_t* offsets, int64_t off_ustride,
+                         int32_t* perm, int64_t perm_ustride, int32_t* chunk_ws,
+                         const Relayout* relayout, uint32_t* err, cudaStream_t s) {
+    const int32_t nch = (int32_t)n_chunks(k.m);
+    cudaError_t e;
+    const size_t hsmem = (size_t)C * sizeof(int32_t);
+    e = cudaFuncSetAttribute(kmeans_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)hsmem);
+    if (e != cudaSuccess) return cuda_fail(e, "count: set smem");
+    e = cudaFuncSetAttribute(kmeans_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)hsmem);
+    if (e != cudaSuccess) return cuda_fail(e, "scatter: set smem");
+    const size_t ssmem = (size_t)(C + 32) * sizeof(int32_t);
+    e = cudaFuncSetAttribute(kmeans_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)ssmem);
+    if (e != cudaSuccess) return cuda_fail(e, "scan: set smem");
+    if (nch > 0) {
+        kmeans_count_kernel<<<dim3(nch, k.U), 256, hsmem, s>>>(assign, assign_ustride, k.m, C, nch,
+                                                               chunk_ws, err);
+    }
+    kmeans_scan_kernel<<<k.U, 1024, ssmem, s>>>(chunk_ws, nch, C, k.m, offsets, off_ustride);
+    if (nch > 0) {
+        kmeans_scatter_kernel<<<dim3(nch, k.U), 32, hsmem, s>>>(assign, assign_ustride, k.m, C, nch,
+                                                                chunk_ws, offsets, off_ustride,
+                                                                perm, perm_ustride);
+    }
+    Relayout rl{};
+    if (relayout) rl = *relayout;
+    kmeans_mean_kernel<<<dim3((C + 7) / 8, k.U), 256, 0, s>>>(k, perm, perm_ustride, offsets,
+                                                              off_ustride, C, mu, mu_ustride,
+                                                              mu_hat, muhat_ustride, rl);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? CKV_OK : cuda_fail(e, "update: launch");
+}
+
+int launch_copy_sinks(const uint16_t* K, const uint16_t* V, int64_t n, int32_t U, int32_t n_sink,
+                      uint16_t* spk, uint16_t* spv, int64_t sp_ustride_rows, cudaStream_t s) {
+    copy_sinks_kernel<<<U, 256, 0, s>>>(K, V, n, n_sink, spk, spv, sp_ustride_rows);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? CKV_OK : cuda_fail(e, "sinks: launch");
+}
+
+}  // namespace ckv

@@ -1,0 +1,174 @@
+"""GPU parity of cluster_prefill and select_and_attend against the oracle.
+
+* prefill: store invariants (ids are a permutation of the non-sink tokens; K/V rows are the
+  inputs permuted; sinks copied); the final centroids are within 1e-3 of the oracle's means
+  of the GPU's final clusters; the free-run agreement with the oracle's own K-means is
+  reported (a single near-tie flip changes later iterations, so it is not bit-exact).
+* decode, stage-wise: the oracle runs select_clusters and attention on the GPU's own store.
+  Selected sets must be equal except at near-ties, and outputs must be within 2e-3.
+* decode edge cases on stores built by the oracle and imported: large cut clusters (radix
+  select in shared and in global memory), duplicate centroids and keys (exact ties), empty
+  clusters, pending tokens, budgets at the sinks, at an exact prefix and beyond n.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth_inputs as si
+from gpu_helpers import (MU_TOL, check_decode_unit, fp32_store, store_from_export, store_to_import,
+                         to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+def _ckv():
+    import recallable_kv_cache_cosine_b200 as ckv
+    return ckv
+
+
+def _layer_data(seed, layer, B, Hkv, n, n_centers):
+    K = np.empty((B, Hkv, n, 128), np.uint16)
+    V = np.empty_like(K)
+    for b in range(B):
+        for h in range(Hkv):
+            K[b, h], V[b, h] = si.keys_values(seed, si.unit_id(layer, b, h, B, Hkv), n, n_centers)
+    return K, V
+
+
+def _decode_and_check(ctx, layer, q_u16, budget, stats, B, Hkv, G):
+    qd = to_dev(q_u16)
+    out = torch.empty(B, Hkv * G, 128, device="cuda", dtype=torch.float32)
+    sel = torch.empty(B, Hkv, budget, device="cuda", dtype=torch.int32)
+    cnt = torch.empty(B, Hkv, device="cuda", dtype=torch.int32)
+    ctx.select_and_attend(layer, qd, budget, out, sel, cnt)
+    torch.cuda.synchronize()
+    ctx.check_device_error()
+    outs, sels, cnts = out.cpu().numpy(), sel.cpu().numpy(), cnt.cpu().numpy()
+    for b in range(B):
+        for h in range(Hkv):
+            st = store_from_export(ctx.export_unit(layer, b, h), n_sink=ctx.cfg.n_sink)
+            check_decode_unit(st, q_u16[b, h * G:(h + 1) * G], budget,
+                              outs[b, h * G:(h + 1) * G], sels[b, h], int(cnts[b, h]), stats)
+
+
+@pytest.mark.parametrize("B,Hkv,G,n,C,n_centers", [(1, 1, 4, 2048, 32, 32), (2, 2, 4, 5000, 60, 50),
+                                                   (1, 2, 1, 3000, 40, 40), (1, 1, 8, 4000, 100, 80)])
+def test_prefill_store_then_decode(B, Hkv, G, n, C, n_centers):
+    ckv = _ckv()
+    seed = 7
+    K, V = _layer_data(seed, 0, B, Hkv, n, n_centers)
+    ctx = ckv.ClusterKV(1, B, Hkv, Hkv * G, capacity=n, max_clusters=C, seed=seed)
+    ctx.cluster_prefill(0, to_dev(K), to_dev(V), C)
+    torch.cuda.synchronize()
+    ctx.check_device_error()
+    agree = []
+    for b in range(B):
+        for h in range(Hkv):
+            ex = ctx.export_unit(0, b, h)
+            st = store_from_export(ex)
+            np.testing.assert_array_equal(np.sort(st.ids), np.arange(16, n))
+            np.testing.assert_array_equal(st.kp, K[b, h][st.ids])
+            np.testing.assert_array_equal(st.vp, V[b, h][st.ids])
+            np.testing.assert_array_equal(st.sp_k, K[b, h, :16])
+            np.testing.assert_array_equal(st.sp_v, V[b, h, :16])
+            a = np.empty(n - 16, np.int32)
+            for c in range(C):
+                seg = st.ids[st.offsets[c]:st.offsets[c + 1]]
+                assert np.all(np.diff(seg) > 0)
+                a[seg - 16] = c
+            w_mu, w_off, _ = oracle.update(K[b, h, 16:], a, C, st.mu)
+            np.testing.assert_array_equal(w_off, st.offsets)
+            assert np.abs(w_mu - st.mu).max() <= MU_TOL
+            # free-run agreement with the oracle's own clustering of the same unit
+            u = si.unit_id(0, b, h, B, Hkv)
+            _, a_or = oracle.prefill_unit(K[b, h], V[b, h], C, oracle.stream_key(seed, u, 0))
+            agree.append(float((a_or == a).mean()))
+    print(f"free-run assignment agreement with the oracle: {agree}")
+    assert min(agree) > 0.5
+    stats = {}
+    for step, budget in enumerate([16, 17, 256, 1000, n - 1, n, n + 100]):
+        q = np.stack([si.queries(seed, 0, b, 1 + step, Hkv * G)[step] for b in range(B)])
+        _decode_and_check(ctx, 0, q, budget, stats, B, Hkv, G)
+    print("decode stats", stats)
+    assert stats["near_tie"] <= 1
+
+
+def _imported_ctx(stores, G=4, budget_pending=0):
+    ckv = _ckv()
+    st0 = stores[0]
+    cap = st0.n_sink + st0.m + 320
+    ctx = ckv.ClusterKV(1, 1, len(stores), len(stores) * G, capacity=cap, max_clusters=st0.C + 8)
+    for h, st in enumerate(stores):
+        ctx.import_unit(0, 0, h, store_to_import(st), pending=st.pending)
+    return ctx
+
+
+def _oracle_store(seed, n, C, n_centers, pending=0, iters=3, sigma=0.3):
+    K, V = si.keys_values(seed, 0, n, n_centers, sigma=sigma)
+    st, _ = oracle.prefill_unit(K, V, C, oracle.stream_key(seed, 0, 0), iters=iters)
+    ka, va = si.appended_tokens(seed, 0, pending, n_centers, sigma=sigma) if pending else (None, None)
+    for j in range(pending):
+        st = oracle.append(st, ka[j], va[j])
+    return fp32_store(st)
+
+
+def _check_imported(stores, budgets, G=4, seed=0):
+    ctx = _imported_ctx(stores, G)
+    stats = {}
+    Hkv = len(stores)
+    for i, budget in enumerate(budgets):
+        q = si.queries(seed, 0, 0, len(budgets), Hkv * G)[i][None]
+        _decode_and_check(ctx, 0, q, budget, stats, 1, Hkv, G)
+    return stats
+
+
+def test_decode_large_cut_clusters_radix_paths():
+    # 2 clusters of ~3000 tokens (radix select in shared memory) and ~6000 (global memory)
+    st_a = _oracle_store(1, 6016, 2, 2, pending=3)
+    st_b = _oracle_store(2, 12016, 2, 2, pending=3)
+    for st in (st_a, st_b):
+        sizes = np.diff(st.offsets)
+        assert sizes.max() > 256
+    assert np.diff(st_b.offsets).max() > 4096
+    stats = _check_imported([st_a], [19, 500, 1000, 2999, 3001, 5000])
+    stats = _check_imported([st_b], [19, 700, 4097, 5000, 9000])
+    assert stats["near_tie"] == 0
+
+
+def test_decode_exact_ties_and_empty_clusters():
+    st = _oracle_store(3, 3000, 40, 30, pending=7)
+    mu = st.mu.copy()
+    mu[20] = mu[3]            # duplicate centroid: equal scores, lower index first
+    mu[21] = mu[3]
+    offs = st.offsets.copy()
+    kp, vp, ids = st.kp.copy(), st.vp.copy(), st.ids.copy()
+    # duplicate keys inside every cluster: equal token scores, lower id first
+    for c in range(st.C):
+        lo, hi = offs[c], offs[c + 1]
+        if hi - lo >= 4:
+            kp[lo + 1] = kp[lo]
+            kp[hi - 1] = kp[lo]
+    # make clusters 10 and 11 empty by merging their rows into cluster 12 (segments stay contiguous)
+    lo10, hi12 = offs[10], offs[13]
+    order = np.argsort(ids[lo10:hi12], kind="stable")
+    kp[lo10:hi12], vp[lo10:hi12], ids[lo10:hi12] = kp[lo10:hi12][order], vp[lo10:hi12][order], ids[lo10:hi12][order]
+    offs[11] = lo10
+    offs[12] = lo10
+    st2 = oracle.Store(st.sp_k, st.sp_v, kp, vp, ids, offs, mu, st.n_sink)
+    budgets = [23, 24, 100, 300, 800, 1500, 2999, 3007, 4000]
+    _check_imported([st2, st2], budgets)
+
+
+def test_decode_exact_prefix_budgets_take_no_partial():
+    st = _oracle_store(4, 4000, 50, 40)
+    q = si.queries(0, 0, 0, 1, 4)[0][None]
+    qbar = oracle.group_query(q[0])
+    s = st.mu @ qbar
+    order = sorted(range(st.C), key=lambda c: (-s[c], c))
+    sizes = np.diff(st.offsets)
+    budgets = [16 + int(sizes[order[:k]].sum()) for k in (1, 2, 5, 11)]
+    ctx = _imported_ctx([st])
+    stats = {}
+    for bud in budgets:
+        _decode_and_check(ctx, 0, q, bud, stats, 1, 1, 4)
