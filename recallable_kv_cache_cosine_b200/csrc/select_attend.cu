@@ -396,12 +396,14 @@ __global__ void __launch_bounds__(kNT) select_attend_kernel(const DecodeArgs a, 
             if (sel_out) sel_out[idx] = oid;
         }
         __syncthreads();
-        for (int j0 = hw; j0 < n; j0 += 4 * (kNT / 16)) {
+        // The trip count is the same for every thread of the CTA: the full-mask shuffles
+        // below need both half-warps of a warp in every iteration.
+        for (int j0 = 0; j0 < n; j0 += 4 * (kNT / 16)) {
             uint4 kw[4], vw[4];
             int valid[4];
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
-                const int j = j0 + t * (kNT / 16);
+                const int j = j0 + hw + t * (kNT / 16);
                 valid[t] = j < n;
                 if (valid[t]) {
                     const int32_t row = sm.rows[j];

@@ -60,8 +60,8 @@ def test_assign_ties_go_to_lower_index():
     Kn, Kd = _keys(U, n, 50, seed=3)
     rng = np.random.default_rng(0)
     mh = rng.standard_normal((C, 128))
-    mh[150:300] = mh[0:150]           # every centroid >= 150 duplicates one below it
     mh[7] = 0.0
+    mh[150:300] = mh[0:150]  # every centroid >= 150 duplicates one below it
     mh_u16 = oracle.normalize(mh)
     ctx = _ctx(U, n, C)
     assign = ctx.kmeans_assign(Kd, 16, m, to_dev(mh_u16[None]))
