@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Benchmark of the ClusterKV hot path on B200.
+
+Metric: select+attend µs per layer-step at a 32k context and a 1k budget, with K-means
+keys/s and the fraction of the HBM roofline.
+
+Workload (one Llama-3.1-8B-shaped layer: 32 query / 8 KV heads, head_dim 128, n = 32768,
+batch 1, C = 400, budget 1024), held as 32 distinct layer stores. Each decode pass then
+reads ~190 MB of selected rows and centroids, more than the 126 MB L2. Inputs are
+synthetic (seeded clustered mixture), already resident in HBM.
+
+One bench step is one pass of the whole hot path:
+  A. cluster_prefill of all 32 layers (sinks, seeded init, 10 Lloyd iterations of tcgen05
+     assignment + counting-sort update, relayout of K and V);
+  B. 64 decode steps x 32 layers of select_and_attend (queries only), one CUDA graph;
+  C. one 320-token incremental window on layer 0: per token append_kv + select_and_attend,
+     then recluster_increment.
+`value` = device time of B / layer-steps (µs, lower is better). Per-section times, keys/s,
+the roofline of the select+attend kernel, an end-to-end figure (eager API calls with the
+query copied in from pinned host memory and the output read back, per layer-step) and the
+CPU oracle's time on a bounded sample of the same workload are added to the JSON line.
+
+--impl reference times the CPU oracle instead, on the same metric.
+N > 1 (torchrun): every rank runs the same workload on its own GPU (weak scaling, no
+data-path collective). Times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth_inputs as si  # noqa: E402
+
+METRIC = "select+attend µs per layer-step @32k ctx/1k budget; k-means keys/s; % HBM roofline"
+UNIT = "us/layer-step"
+
+# workload: one Llama-3.1-8B-shaped layer, 32 distinct layer stores
+B, HKV, HQ, N_CTX, C_CLUSTERS, BUDGET, N_CENTERS = 1, 8, 32, 32768, 400, 1024, 400
+N_SINK, WINDOW, ITERS, SEED = 16, 320, 10, 1
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+
+# DRAM bytes per select+attend launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum)
+# for the current kernel, or None when the kernel changed after the counters were taken.
+SELECT_ATTEND_TRAFFIC = None
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def select_attend_bytes(units, budget, C, m, G):
+    """Algorithmic bytes of one select+attend launch: per unit the budget's K and V rows
+    (256 B each), the fp32 centroids (512 B each), the offsets, the cut cluster's K rows
+    (mean cluster size m/C, 256 B each), q (bf16) and o (fp32)."""
+    per_unit = budget * 512 + C * 512 + (C + 1) * 4 + (m / C) * 256 + G * 128 * 2 + G * 128 * 4
+    return units * per_unit
+
+
+class Clocks:
+    """nvidia-smi sampler running during the timed region."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local_index):
+        # address the GPU by UUID: CUDA_VISIBLE_DEVICES may renumber devices
+        try:
+            u = str(torch.cuda.get_device_properties(local_index).uuid)
+            self.index = u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            self.index = str(local_index)
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.rows = []
+        if self.proc is None:
+            return False
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        for line in out.splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 8:
+                self.rows.append(parts)
+        return False
+
+    def summary(self):
+        if not getattr(self, "rows", None):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[4 + i].lower() == "active"})
+        busy = [s for s in sm if s > 0.5 * (max(mx) if mx else 1)]
+        return {"sm_mhz": statistics.median(busy or sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------- CPU oracle leg
+
+def oracle_sample_stores(units=HKV):
+    """Stores for a bounded CPU sample: layer-0 units of the workload whose clusters are the
+    generator's mixture components, with centroids from one oracle mean update. The decode
+    work is the same size as the GPU's (C = 400 clusters of ~82 tokens, budget 1024)."""
+    import oracle
+    stores = []
+    for h in range(units):
+        K, V, lab = si.keys_values_labeled(SEED, si.unit_id(0, 0, h, B, HKV), N_CTX, N_CENTERS)
+        keys = np.ascontiguousarray(K[N_SINK:])
+        mu, offs, perm = oracle.update(keys, lab[N_SINK:], C_CLUSTERS, np.zeros((C_CLUSTERS, 128)))
+        stores.append((K[:N_SINK], V[:N_SINK], K[N_SINK:][perm], V[N_SINK:][perm],
+                       (perm + N_SINK).astype(np.int32), offs, mu))
+    st = [np.stack([s[i] for s in stores]) for i in range(7)]
+    q = np.stack([si.queries(SEED, 0, 0, 64, HQ)[:, h * (HQ // HKV):(h + 1) * (HQ // HKV)]
+                  for h in range(units)], axis=1)  # [steps, units, G, 128]
+    return st, q
+
+
+def oracle_time_layer_steps(st, q, n_layer_steps):
+    import oracle
+    t0 = time.perf_counter()
+    for i in range(n_layer_steps):
+        oracle.select_attend_batch(*st, q[i % q.shape[0]], BUDGET)
+    return (time.perf_counter() - t0) / n_layer_steps
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import oracle
+    cores = oracle.omp_threads()
+    st, q = oracle_sample_stores()
+    per_step = 8  # layer-steps per bench step
+    for _ in range(args.warmup):
+        oracle_time_layer_steps(st, q, per_step)
+    times = [oracle_time_layer_steps(st, q, per_step) for _ in range(args.steps)]
+    us = statistics.mean(times) * 1e6
+    sample = (f"oracle select+attend of one 32k-token layer (8 KV heads, G=4, C=400, budget 1024), "
+              f"{per_step} layer-steps per bench step, OpenMP over the 8 units on {cores} threads")
+    line = {"impl": "reference", "metric": METRIC, "value": us, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": us * per_step / 1e3,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": "llama3.1-8b-shaped layer, n=32768, B=1, 8 kv / 32 q heads, "
+                                   "C=400, budget=1024 (CPU oracle sample)"},
+            "cpu_baseline": {"value": us, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": us, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------- GPU leg
+
+def launches_per_prefill(C, iters):
+    assign_launches = (C + 511) // 512
+    return 1 + iters * (assign_launches + 4) + 1
+
+
+def run_gpu(args, world, rank, local):
+    import recallable_kv_cache_cosine_b200 as ckv
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    L, D, W = args.layers, args.decode_steps, WINDOW
+    G = HQ // HKV
+    units = B * HKV
+    hbm_gbs, bf16_tflops, peak_kind = peaks()
+
+    # ------------------------------------------------------------ inputs (resident in HBM)
+    K = torch.empty(L, B, HKV, N_CTX, 128, dtype=torch.bfloat16, device=dev)
+    V = torch.empty_like(K)
+    for l in range(L):
+        for h in range(HKV):
+            K[l, 0, h], V[l, 0, h] = si.keys_values_torch(SEED + rank, si.unit_id(l, 0, h, B, HKV),
+                                                          N_CTX, N_CENTERS, dev)
+    q = torch.empty(D, L, B, HQ, 128, dtype=torch.bfloat16, device=dev)
+    for l in range(L):
+        q[:, l, 0] = si.queries_torch(SEED + rank, l, 0, D, HQ, dev)
+    out = torch.empty(D, L, B, HQ, 128, dtype=torch.float32, device=dev)
+    app_k = torch.empty(W, B, HKV, 128, dtype=torch.bfloat16, device=dev)
+    app_v = torch.empty_like(app_k)
+    for h in range(HKV):
+        app_k[:, 0, h], app_v[:, 0, h] = si.appended_tokens_torch(SEED + rank, si.unit_id(0, 0, h, B, HKV),
+                                                                   W, N_CENTERS, dev)
+    out_c = torch.empty(B, HQ, 128, dtype=torch.float32, device=dev)
+
+    ctx = ckv.ClusterKV(n_layers=L, batch=B, n_kv_heads=HKV, n_q_heads=HQ, capacity=N_CTX + W,
+                        max_clusters=C_CLUSTERS + 4, seed=SEED)
+    s = torch.cuda.Stream(device=dev)
+    launches = {"A": 0, "B": 0, "C": 0}
+
+    def section_a():
+        for l in range(L):
+            ctx.cluster_prefill(l, K[l], V[l], C_CLUSTERS, stream=s)
+
+    def section_b():
+        for d in range(D):
+            for l in range(L):
+                ctx.select_and_attend(l, q[d, l], BUDGET, out[d, l], stream=s)
+
+    def section_c():
+        for t in range(W):
+            ctx.append_kv(0, app_k[t], app_v[t], stream=s)
+            ctx.select_and_attend(0, q[t % D, 0], BUDGET, out_c, stream=s)
+        ctx.recluster_increment(0, stream=s)
+
+    launches["A"] = L * launches_per_prefill(C_CLUSTERS, ITERS)
+    launches["B"] = D * L
+    launches["C"] = 2 * W + 1
+
+    # ------------------------------------------------------------ capture B and C
+    with torch.cuda.stream(s):
+        section_a()
+    s.synchronize()
+    ctx.check_device_error(stream=s)
+    gB, gC = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gB, stream=s, capture_error_mode="thread_local"):
+        section_b()
+    with torch.cuda.graph(gC, stream=s, capture_error_mode="thread_local"):
+        section_c()
+    torch.cuda.synchronize()
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def one_step(record):
+        e = [ev() for _ in range(4)]
+        with torch.cuda.stream(s):
+            e[0].record(s)
+            section_a()
+            e[1].record(s)
+            gB.replay()
+            e[2].record(s)
+            gC.replay()
+            e[3].record(s)
+        record.append(e)
+
+    warm = []
+    for _ in range(args.warmup):
+        one_step(warm)
+    torch.cuda.synchronize()
+    ctx.check_device_error(stream=s)
+
+    # ------------------------------------------------------------ timed region
+    rec = []
+    barrier(world)
+    torch.cuda.synchronize()
+    with Clocks(local) as clk:
+        for _ in range(args.steps):
+            one_step(rec)
+        torch.cuda.synchronize()
+    barrier(world)
+    ctx.check_device_error(stream=s)
+    tA = sum(e[0].elapsed_time(e[1]) for e in rec) / 1e3
+    tB = sum(e[1].elapsed_time(e[2]) for e in rec) / 1e3
+    tC = sum(e[2].elapsed_time(e[3]) for e in rec) / 1e3
+    t_step = sum(e[0].elapsed_time(e[3]) for e in rec) / 1e3
+    tA, tB, tC, t_step = (max_over_ranks(x, world) for x in (tA, tB, tC, t_step))
+
+    K_steps = args.steps
+    layer_steps = K_steps * D * L * world
+    value = tB / layer_steps * 1e6
+    keys = K_steps * L * units * (N_CTX - N_SINK) * world
+    keys_per_s = keys / tA
+    keys_roof = min(bf16_tflops * 1e12 / (2 * C_CLUSTERS * 128), hbm_gbs * 1e9 / 512) / ITERS
+    launch_us = tB / (K_steps * D * L) * 1e6
+    m = N_CTX - N_SINK
+    bytes_launch = select_attend_bytes(units, BUDGET, C_CLUSTERS, m, G)
+    achieved = bytes_launch / (launch_us * 1e-6) / 1e9
+    inc_us = tC / (K_steps * W * world) * 1e6
+
+    # ------------------------------------------------------------ end to end (host buffers)
+    with torch.cuda.stream(s):
+        section_a()
+    q_host = q[: min(D, 16)].cpu().pin_memory()
+    o_host = torch.empty(q_host.shape[:3] + (HQ, 128), dtype=torch.float32).pin_memory()
+    q_dev = torch.empty(B, HQ, 128, dtype=torch.bfloat16, device=dev)
+    o_dev = torch.empty(B, HQ, 128, dtype=torch.float32, device=dev)
+    De = q_host.shape[0]
+
+    def e2e_pass():
+        with torch.cuda.stream(s):
+            for d in range(De):
+                for l in range(L):
+                    q_dev.copy_(q_host[d, l], non_blocking=True)
+                    ctx.select_and_attend(l, q_dev, BUDGET, o_dev, stream=s)
+                    o_host[d, l].copy_(o_dev, non_blocking=True)
+
+    e2e_pass()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = ev(), ev()
+    e0.record(s)
+    for _ in range(max(1, args.steps)):
+        e2e_pass()
+    e1.record(s)
+    torch.cuda.synchronize()
+    t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+    e2e_value = t_e2e / (max(1, args.steps) * De * L * world) * 1e6
+    launches_e2e = max(1, args.steps) * De * L
+    ctx.check_device_error(stream=s)
+
+    # ------------------------------------------------------------ CPU baseline (rank 0, N = 1)
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        st, qo = oracle_sample_stores()
+        oracle_time_layer_steps(st, qo, 2)
+        n_ls = args.cpu_layer_steps
+        t = oracle_time_layer_steps(st, qo, n_ls)
+        cpu = {"value": t * 1e6, "unit": UNIT, "cores": oracle.omp_threads(), "kind": "oracle",
+               "sample": (f"{n_ls} layer-steps of select+attend over one 32k-token layer (8 KV heads, "
+                          f"G=4, C=400, budget 1024); clusters = the generator's mixture components "
+                          f"with one oracle mean update; OpenMP over the 8 units")}
+
+    if rank == 0:
+        clocks = clk.summary()
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K_steps,
+            "warmup": args.warmup, "ms_per_step": t_step / K_steps * 1e3, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "llama3.1-8b-shaped layer (32 q / 8 kv heads, d=128), n=32768, "
+                                   "batch 1, C=400, budget=1024, held as 32 distinct layer stores",
+                       "layer_stores": L, "decode_steps": D, "n": N_CTX, "batch": B, "kv_heads": HKV,
+                       "q_heads": HQ, "C": C_CLUSTERS, "budget": BUDGET, "iters": ITERS,
+                       "window": W, "parallelism": f"replicas x{world} (units independent)",
+                       "l2": "inputs larger than L2: 32 layer stores, ~193 MB selected per decode pass"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                         "frac": achieved / hbm_gbs, "traffic": SELECT_ATTEND_TRAFFIC,
+                         "kernel": "select_attend_kernel<4>", "bytes_per_launch": bytes_launch,
+                         "us_per_launch": launch_us, "peak_kind": peak_kind},
+            "kmeans": {"keys_per_s": keys_per_s, "roofline_keys_per_s": keys_roof,
+                       "frac": keys_per_s / keys_roof, "prefill_ms_per_layer": tA / (K_steps * L) * 1e3,
+                       "bound": "min(tensor at 2*C*128 flop/key, HBM at 2 key reads)/iters"},
+            "incremental": {"us_per_token_layer": inc_us,
+                            "what": "append_kv + select_and_attend per token, recluster every 320"},
+            "sections_ms_per_step": {"prefill": tA / K_steps * 1e3, "decode": tB / K_steps * 1e3,
+                                     "incremental": tC / K_steps * 1e3},
+            "e2e": {"value": e2e_value, "unit": UNIT,
+                    "h2d_bytes_per_step": De * L * B * HQ * 128 * 2,
+                    "d2h_bytes_per_step": De * L * B * HQ * 128 * 4,
+                    "what": "eager API calls, q copied from pinned host memory and the output read "
+                            "back every layer-step"},
+            "gpu_launches": (launches["A"] + launches["B"] + launches["C"]) * K_steps,
+            "gpu_launches_e2e": launches_e2e,
+            "cpu_baseline": cpu,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    del gB, gC
+    ctx.close()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--decode-steps", type=int, default=64)
+    ap.add_argument("--cpu-layer-steps", type=int, default=256)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        run_gpu(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -130,10 +130,16 @@ __global__ void __launch_bounds__(1024) kmeans_scan_kernel(int32_t* chunk, int32
     int32_t* ck = chunk + (int64_t)u * nch * C;
     for (int c = threadIdx.x; c < C; c += blockDim.x) {
         int32_t run = 0;
-        for (int ch = 0; ch < nch; ++ch) {
-            const int32_t h = ck[(int64_t)ch * C + c];
-            ck[(int64_t)ch * C + c] = run;
-            run += h;
+        for (int ch0 = 0; ch0 < nch; ch0 += 16) {
+            int32_t h[16];  // 16 loads in flight per batch
+#pragma unroll
+            for (int t = 0; t < 16; ++t) h[t] = ch0 + t < nch ? ck[(int64_t)(ch0 + t) * C + c] : 0;
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+                if (ch0 + t < nch) {
+                    ck[(int64_t)(ch0 + t) * C + c] = run;
+                    run += h[t];
+                }
         }
         sz[c] = run;
     }
@@ -182,21 +188,39 @@ __global__ void __launch_bounds__(32) kmeans_scatter_kernel(const int32_t* assig
                                                             const int32_t* offsets,
                                                             int64_t off_ustride, int32_t* perm,
                                                             int64_t perm_ustride) {
-    extern __shared__ int32_t cnt[];
+    extern __shared__ int32_t cnt[];  // [C] counters, then [kChunk] assignments
+    int32_t* sa = cnt + C;
     const int ch = blockIdx.x, u = blockIdx.y;
     const int lane = threadIdx.x;
     const int32_t* base = chunk + ((int64_t)u * nch + ch) * C;
     const int32_t* off = offsets + (int64_t)u * off_ustride;
-    for (int c = lane; c < C; c += 32) cnt[c] = off[c] + base[c];
-    __syncwarp();
     const int32_t* a = assign + (int64_t)u * a_ustride;
     int32_t* pm = perm + (int64_t)u * perm_ustride;
     const int64_t lo = (int64_t)ch * kChunk;
     const int64_t hi = lo + kChunk < m ? lo + kChunk : m;
+    // Stage the counters and the chunk's assignments in shared memory with all loads in
+    // flight, so the sequential loop below touches shared memory only.
+    for (int c0 = 0; c0 < C; c0 += 32 * 8) {
+        int32_t o[8], bb[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            const int c = c0 + t * 32 + lane;
+            o[t] = c < C ? off[c] : 0;
+            bb[t] = c < C ? base[c] : 0;
+        }
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            const int c = c0 + t * 32 + lane;
+            if (c < C) cnt[c] = o[t] + bb[t];
+        }
+    }
+#pragma unroll 8
+    for (int j = lane; j < kChunk; j += 32) sa[j] = lo + j < hi ? a[lo + j] : -1;
+    __syncwarp();
     const uint32_t lt = (1u << lane) - 1u;
     for (int64_t i0 = lo; i0 < hi; i0 += 32) {
         const int64_t i = i0 + lane;
-        int32_t c = i < hi ? a[i] : -1;
+        int32_t c = sa[i - lo];
         if ((uint32_t)c >= (uint32_t)C) c = -1;  // out of range (flagged by the count kernel)
         const uint32_t same = __match_any_sync(0xffffffffu, c);
         const int32_t pos = c >= 0 ? cnt[c] + __popc(same & lt) : 0;
@@ -230,17 +254,25 @@ __global__ void __launch_bounds__(256) kmeans_mean_kernel(KeysView k, const int3
     const bool relay = rl.kp != nullptr;
     const uint16_t* vals = relay ? rl.V + ubase * kD : nullptr;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    int32_t j = lo;
-    for (; j + 4 <= hi; j += 4) {
-        int32_t idx[4];
-        uint2 w[4];
+    // Rows in batches of 8 (8 loads in flight per lane); the next batch's member indices are
+    // fetched while the current batch's rows are loading. Accumulation stays in member order.
+    constexpr int kB = 8;
+    int32_t nxt[kB];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) idx[t] = pm[j + t];
+    for (int t = 0; t < kB; ++t) nxt[t] = lo + t < hi ? pm[lo + t] : 0;
+    for (int32_t j = lo; j < hi; j += kB) {
+        int32_t idx[kB];
 #pragma unroll
-        for (int t = 0; t < 4; ++t)
-            w[t] = reinterpret_cast<const uint2*>(keys + (int64_t)idx[t] * kD)[lane];
+        for (int t = 0; t < kB; ++t) idx[t] = nxt[t];
+        uint2 w[kB];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
+        for (int t = 0; t < kB; ++t)
+            if (j + t < hi) w[t] = reinterpret_cast<const uint2*>(keys + (int64_t)idx[t] * kD)[lane];
+#pragma unroll
+        for (int t = 0; t < kB; ++t) nxt[t] = j + kB + t < hi ? pm[j + kB + t] : 0;
+#pragma unroll
+        for (int t = 0; t < kB; ++t) {
+            if (j + t >= hi) break;
             acc.x += bf16_lo(w[t].x);
             acc.y += bf16_hi(w[t].x);
             acc.z += bf16_lo(w[t].y);
@@ -248,28 +280,14 @@ __global__ void __launch_bounds__(256) kmeans_mean_kernel(KeysView k, const int3
         }
         if (relay) {
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
+            for (int t = 0; t < kB; ++t) {
+                if (j + t >= hi) break;
                 const int64_t dst = (int64_t)u * rl.ustride_rows + j + t;
                 reinterpret_cast<uint2*>(rl.kp + dst * kD)[lane] = w[t];
                 reinterpret_cast<uint2*>(rl.vp + dst * kD)[lane] =
                     reinterpret_cast<const uint2*>(vals + (int64_t)idx[t] * kD)[lane];
                 if (lane == 0) rl.ids[dst] = rl.id_base + idx[t];
             }
-        }
-    }
-    for (; j < hi; ++j) {
-        const int32_t idx = pm[j];
-        const uint2 w = reinterpret_cast<const uint2*>(keys + (int64_t)idx * kD)[lane];
-        acc.x += bf16_lo(w.x);
-        acc.y += bf16_hi(w.x);
-        acc.z += bf16_lo(w.y);
-        acc.w += bf16_hi(w.y);
-        if (relay) {
-            const int64_t dst = (int64_t)u * rl.ustride_rows + j;
-            reinterpret_cast<uint2*>(rl.kp + dst * kD)[lane] = w;
-            reinterpret_cast<uint2*>(rl.vp + dst * kD)[lane] =
-                reinterpret_cast<const uint2*>(vals + (int64_t)idx * kD)[lane];
-            if (lane == 0) rl.ids[dst] = rl.id_base + idx;
         }
     }
     float* mrow = mu + ((int64_t)u * mu_ustride + c) * kD;
@@ -324,11 +342,12 @@ int launch_kmeans_update(const KeysView& k, const int32_t* assign, int64_t assig
     const int32_t nch = (int32_t)n_chunks(k.m);
     cudaError_t e;
     const size_t hsmem = (size_t)C * sizeof(int32_t);
+    const size_t scsmem = (size_t)(C + kChunk) * sizeof(int32_t);
     e = cudaFuncSetAttribute(kmeans_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)hsmem);
     if (e != cudaSuccess) return cuda_fail(e, "count: set smem");
     e = cudaFuncSetAttribute(kmeans_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)hsmem);
+                             (int)scsmem);
     if (e != cudaSuccess) return cuda_fail(e, "scatter: set smem");
     const size_t ssmem = (size_t)(C + 32) * sizeof(int32_t);
     e = cudaFuncSetAttribute(kmeans_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -340,7 +359,7 @@ int launch_kmeans_update(const KeysView& k, const int32_t* assign, int64_t assig
     }
     kmeans_scan_kernel<<<k.U, 1024, ssmem, s>>>(chunk_ws, nch, C, k.m, offsets, off_ustride);
     if (nch > 0) {
-        kmeans_scatter_kernel<<<dim3(nch, k.U), 32, hsmem, s>>>(assign, assign_ustride, k.m, C, nch,
+        kmeans_scatter_kernel<<<dim3(nch, k.U), 32, scsmem, s>>>(assign, assign_ustride, k.m, C, nch,
                                                                 chunk_ws, offsets, off_ustride,
                                                                 perm, perm_ustride);
     }

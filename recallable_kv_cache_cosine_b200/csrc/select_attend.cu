@@ -30,6 +30,10 @@
 // slice into L2 before waiting on the previous grid.
 #include <float.h>
 
+#include <map>
+#include <mutex>
+#include <tuple>
+
 #include "ckv_common.cuh"
 #include "ckv_internal.h"
 
@@ -50,6 +54,33 @@ CKV_DEV uint32_t orderable(float f) {
     f = f + 0.0f;  // -0 -> +0
     const uint32_t u = __float_as_uint(f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Orderable key of qbar . k for one 256-byte key row, computed by one thread: 16 independent
+// 16-byte loads, then an fp32 dot product in dimension order.
+CKV_DEV uint32_t row_key(const uint16_t* row, const float* qbar) {
+    float s = 0.f;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+    uint4 w[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) w[t] = ldg_nc_v4(row + 64 * half + 8 * t);
+#pragma unroll
+    for (int t0 = 0; t0 < 8; ++t0) {
+        const int t = 8 * half + t0;
+        const float4 qa = reinterpret_cast<const float4*>(qbar)[2 * t];
+        const float4 qb = reinterpret_cast<const float4*>(qbar)[2 * t + 1];
+        s = fmaf(qa.x, bf16_lo(w[t0].x), s);
+        s = fmaf(qa.y, bf16_hi(w[t0].x), s);
+        s = fmaf(qa.z, bf16_lo(w[t0].y), s);
+        s = fmaf(qa.w, bf16_hi(w[t0].y), s);
+        s = fmaf(qb.x, bf16_lo(w[t0].z), s);
+        s = fmaf(qb.y, bf16_hi(w[t0].z), s);
+        s = fmaf(qb.z, bf16_lo(w[t0].w), s);
+        s = fmaf(qb.w, bf16_hi(w[t0].w), s);
+    }
+    }
+    return orderable(s);
 }
 
 // Exclusive block scan of one int per thread. `tot` receives the block total.
@@ -92,7 +123,7 @@ struct Smem {
 };
 
 template <int G>
-__global__ void __launch_bounds__(kNT) select_attend_kernel(const DecodeArgs a, int32_t S,
+__global__ void __launch_bounds__(kNT, (G <= 4) ? 2 : 1) select_attend_kernel(const DecodeArgs a, int32_t S,
                                                             int32_t prow_cap) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     const int C = a.C;
@@ -140,8 +171,28 @@ __global__ void __launch_bounds__(kNT) select_attend_kernel(const DecodeArgs a, 
     pdl_wait();
 
     // ---------------------------------------------------------------- phase 1: scores
+    // A quarter-warp (8 lanes) per centroid, 16 dimensions per lane: 32 centroids per CTA
+    // per round. The first round's centroid and size loads are issued before the query
+    // loads, so both share one memory round trip.
     const int32_t pend = a.pending;
     const int64_t R = (int64_t)a.budget - a.n_sink - pend;  // >= 0 (host-checked)
+    const int q8 = lane >> 3, l8 = lane & 7;
+    constexpr int kPerRound = kWarps * 4;
+    float4 mv[4];
+    int32_t csize = 0;
+    auto load_centroid = [&](int c) {
+        if (c < c_end) {
+            const float4* row = reinterpret_cast<const float4*>(mu + (int64_t)c * kD) + l8 * 4;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) mv[t] = row[t];
+            csize = off[c + 1] - off[c];
+        } else {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) mv[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+            csize = 0;
+        }
+    };
+    load_centroid(c_begin + warp * 4 + q8);
     {
         const uint16_t* q = a.q + ((int64_t)b * a.Hkv * G + (int64_t)h * G) * kD;
         const float scale = kLog2e * rsqrtf((float)kD);
@@ -159,17 +210,23 @@ __global__ void __launch_bounds__(kNT) select_attend_kernel(const DecodeArgs a, 
     if (threadIdx.x == 0) sm.cut->c = -1;
     __syncthreads();
     cluster_wait_acquire();  // every CTA of the cluster is running
-    {
-        const float4 qb = reinterpret_cast<const float4*>(sm.qbar)[lane];
-        for (int c = c_begin + warp; c < c_end; c += kWarps) {
-            const float4 m4 = reinterpret_cast<const float4*>(mu + (int64_t)c * kD)[lane];
-            float s = qb.x * m4.x + qb.y * m4.y + qb.z * m4.z + qb.w * m4.w;
+    for (int r0 = 0; r0 < c_end - c_begin; r0 += kPerRound) {
+        const int c = c_begin + r0 + warp * 4 + q8;
+        if (r0 > 0) load_centroid(c);
+        const float4* qb4 = reinterpret_cast<const float4*>(sm.qbar) + l8 * 4;
+        float s = 0.f;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-            const int32_t size = off[c + 1] - off[c];
-            if (lane < S) {
-                st_cluster_f32(map_shared_rank(smem_u32(&sm.sc[c]), lane), s);
-                st_cluster_u32(map_shared_rank(smem_u32(&sm.sz[c]), lane), (uint32_t)size);
+        for (int t = 0; t < 4; ++t) {
+            const float4 qv4 = qb4[t];
+            s += qv4.x * mv[t].x + qv4.y * mv[t].y + qv4.z * mv[t].z + qv4.w * mv[t].w;
+        }
+        s += __shfl_xor_sync(0xffffffffu, s, 4);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        if (c < c_end) {
+            for (int r = l8; r < S; r += 8) {
+                st_cluster_f32(map_shared_rank(smem_u32(&sm.sc[c]), r), s);
+                st_cluster_u32(map_shared_rank(smem_u32(&sm.sz[c]), r), (uint32_t)csize);
             }
         }
     }
@@ -234,16 +291,9 @@ __global__ void __launch_bounds__(kNT) select_attend_kernel(const DecodeArgs a, 
     if (r_part > 0 && big_cut) {
         // Keys of a large cut cluster are written once, split across the cluster's CTAs.
         const int32_t crow = sm.cut->row;
-        const float4 qb = reinterpret_cast<const float4*>(sm.qbar)[lane];
         const int64_t k0 = (int64_t)csz * rank / S, k1 = (int64_t)csz * (rank + 1) / S;
-        for (int64_t i = k0 + warp; i < k1; i += kWarps) {
-            const uint2 w = reinterpret_cast<const uint2*>(a.kp + (kp_base + crow + i) * kD)[lane];
-            float s = qb.x * bf16_lo(w.x) + qb.y * bf16_hi(w.x) + qb.z * bf16_lo(w.y) +
-                      qb.w * bf16_hi(w.y);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-            if (lane == 0) gkeys[i] = orderable(s);
-        }
+        for (int64_t i = k0 + threadIdx.x; i < k1; i += kNT)
+            gkeys[i] = row_key(a.kp + (kp_base + crow + i) * kD, sm.qbar);
         cluster_arrive_release();
         cluster_wait_acquire();
     }
@@ -252,16 +302,8 @@ __global__ void __launch_bounds__(kNT) select_attend_kernel(const DecodeArgs a, 
         const uint32_t* skeys = sm.pkey;
         auto key_at = [&](int i) -> uint32_t { return big_cut ? __ldcg(gkeys + i) : skeys[i]; };
         if (!big_cut) {
-            const float4 qb = reinterpret_cast<const float4*>(sm.qbar)[lane];
-            for (int i = warp; i < csz; i += kWarps) {
-                const uint2 w =
-                    reinterpret_cast<const uint2*>(a.kp + (kp_base + crow + i) * kD)[lane];
-                float s = qb.x * bf16_lo(w.x) + qb.y * bf16_hi(w.x) + qb.z * bf16_lo(w.y) +
-                          qb.w * bf16_hi(w.y);
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-                if (lane == 0) sm.pkey[i] = orderable(s);
-            }
+            for (int i = threadIdx.x; i < csz; i += kNT)
+                sm.pkey[i] = row_key(a.kp + (kp_base + crow + i) * kD, sm.qbar);
         }
         __syncthreads();
         // Threshold: key theta and `need` = how many keys equal to theta are taken (the
@@ -356,11 +398,7 @@ __global__ void __launch_bounds__(kNT) select_attend_kernel(const DecodeArgs a, 
 
     // ---------------------------------------------------------------- phase 4: gather + attend
     const int hw = threadIdx.x >> 4, l16 = threadIdx.x & 15;
-    float qv[G][8];
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) qv[g][e] = sm.qg[g * kD + l16 * 8 + e];
+    const float4* qg4 = reinterpret_cast<const float4*>(sm.qg) + l16 * 2;  // this lane's 8 dims
     float mrun[G], lrun[G], acc[G][8];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -436,9 +474,16 @@ __global__ void __launch_bounds__(kNT) select_attend_kernel(const DecodeArgs a, 
                 float z[G];
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
-                    float s = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) s = fmaf(qv[g][e], kf[e], s);
+                    const float4 qa = qg4[g * (kD / 4)];
+                    const float4 qb = qg4[g * (kD / 4) + 1];
+                    float s = qa.x * kf[0];
+                    s = fmaf(qa.y, kf[1], s);
+                    s = fmaf(qa.z, kf[2], s);
+                    s = fmaf(qa.w, kf[3], s);
+                    s = fmaf(qb.x, kf[4], s);
+                    s = fmaf(qb.y, kf[5], s);
+                    s = fmaf(qb.z, kf[6], s);
+                    s = fmaf(qb.w, kf[7], s);
                     z[g] = s;
                 }
 #pragma unroll
@@ -537,54 +582,113 @@ __global__ void __launch_bounds__(kNT) select_attend_kernel(const DecodeArgs a, 
     }
 }
 
+size_t smem_bytes(int G, int S, int C, int budget) {
+    const int32_t pc = (int32_t)((int64_t)budget / S + 2);
+    size_t b = 0;
+    auto add = [&](size_t x) { b += (x + 15) & ~(size_t)15; };
+    add(sizeof(float) * G * kD);
+    add(sizeof(float) * kD);
+    add(sizeof(float) * C);
+    add(sizeof(int32_t) * C);
+    add(sizeof(int32_t) * (C + 1));
+    add(sizeof(int32_t) * (C + 1));
+    add(sizeof(uint32_t) * kPartCap);
+    add(sizeof(int32_t) * pc);
+    add(sizeof(int32_t) * kRowChunk);
+    add(sizeof(int32_t) * 64);
+    add(sizeof(float) * kWarps * G * 130);
+    add(sizeof(float) * S * G * 130);
+    add(sizeof(CutInfo));
+    return b;
+}
+
+struct Plan {
+    int S = 0;
+    size_t smem = 0;
+};
+
+// One launch plan per (device, group size, units, C, budget), found once. The cluster size S
+// is the largest power of two <= 16 whose clusters for all units are resident at once (one
+// wave), with U * S <= 2 * SMs; otherwise the smallest S that fits in shared memory.
 template <int G>
-int launch_g(const DecodeArgs& a, int num_sms, cudaStream_t s) {
+int plan_for(const DecodeArgs& a, int num_sms, Plan* out) {
+    static std::mutex mtx;
+    static std::map<std::tuple<int, int, int, int>, Plan> cache;
+    static size_t smem_set = 0;
+    static bool nonportable_set = false;
+    int dev = 0;
+    cudaGetDevice(&dev);
     const int U = a.B * a.Hkv;
-    int S = 1;
-    while (S * 2 <= 16 && (int64_t)U * S * 2 <= 2 * (int64_t)num_sms) S *= 2;
-    // rows of the partial share handled by one CTA: at most its share of the budget
-    const int32_t prow_cap = (int32_t)((int64_t)a.budget / S + 2);
-    auto smem_for = [&](int S_) {
-        const int32_t pc = (int32_t)((int64_t)a.budget / S_ + 2);
-        size_t b = 0;
-        auto add = [&](size_t x) { b += (x + 15) & ~(size_t)15; };
-        add(sizeof(float) * G * kD);
-        add(sizeof(float) * kD);
-        add(sizeof(float) * a.C);
-        add(sizeof(int32_t) * a.C);
-        add(sizeof(int32_t) * (a.C + 1));
-        add(sizeof(int32_t) * (a.C + 1));
-        add(sizeof(uint32_t) * kPartCap);
-        add(sizeof(int32_t) * pc);
-        add(sizeof(int32_t) * kRowChunk);
-        add(sizeof(int32_t) * 64);
-        add(sizeof(float) * kWarps * G * 130);
-        add(sizeof(float) * S_ * G * 130);
-        add(sizeof(CutInfo));
-        return b;
-    };
-    size_t smem = smem_for(S);
-    while (smem > 227 * 1024 && S > 1) {
-        S /= 2;
-        smem = smem_for(S);
+    const auto key = std::make_tuple(dev, U, a.C, a.budget);
+    std::lock_guard<std::mutex> lock(mtx);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+        *out = it->second;
+        return CKV_OK;
     }
-    if (smem > 227 * 1024) {
-        set_error("select_and_attend: shared memory need exceeds 227 KB (budget or C too large)");
+    auto kern = select_attend_kernel<G>;
+    Plan best{};
+    for (int S = 16; S >= 1; S /= 2) {
+        const size_t smem = smem_bytes(G, S, a.C, a.budget);
+        if (smem > 227 * 1024) continue;
+        if ((int64_t)U * S > 2 * (int64_t)num_sms && S > 1) continue;
+        if (smem > smem_set) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)smem);
+            if (e != cudaSuccess) return cuda_fail(e, "select_attend: set smem");
+            smem_set = smem;
+        }
+        if (S > 8 && !nonportable_set) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (e != cudaSuccess) return cuda_fail(e, "select_attend: non-portable cluster");
+            nonportable_set = true;
+        }
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3((unsigned)(U * S));
+        cfg.blockDim = dim3(kNT);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)S;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int nclusters = 0;
+        cudaError_t e = cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg);
+        if (e != cudaSuccess) {
+            (void)cudaGetLastError();
+            continue;
+        }
+        if (nclusters <= 0) continue;
+        if (best.S == 0) best = Plan{S, smem};  // fallback: fits, maybe several waves
+        if (nclusters >= U) {
+            best = Plan{S, smem};
+            break;
+        }
+        best = Plan{S, smem};
+    }
+    if (best.S == 0) {
+        set_error("select_and_attend: no launch shape fits (budget or C too large for shared memory)");
         return CKV_ECAPACITY;
     }
+    cache[key] = best;
+    *out = best;
+    return CKV_OK;
+}
+
+template <int G>
+int launch_g(const DecodeArgs& a, int num_sms, cudaStream_t s) {
+    Plan plan;
+    int rc = plan_for<G>(a, num_sms, &plan);
+    if (rc != CKV_OK) return rc;
+    const int U = a.B * a.Hkv;
+    const int S = plan.S;
     const int32_t pc = (int32_t)((int64_t)a.budget / S + 2);
-    (void)prow_cap;
-    auto kern = select_attend_kernel<G>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_fail(e, "select_attend: set smem");
-    if (S > 8) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return cuda_fail(e, "select_attend: non-portable cluster");
-    }
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)(U * S));
     cfg.blockDim = dim3(kNT);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = plan.smem;
     cfg.stream = s;
     cudaLaunchAttribute attrs[2];
     attrs[0].id = cudaLaunchAttributeClusterDimension;
@@ -595,24 +699,7 @@ int launch_g(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     attrs[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attrs;
     cfg.numAttrs = 2;
-    // A 16-CTA cluster must fit on one GPC. Fall back to 8 if the device cannot place it.
-    if (S > 8) {
-        int nclusters = 0;
-        e = cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg);
-        if (e != cudaSuccess || nclusters <= 0) {
-            (void)cudaGetLastError();
-            S = 8;
-            smem = smem_for(S);
-            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return cuda_fail(e, "select_attend: set smem");
-            cfg.gridDim = dim3((unsigned)(U * S));
-            cfg.dynamicSmemBytes = smem;
-            attrs[0].val.clusterDim.x = (unsigned)S;
-        }
-    }
-    const int32_t pc2 = (int32_t)((int64_t)a.budget / S + 2);
-    (void)pc;
-    e = cudaLaunchKernelEx(&cfg, kern, a, (int32_t)S, pc2);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, select_attend_kernel<G>, a, (int32_t)S, pc);
     if (e != cudaSuccess) return cuda_fail(e, "select_attend: launch");
     return CKV_OK;
 }

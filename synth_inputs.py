@@ -56,18 +56,26 @@ def centers(config_seed: int, unit: int, n_centers: int) -> np.ndarray:
     return c / np.linalg.norm(c, axis=1, keepdims=True)
 
 
-def _mixture(g: np.random.Generator, cen: np.ndarray, count: int, sigma: float, scale: float):
+def _mixture(g: np.random.Generator, cen: np.ndarray, count: int, sigma: float, scale: float,
+             labels: bool = False):
     j = g.integers(0, cen.shape[0], size=count)
-    return scale * (cen[j] + sigma * g.standard_normal((count, D)))
+    k = scale * (cen[j] + sigma * g.standard_normal((count, D)))
+    return (k, j) if labels else k
 
 
 def keys_values(config_seed: int, unit: int, n: int, n_centers: int,
                 sigma: float = 0.3, scale: float = 8.0):
     """K, V of one unit: ``[n, 128]`` bf16 bit patterns each."""
+    return keys_values_labeled(config_seed, unit, n, n_centers, sigma, scale)[:2]
+
+
+def keys_values_labeled(config_seed: int, unit: int, n: int, n_centers: int,
+                        sigma: float = 0.3, scale: float = 8.0):
+    """K, V of one unit plus the mixture component each token was drawn from."""
     cen = centers(config_seed, unit, n_centers)
-    k = _mixture(_rng(config_seed, TAG_KEYS, unit), cen, n, sigma, scale)
+    k, j = _mixture(_rng(config_seed, TAG_KEYS, unit), cen, n, sigma, scale, labels=True)
     v = _rng(config_seed, TAG_VALUES, unit).standard_normal((n, D))
-    return to_bf16_bits(k), to_bf16_bits(v)
+    return to_bf16_bits(k), to_bf16_bits(v), j.astype(np.int32)
 
 
 def appended_tokens(config_seed: int, unit: int, count: int, n_centers: int,
@@ -124,3 +132,16 @@ def keys_values_torch(config_seed: int, unit: int, n: int, n_centers: int, devic
 def queries_torch(config_seed: int, layer: int, b: int, steps: int, n_q_heads: int, device):
     g = _torch_gen(config_seed, TAG_QUERIES, (layer << 20) | b, device)
     return torch.randn(steps, n_q_heads, D, generator=g, device=device).to(torch.bfloat16)
+
+
+def appended_tokens_torch(config_seed: int, unit: int, count: int, n_centers: int, device,
+                          sigma: float = 0.3, scale: float = 8.0):
+    """Same recipe as :func:`appended_tokens` drawn with ``torch.Generator`` on ``device``."""
+    g = _torch_gen(config_seed, TAG_CENTERS, unit, device)
+    cen = torch.randn(n_centers, D, generator=g, device=device)
+    cen = cen / cen.norm(dim=1, keepdim=True)
+    g = _torch_gen(config_seed, TAG_APPEND, unit, device)
+    j = torch.randint(0, n_centers, (count,), generator=g, device=device)
+    k = scale * (cen[j] + sigma * torch.randn(count, D, generator=g, device=device))
+    v = torch.randn(count, D, generator=g, device=device)
+    return k.to(torch.bfloat16), v.to(torch.bfloat16)
