@@ -206,6 +206,27 @@ CKV_API int ckv_kmeans_update(ckv_ctx* ctx, const void* keys, int64_t n_rows, in
                       int32_t U, const int32_t* assign, int32_t C, float* mu, void* mu_hat,
                       int32_t* offsets, int32_t* perm, void* stream);
 
+/* ---- Allocation-free variant of ckv_kmeans_update. The pages have no counterpart for this
+ * call: it exists for callers that cannot allocate device memory, such as an engine that
+ * takes all of its memory from its own pool at start-up, a decode loop that must not stall
+ * on cudaMalloc/cudaFree (they can synchronise the device), or a plugin whose host
+ * application owns the device memory. It needs no context. The inputs and outputs are the
+ * caller's, exactly as for ckv_kmeans_update (keys bf16 [U, n_rows, 128]; assign int32
+ * [U, m]; mu fp32 [U, C, 128] in/out; mu_hat bf16 [U, C, 128]; offsets int32 [U, C + 1];
+ * perm int32 [U, m]), and so are the results.
+ * The kernels' scratch, the per-chunk cluster counts of the counting sort, is a fixed
+ * array of 2^21 int32 (8 MiB) compiled into the library. Every GPU that loads the library
+ * holds it until the process exits. A call needs U * ceil(m / 1024) * C counts. Larger
+ * requests return CKV_EINVAL with the sizes in ckv_last_error(), and nothing is enqueued.
+ * The call allocates nothing. On a device's first call it looks up the array's device
+ * address (cudaGetSymbolAddress), so make that first call before any stream capture.
+ * All calls on a device share the array: calls whose kernels overlap on the GPU (for
+ * example on two streams) race. Each call writes every count it reads, so one call's
+ * leftovers never reach the next call's results. */
+CKV_API int ckv_kmeans_update_noalloc(const void* keys, int64_t n_rows, int64_t row0, int64_t m,
+                                      int32_t U, const int32_t* assign, int32_t C, float* mu,
+                                      void* mu_hat, int32_t* offsets, int32_t* perm, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

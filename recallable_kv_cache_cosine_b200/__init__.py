@@ -66,6 +66,7 @@ SIGNATURES = {
     "ckv_kmeans_init": (C.c_int, [P, P, I64, I64, I64, I32, I32, U64, I64, U64, P, P, P, P]),
     "ckv_kmeans_assign": (C.c_int, [P, P, I64, I64, I64, I32, P, I32, P, P]),
     "ckv_kmeans_update": (C.c_int, [P, P, I64, I64, I64, I32, P, I32, P, P, P, P, P]),
+    "ckv_kmeans_update_noalloc": (C.c_int, [P, I64, I64, I64, I32, P, I32, P, P, P, P, P]),
 }
 
 _lib = None
