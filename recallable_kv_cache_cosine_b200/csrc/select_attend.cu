@@ -13,17 +13,18 @@
 // attended and counted against the budget.
 //
 // One unit (sequence b, KV head h) is served by a thread-block cluster of S CTAs:
-//   1. each CTA scores a slice of the C centroids (fp32) and broadcasts (score, size) to every
-//      CTA of the cluster through distributed shared memory;
-//   2. each CTA ranks its own slice against all C scores, which gives each cluster's rank and
-//      the number of tokens ranked before it. Whole clusters and the cut cluster follow
-//      without a sort. The whole clusters' (prefix, first row) are broadcast, indexed by rank;
+//   1. each CTA scores a slice of the C centroids (fp32; a quarter-warp per centroid) and
+//      broadcasts (score, size) to every CTA of the cluster through distributed shared memory;
+//   2. each CTA ranks its slice against all C scores (8 threads per cluster). The rank and
+//      the number of tokens ranked before each cluster give the whole clusters and the cut
+//      cluster without a sort. The whole clusters' (prefix, first row) are broadcast,
+//      indexed by rank;
 //   3. the selected rows form one index space: sinks, pending, whole clusters by rank, then
-//      the partial tokens. CTA r takes an equal share of it. The CTAs whose share reaches
-//      the partial tokens rank the cut cluster's tokens by qbar . k (comparison rank for
-//      small clusters, radix select for large ones);
-//   4. half-warps stream their rows with 16-byte loads and run an online softmax for the
-//      G query heads;
+//      the partial tokens of the cut cluster. With a partial fill and S > 1, CTA S-1 takes
+//      exactly the partial tokens and ranks the cut cluster's tokens by qbar . k (comparison
+//      rank for small clusters, radix select for large ones); the other CTAs split the rest;
+//   4. half-warps stream their rows with 16-byte loads, 4 rows per group, and run one online
+//      softmax update per group for the G query heads;
 //   5. the CTA partials (max, sum, accumulator) are merged in CTA 0 through distributed
 //      shared memory, which writes the fp32 output.
 // The kernel triggers programmatic dependent launch at entry and prefetches its centroid
@@ -56,31 +57,27 @@ CKV_DEV uint32_t orderable(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Orderable key of qbar . k for one 256-byte key row, computed by one thread: 16 independent
-// 16-byte loads, then an fp32 dot product in dimension order.
-CKV_DEV uint32_t row_key(const uint16_t* row, const float* qbar) {
-    float s = 0.f;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
+// qbar . k over one half (64 dims) of a 256-byte key row: 8 independent 16-byte loads, then
+// fp32 FMAs in dimension order.
+CKV_DEV float half_row_dot(const uint16_t* row, int half, const float* qbar) {
     uint4 w[8];
 #pragma unroll
     for (int t = 0; t < 8; ++t) w[t] = ldg_nc_v4(row + 64 * half + 8 * t);
+    const float4* q4 = reinterpret_cast<const float4*>(qbar + 64 * half);
+    float s = 0.f;
 #pragma unroll
-    for (int t0 = 0; t0 < 8; ++t0) {
-        const int t = 8 * half + t0;
-        const float4 qa = reinterpret_cast<const float4*>(qbar)[2 * t];
-        const float4 qb = reinterpret_cast<const float4*>(qbar)[2 * t + 1];
-        s = fmaf(qa.x, bf16_lo(w[t0].x), s);
-        s = fmaf(qa.y, bf16_hi(w[t0].x), s);
-        s = fmaf(qa.z, bf16_lo(w[t0].y), s);
-        s = fmaf(qa.w, bf16_hi(w[t0].y), s);
-        s = fmaf(qb.x, bf16_lo(w[t0].z), s);
-        s = fmaf(qb.y, bf16_hi(w[t0].z), s);
-        s = fmaf(qb.z, bf16_lo(w[t0].w), s);
-        s = fmaf(qb.w, bf16_hi(w[t0].w), s);
+    for (int t = 0; t < 8; ++t) {
+        const float4 qa = q4[2 * t], qb = q4[2 * t + 1];
+        s = fmaf(qa.x, bf16_lo(w[t].x), s);
+        s = fmaf(qa.y, bf16_hi(w[t].x), s);
+        s = fmaf(qa.z, bf16_lo(w[t].y), s);
+        s = fmaf(qa.w, bf16_hi(w[t].y), s);
+        s = fmaf(qb.x, bf16_lo(w[t].z), s);
+        s = fmaf(qb.y, bf16_hi(w[t].z), s);
+        s = fmaf(qb.z, bf16_lo(w[t].w), s);
+        s = fmaf(qb.w, bf16_hi(w[t].w), s);
     }
-    }
-    return orderable(s);
+    return s;
 }
 
 // Exclusive block scan of one int per thread. `tot` receives the block total.
@@ -109,22 +106,23 @@ CKV_DEV int32_t block_excl_scan(int32_t v, int32_t* wbuf, int32_t* tot) {
 struct Smem {
     float* qg;        // [G][128], scaled by log2(e)/sqrt(128)
     float* qbar;      // [128]
-    float* sc;        // [C] scores
-    int32_t* sz;      // [C] sizes
-    int32_t* spre;    // [C] prefix of the whole cluster of rank k
-    int32_t* srow;    // [C] first store row of the whole cluster of rank k
+    int2* scsz;       // [C] (score bits, size) of every cluster
+    int32_t* crow;    // [C] first store row of the clusters this CTA scored
+    int32_t* spre;    // [C + 1] prefix of the whole cluster of rank k
+    int32_t* srow;    // [C + 1] first store row of the whole cluster of rank k
     uint32_t* pkey;   // [kPartCap] cut-cluster token keys
-    int32_t* prow;    // [kRowChunk.. ] partial rows for this CTA's share
+    int32_t* prow;    // [prow_cap] partial rows of this CTA's share
     int32_t* rows;    // [kRowChunk] row list of the current chunk
     int32_t* wbuf;    // [64] scan / misc scratch
     float* wcomb;     // [kWarps][G][130]
+    float* scl;       // [(kWarps + S) * G] merge scales, then [2 * G] sums
     float* ccomb;     // [S][G][130] (filled in CTA 0)
     CutInfo* cut;
 };
 
 template <int G>
-__global__ void __launch_bounds__(kNT, (G <= 4) ? 2 : 1) select_attend_kernel(const DecodeArgs a, int32_t S,
-                                                            int32_t prow_cap) {
+__global__ void __launch_bounds__(kNT, (G <= 4) ? 2 : 1)
+    select_attend_kernel(const DecodeArgs a, int32_t S, int32_t prow_cap) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     const int C = a.C;
     const uint32_t rank = cluster_ctarank();
@@ -142,8 +140,8 @@ __global__ void __launch_bounds__(kNT, (G <= 4) ? 2 : 1) select_attend_kernel(co
         };
         sm.qg = (float*)take(sizeof(float) * G * kD);
         sm.qbar = (float*)take(sizeof(float) * kD);
-        sm.sc = (float*)take(sizeof(float) * C);
-        sm.sz = (int32_t*)take(sizeof(int32_t) * C);
+        sm.scsz = (int2*)take(sizeof(int2) * C);
+        sm.crow = (int32_t*)take(sizeof(int32_t) * C);
         sm.spre = (int32_t*)take(sizeof(int32_t) * (C + 1));
         sm.srow = (int32_t*)take(sizeof(int32_t) * (C + 1));
         sm.pkey = (uint32_t*)take(sizeof(uint32_t) * kPartCap);
@@ -151,6 +149,7 @@ __global__ void __launch_bounds__(kNT, (G <= 4) ? 2 : 1) select_attend_kernel(co
         sm.rows = (int32_t*)take(sizeof(int32_t) * kRowChunk);
         sm.wbuf = (int32_t*)take(sizeof(int32_t) * 64);
         sm.wcomb = (float*)take(sizeof(float) * kWarps * G * 130);
+        sm.scl = (float*)take(sizeof(float) * ((kWarps + S) * G + 2 * G));
         sm.ccomb = (float*)take(sizeof(float) * S * G * 130);
         sm.cut = (CutInfo*)take(sizeof(CutInfo));
     }
@@ -172,24 +171,25 @@ __global__ void __launch_bounds__(kNT, (G <= 4) ? 2 : 1) select_attend_kernel(co
 
     // ---------------------------------------------------------------- phase 1: scores
     // A quarter-warp (8 lanes) per centroid, 16 dimensions per lane: 32 centroids per CTA
-    // per round. The first round's centroid and size loads are issued before the query
+    // per round. The first round's centroid and offset loads are issued before the query
     // loads, so both share one memory round trip.
     const int32_t pend = a.pending;
-    const int64_t R = (int64_t)a.budget - a.n_sink - pend;  // >= 0 (host-checked)
+    const int32_t R = a.budget - a.n_sink - pend;  // >= 0 (host-checked)
     const int q8 = lane >> 3, l8 = lane & 7;
     constexpr int kPerRound = kWarps * 4;
     float4 mv[4];
-    int32_t csize = 0;
+    int32_t c_lo_row = 0, c_hi_row = 0;
     auto load_centroid = [&](int c) {
         if (c < c_end) {
             const float4* row = reinterpret_cast<const float4*>(mu + (int64_t)c * kD) + l8 * 4;
 #pragma unroll
             for (int t = 0; t < 4; ++t) mv[t] = row[t];
-            csize = off[c + 1] - off[c];
+            c_lo_row = off[c];
+            c_hi_row = off[c + 1];
         } else {
 #pragma unroll
             for (int t = 0; t < 4; ++t) mv[t] = make_float4(0.f, 0.f, 0.f, 0.f);
-            csize = 0;
+            c_lo_row = c_hi_row = 0;
         }
     };
     load_centroid(c_begin + warp * 4 + q8);
@@ -224,9 +224,13 @@ __global__ void __launch_bounds__(kNT, (G <= 4) ? 2 : 1) select_attend_kernel(co
         s += __shfl_xor_sync(0xffffffffu, s, 2);
         s += __shfl_xor_sync(0xffffffffu, s, 1);
         if (c < c_end) {
+            if (l8 == 0) sm.crow[c] = c_lo_row;
+            const uint32_t sz = (uint32_t)(c_hi_row - c_lo_row);
             for (int r = l8; r < S; r += 8) {
-                st_cluster_f32(map_shared_rank(smem_u32(&sm.sc[c]), r), s);
-                st_cluster_u32(map_shared_rank(smem_u32(&sm.sz[c]), r), (uint32_t)csize);
+                const uint32_t dst = map_shared_rank(smem_u32(&sm.scsz[c]), r);
+                asm volatile("st.shared::cluster.v2.u32 [%0], {%1, %2};" ::"r"(dst),
+                             "r"(__float_as_uint(s)), "r"(sz)
+                             : "memory");
             }
         }
     }
@@ -234,36 +238,48 @@ __global__ void __launch_bounds__(kNT, (G <= 4) ? 2 : 1) select_attend_kernel(co
     cluster_wait_acquire();
 
     // ---------------------------------------------------------------- phase 2: ranks
-    for (int c = c_begin + warp; c < c_end; c += kWarps) {
-        const float s = sm.sc[c];
-        int32_t rk = 0;
-        int64_t pre = 0;
-        for (int j = lane; j < C; j += 32) {
-            const float t = sm.sc[j];
-            if (t > s || (t == s && j < c)) {
-                ++rk;
-                pre += sm.sz[j];
-            }
+    // 8 threads per cluster of this CTA's slice; each compares 1/8 of all C clusters.
+    for (int c0 = c_begin; c0 < c_end; c0 += kNT / 8) {
+        const int c = c0 + (threadIdx.x >> 3);
+        const int sub = threadIdx.x & 7;
+        float s = 0.f;
+        int32_t size = 0;
+        if (c < c_end) {
+            const int2 me = sm.scsz[c];
+            s = __int_as_float(me.x);
+            size = me.y;
+        }
+        int32_t rk = 0, pre = 0;
+#pragma unroll 4
+        for (int j = sub; j < C; j += 8) {
+            const int2 o = sm.scsz[j];
+            const float t = __int_as_float(o.x);
+            const bool before = (t > s) || (t == s && j < c);
+            rk += before ? 1 : 0;
+            pre += before ? o.y : 0;
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
+        for (int o = 4; o > 0; o >>= 1) {
             rk += __shfl_xor_sync(0xffffffffu, rk, o);
             pre += __shfl_xor_sync(0xffffffffu, pre, o);
         }
-        const int32_t size = sm.sz[c];
-        if (pre + size <= R) {  // whole cluster
-            if (lane < S) {
-                st_cluster_u32(map_shared_rank(smem_u32(&sm.spre[rk]), lane), (uint32_t)pre);
-                st_cluster_u32(map_shared_rank(smem_u32(&sm.srow[rk]), lane), (uint32_t)off[c]);
-            }
-        } else if (pre <= R) {  // the cut cluster (R < pre + size)
-            if (lane < S) {
-                const uint32_t base = map_shared_rank(smem_u32(sm.cut), lane);
-                st_cluster_u32(base + 0, (uint32_t)c);
-                st_cluster_u32(base + 4, (uint32_t)pre);
-                st_cluster_u32(base + 8, (uint32_t)rk);
-                st_cluster_u32(base + 12, (uint32_t)off[c]);
-                st_cluster_u32(base + 16, (uint32_t)size);
+        if (c < c_end) {
+            if (pre + size <= R) {  // whole cluster
+                const int32_t row = sm.crow[c];
+                for (int r = sub; r < S; r += 8) {
+                    st_cluster_u32(map_shared_rank(smem_u32(&sm.spre[rk]), r), (uint32_t)pre);
+                    st_cluster_u32(map_shared_rank(smem_u32(&sm.srow[rk]), r), (uint32_t)row);
+                }
+            } else if (pre <= R) {  // the cut cluster (R < pre + size)
+                const int32_t row = sm.crow[c];
+                for (int r = sub; r < S; r += 8) {
+                    const uint32_t base = map_shared_rank(smem_u32(sm.cut), r);
+                    st_cluster_u32(base + 0, (uint32_t)c);
+                    st_cluster_u32(base + 4, (uint32_t)pre);
+                    st_cluster_u32(base + 8, (uint32_t)rk);
+                    st_cluster_u32(base + 12, (uint32_t)row);
+                    st_cluster_u32(base + 16, (uint32_t)size);
+                }
             }
         }
     }
@@ -277,7 +293,21 @@ __global__ void __launch_bounds__(kNT, (G <= 4) ? 2 : 1) select_attend_kernel(co
     const int64_t base_w = (int64_t)a.n_sink + pend;
     const int64_t base_p = base_w + W;
     const int64_t T = base_p + r_part;
-    const int64_t lo = T * rank / S, hi = T * (rank + 1) / S;
+    // Work split of the selection index space [0, T). With a partial fill, CTA S-1 takes
+    // exactly the partial tokens (it also ranks them) and the other CTAs split the rest.
+    int64_t lo, hi;
+    if (r_part > 0 && S > 1 && r_part <= prow_cap) {
+        if ((int)rank == S - 1) {
+            lo = base_p;
+            hi = T;
+        } else {
+            lo = base_p * rank / (S - 1);
+            hi = base_p * (rank + 1) / (S - 1);
+        }
+    } else {
+        lo = T * rank / S;
+        hi = T * (rank + 1) / S;
+    }
 
     // ---------------------------------------------------------------- phase 3: partial
     // This CTA's share of the partial tokens: positions [p_lo, p_hi) in store order.
@@ -288,12 +318,21 @@ __global__ void __launch_bounds__(kNT, (G <= 4) ? 2 : 1) select_attend_kernel(co
     uint32_t* gkeys = a.part_scratch ? reinterpret_cast<uint32_t*>(a.part_scratch) +
                                            (int64_t)unit * a.part_ustride
                                      : nullptr;
+    auto score_keys = [&](int64_t k0, int64_t k1, uint32_t* dst, int32_t crow) {
+        // two threads per row, one memory round trip per pass
+        for (int64_t i0 = k0; i0 < k1; i0 += kNT / 2) {
+            const int64_t i = i0 + (threadIdx.x >> 1);
+            const int half = threadIdx.x & 1;
+            float s = 0.f;
+            if (i < k1) s = half_row_dot(a.kp + (kp_base + crow + i) * kD, half, sm.qbar);
+            s += __shfl_xor_sync(0xffffffffu, s, 1);
+            if (i < k1 && half == 0) dst[i] = orderable(s);
+        }
+    };
     if (r_part > 0 && big_cut) {
         // Keys of a large cut cluster are written once, split across the cluster's CTAs.
-        const int32_t crow = sm.cut->row;
         const int64_t k0 = (int64_t)csz * rank / S, k1 = (int64_t)csz * (rank + 1) / S;
-        for (int64_t i = k0 + threadIdx.x; i < k1; i += kNT)
-            gkeys[i] = row_key(a.kp + (kp_base + crow + i) * kD, sm.qbar);
+        score_keys(k0, k1, gkeys, sm.cut->row);
         cluster_arrive_release();
         cluster_wait_acquire();
     }
@@ -302,37 +341,44 @@ __global__ void __launch_bounds__(kNT, (G <= 4) ? 2 : 1) select_attend_kernel(co
         const uint32_t* skeys = sm.pkey;
         auto key_at = [&](int i) -> uint32_t { return big_cut ? __ldcg(gkeys + i) : skeys[i]; };
         if (!big_cut) {
-            for (int i = threadIdx.x; i < csz; i += kNT)
-                sm.pkey[i] = row_key(a.kp + (kp_base + crow + i) * kD, sm.qbar);
+            score_keys(0, csz, sm.pkey, crow);
+            if (threadIdx.x < 4) sm.pkey[csz + threadIdx.x] = 0u;  // pad: never outranks a key
         }
         __syncthreads();
-        // Threshold: key theta and `need` = how many keys equal to theta are taken (the
-        // lowest-index ones), so that exactly r_part tokens are selected.
-        uint32_t theta;
-        int32_t need;
-        if (csz <= kNT) {
-            // comparison rank (ties: lower index)
-            int32_t sel = 0;
-            if (threadIdx.x < csz) {
-                const uint32_t ki = key_at(threadIdx.x);
-                int32_t rk = 0;
-                for (int j = 0; j < csz; ++j) {
-                    const uint32_t kj = key_at(j);
-                    rk += (kj > ki) || (kj == ki && j < (int)threadIdx.x);
+        if (!big_cut && csz <= kNT) {
+            // comparison rank (ties: lower index), tpe threads per token, 4 keys per load
+            const int tpe = csz <= 32 ? 8 : (csz <= 64 ? 4 : (csz <= 128 ? 2 : 1));
+            const int e = threadIdx.x / tpe, sub = threadIdx.x % tpe;
+            int32_t rk = 0;
+            if (e < csz) {
+                const uint32_t ke = sm.pkey[e];
+                const uint4* k4 = reinterpret_cast<const uint4*>(sm.pkey);
+                const int n4 = (csz + 3) >> 2;
+#pragma unroll 4
+                for (int j4 = sub; j4 < n4; j4 += tpe) {
+                    const uint4 v = k4[j4];
+                    const int j = 4 * j4;
+                    rk += (v.x > ke) || (v.x == ke && j < e);
+                    rk += (v.y > ke) || (v.y == ke && j + 1 < e);
+                    rk += (v.z > ke) || (v.z == ke && j + 2 < e);
+                    rk += (v.w > ke) || (v.w == ke && j + 3 < e);
                 }
-                sel = rk < r_part;
             }
+#pragma unroll
+            for (int o = 4; o > 0; o >>= 1) {
+                const int32_t y = __shfl_xor_sync(0xffffffffu, rk, o);
+                if (o < tpe) rk += y;
+            }
+            const int32_t sel = (e < csz && sub == 0 && rk < r_part) ? 1 : 0;
             int32_t tot;
             const int32_t pos = block_excl_scan(sel, sm.wbuf, &tot);
-            if (sel && pos >= p_lo && pos < p_hi) sm.prow[pos - p_lo] = crow + threadIdx.x;
-            theta = 0;
-            need = 0;
-            (void)theta;
-            (void)need;
+            if (sel && pos >= p_lo && pos < p_hi) sm.prow[pos - p_lo] = crow + e;
         } else {
-            // radix select over 4 digits of 8 bits, most significant first
+            // radix select over 4 digits of 8 bits, most significant first: the threshold key
+            // theta and `need` = how many keys equal to theta are taken (the lowest-index
+            // ones), so that exactly r_part tokens are selected.
             uint32_t prefix = 0, mask = 0;
-            need = r_part;
+            int32_t need = r_part;
             int32_t* hist = (int32_t*)sm.wcomb;  // 256 counters (scratch, unused until phase 5)
             for (int pass = 0; pass < 4; ++pass) {
                 const int shift = 24 - 8 * pass;
@@ -376,8 +422,7 @@ __global__ void __launch_bounds__(kNT, (G <= 4) ? 2 : 1) select_attend_kernel(co
                 mask |= 255u << shift;
                 __syncthreads();
             }
-            theta = prefix;
-            // select: key > theta, or key == theta among the first `need` such keys
+            const uint32_t theta = prefix;
             int32_t eq_run = 0, sel_run = 0;
             for (int base = 0; base < csz; base += kNT) {
                 const int i = base + threadIdx.x;
@@ -425,10 +470,10 @@ __global__ void __launch_bounds__(kNT, (G <= 4) ? 2 : 1) select_attend_kernel(co
                     if (sm.spre[mid] <= x) lo2 = mid; else hi2 = mid - 1;
                 }
                 row = sm.srow[lo2] + (x - sm.spre[lo2]);
-                oid = ids[row];
+                oid = sel_out ? ids[row] : 0;
             } else {
                 row = sm.prow[idx - base_p - p_lo];
-                oid = ids[row];
+                oid = sel_out ? ids[row] : 0;
             }
             sm.rows[threadIdx.x] = row;
             if (sel_out) sel_out[idx] = oid;
@@ -438,11 +483,13 @@ __global__ void __launch_bounds__(kNT, (G <= 4) ? 2 : 1) select_attend_kernel(co
         // below need both half-warps of a warp in every iteration.
         for (int j0 = 0; j0 < n; j0 += 4 * (kNT / 16)) {
             uint4 kw[4], vw[4];
-            int valid[4];
+            bool valid[4];
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
                 const int j = j0 + hw + t * (kNT / 16);
                 valid[t] = j < n;
+                kw[t] = make_uint4(0u, 0u, 0u, 0u);
+                vw[t] = kw[t];
                 if (valid[t]) {
                     const int32_t row = sm.rows[j];
                     const uint16_t* kr = row >= 0 ? a.kp + (kp_base + row) * kD
@@ -453,53 +500,62 @@ __global__ void __launch_bounds__(kNT, (G <= 4) ? 2 : 1) select_attend_kernel(co
                     vw[t] = ldg_nc_v4(vr + l16 * 8);
                 }
             }
+            // logits of the 4 rows for every head (full-mask shuffles: all lanes)
+            float z[4][G];
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
-                // Every lane runs the shuffles below; rows past the chunk end only skip
-                // the state update.
-                if (!valid[t]) {
-                    kw[t] = make_uint4(0u, 0u, 0u, 0u);
-                    vw[t] = kw[t];
-                }
-                float kf[8], vf[8];
-                const uint32_t kk[4] = {kw[t].x, kw[t].y, kw[t].z, kw[t].w};
-                const uint32_t vv[4] = {vw[t].x, vw[t].y, vw[t].z, vw[t].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    kf[2 * e] = bf16_lo(kk[e]);
-                    kf[2 * e + 1] = bf16_hi(kk[e]);
-                    vf[2 * e] = bf16_lo(vv[e]);
-                    vf[2 * e + 1] = bf16_hi(vv[e]);
-                }
-                float z[G];
+                const float k0 = bf16_lo(kw[t].x), k1 = bf16_hi(kw[t].x), k2 = bf16_lo(kw[t].y),
+                            k3 = bf16_hi(kw[t].y), k4 = bf16_lo(kw[t].z), k5 = bf16_hi(kw[t].z),
+                            k6 = bf16_lo(kw[t].w), k7 = bf16_hi(kw[t].w);
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
                     const float4 qa = qg4[g * (kD / 4)];
                     const float4 qb = qg4[g * (kD / 4) + 1];
-                    float s = qa.x * kf[0];
-                    s = fmaf(qa.y, kf[1], s);
-                    s = fmaf(qa.z, kf[2], s);
-                    s = fmaf(qa.w, kf[3], s);
-                    s = fmaf(qb.x, kf[4], s);
-                    s = fmaf(qb.y, kf[5], s);
-                    s = fmaf(qb.z, kf[6], s);
-                    s = fmaf(qb.w, kf[7], s);
-                    z[g] = s;
+                    float s = qa.x * k0;
+                    s = fmaf(qa.y, k1, s);
+                    s = fmaf(qa.z, k2, s);
+                    s = fmaf(qa.w, k3, s);
+                    s = fmaf(qb.x, k4, s);
+                    s = fmaf(qb.y, k5, s);
+                    s = fmaf(qb.z, k6, s);
+                    s = fmaf(qb.w, k7, s);
+                    z[t][g] = s;
                 }
+            }
 #pragma unroll
-                for (int o = 8; o > 0; o >>= 1)
+            for (int o = 8; o > 0; o >>= 1)
 #pragma unroll
-                    for (int g = 0; g < G; ++g) z[g] += __shfl_xor_sync(0xffffffffu, z[g], o);
-                if (!valid[t]) continue;
+                for (int t = 0; t < 4; ++t)
 #pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float mn = fmaxf(mrun[g], z[g]);
-                    const float corr = exp2f(mrun[g] - mn);
-                    const float pz = exp2f(z[g] - mn);
-                    lrun[g] = lrun[g] * corr + pz;
+                    for (int g = 0; g < G; ++g) z[t][g] += __shfl_xor_sync(0xffffffffu, z[t][g], o);
+            if (!valid[0]) continue;  // no row of this group for this half-warp
+            // one online-softmax update per head for the whole group
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(pz, vf[e], acc[g][e] * corr);
-                    mrun[g] = mn;
+            for (int g = 0; g < G; ++g) {
+                float mx = mrun[g];
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+                    if (valid[t]) mx = fmaxf(mx, z[t][g]);
+                const float corr = mrun[g] == -INFINITY ? 0.f : exp2f(mrun[g] - mx);
+                float p[4];
+                float psum = 0.f;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    p[t] = valid[t] ? exp2f(z[t][g] - mx) : 0.f;
+                    psum += p[t];
+                }
+                lrun[g] = lrun[g] * corr + psum;
+                mrun[g] = mx;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[g][e] *= corr;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const uint32_t vv[4] = {vw[t].x, vw[t].y, vw[t].z, vw[t].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        acc[g][2 * e] = fmaf(p[t], bf16_lo(vv[e]), acc[g][2 * e]);
+                        acc[g][2 * e + 1] = fmaf(p[t], bf16_hi(vv[e]), acc[g][2 * e + 1]);
+                    }
                 }
             }
         }
@@ -536,24 +592,46 @@ __global__ void __launch_bounds__(kNT, (G <= 4) ? 2 : 1) select_attend_kernel(co
         }
     }
     __syncthreads();
+    // per-head merge scales of the 8 warps, computed once
+    float* wsc = sm.scl;                     // [kWarps][G]
+    float* rsc = sm.scl + kWarps * G;        // [S][G]
+    float* sums = sm.scl + (kWarps + S) * G; // [G] max, [G] sum
+    // thread (g, w) in groups of 8 lanes: warp w's state for head g
+    static_assert(kWarps == 8, "the merge below maps one lane per warp in groups of 8");
+    if (threadIdx.x < 8 * G) {
+        // lanes of this warp taking part: 8 per head, heads in order (groups stay aligned)
+        const int active = min(32, 8 * G - 32 * warp);
+        const uint32_t gmask = active >= 32 ? 0xffffffffu : ((1u << active) - 1u);
+        const int g = threadIdx.x >> 3, w = threadIdx.x & 7;
+        const float mw = sm.wcomb[(w * G + g) * 130 + 128];
+        float mx = mw;
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(gmask, mx, o));
+        const float sc = mw == -INFINITY ? 0.f : exp2f(mw - mx);
+        wsc[w * G + g] = sc;
+        float l = sm.wcomb[(w * G + g) * 130 + 129] * sc;
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) l += __shfl_xor_sync(gmask, l, o);
+        if (w == 0) {
+            sums[g] = mx;
+            sums[G + g] = l;
+        }
+    }
+    __syncthreads();
     // warps -> CTA partial, written into CTA 0's combine buffer
     {
         const uint32_t dst0 = map_shared_rank(smem_u32(sm.ccomb), 0);
         for (int t = threadIdx.x; t < G * 130; t += kNT) {
             const int g = t / 130, e = t % 130;
-            float mx = -INFINITY;
-            for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, sm.wcomb[(w * G + g) * 130 + 128]);
             float v;
             if (e == 128) {
-                v = mx;
+                v = sums[g];
+            } else if (e == 129) {
+                v = sums[G + g];
             } else {
-                float sacc = 0.f;
-                for (int w = 0; w < kWarps; ++w) {
-                    const float mw = sm.wcomb[(w * G + g) * 130 + 128];
-                    const float cw = mw == -INFINITY ? 0.f : exp2f(mw - mx);
-                    sacc += sm.wcomb[(w * G + g) * 130 + e] * cw;
-                }
-                v = sacc;
+                v = 0.f;
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) v = fmaf(sm.wcomb[(w * G + g) * 130 + e], wsc[w * G + g], v);
             }
             st_cluster_f32(dst0 + (uint32_t)(((rank * G + g) * 130 + e) * 4), v);
         }
@@ -561,19 +639,27 @@ __global__ void __launch_bounds__(kNT, (G <= 4) ? 2 : 1) select_attend_kernel(co
     cluster_arrive_release();
     cluster_wait_acquire();
     if (rank == 0) {
+        // thread (g, r) in groups of S lanes (S is a power of two <= 16)
+        if (threadIdx.x < S * G) {
+            const int active = min(32, S * G - 32 * warp);
+            const uint32_t gmask = active >= 32 ? 0xffffffffu : ((1u << active) - 1u);
+            const int g = threadIdx.x / S, r = threadIdx.x % S;
+            const float mr = sm.ccomb[(r * G + g) * 130 + 128];
+            float mx = mr;
+            for (int o = S >> 1; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(gmask, mx, o));
+            const float sc = mr == -INFINITY ? 0.f : exp2f(mr - mx);
+            rsc[r * G + g] = sc;
+            float l = sm.ccomb[(r * G + g) * 130 + 129] * sc;
+            for (int o = S >> 1; o > 0; o >>= 1) l += __shfl_xor_sync(gmask, l, o);
+            if (r == 0) sums[G + g] = 1.f / l;
+        }
+        __syncthreads();
         float* o = a.out + ((int64_t)b * a.Hkv * G + (int64_t)h * G) * kD;
         for (int t = threadIdx.x; t < G * kD; t += kNT) {
             const int g = t / kD, d = t % kD;
-            float mx = -INFINITY;
-            for (int r = 0; r < S; ++r) mx = fmaxf(mx, sm.ccomb[(r * G + g) * 130 + 128]);
-            float num = 0.f, den = 0.f;
-            for (int r = 0; r < S; ++r) {
-                const float* pr = sm.ccomb + (r * G + g) * 130;
-                const float cw = pr[128] == -INFINITY ? 0.f : exp2f(pr[128] - mx);
-                num += pr[d] * cw;
-                den += pr[129] * cw;
-            }
-            o[t] = num / den;
+            float num = 0.f;
+            for (int r = 0; r < S; ++r) num = fmaf(sm.ccomb[(r * G + g) * 130 + d], rsc[r * G + g], num);
+            o[t] = num * sums[G + g];
         }
         if (a.sel_count && threadIdx.x == 0) a.sel_count[unit] = (int32_t)T;
     }
@@ -582,13 +668,18 @@ __global__ void __launch_bounds__(kNT, (G <= 4) ? 2 : 1) select_attend_kernel(co
     }
 }
 
+// Rows of partial tokens one CTA may own: twice the even share of the budget. The dedicated
+// partial CTA is used only when the partial fill fits it; otherwise the even split applies,
+// whose share is at most budget / S + 1.
+int32_t prow_capacity(int budget, int S) { return (int32_t)(2 * ((int64_t)budget / S) + 2); }
+
 size_t smem_bytes(int G, int S, int C, int budget) {
-    const int32_t pc = (int32_t)((int64_t)budget / S + 2);
+    const int32_t pc = prow_capacity(budget, S);
     size_t b = 0;
     auto add = [&](size_t x) { b += (x + 15) & ~(size_t)15; };
     add(sizeof(float) * G * kD);
     add(sizeof(float) * kD);
-    add(sizeof(float) * C);
+    add(sizeof(int2) * C);
     add(sizeof(int32_t) * C);
     add(sizeof(int32_t) * (C + 1));
     add(sizeof(int32_t) * (C + 1));
@@ -597,6 +688,7 @@ size_t smem_bytes(int G, int S, int C, int budget) {
     add(sizeof(int32_t) * kRowChunk);
     add(sizeof(int32_t) * 64);
     add(sizeof(float) * kWarps * G * 130);
+    add(sizeof(float) * ((kWarps + S) * G + 2 * G));
     add(sizeof(float) * S * G * 130);
     add(sizeof(CutInfo));
     return b;
@@ -684,7 +776,7 @@ int launch_g(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     if (rc != CKV_OK) return rc;
     const int U = a.B * a.Hkv;
     const int S = plan.S;
-    const int32_t pc = (int32_t)((int64_t)a.budget / S + 2);
+    const int32_t pc = prow_capacity(a.budget, S);
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)(U * S));
     cfg.blockDim = dim3(kNT);
