@@ -3,8 +3,10 @@
 #include <cudaTypedefs.h>
 #include <stdio.h>
 
+#include <map>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "ckv_common.cuh"
 #include "ckv_internal.h"
@@ -31,6 +33,20 @@ int num_sms_of_current_device() {
         cache[dev] = v > 0 ? v : 148;
     }
     return cache[dev];
+}
+
+int ensure_smem(const void* func, size_t bytes, const char* what) {
+    static std::mutex mtx;
+    static std::map<std::pair<int, const void*>, size_t> done;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mtx);
+    size_t& cur = done[std::make_pair(dev, func)];
+    if (bytes <= cur) return CKV_OK;
+    cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    cur = bytes;
+    return CKV_OK;
 }
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -266,9 +282,12 @@ int cluster_prefill(ckv_ctx* ctx, int32_t layer, const void* K, const void* V, i
     rl.ids = c->ids + c->rows_kp(layer, 0);
     rl.ustride_rows = c->cap_c;
     rl.id_base = ns;
+    AssignPlan plan;
+    rc = prepare_kmeans_assign(kv, c->ws.mu_hat, cmax, C, c->ws.assign, c->cap_c, c->ws.best,
+                               c->cap_c, c->err, &plan);
+    if (rc) return rc;
     for (int it = 0; it < c->cfg.iters; ++it) {
-        rc = launch_kmeans_assign(kv, c->ws.mu_hat, cmax, C, c->ws.assign, c->cap_c, c->ws.best,
-                                  c->cap_c, c->err, s);
+        rc = run_kmeans_assign(plan, s);
         if (rc) return rc;
         const bool last = it + 1 == c->cfg.iters;
         rc = launch_kmeans_update(kv, c->ws.assign, c->cap_c, C, mu, cmax, c->ws.mu_hat, cmax,
@@ -450,11 +469,11 @@ int ckv_export_unit(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h,
     cudaStream_t s = (cudaStream_t)stream;
     const int64_t sp = c->cfg.n_sink + L.pending;
     struct Item { void* d; const void* s; size_t n; } items[] = {
-        {dst->mu, c->mu + c->mu_rows(layer, u) * kD, sizeof(float) * L.C * kD},
-        {dst->offsets, c->offsets + c->off_base(layer, u), sizeof(int32_t) * (L.C + 1)},
-        {dst->ids, c->ids + c->rows_kp(layer, u), sizeof(int32_t) * L.m},
-        {dst->kp, c->kp + c->rows_kp(layer, u) * kD, 2 * L.m * kD},
-        {dst->vp, c->vp + c->rows_kp(layer, u) * kD, 2 * L.m * kD},
+        {dst->mu, c->mu + c->mu_rows(layer, u) * kD, sizeof(float) * (size_t)L.C * kD},
+        {dst->offsets, c->offsets + c->off_base(layer, u), sizeof(int32_t) * (size_t)(L.C + 1)},
+        {dst->ids, c->ids + c->rows_kp(layer, u), sizeof(int32_t) * (size_t)L.m},
+        {dst->kp, c->kp + c->rows_kp(layer, u) * kD, (size_t)(2 * L.m * kD)},
+        {dst->vp, c->vp + c->rows_kp(layer, u) * kD, (size_t)(2 * L.m * kD)},
         {dst->sp_k, c->spk + c->rows_sp(layer, u) * kD, (size_t)(2 * sp * kD)},
         {dst->sp_v, c->spv + c->rows_sp(layer, u) * kD, (size_t)(2 * sp * kD)},
     };
@@ -500,9 +519,9 @@ int ckv_import_unit(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h, int64_t m
     const int u = b * c->cfg.n_kv_heads + h;
     const int64_t sp = c->cfg.n_sink + pending;
     struct Item { void* d; const void* s; size_t n; } items[] = {
-        {c->mu + c->mu_rows(layer, u) * kD, src->mu, sizeof(float) * C * kD},
-        {c->offsets + c->off_base(layer, u), src->offsets, sizeof(int32_t) * (C + 1)},
-        {c->ids + c->rows_kp(layer, u), src->ids, sizeof(int32_t) * m},
+        {c->mu + c->mu_rows(layer, u) * kD, src->mu, sizeof(float) * (size_t)C * kD},
+        {c->offsets + c->off_base(layer, u), src->offsets, sizeof(int32_t) * (size_t)(C + 1)},
+        {c->ids + c->rows_kp(layer, u), src->ids, sizeof(int32_t) * (size_t)m},
         {c->kp + c->rows_kp(layer, u) * kD, src->kp, (size_t)(2 * m * kD)},
         {c->vp + c->rows_kp(layer, u) * kD, src->vp, (size_t)(2 * m * kD)},
         {c->spk + c->rows_sp(layer, u) * kD, src->sp_k, (size_t)(2 * sp * kD)},

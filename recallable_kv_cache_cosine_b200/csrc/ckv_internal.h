@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <memory>
 #include <string>
 #include <vector>
 
@@ -86,6 +87,10 @@ int encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
 
 int num_sms_of_current_device();
 
+// Raises a kernel's dynamic shared-memory limit to at least `bytes` on the current device.
+// The attribute is set once per (device, kernel, size increase), not on every launch.
+int ensure_smem(const void* func, size_t bytes, const char* what);
+
 // ---- launchers (each returns CKV_OK or an error code; all asynchronous on `stream`)
 int launch_kmeans_init(const KeysView& k, int32_t C, uint64_t seed, int64_t unit_base,
                        uint64_t window, int32_t* init_idx, float* mu, int64_t mu_ustride,
@@ -94,6 +99,18 @@ int launch_kmeans_init(const KeysView& k, int32_t C, uint64_t seed, int64_t unit
 int launch_kmeans_assign(const KeysView& k, const uint16_t* mu_hat, int64_t muhat_ustride,
                          int32_t C, int32_t* assign, int64_t assign_ustride, float* best,
                          int64_t best_ustride, uint32_t* err, cudaStream_t s);
+
+// The same launch split in two: prepare encodes the tensor maps and launch shapes once (they
+// depend only on pointers and sizes), run launches them. cluster_prefill prepares once and
+// runs once per Lloyd iteration.
+struct AssignPlanImpl;
+struct AssignPlan {
+    std::shared_ptr<AssignPlanImpl> impl;
+};
+int prepare_kmeans_assign(const KeysView& k, const uint16_t* mu_hat, int64_t muhat_ustride,
+                          int32_t C, int32_t* assign, int64_t assign_ustride, float* best,
+                          int64_t best_ustride, uint32_t* err, AssignPlan* out);
+int run_kmeans_assign(const AssignPlan& plan, cudaStream_t s);
 
 struct Relayout {  // final-iteration relayout of K and V into the cluster-major store
     const uint16_t* V = nullptr;  // same shape as the keys tensor

@@ -46,39 +46,63 @@ CKV_DEV float4 load_row4_bf16(const uint16_t* row) {
 // ---------------------------------------------------------------------- init
 // Seeded init: the first C entries of a Fisher-Yates shuffle of 0..m-1, driven by SplitMix64
 // with key seed ^ (unit << 32) ^ window, each draw mapped into [0, m-i) by Lemire's
-// multiply-shift. Only the <= C displaced positions of the virtual array are stored, in a
-// shared-memory open-addressing table.
+// multiply-shift. SplitMix64 is counter-based (draw i mixes key + (i+1) * gamma), so the C
+// swap targets are computed in parallel. Only the swaps run in order, on a dense
+// shared-memory copy of the index array when it fits (`dense`, chosen by the host from the
+// shared-memory size), otherwise on an open-addressing table of the <= C displaced positions.
+constexpr size_t kInitSmemLimit = 200 * 1024;
+
 __global__ void __launch_bounds__(256) kmeans_init_kernel(KeysView k, int32_t C, uint64_t seed,
                                                           int64_t unit_base, uint64_t window,
                                                           int32_t* init_idx, float* mu,
                                                           int64_t mu_ustride, uint16_t* mu_hat,
-                                                          int64_t muhat_ustride, int32_t tbits) {
+                                                          int64_t muhat_ustride, int32_t tbits,
+                                                          int32_t dense) {
     extern __shared__ int32_t sm[];
-    const int32_t tsize = 1 << tbits;
-    int32_t* tkey = sm;
-    int32_t* tval = sm + tsize;
-    int32_t* chosen = sm + 2 * tsize;
     const int u = blockIdx.x;
-    for (int i = threadIdx.x; i < tsize; i += blockDim.x) tkey[i] = -1;
+    const int32_t m = (int32_t)k.m;
+    int32_t* target = sm;          // [C] swap target of step i
+    int32_t* chosen = sm + C;      // [C]
+    int32_t* work = sm + 2 * C;    // dense [m] array, or table keys [2^tbits] + values [2^tbits]
+    const uint64_t key = seed ^ ((uint64_t)(unit_base + u) << 32) ^ window;
+    for (int i = threadIdx.x; i < C; i += blockDim.x) {
+        uint64_t st = key + (uint64_t)i * 0x9E3779B97F4A7C15ull;  // state before draw i
+        const uint64_t x = splitmix64_next(st);
+        target[i] = i + (int32_t)bounded_draw(x, (uint32_t)(m - i));
+    }
+    const int32_t tsize = 1 << tbits;
+    if (dense) {
+        for (int i = threadIdx.x; i < m; i += blockDim.x) work[i] = i;
+    } else {
+        for (int i = threadIdx.x; i < tsize; i += blockDim.x) work[i] = -1;
+    }
     __syncthreads();
     if (threadIdx.x == 0) {
-        uint64_t state = seed ^ ((uint64_t)(unit_base + u) << 32) ^ window;
-        auto slot = [&](int32_t pos) -> int32_t {
-            uint32_t hsh = ((uint32_t)pos * 2654435761u) >> (32 - tbits);
-            while (tkey[hsh] != -1 && tkey[hsh] != pos) hsh = (hsh + 1) & (uint32_t)(tsize - 1);
-            return (int32_t)hsh;
-        };
-        for (int32_t i = 0; i < C; ++i) {
-            const uint64_t x = splitmix64_next(state);
-            const int32_t j = i + (int32_t)bounded_draw(x, (uint32_t)(k.m - i));
-            const int32_t si = slot(i);
-            const int32_t vi = tkey[si] == i ? tval[si] : i;
-            const int32_t sj = slot(j);
-            const int32_t vj = tkey[sj] == j ? tval[sj] : j;
-            // a[i] <- a[j] (position i is never read again), a[j] <- old a[i]
-            tkey[sj] = j;
-            tval[sj] = vi;
-            chosen[i] = vj;
+        if (dense) {
+            for (int32_t i = 0; i < C; ++i) {
+                const int32_t j = target[i];
+                const int32_t vj = work[j];
+                work[j] = work[i];  // position i is never read again
+                chosen[i] = vj;
+            }
+        } else {
+            int32_t* tkey = work;
+            int32_t* tval = work + tsize;
+            auto slot = [&](int32_t pos) -> int32_t {
+                uint32_t hsh = ((uint32_t)pos * 2654435761u) >> (32 - tbits);
+                while (tkey[hsh] != -1 && tkey[hsh] != pos) hsh = (hsh + 1) & (uint32_t)(tsize - 1);
+                return (int32_t)hsh;
+            };
+            for (int32_t i = 0; i < C; ++i) {
+                const int32_t j = target[i];
+                const int32_t si = slot(i);
+                const int32_t vi = tkey[si] == i ? tval[si] : i;
+                const int32_t sj = slot(j);
+                const int32_t vj = tkey[sj] == j ? tval[sj] : j;
+                tkey[sj] = j;  // a[j] <- old a[i]; position i is never read again
+                tval[sj] = vi;
+                chosen[i] = vj;
+            }
         }
     }
     __syncthreads();
@@ -200,22 +224,29 @@ __global__ void __launch_bounds__(32) kmeans_scatter_kernel(const int32_t* assig
     const int64_t hi = lo + kChunk < m ? lo + kChunk : m;
     // Stage the counters and the chunk's assignments in shared memory with all loads in
     // flight, so the sequential loop below touches shared memory only.
-    for (int c0 = 0; c0 < C; c0 += 32 * 8) {
-        int32_t o[8], bb[8];
+    static_assert(kChunk == 1024, "the staging below loads 32 assignments per lane");
+    int32_t av[32];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
+    for (int t = 0; t < 32; ++t) {
+        const int64_t i = lo + t * 32 + lane;
+        av[t] = i < hi ? a[i] : -1;
+    }
+    for (int c0 = 0; c0 < C; c0 += 32 * 16) {
+        int32_t o[16], bb[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
             const int c = c0 + t * 32 + lane;
             o[t] = c < C ? off[c] : 0;
             bb[t] = c < C ? base[c] : 0;
         }
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
+        for (int t = 0; t < 16; ++t) {
             const int c = c0 + t * 32 + lane;
             if (c < C) cnt[c] = o[t] + bb[t];
         }
     }
-#pragma unroll 8
-    for (int j = lane; j < kChunk; j += 32) sa[j] = lo + j < hi ? a[lo + j] : -1;
+#pragma unroll
+    for (int t = 0; t < 32; ++t) sa[t * 32 + lane] = av[t];
     __syncwarp();
     const uint32_t lt = (1u << lane) - 1u;
     for (int64_t i0 = lo; i0 < hi; i0 += 32) {
@@ -232,9 +263,13 @@ __global__ void __launch_bounds__(32) kmeans_scatter_kernel(const int32_t* assig
 }
 
 // ---------------------------------------------------------------------- mean
-// One warp per cluster: mu_c = (1/|c|) sum of member keys (fp32, ascending member order),
-// empty clusters keep mu_c; then mu_hat. With a relayout, the same pass copies the member K
-// rows and their V rows into the cluster-major store and records the original token ids.
+// One CTA (8 warps) per cluster: mu_c = (1/|c|) sum of member keys (fp32); empty clusters
+// keep mu_c; then mu_hat. The CTA is 32 row groups of 8 lanes: group g (warp g/4) sums the
+// members g, g+32, g+64, ... in order, each lane holding 16 dimensions, with 4 rows per group
+// in flight, so a cluster of up to 128 members is read in one memory round trip. The group
+// sums are added in a fixed order (a butterfly inside each warp, then warps 0..7), so the
+// result is run-to-run exact. With a relayout, the same pass copies each member's K row and
+// its V row into the cluster-major store and records the original token ids.
 __global__ void __launch_bounds__(256) kmeans_mean_kernel(KeysView k, const int32_t* perm,
                                                           int64_t perm_ustride,
                                                           const int32_t* offsets,
@@ -242,10 +277,11 @@ __global__ void __launch_bounds__(256) kmeans_mean_kernel(KeysView k, const int3
                                                           float* mu, int64_t mu_ustride,
                                                           uint16_t* mu_hat, int64_t muhat_ustride,
                                                           Relayout rl) {
+    __shared__ __align__(16) float part[8][kD];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int c = blockIdx.x * (blockDim.x >> 5) + warp;
+    const int c = blockIdx.x;
     const int u = blockIdx.y;
-    if (c >= C) return;
+    const int grp = threadIdx.x >> 3, l8 = lane & 7;  // row group 0..31, dims [16*l8, 16*l8+16)
     const int32_t* off = offsets + (int64_t)u * off_ustride;
     const int32_t lo = off[c], hi = off[c + 1];
     const int32_t* pm = perm + (int64_t)u * perm_ustride;
@@ -253,49 +289,80 @@ __global__ void __launch_bounds__(256) kmeans_mean_kernel(KeysView k, const int3
     const uint16_t* keys = k.base + ubase * kD;
     const bool relay = rl.kp != nullptr;
     const uint16_t* vals = relay ? rl.V + ubase * kD : nullptr;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    // Rows in batches of 8 (8 loads in flight per lane); the next batch's member indices are
-    // fetched while the current batch's rows are loading. Accumulation stays in member order.
-    constexpr int kB = 8;
-    int32_t nxt[kB];
+    float acc[16];
 #pragma unroll
-    for (int t = 0; t < kB; ++t) nxt[t] = lo + t < hi ? pm[lo + t] : 0;
-    for (int32_t j = lo; j < hi; j += kB) {
+    for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+    constexpr int kB = 4;  // rows in flight per row group
+    for (int32_t j0 = lo; j0 < hi; j0 += 32 * kB) {
         int32_t idx[kB];
-#pragma unroll
-        for (int t = 0; t < kB; ++t) idx[t] = nxt[t];
-        uint2 w[kB];
-#pragma unroll
-        for (int t = 0; t < kB; ++t)
-            if (j + t < hi) w[t] = reinterpret_cast<const uint2*>(keys + (int64_t)idx[t] * kD)[lane];
-#pragma unroll
-        for (int t = 0; t < kB; ++t) nxt[t] = j + kB + t < hi ? pm[j + kB + t] : 0;
+        bool ok[kB];
 #pragma unroll
         for (int t = 0; t < kB; ++t) {
-            if (j + t >= hi) break;
-            acc.x += bf16_lo(w[t].x);
-            acc.y += bf16_hi(w[t].x);
-            acc.z += bf16_lo(w[t].y);
-            acc.w += bf16_hi(w[t].y);
+            const int32_t j = j0 + grp + 32 * t;
+            ok[t] = j < hi;
+            idx[t] = ok[t] ? pm[j] : 0;
         }
+        uint4 w[kB][2];
+#pragma unroll
+        for (int t = 0; t < kB; ++t)
+            if (ok[t]) {
+                const uint4* row = reinterpret_cast<const uint4*>(keys + (int64_t)idx[t] * kD) + 2 * l8;
+                w[t][0] = row[0];
+                w[t][1] = row[1];
+            }
+#pragma unroll
+        for (int t = 0; t < kB; ++t)
+            if (ok[t]) {
+                const uint32_t ww[8] = {w[t][0].x, w[t][0].y, w[t][0].z, w[t][0].w,
+                                        w[t][1].x, w[t][1].y, w[t][1].z, w[t][1].w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    acc[2 * e] += bf16_lo(ww[e]);
+                    acc[2 * e + 1] += bf16_hi(ww[e]);
+                }
+            }
         if (relay) {
 #pragma unroll
-            for (int t = 0; t < kB; ++t) {
-                if (j + t >= hi) break;
-                const int64_t dst = (int64_t)u * rl.ustride_rows + j + t;
-                reinterpret_cast<uint2*>(rl.kp + dst * kD)[lane] = w[t];
-                reinterpret_cast<uint2*>(rl.vp + dst * kD)[lane] =
-                    reinterpret_cast<const uint2*>(vals + (int64_t)idx[t] * kD)[lane];
-                if (lane == 0) rl.ids[dst] = rl.id_base + idx[t];
-            }
+            for (int t = 0; t < kB; ++t)
+                if (ok[t]) {
+                    const int64_t dst = (int64_t)u * rl.ustride_rows + j0 + grp + 32 * t;
+                    uint4* kd = reinterpret_cast<uint4*>(rl.kp + dst * kD) + 2 * l8;
+                    kd[0] = w[t][0];
+                    kd[1] = w[t][1];
+                    const uint4* vs = reinterpret_cast<const uint4*>(vals + (int64_t)idx[t] * kD) + 2 * l8;
+                    uint4* vd = reinterpret_cast<uint4*>(rl.vp + dst * kD) + 2 * l8;
+                    vd[0] = vs[0];
+                    vd[1] = vs[1];
+                    if (l8 == 0) rl.ids[dst] = rl.id_base + idx[t];
+                }
         }
     }
+    // fixed-order sum: the four row groups of each warp, then the eight warps
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 8);
+        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+    }
+    if (lane < 8) {
+        float4* dst = reinterpret_cast<float4*>(&part[warp][16 * l8]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
+    }
+    __syncthreads();
+    if (warp != 0) return;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w8 = 0; w8 < 8; ++w8) {
+        const float4 p4 = reinterpret_cast<const float4*>(part[w8])[lane];
+        v.x += p4.x;
+        v.y += p4.y;
+        v.z += p4.z;
+        v.w += p4.w;
+    }
     float* mrow = mu + ((int64_t)u * mu_ustride + c) * kD;
-    float4 v;
     if (hi > lo) {
         const float n = (float)(hi - lo);
-        v = make_float4(__fdiv_rn(acc.x, n), __fdiv_rn(acc.y, n), __fdiv_rn(acc.z, n),
-                        __fdiv_rn(acc.w, n));
+        v = make_float4(__fdiv_rn(v.x, n), __fdiv_rn(v.y, n), __fdiv_rn(v.z, n), __fdiv_rn(v.w, n));
     } else {
         v = reinterpret_cast<const float4*>(mrow)[lane];
     }
@@ -324,12 +391,15 @@ int launch_kmeans_init(const KeysView& k, int32_t C, uint64_t seed, int64_t unit
     (void)err;
     int tbits = 6;
     while ((1 << tbits) < 2 * C) ++tbits;
-    const size_t smem = (size_t)(2 * (1 << tbits) + C) * sizeof(int32_t);
-    cudaError_t e = cudaFuncSetAttribute(kmeans_init_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_fail(e, "init: set smem");
+    const bool dense = (2 * (size_t)C + (size_t)k.m) * sizeof(int32_t) <= kInitSmemLimit;
+    const size_t work = dense ? (size_t)k.m : (size_t)2 * (1 << tbits);
+    const size_t smem = (2 * (size_t)C + work) * sizeof(int32_t);
+    int rc = ensure_smem((const void*)kmeans_init_kernel, smem, "init: set smem");
+    if (rc != CKV_OK) return rc;
+    cudaError_t e;
     kmeans_init_kernel<<<k.U, 256, smem, s>>>(k, C, seed, unit_base, window, init_idx, mu,
-                                              mu_ustride, mu_hat, muhat_ustride, tbits);
+                                              mu_ustride, mu_hat, muhat_ustride, tbits,
+                                              dense ? 1 : 0);
     e = cudaGetLastError();
     return e == cudaSuccess ? CKV_OK : cuda_fail(e, "init: launch");
 }
@@ -343,16 +413,11 @@ int launch_kmeans_update(const KeysView& k, const int32_t* assign, int64_t assig
     cudaError_t e;
     const size_t hsmem = (size_t)C * sizeof(int32_t);
     const size_t scsmem = (size_t)(C + kChunk) * sizeof(int32_t);
-    e = cudaFuncSetAttribute(kmeans_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)hsmem);
-    if (e != cudaSuccess) return cuda_fail(e, "count: set smem");
-    e = cudaFuncSetAttribute(kmeans_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)scsmem);
-    if (e != cudaSuccess) return cuda_fail(e, "scatter: set smem");
     const size_t ssmem = (size_t)(C + 32) * sizeof(int32_t);
-    e = cudaFuncSetAttribute(kmeans_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)ssmem);
-    if (e != cudaSuccess) return cuda_fail(e, "scan: set smem");
+    int rc = ensure_smem((const void*)kmeans_count_kernel, hsmem, "count: set smem");
+    if (rc == CKV_OK) rc = ensure_smem((const void*)kmeans_scatter_kernel, scsmem, "scatter: set smem");
+    if (rc == CKV_OK) rc = ensure_smem((const void*)kmeans_scan_kernel, ssmem, "scan: set smem");
+    if (rc != CKV_OK) return rc;
     if (nch > 0) {
         kmeans_count_kernel<<<dim3(nch, k.U), 256, hsmem, s>>>(assign, assign_ustride, k.m, C, nch,
                                                                chunk_ws, err);
@@ -365,7 +430,7 @@ int launch_kmeans_update(const KeysView& k, const int32_t* assign, int64_t assig
     }
     Relayout rl{};
     if (relayout) rl = *relayout;
-    kmeans_mean_kernel<<<dim3((C + 7) / 8, k.U), 256, 0, s>>>(k, perm, perm_ustride, offsets,
+    kmeans_mean_kernel<<<dim3(C, k.U), 256, 0, s>>>(k, perm, perm_ustride, offsets,
                                                               off_ustride, C, mu, mu_ustride,
                                                               mu_hat, muhat_ustride, rl);
     e = cudaGetLastError();

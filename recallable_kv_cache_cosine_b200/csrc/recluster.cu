@@ -171,11 +171,10 @@ int launch_recluster(const ReclusterArgs& a, cudaStream_t s) {
         set_error("recluster: window too large for shared memory");
         return CKV_EINVAL;
     }
-    cudaError_t e = cudaFuncSetAttribute(recluster_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_fail(e, "recluster: set smem");
+    const int rc = ensure_smem((const void*)recluster_kernel, smem, "recluster: set smem");
+    if (rc != CKV_OK) return rc;
     recluster_kernel<<<a.U, kRT, smem, s>>>(a);
-    e = cudaGetLastError();
+    cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? CKV_OK : cuda_fail(e, "recluster: launch");
 }
 

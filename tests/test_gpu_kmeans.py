@@ -31,7 +31,8 @@ def _keys(U, n, n_centers, seed):
 
 
 @pytest.mark.parametrize("m,C", [(40, 3), (127, 8), (300, 4), (2032, 32), (5000, 200), (5000, 256),
-                                 (5000, 257), (4000, 400), (3000, 512), (3000, 513), (6000, 1100)])
+                                 (5000, 257), (4000, 400), (3000, 512), (3000, 513), (6000, 1100),
+                                 (60000, 40)])
 def test_init_and_assign_stage(m, C):
     U, n = 2, m + 16
     Kn, Kd = _keys(U, n, max(C, 4), seed=m + C)
