@@ -747,6 +747,7 @@ __global__ void __launch_bounds__(kNT, 2)
                     s[k] = fmaf(qb4.w, bf16_hi(w.w), t);
                 }
             }
+            __syncwarp();  // all 8 rows' products first, then the reductions
 #pragma unroll
             for (int o = 8; o > 0; o >>= 1)
 #pragma unroll
