@@ -263,25 +263,35 @@ __global__ void __launch_bounds__(32) kmeans_scatter_kernel(const int32_t* assig
 }
 
 // ---------------------------------------------------------------------- mean
-// One CTA (8 warps) per cluster: mu_c = (1/|c|) sum of member keys (fp32); empty clusters
-// keep mu_c; then mu_hat. The CTA is 32 row groups of 8 lanes: group g (warp g/4) sums the
-// members g, g+32, g+64, ... in order, each lane holding 16 dimensions, with 4 rows per group
-// in flight, so a cluster of up to 128 members is read in one memory round trip. The group
-// sums are added in a fixed order (a butterfly inside each warp, then warps 0..7), so the
-// result is run-to-run exact. With a relayout, the same pass copies each member's K row and
-// its V row into the cluster-major store and records the original token ids.
-__global__ void __launch_bounds__(256) kmeans_mean_kernel(KeysView k, const int32_t* perm,
-                                                          int64_t perm_ustride,
-                                                          const int32_t* offsets,
-                                                          int64_t off_ustride, int32_t C,
-                                                          float* mu, int64_t mu_ustride,
-                                                          uint16_t* mu_hat, int64_t muhat_ustride,
-                                                          Relayout rl) {
-    __shared__ __align__(16) float part[8][kD];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// One CTA (4 warps) per cluster: mu_c = (1/|c|) sum of the member keys (fp32); empty clusters
+// keep mu_c; then mu_hat. The member list, then the members' key rows, are gathered into
+// shared memory (cp.async, 16 bytes per thread, up to kMeanRows rows per pass, one memory
+// round trip per pass). Thread d sums dimension d over the rows in member order into four
+// partial sums (rows 4i, 4i+1, 4i+2, 4i+3 of each pass), added in a fixed order, so the
+// result is run-to-run exact. With a relayout the pass also writes the key rows, their V rows
+// and the original token ids into the cluster-major store.
+constexpr int kMeanThreads = 128;  // one thread per dimension
+constexpr int kMeanRows = 128;
+
+CKV_DEV void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+__global__ void __launch_bounds__(kMeanThreads) kmeans_mean_kernel(KeysView k, const int32_t* perm,
+                                                                   int64_t perm_ustride,
+                                                                   const int32_t* offsets,
+                                                                   int64_t off_ustride, int32_t C,
+                                                                   float* mu, int64_t mu_ustride,
+                                                                   uint16_t* mu_hat,
+                                                                   int64_t muhat_ustride,
+                                                                   Relayout rl) {
+    static_assert(kMeanThreads == kD, "one thread per dimension");
+    __shared__ __align__(16) uint16_t srow[kMeanRows * kD];
+    __shared__ int32_t sidx[kMeanRows];
+    __shared__ __align__(16) float ssum[kD];
+    const int tid = threadIdx.x;
     const int c = blockIdx.x;
     const int u = blockIdx.y;
-    const int grp = threadIdx.x >> 3, l8 = lane & 7;  // row group 0..31, dims [16*l8, 16*l8+16)
     const int32_t* off = offsets + (int64_t)u * off_ustride;
     const int32_t lo = off[c], hi = off[c + 1];
     const int32_t* pm = perm + (int64_t)u * perm_ustride;
@@ -289,76 +299,52 @@ __global__ void __launch_bounds__(256) kmeans_mean_kernel(KeysView k, const int3
     const uint16_t* keys = k.base + ubase * kD;
     const bool relay = rl.kp != nullptr;
     const uint16_t* vals = relay ? rl.V + ubase * kD : nullptr;
-    float acc[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-    constexpr int kB = 4;  // rows in flight per row group
-    for (int32_t j0 = lo; j0 < hi; j0 += 32 * kB) {
-        int32_t idx[kB];
-        bool ok[kB];
-#pragma unroll
-        for (int t = 0; t < kB; ++t) {
-            const int32_t j = j0 + grp + 32 * t;
-            ok[t] = j < hi;
-            idx[t] = ok[t] ? pm[j] : 0;
+    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+    for (int32_t j0 = lo; j0 < hi; j0 += kMeanRows) {
+        const int n = (hi - j0) < kMeanRows ? (hi - j0) : kMeanRows;
+        if (j0 > lo) __syncthreads();  // the previous pass is done with srow and sidx
+        for (int r = tid; r < n; r += kMeanThreads) sidx[r] = pm[j0 + r];
+        __syncthreads();
+        for (int i = tid; i < n * 16; i += kMeanThreads) {
+            const int r = i >> 4, ch = i & 15;
+            cp_async16(srow + r * kD + ch * 8, keys + (int64_t)sidx[r] * kD + ch * 8);
         }
-        uint4 w[kB][2];
-#pragma unroll
-        for (int t = 0; t < kB; ++t)
-            if (ok[t]) {
-                const uint4* row = reinterpret_cast<const uint4*>(keys + (int64_t)idx[t] * kD) + 2 * l8;
-                w[t][0] = row[0];
-                w[t][1] = row[1];
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        if (relay) {  // V rows and token ids while the key rows arrive
+            for (int i = tid; i < n * 16; i += kMeanThreads) {
+                const int r = i >> 4, ch = i & 15;
+                const int64_t dst = (int64_t)u * rl.ustride_rows + j0 + r;
+                reinterpret_cast<uint4*>(rl.vp + dst * kD)[ch] =
+                    reinterpret_cast<const uint4*>(vals + (int64_t)sidx[r] * kD)[ch];
             }
-#pragma unroll
-        for (int t = 0; t < kB; ++t)
-            if (ok[t]) {
-                const uint32_t ww[8] = {w[t][0].x, w[t][0].y, w[t][0].z, w[t][0].w,
-                                        w[t][1].x, w[t][1].y, w[t][1].z, w[t][1].w};
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    acc[2 * e] += bf16_lo(ww[e]);
-                    acc[2 * e + 1] += bf16_hi(ww[e]);
-                }
-            }
+            for (int r = tid; r < n; r += kMeanThreads)
+                rl.ids[(int64_t)u * rl.ustride_rows + j0 + r] = rl.id_base + sidx[r];
+        }
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncthreads();
+        const uint16_t* col = srow + tid;
+        int r = 0;
+        for (; r + 4 <= n; r += 4) {
+            acc0 += __uint_as_float((uint32_t)col[(r + 0) * kD] << 16);
+            acc1 += __uint_as_float((uint32_t)col[(r + 1) * kD] << 16);
+            acc2 += __uint_as_float((uint32_t)col[(r + 2) * kD] << 16);
+            acc3 += __uint_as_float((uint32_t)col[(r + 3) * kD] << 16);
+        }
+        for (; r < n; ++r) acc0 += __uint_as_float((uint32_t)col[r * kD] << 16);
         if (relay) {
-#pragma unroll
-            for (int t = 0; t < kB; ++t)
-                if (ok[t]) {
-                    const int64_t dst = (int64_t)u * rl.ustride_rows + j0 + grp + 32 * t;
-                    uint4* kd = reinterpret_cast<uint4*>(rl.kp + dst * kD) + 2 * l8;
-                    kd[0] = w[t][0];
-                    kd[1] = w[t][1];
-                    const uint4* vs = reinterpret_cast<const uint4*>(vals + (int64_t)idx[t] * kD) + 2 * l8;
-                    uint4* vd = reinterpret_cast<uint4*>(rl.vp + dst * kD) + 2 * l8;
-                    vd[0] = vs[0];
-                    vd[1] = vs[1];
-                    if (l8 == 0) rl.ids[dst] = rl.id_base + idx[t];
-                }
+            for (int i = tid; i < n * 16; i += kMeanThreads) {
+                const int rr = i >> 4, ch = i & 15;
+                const int64_t dst = (int64_t)u * rl.ustride_rows + j0 + rr;
+                reinterpret_cast<uint4*>(rl.kp + dst * kD)[ch] =
+                    reinterpret_cast<const uint4*>(srow + rr * kD)[ch];
+            }
         }
     }
-    // fixed-order sum: the four row groups of each warp, then the eight warps
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 8);
-        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
-    }
-    if (lane < 8) {
-        float4* dst = reinterpret_cast<float4*>(&part[warp][16 * l8]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dst[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
-    }
+    ssum[tid] = (acc0 + acc1) + (acc2 + acc3);
     __syncthreads();
-    if (warp != 0) return;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int w8 = 0; w8 < 8; ++w8) {
-        const float4 p4 = reinterpret_cast<const float4*>(part[w8])[lane];
-        v.x += p4.x;
-        v.y += p4.y;
-        v.z += p4.z;
-        v.w += p4.w;
-    }
+    if (tid >= 32) return;
+    const int lane = tid;
+    float4 v = reinterpret_cast<const float4*>(ssum)[lane];
     float* mrow = mu + ((int64_t)u * mu_ustride + c) * kD;
     if (hi > lo) {
         const float n = (float)(hi - lo);
@@ -430,7 +416,7 @@ int launch_kmeans_update(const KeysView& k, const int32_t* assign, int64_t assig
     }
     Relayout rl{};
     if (relayout) rl = *relayout;
-    kmeans_mean_kernel<<<dim3(C, k.U), 256, 0, s>>>(k, perm, perm_ustride, offsets,
+    kmeans_mean_kernel<<<dim3(C, k.U), kMeanThreads, 0, s>>>(k, perm, perm_ustride, offsets,
                                                               off_ustride, C, mu, mu_ustride,
                                                               mu_hat, muhat_ustride, rl);
     e = cudaGetLastError();
