@@ -2,6 +2,8 @@
 // the kernel launchers. Not part of the public ABI.
 #pragma once
 
+#include <utility>
+
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -154,6 +156,25 @@ struct DecodeArgs {
     int64_t part_ustride;
     uint32_t* err;
 };
+// Launch with programmatic dependent launch allowed: the kernel may be scheduled while the
+// previous kernel in the stream is still running. Every kernel launched this way calls
+// pdl_wait() before it touches memory that earlier work writes, so stream order holds.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 int launch_select_attend(const DecodeArgs& a, int num_sms, cudaStream_t s);
 
 int launch_append(const uint16_t* k, const uint16_t* v, int32_t U, uint16_t* spk, uint16_t* spv,

@@ -100,6 +100,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     assign_tc_kernel(const __grid_constant__ CUtensorMap map_a,
                      const __grid_constant__ CUtensorMap map_b0,
                      const __grid_constant__ CUtensorMap map_b1, const AssignParams p) {
+    pdl_launch_dependents();  // let the next kernel in the stream be scheduled early
+    pdl_wait();               // the previous kernel's writes are visible from here on
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     // centroid slots: slot h holds n_h rows as two 64-column halves of n_h x 128 B each
@@ -412,9 +414,8 @@ int run_kmeans_assign(const AssignPlan& plan, cudaStream_t s) {
     const AssignPlanImpl* impl = plan.impl.get();
     if (!impl) return CKV_EINVAL;
     for (size_t ch = 0; ch < impl->params.size(); ++ch) {
-        assign_tc_kernel<<<impl->grid, kThreads, impl->smem[ch], s>>>(
-            impl->map_a, impl->map_b0[ch], impl->map_b1[ch], impl->params[ch]);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = launch_pdl(assign_tc_kernel, dim3(impl->grid), dim3(kThreads), impl->smem[ch], s,
+                                   impl->map_a, impl->map_b0[ch], impl->map_b1[ch], impl->params[ch]);
         if (e != cudaSuccess) return cuda_fail(e, "assign: launch");
     }
     return CKV_OK;

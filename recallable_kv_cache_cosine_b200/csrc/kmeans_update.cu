@@ -58,6 +58,8 @@ __global__ void __launch_bounds__(256) kmeans_init_kernel(KeysView k, int32_t C,
                                                           int64_t mu_ustride, uint16_t* mu_hat,
                                                           int64_t muhat_ustride, int32_t tbits,
                                                           int32_t dense) {
+    pdl_launch_dependents();  // let the next kernel in the stream be scheduled early
+    pdl_wait();               // the previous kernel's writes are visible from here on
     extern __shared__ int32_t sm[];
     const int u = blockIdx.x;
     const int32_t m = (int32_t)k.m;
@@ -122,6 +124,8 @@ __global__ void __launch_bounds__(256) kmeans_init_kernel(KeysView k, int32_t C,
 __global__ void __launch_bounds__(256) kmeans_count_kernel(const int32_t* assign, int64_t a_ustride,
                                                            int64_t m, int32_t C, int32_t nch,
                                                            int32_t* chunk, uint32_t* err) {
+    pdl_launch_dependents();  // let the next kernel in the stream be scheduled early
+    pdl_wait();               // the previous kernel's writes are visible from here on
     extern __shared__ int32_t hist[];
     const int ch = blockIdx.x, u = blockIdx.y;
     for (int c = threadIdx.x; c < C; c += blockDim.x) hist[c] = 0;
@@ -148,6 +152,8 @@ __global__ void __launch_bounds__(256) kmeans_count_kernel(const int32_t* assign
 __global__ void __launch_bounds__(1024) kmeans_scan_kernel(int32_t* chunk, int32_t nch, int32_t C,
                                                            int64_t m, int32_t* offsets,
                                                            int64_t off_ustride) {
+    pdl_launch_dependents();  // let the next kernel in the stream be scheduled early
+    pdl_wait();               // the previous kernel's writes are visible from here on
     extern __shared__ int32_t sz[];  // [C] then [32] warp totals
     int32_t* wsum = sz + C;
     const int u = blockIdx.x;
@@ -212,6 +218,8 @@ __global__ void __launch_bounds__(32) kmeans_scatter_kernel(const int32_t* assig
                                                             const int32_t* offsets,
                                                             int64_t off_ustride, int32_t* perm,
                                                             int64_t perm_ustride) {
+    pdl_launch_dependents();  // let the next kernel in the stream be scheduled early
+    pdl_wait();               // the previous kernel's writes are visible from here on
     extern __shared__ int32_t cnt[];  // [C] counters, then [kChunk] assignments
     int32_t* sa = cnt + C;
     const int ch = blockIdx.x, u = blockIdx.y;
@@ -285,6 +293,8 @@ __global__ void __launch_bounds__(kMeanThreads) kmeans_mean_kernel(KeysView k, c
                                                                    uint16_t* mu_hat,
                                                                    int64_t muhat_ustride,
                                                                    Relayout rl) {
+    pdl_launch_dependents();  // let the next kernel in the stream be scheduled early
+    pdl_wait();               // the previous kernel's writes are visible from here on
     static_assert(kMeanThreads == kD, "one thread per dimension");
     __shared__ __align__(16) uint16_t srow[kMeanRows * kD];
     __shared__ int32_t sidx[kMeanRows];
@@ -357,6 +367,8 @@ __global__ void __launch_bounds__(kMeanThreads) kmeans_mean_kernel(KeysView k, c
 
 __global__ void copy_sinks_kernel(const uint16_t* K, const uint16_t* V, int64_t n, int32_t n_sink,
                                   uint16_t* spk, uint16_t* spv, int64_t sp_ustride) {
+    pdl_launch_dependents();  // let the next kernel in the stream be scheduled early
+    pdl_wait();               // the previous kernel's writes are visible from here on
     const int u = blockIdx.x;
     const int64_t words = (int64_t)n_sink * kD / 8;  // 16-byte words
     const uint4* ks = reinterpret_cast<const uint4*>(K + (int64_t)u * n * kD);
@@ -383,10 +395,8 @@ int launch_kmeans_init(const KeysView& k, int32_t C, uint64_t seed, int64_t unit
     int rc = ensure_smem((const void*)kmeans_init_kernel, smem, "init: set smem");
     if (rc != CKV_OK) return rc;
     cudaError_t e;
-    kmeans_init_kernel<<<k.U, 256, smem, s>>>(k, C, seed, unit_base, window, init_idx, mu,
-                                              mu_ustride, mu_hat, muhat_ustride, tbits,
-                                              dense ? 1 : 0);
-    e = cudaGetLastError();
+    e = launch_pdl(kmeans_init_kernel, dim3(k.U), dim3(256), smem, s, k, C, seed, unit_base, window,
+                   init_idx, mu, mu_ustride, mu_hat, muhat_ustride, tbits, dense ? 1 : 0);
     return e == cudaSuccess ? CKV_OK : cuda_fail(e, "init: launch");
 }
 
@@ -405,28 +415,30 @@ int launch_kmeans_update(const KeysView& k, const int32_t* assign, int64_t assig
     if (rc == CKV_OK) rc = ensure_smem((const void*)kmeans_scan_kernel, ssmem, "scan: set smem");
     if (rc != CKV_OK) return rc;
     if (nch > 0) {
-        kmeans_count_kernel<<<dim3(nch, k.U), 256, hsmem, s>>>(assign, assign_ustride, k.m, C, nch,
-                                                               chunk_ws, err);
+        e = launch_pdl(kmeans_count_kernel, dim3(nch, k.U), dim3(256), hsmem, s, assign,
+                       assign_ustride, k.m, C, nch, chunk_ws, err);
+        if (e != cudaSuccess) return cuda_fail(e, "update: count launch");
     }
-    kmeans_scan_kernel<<<k.U, 1024, ssmem, s>>>(chunk_ws, nch, C, k.m, offsets, off_ustride);
+    e = launch_pdl(kmeans_scan_kernel, dim3(k.U), dim3(1024), ssmem, s, chunk_ws, nch, C, k.m,
+                   offsets, off_ustride);
+    if (e != cudaSuccess) return cuda_fail(e, "update: scan launch");
     if (nch > 0) {
-        kmeans_scatter_kernel<<<dim3(nch, k.U), 32, scsmem, s>>>(assign, assign_ustride, k.m, C, nch,
-                                                                chunk_ws, offsets, off_ustride,
-                                                                perm, perm_ustride);
+        e = launch_pdl(kmeans_scatter_kernel, dim3(nch, k.U), dim3(32), scsmem, s, assign,
+                       assign_ustride, k.m, C, nch, chunk_ws, offsets, off_ustride, perm,
+                       perm_ustride);
+        if (e != cudaSuccess) return cuda_fail(e, "update: scatter launch");
     }
     Relayout rl{};
     if (relayout) rl = *relayout;
-    kmeans_mean_kernel<<<dim3(C, k.U), kMeanThreads, 0, s>>>(k, perm, perm_ustride, offsets,
-                                                              off_ustride, C, mu, mu_ustride,
-                                                              mu_hat, muhat_ustride, rl);
-    e = cudaGetLastError();
+    e = launch_pdl(kmeans_mean_kernel, dim3(C, k.U), dim3(kMeanThreads), 0, s, k, perm, perm_ustride,
+                   offsets, off_ustride, C, mu, mu_ustride, mu_hat, muhat_ustride, rl);
     return e == cudaSuccess ? CKV_OK : cuda_fail(e, "update: launch");
 }
 
 int launch_copy_sinks(const uint16_t* K, const uint16_t* V, int64_t n, int32_t U, int32_t n_sink,
                       uint16_t* spk, uint16_t* spv, int64_t sp_ustride_rows, cudaStream_t s) {
-    copy_sinks_kernel<<<U, 256, 0, s>>>(K, V, n, n_sink, spk, spv, sp_ustride_rows);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(copy_sinks_kernel, dim3(U), dim3(256), 0, s, K, V, n, n_sink, spk,
+                               spv, sp_ustride_rows);
     return e == cudaSuccess ? CKV_OK : cuda_fail(e, "sinks: launch");
 }
 

@@ -20,6 +20,8 @@ namespace {
 constexpr int kRT = 512;
 
 __global__ void __launch_bounds__(kRT) recluster_kernel(const ReclusterArgs a) {
+    pdl_launch_dependents();  // let the next kernel in the stream be scheduled early
+    pdl_wait();               // the previous kernel's writes are visible from here on
     extern __shared__ __align__(16) uint8_t smem_raw[];
     const int W = a.window, Cn = a.C_new;
     uint16_t* skey = (uint16_t*)smem_raw;                         // [W][128] bf16
@@ -156,6 +158,8 @@ __global__ void __launch_bounds__(kRT) recluster_kernel(const ReclusterArgs a) {
 
 __global__ void append_kernel(const uint16_t* k, const uint16_t* v, uint16_t* spk, uint16_t* spv,
                               int64_t sp_ustride, int32_t row) {
+    pdl_launch_dependents();  // let the next kernel in the stream be scheduled early
+    pdl_wait();               // the previous kernel's writes are visible from here on
     const int u = blockIdx.x, t = threadIdx.x;  // 16 threads x 16 bytes per row
     const int64_t dst = ((int64_t)u * sp_ustride + row) * kD;
     reinterpret_cast<uint4*>(spk + dst)[t] = reinterpret_cast<const uint4*>(k + (int64_t)u * kD)[t];
@@ -173,15 +177,14 @@ int launch_recluster(const ReclusterArgs& a, cudaStream_t s) {
     }
     const int rc = ensure_smem((const void*)recluster_kernel, smem, "recluster: set smem");
     if (rc != CKV_OK) return rc;
-    recluster_kernel<<<a.U, kRT, smem, s>>>(a);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(recluster_kernel, dim3(a.U), dim3(kRT), smem, s, a);
     return e == cudaSuccess ? CKV_OK : cuda_fail(e, "recluster: launch");
 }
 
 int launch_append(const uint16_t* k, const uint16_t* v, int32_t U, uint16_t* spk, uint16_t* spv,
                   int64_t sp_ustride_rows, int32_t row, cudaStream_t s) {
-    append_kernel<<<U, 16, 0, s>>>(k, v, spk, spv, sp_ustride_rows, row);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(append_kernel, dim3(U), dim3(16), 0, s, k, v, spk, spv,
+                               sp_ustride_rows, row);
     return e == cudaSuccess ? CKV_OK : cuda_fail(e, "append: launch");
 }
 
