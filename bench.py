@@ -16,8 +16,8 @@ One bench step is one pass of the whole hot path:
   C. one 320-token incremental window on layer 0: per token append_kv + select_and_attend,
      then recluster_increment.
 `value` = device time of B / layer-steps (µs, lower is better). Per-section times, keys/s,
-the roofline of the select+attend kernel, an end-to-end figure (eager API calls with the
-query copied in from pinned host memory and the output read back, per layer-step) and the
+the roofline of the select+attend kernel, an end-to-end figure (eager API calls; per decode
+step the queries copied in from pinned host memory and the outputs read back) and the
 CPU oracle's time on a bounded sample of the same workload are added to the JSON line.
 
 --impl reference times the CPU oracle instead, on the same metric.
@@ -323,19 +323,21 @@ def run_gpu(args, world, rank, local):
     # ------------------------------------------------------------ end to end (host buffers)
     with torch.cuda.stream(s):
         section_a()
-    q_host = q[: min(D, 16)].cpu().pin_memory()
+    q_host = q[: min(D, 16)].cpu().pin_memory()  # [De, L, B, HQ, 128]
     o_host = torch.empty(q_host.shape[:3] + (HQ, 128), dtype=torch.float32).pin_memory()
-    q_dev = torch.empty(B, HQ, 128, dtype=torch.bfloat16, device=dev)
-    o_dev = torch.empty(B, HQ, 128, dtype=torch.float32, device=dev)
+    q_dev = torch.empty(q_host.shape[1:], dtype=torch.bfloat16, device=dev)
+    o_dev = torch.empty(o_host.shape[1:], dtype=torch.float32, device=dev)
     De = q_host.shape[0]
 
     def e2e_pass():
+        # per decode step: one copy of every layer's queries in, a select_and_attend per layer,
+        # one copy of every layer's output back
         with torch.cuda.stream(s):
             for d in range(De):
+                q_dev.copy_(q_host[d], non_blocking=True)
                 for l in range(L):
-                    q_dev.copy_(q_host[d, l], non_blocking=True)
-                    ctx.select_and_attend(l, q_dev, BUDGET, o_dev, stream=s)
-                    o_host[d, l].copy_(o_dev, non_blocking=True)
+                    ctx.select_and_attend(l, q_dev[l], BUDGET, o_dev[l], stream=s)
+                o_host[d].copy_(o_dev, non_blocking=True)
 
     e2e_pass()
     torch.cuda.synchronize()
@@ -390,8 +392,9 @@ def run_gpu(args, world, rank, local):
             "e2e": {"value": e2e_value, "unit": UNIT,
                     "h2d_bytes_per_step": De * L * B * HQ * 128 * 2,
                     "d2h_bytes_per_step": De * L * B * HQ * 128 * 4,
-                    "what": "eager API calls, q copied from pinned host memory and the output read "
-                            "back every layer-step"},
+                    "what": "eager API calls on one stream; per decode step the queries of all "
+                            "layers are copied in from pinned host memory and all outputs are "
+                            "read back"},
             "gpu_launches": (launches["A"] + launches["B"] + launches["C"]) * K_steps,
             "gpu_launches_e2e": launches_e2e,
             "cpu_baseline": cpu,
