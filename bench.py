@@ -204,6 +204,111 @@ def run_reference(args, world, rank):
 
 # ---------------------------------------------------------------------- GPU leg
 
+def extra_measurements(ckv, ctx, q, out, s, L, dev, hbm_gbs, bf16_tflops):
+    """Single-launch latency with L2 flushed, the batch-8 / budget-2048 shape, and the prefill
+    keys/s sweep over n in {8k, 32k, 128k}."""
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    G = HQ // HKV
+    res = {}
+    # one select+attend launch after a 256 MB write (more than the 126 MB L2)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    single = []
+    for i in range(9):
+        with torch.cuda.stream(s):
+            flush.zero_()
+            e0, e1 = ev(), ev()
+            e0.record(s)
+            ctx.select_and_attend(i % L, q[0, i % L], BUDGET, out[0, i % L], stream=s)
+            e1.record(s)
+        s.synchronize()
+        single.append(e0.elapsed_time(e1) * 1e3)
+    res["single_launch_us_l2_flushed"] = statistics.median(single[1:])
+    del flush
+
+    # batch 8, budget 2048: 64 units per launch, 4 layer stores (320 MB per decode pass)
+    B8, L8, D8, BUD8 = 8, 4, 8, 2048
+    c8 = ckv.ClusterKV(n_layers=L8, batch=B8, n_kv_heads=HKV, n_q_heads=HQ, capacity=N_CTX,
+                       max_clusters=C_CLUSTERS, seed=SEED)
+    K8 = torch.empty(B8, HKV, N_CTX, 128, dtype=torch.bfloat16, device=dev)
+    V8 = torch.empty_like(K8)
+    q8 = torch.empty(D8, L8, B8, HQ, 128, dtype=torch.bfloat16, device=dev)
+    o8 = torch.empty(D8, L8, B8, HQ, 128, dtype=torch.float32, device=dev)
+    for l in range(L8):
+        for b in range(B8):
+            for h in range(HKV):
+                K8[b, h], V8[b, h] = si.keys_values_torch(SEED + 7, si.unit_id(l, b, h, B8, HKV), N_CTX,
+                                                          N_CENTERS, dev)
+            q8[:, l, b] = si.queries_torch(SEED + 7, l, b, D8, HQ, dev)
+        with torch.cuda.stream(s):
+            c8.cluster_prefill(l, K8, V8, C_CLUSTERS, stream=s)
+    s.synchronize()
+    del K8, V8
+
+    def dec8():
+        for d in range(D8):
+            for l in range(L8):
+                c8.select_and_attend(l, q8[d, l], BUD8, o8[d, l], stream=s)
+    with torch.cuda.stream(s):
+        dec8()
+    s.synchronize()
+    g8 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g8, stream=s, capture_error_mode="thread_local"):
+        dec8()
+    for _ in range(3):
+        g8.replay()
+    torch.cuda.synchronize()
+    e0, e1 = ev(), ev()
+    with torch.cuda.stream(s):
+        e0.record(s)
+        for _ in range(5):
+            g8.replay()
+        e1.record(s)
+    torch.cuda.synchronize()
+    c8.check_device_error(stream=s)
+    us8 = e0.elapsed_time(e1) * 1e3 / (5 * D8 * L8)
+    by8 = select_attend_bytes(B8 * HKV, BUD8, C_CLUSTERS, N_CTX - N_SINK, G)
+    res["batch8_budget2k"] = {"us_per_layer_step": us8, "units": B8 * HKV, "bytes_per_launch": by8,
+                              "achieved_gbs": by8 / (us8 * 1e-6) / 1e9,
+                              "frac": by8 / (us8 * 1e-6) / 1e9 / hbm_gbs,
+                              "what": "batch 8 x 8 KV heads, n=32768, C=400, budget 2048, 4 layer "
+                                      "stores (320 MB per decode pass), CUDA graph of 32 launches"}
+    del g8
+    c8.close()
+    del q8, o8
+
+    # prefill keys/s sweep, one layer of 8 KV heads each
+    sweep = []
+    for n_s, c_s in ((8192, 100), (32768, 400), (131072, 1600)):
+        Ks = torch.empty(1, HKV, n_s, 128, dtype=torch.bfloat16, device=dev)
+        Vs = torch.empty_like(Ks)
+        for h in range(HKV):
+            Ks[0, h], Vs[0, h] = si.keys_values_torch(SEED + 11, h, n_s, c_s, dev)
+        cs = ckv.ClusterKV(n_layers=1, batch=1, n_kv_heads=HKV, n_q_heads=HQ, capacity=n_s,
+                           max_clusters=c_s, seed=SEED)
+        with torch.cuda.stream(s):
+            cs.cluster_prefill(0, Ks, Vs, c_s, stream=s)
+        s.synchronize()
+        ts = []
+        for _ in range(3):
+            e0, e1 = ev(), ev()
+            with torch.cuda.stream(s):
+                e0.record(s)
+                cs.cluster_prefill(0, Ks, Vs, c_s, stream=s)
+                e1.record(s)
+            s.synchronize()
+            ts.append(e0.elapsed_time(e1) / 1e3)
+        cs.check_device_error(stream=s)
+        t = statistics.median(ts)
+        kps = HKV * (n_s - N_SINK) / t
+        roof = min(bf16_tflops * 1e12 / (2 * c_s * 128), hbm_gbs * 1e9 / 512) / ITERS
+        sweep.append({"n": n_s, "C": c_s, "ms_per_layer": t * 1e3, "keys_per_s": kps,
+                      "roofline_keys_per_s": roof, "frac": kps / roof})
+        cs.close()
+        del Ks, Vs
+    res["prefill_sweep"] = sweep
+    return res
+
+
 def launches_per_prefill(C, iters):
     assign_launches = (C + 511) // 512
     return 1 + iters * (assign_launches + 4) + 1
@@ -353,6 +458,11 @@ def run_gpu(args, world, rank, local):
     launches_e2e = max(1, args.steps) * De * L
     ctx.check_device_error(stream=s)
 
+    # ------------------------------------------------------------ more shapes (rank 0)
+    extra = {}
+    if rank == 0:
+        extra = extra_measurements(ckv, ctx, q, out, s, L, dev, hbm_gbs, bf16_tflops)
+
     # ------------------------------------------------------------ CPU baseline (rank 0, N = 1)
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
@@ -400,6 +510,7 @@ def run_gpu(args, world, rank, local):
             "cpu_baseline": cpu,
             "clocks": clocks,
         }
+        line.update(extra)
         print(json.dumps(line), flush=True)
     del gB, gC
     ctx.close()
