@@ -119,10 +119,12 @@ CKV_API int select_and_attend(ckv_ctx* ctx, int32_t layer, const void* q, int32_
                       int32_t* sel_idx, int32_t* sel_count, void* stream);
 
 /* Appends one generated token's K/V per unit to the layer's pending rows (the tokens a
- * later recluster_increment will cluster).
+ * later re-clustering will cluster). The pending rows form a ring of 2 x window rows per
+ * unit: one window can be re-clustering (recluster_begin) while the next one fills.
  *   k, v : device bf16 [batch, n_kv_heads, 128].
- * CKV_ECAPACITY if the layer already holds `window` pending tokens (call
- * recluster_increment first) or if the unit capacity would be exceeded. */
+ * CKV_ECAPACITY if the layer already holds `window` pending tokens and no re-clustering is
+ * in flight (call recluster_increment or recluster_begin first), if it holds 2 x window
+ * pending tokens (call recluster_finish first), or if the unit capacity would be exceeded. */
 CKV_API int ckv_append_kv(ckv_ctx* ctx, int32_t layer, const void* k, const void* v, void* stream);
 
 /* Incremental clustering of one layer ([EXPL] 3.2, every 320 new tokens): cosine K-means
@@ -137,6 +139,25 @@ CKV_API int ckv_append_kv(ckv_ctx* ctx, int32_t layer, const void* k, const void
 CKV_API int recluster_increment(ckv_ctx* ctx, int32_t layer, void* stream);
 CKV_API int recluster_increment_traced(ckv_ctx* ctx, int32_t layer, float* mu_trace,
                                int32_t* assign_trace, void* stream);
+
+/* The same incremental clustering, overlapped with decoding ([EXPL] 4.1: clustering runs
+ * asynchronously with decode). recluster_begin launches it on `stream`, usually a second
+ * stream. The caller orders `stream` after the appends that filled the window (an event or
+ * a stream wait). Until recluster_finish, the layer keeps its clusters and still attends the
+ * window as pending tokens. Tokens appended meanwhile join the pending rows in the ring's
+ * other half. The decode kernels read only the existing clusters and rows, and the
+ * re-clustering writes only rows, offsets and centroids past them, so the two never touch
+ * the same memory.
+ * recluster_finish makes `stream` wait for the re-clustering. The window's tokens then join
+ * the cluster store (4 new clusters), and the tokens appended since begin stay pending. The
+ * final store is identical to that of recluster_increment called at begin's position.
+ * recluster_begin: CKV_ESTATE unless exactly `window` tokens are pending and none is in
+ * flight. CKV_ECAPACITY if the store is full.
+ * recluster_finish: CKV_ESTATE without a recluster_begin in flight.
+ * While a re-clustering is in flight, cluster_prefill, recluster_increment and
+ * ckv_import_unit of the layer return CKV_ESTATE. */
+CKV_API int recluster_begin(ckv_ctx* ctx, int32_t layer, void* stream);
+CKV_API int recluster_finish(ckv_ctx* ctx, int32_t layer, void* stream);
 
 typedef struct ckv_layer_info {
     int64_t n_total;   /* tokens per unit: n_sink + m + pending */

@@ -59,6 +59,8 @@ SIGNATURES = {
     "ckv_append_kv": (C.c_int, [P, I32, P, P, P]),
     "recluster_increment": (C.c_int, [P, I32, P]),
     "recluster_increment_traced": (C.c_int, [P, I32, P, P, P]),
+    "recluster_begin": (C.c_int, [P, I32, P]),
+    "recluster_finish": (C.c_int, [P, I32, P]),
     "ckv_get_layer_info": (C.c_int, [P, I32, P]),
     "ckv_export_unit": (C.c_int, [P, I32, I32, I32, P, P]),
     "ckv_import_unit": (C.c_int, [P, I32, I32, I32, I64, I32, I32, P, P]),
@@ -176,6 +178,14 @@ class ClusterKV:
     def recluster_increment(self, layer: int, mu_trace=None, assign_trace=None, stream=None):
         _check(lib().recluster_increment_traced(self._ctx, layer, _ptr(mu_trace), _ptr(assign_trace),
                                                 _stream(stream)), "recluster_increment")
+
+    def recluster_begin(self, layer: int, stream=None):
+        """Starts re-clustering the full pending window on `stream`, overlapped with decode."""
+        _check(lib().recluster_begin(self._ctx, layer, _stream(stream)), "recluster_begin")
+
+    def recluster_finish(self, layer: int, stream=None):
+        """Makes `stream` wait for that re-clustering and switches the layer to its clusters."""
+        _check(lib().recluster_finish(self._ctx, layer, _stream(stream)), "recluster_finish")
 
     # -- inspection
     def layer_info(self, layer: int) -> LayerInfo:

@@ -1,5 +1,6 @@
 // C-ABI of the ClusterKV hot path: context, argument checks and orchestration of the
 // kernels. The ABI is declared and documented in include/ckv.h.
+#include <algorithm>
 #include <cudaTypedefs.h>
 #include <stdio.h>
 
@@ -138,6 +139,58 @@ void free_all(Ctx* c) {
         if (p) cudaFree(p);
 }
 
+// Checks and launches the re-clustering of layer's full window (the `window` oldest pending
+// tokens, at ring position L.pstart). The host state is left to the caller.
+int launch_window_recluster(Ctx* c, int32_t layer, float* mu_trace, int32_t* assign_trace,
+                            cudaStream_t stream) {
+    LayerState& L = c->layers[(size_t)layer];
+    if (!L.prefilled || L.in_flight || L.pending != c->cfg.window) {
+        set_error(L.in_flight ? "a re-clustering of this layer is in flight; call recluster_finish"
+                              : "re-clustering needs exactly `window` pending tokens");
+        return CKV_ESTATE;
+    }
+    if (L.m + c->cfg.window > c->cap_c || L.C + c->cfg.new_clusters > c->cfg.max_clusters) {
+        set_error("cluster store full (tokens or clusters)");
+        return CKV_ECAPACITY;
+    }
+    if ((mu_trace && ((uintptr_t)mu_trace & 15u)) || (assign_trace && ((uintptr_t)assign_trace & 3u)))
+        return einval("misaligned trace buffer");
+    ReclusterArgs a{};
+    a.U = c->units;
+    a.n_sink = c->cfg.n_sink;
+    a.window = c->cfg.window;
+    a.win_row0 = c->cfg.n_sink + L.pstart;
+    a.C_new = c->cfg.new_clusters;
+    a.iters = c->cfg.iters;
+    a.C_old = L.C;
+    a.m_old = L.m;
+    a.seed = c->cfg.seed;
+    a.unit_base = (int64_t)layer * c->units;
+    a.window_no = (uint64_t)L.windows + 1;
+    a.spk = c->spk + c->rows_sp(layer, 0) * kD;
+    a.spv = c->spv + c->rows_sp(layer, 0) * kD;
+    a.sp_ustride = c->sp_rows;
+    a.kp = c->kp + c->rows_kp(layer, 0) * kD;
+    a.vp = c->vp + c->rows_kp(layer, 0) * kD;
+    a.ids = c->ids + c->rows_kp(layer, 0);
+    a.kp_ustride = c->cap_c;
+    a.offsets = c->offsets + c->off_base(layer, 0);
+    a.off_ustride = c->cfg.max_clusters + 1;
+    a.mu = c->mu + c->mu_rows(layer, 0) * kD;
+    a.mu_ustride = c->cfg.max_clusters;
+    a.mu_trace = mu_trace;
+    a.assign_trace = assign_trace;
+    return launch_recluster(a, stream);
+}
+
+// The window's tokens join the cluster store: the layer's host state after a re-clustering.
+void commit_window(Ctx* c, LayerState& L) {
+    L.m += c->cfg.window;
+    L.C += c->cfg.new_clusters;
+    L.pending -= c->cfg.window;
+    L.pstart = (L.pstart + c->cfg.window) % c->ring;
+    L.windows += 1;
+}
 }  // namespace
 
 extern "C" {
@@ -197,7 +250,8 @@ int ckv_create(const ckv_config* cfg, ckv_ctx** out) {
     c->units = f.batch * f.n_kv_heads;
     c->group = group;
     c->cap_c = f.capacity - f.n_sink;
-    c->sp_rows = f.n_sink + f.window;
+    c->ring = 2 * f.window;
+    c->sp_rows = f.n_sink + c->ring;
     c->device = dev;
     c->num_sms = num_sms_of_current_device();
     c->layers.assign((size_t)f.n_layers, LayerState{});
@@ -244,6 +298,8 @@ int ckv_destroy(ckv_ctx* ctx) {
     cudaGetDevice(&cur);
     cudaSetDevice(c->device);
     cudaDeviceSynchronize();
+    for (LayerState& L : c->layers)
+        if (L.done) cudaEventDestroy(L.done);
     free_all(c);
     cudaSetDevice(cur);
     delete c;
@@ -259,6 +315,10 @@ int cluster_prefill(ckv_ctx* ctx, int32_t layer, const void* K, const void* V, i
     Ctx* c = C_(ctx);
     if ((rc = check_layer(c, layer))) return rc;
     if (!aligned16(K) || !aligned16(V)) return einval("K and V must be non-null and 16-byte aligned");
+    if (c->layers[(size_t)layer].in_flight) {
+        set_error("a re-clustering of this layer is in flight; call recluster_finish");
+        return CKV_ESTATE;
+    }
     const int32_t ns = c->cfg.n_sink;
     if (n > c->cfg.capacity) {
         set_error("n exceeds the context capacity");
@@ -307,6 +367,7 @@ int cluster_prefill(ckv_ctx* ctx, int32_t layer, const void* K, const void* V, i
     L.C = C;
     L.pending = 0;
     L.windows = 0;
+    L.pstart = 0;
     return CKV_OK;
 }
 
@@ -337,6 +398,8 @@ int select_and_attend(ckv_ctx* ctx, int32_t layer, const void* q, int32_t budget
     a.G = c->group;
     a.n_sink = c->cfg.n_sink;
     a.pending = L.pending;
+    a.pstart = L.pstart;
+    a.pring = c->ring;
     a.C = L.C;
     a.m = L.m;
     a.kp = c->kp + c->rows_kp(layer, 0) * kD;
@@ -367,8 +430,9 @@ int ckv_append_kv(ckv_ctx* ctx, int32_t layer, const void* k, const void* v, voi
         return CKV_ESTATE;
     }
     if (!aligned16(k) || !aligned16(v)) return einval("k and v must be non-null and 16-byte aligned");
-    if (L.pending >= c->cfg.window) {
-        set_error("pending window is full; call recluster_increment first");
+    if (L.pending >= (L.in_flight ? c->ring : c->cfg.window)) {
+        set_error(L.in_flight ? "pending ring is full; call recluster_finish first"
+                              : "pending window is full; call recluster_increment or recluster_begin first");
         return CKV_ECAPACITY;
     }
     if ((int64_t)c->cfg.n_sink + L.m + L.pending + 1 > c->cfg.capacity) {
@@ -377,7 +441,8 @@ int ckv_append_kv(ckv_ctx* ctx, int32_t layer, const void* k, const void* v, voi
     }
     rc = launch_append((const uint16_t*)k, (const uint16_t*)v, c->units,
                        c->spk + c->rows_sp(layer, 0) * kD, c->spv + c->rows_sp(layer, 0) * kD,
-                       c->sp_rows, c->cfg.n_sink + L.pending, (cudaStream_t)stream);
+                       c->sp_rows, c->cfg.n_sink + (L.pstart + L.pending) % c->ring,
+                       (cudaStream_t)stream);
     if (rc) return rc;
     L.pending += 1;
     return CKV_OK;
@@ -389,52 +454,52 @@ int recluster_increment_traced(ckv_ctx* ctx, int32_t layer, float* mu_trace,
     if (rc) return rc;
     Ctx* c = C_(ctx);
     if ((rc = check_layer(c, layer))) return rc;
-    LayerState& L = c->layers[(size_t)layer];
-    if (!L.prefilled || L.pending != c->cfg.window) {
-        set_error("recluster_increment needs exactly `window` pending tokens");
-        return CKV_ESTATE;
-    }
-    if (L.m + c->cfg.window > c->cap_c || L.C + c->cfg.new_clusters > c->cfg.max_clusters) {
-        set_error("cluster store full (tokens or clusters)");
-        return CKV_ECAPACITY;
-    }
-    if ((mu_trace && ((uintptr_t)mu_trace & 15u)) || (assign_trace && ((uintptr_t)assign_trace & 3u)))
-        return einval("misaligned trace buffer");
-    ReclusterArgs a{};
-    a.U = c->units;
-    a.n_sink = c->cfg.n_sink;
-    a.window = c->cfg.window;
-    a.C_new = c->cfg.new_clusters;
-    a.iters = c->cfg.iters;
-    a.C_old = L.C;
-    a.m_old = L.m;
-    a.seed = c->cfg.seed;
-    a.unit_base = (int64_t)layer * c->units;
-    a.window_no = (uint64_t)L.windows + 1;
-    a.spk = c->spk + c->rows_sp(layer, 0) * kD;
-    a.spv = c->spv + c->rows_sp(layer, 0) * kD;
-    a.sp_ustride = c->sp_rows;
-    a.kp = c->kp + c->rows_kp(layer, 0) * kD;
-    a.vp = c->vp + c->rows_kp(layer, 0) * kD;
-    a.ids = c->ids + c->rows_kp(layer, 0);
-    a.kp_ustride = c->cap_c;
-    a.offsets = c->offsets + c->off_base(layer, 0);
-    a.off_ustride = c->cfg.max_clusters + 1;
-    a.mu = c->mu + c->mu_rows(layer, 0) * kD;
-    a.mu_ustride = c->cfg.max_clusters;
-    a.mu_trace = mu_trace;
-    a.assign_trace = assign_trace;
-    rc = launch_recluster(a, (cudaStream_t)stream);
+    rc = launch_window_recluster(c, layer, mu_trace, assign_trace, (cudaStream_t)stream);
     if (rc) return rc;
-    L.m += c->cfg.window;
-    L.C += c->cfg.new_clusters;
-    L.pending = 0;
-    L.windows += 1;
+    commit_window(c, c->layers[(size_t)layer]);
     return CKV_OK;
 }
 
 int recluster_increment(ckv_ctx* ctx, int32_t layer, void* stream) {
     return recluster_increment_traced(ctx, layer, nullptr, nullptr, stream);
+}
+
+int recluster_begin(ckv_ctx* ctx, int32_t layer, void* stream) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    Ctx* c = C_(ctx);
+    if ((rc = check_layer(c, layer))) return rc;
+    LayerState& L = c->layers[(size_t)layer];
+    if (!L.done) {
+        cudaError_t e = cudaEventCreateWithFlags(&L.done, cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            L.done = nullptr;
+            return cuda_fail(e, "recluster_begin: event");
+        }
+    }
+    rc = launch_window_recluster(c, layer, nullptr, nullptr, (cudaStream_t)stream);
+    if (rc) return rc;
+    cudaError_t e = cudaEventRecord(L.done, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "recluster_begin: record");
+    L.in_flight = 1;
+    return CKV_OK;
+}
+
+int recluster_finish(ckv_ctx* ctx, int32_t layer, void* stream) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    Ctx* c = C_(ctx);
+    if ((rc = check_layer(c, layer))) return rc;
+    LayerState& L = c->layers[(size_t)layer];
+    if (!L.in_flight) {
+        set_error("recluster_finish without recluster_begin");
+        return CKV_ESTATE;
+    }
+    cudaError_t e = cudaStreamWaitEvent((cudaStream_t)stream, L.done, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "recluster_finish: wait");
+    L.in_flight = 0;
+    commit_window(c, L);
+    return CKV_OK;
 }
 
 int ckv_get_layer_info(const ckv_ctx* ctx, int32_t layer, ckv_layer_info* out) {
@@ -467,15 +532,25 @@ int ckv_export_unit(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h,
     }
     const int u = b * c->cfg.n_kv_heads + h;
     cudaStream_t s = (cudaStream_t)stream;
-    const int64_t sp = c->cfg.n_sink + L.pending;
+    // sinks, then the pending tokens in append order (up to two runs of the ring)
+    const int64_t ns = c->cfg.n_sink;
+    const int64_t run1 = std::min<int64_t>(L.pending, c->ring - L.pstart), run2 = L.pending - run1;
+    const uint16_t* spk_u = c->spk + c->rows_sp(layer, u) * kD;
+    const uint16_t* spv_u = c->spv + c->rows_sp(layer, u) * kD;
+    uint16_t* dk = (uint16_t*)dst->sp_k;
+    uint16_t* dv = (uint16_t*)dst->sp_v;
     struct Item { void* d; const void* s; size_t n; } items[] = {
         {dst->mu, c->mu + c->mu_rows(layer, u) * kD, sizeof(float) * (size_t)L.C * kD},
         {dst->offsets, c->offsets + c->off_base(layer, u), sizeof(int32_t) * (size_t)(L.C + 1)},
         {dst->ids, c->ids + c->rows_kp(layer, u), sizeof(int32_t) * (size_t)L.m},
         {dst->kp, c->kp + c->rows_kp(layer, u) * kD, (size_t)(2 * L.m * kD)},
         {dst->vp, c->vp + c->rows_kp(layer, u) * kD, (size_t)(2 * L.m * kD)},
-        {dst->sp_k, c->spk + c->rows_sp(layer, u) * kD, (size_t)(2 * sp * kD)},
-        {dst->sp_v, c->spv + c->rows_sp(layer, u) * kD, (size_t)(2 * sp * kD)},
+        {dk, spk_u, (size_t)(2 * ns * kD)},
+        {dv, spv_u, (size_t)(2 * ns * kD)},
+        {dk ? dk + ns * kD : nullptr, spk_u + (ns + L.pstart) * kD, (size_t)(2 * run1 * kD)},
+        {dv ? dv + ns * kD : nullptr, spv_u + (ns + L.pstart) * kD, (size_t)(2 * run1 * kD)},
+        {dk ? dk + (ns + run1) * kD : nullptr, spk_u + ns * kD, (size_t)(2 * run2 * kD)},
+        {dv ? dv + (ns + run1) * kD : nullptr, spv_u + ns * kD, (size_t)(2 * run2 * kD)},
     };
     for (auto& it : items) {
         if (!it.d || it.n == 0) continue;
@@ -499,7 +574,12 @@ int ckv_import_unit(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h, int64_t m
         pending > c->cfg.window || c->cfg.n_sink + m + pending > c->cfg.capacity)
         return einval("import sizes out of range");
     LayerState& L = c->layers[(size_t)layer];
+    if (L.in_flight) {
+        set_error("a re-clustering of this layer is in flight; call recluster_finish");
+        return CKV_ESTATE;
+    }
     const bool first = !L.prefilled || (L.m != m || L.C != C || L.pending != pending);
+    const int64_t pstart = first ? 0 : L.pstart;  // pending rows go to ring position pstart
     cudaStream_t s = (cudaStream_t)stream;
     // content checks on a host copy of offsets and ids
     std::vector<int32_t> off((size_t)C + 1), ids((size_t)m);
@@ -517,15 +597,21 @@ int ckv_import_unit(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h, int64_t m
     for (int64_t i = 0; i < m; ++i)
         if (ids[(size_t)i] < c->cfg.n_sink || ids[(size_t)i] >= n_total) return einval("id out of range");
     const int u = b * c->cfg.n_kv_heads + h;
-    const int64_t sp = c->cfg.n_sink + pending;
+    const int64_t ns = c->cfg.n_sink;  // pending <= window and pstart is 0 or window: no wrap
+    uint16_t* spk_u = c->spk + c->rows_sp(layer, u) * kD;
+    uint16_t* spv_u = c->spv + c->rows_sp(layer, u) * kD;
+    const uint16_t* sk = (const uint16_t*)src->sp_k;
+    const uint16_t* sv = (const uint16_t*)src->sp_v;
     struct Item { void* d; const void* s; size_t n; } items[] = {
         {c->mu + c->mu_rows(layer, u) * kD, src->mu, sizeof(float) * (size_t)C * kD},
         {c->offsets + c->off_base(layer, u), src->offsets, sizeof(int32_t) * (size_t)(C + 1)},
         {c->ids + c->rows_kp(layer, u), src->ids, sizeof(int32_t) * (size_t)m},
         {c->kp + c->rows_kp(layer, u) * kD, src->kp, (size_t)(2 * m * kD)},
         {c->vp + c->rows_kp(layer, u) * kD, src->vp, (size_t)(2 * m * kD)},
-        {c->spk + c->rows_sp(layer, u) * kD, src->sp_k, (size_t)(2 * sp * kD)},
-        {c->spv + c->rows_sp(layer, u) * kD, src->sp_v, (size_t)(2 * sp * kD)},
+        {spk_u, sk, (size_t)(2 * ns * kD)},
+        {spv_u, sv, (size_t)(2 * ns * kD)},
+        {spk_u + (ns + pstart) * kD, sk + ns * kD, (size_t)(2 * pending * kD)},
+        {spv_u + (ns + pstart) * kD, sv + ns * kD, (size_t)(2 * pending * kD)},
     };
     for (auto& it : items) {
         if (it.n == 0) continue;
@@ -540,6 +626,7 @@ int ckv_import_unit(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h, int64_t m
         L.C = C;
         L.pending = pending;
         L.windows = 0;
+        L.pstart = 0;
     }
     return CKV_OK;
 }

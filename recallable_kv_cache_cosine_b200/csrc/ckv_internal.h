@@ -20,8 +20,11 @@ struct LayerState {
     int prefilled = 0;
     int64_t m = 0;
     int32_t C = 0;
-    int32_t pending = 0;
+    int32_t pending = 0;    // pending tokens, in append order from ring position pstart
     int32_t windows = 0;
+    int32_t pstart = 0;     // ring position of the oldest pending token (0 or window)
+    int in_flight = 0;      // a re-clustering started by recluster_begin is not finished
+    cudaEvent_t done = nullptr;  // recorded after that re-clustering
 };
 
 // Keys of U units: rows [row0, row0 + m) of a [U, n_rows, 128] bf16 tensor.
@@ -50,7 +53,8 @@ struct Ctx {
     int32_t units = 0;   // batch * n_kv_heads
     int32_t group = 0;   // n_q_heads / n_kv_heads
     int64_t cap_c = 0;   // clustered-row capacity per unit
-    int32_t sp_rows = 0; // n_sink + window
+    int32_t sp_rows = 0; // n_sink + ring
+    int32_t ring = 0;    // pending ring rows: 2 * window (one window re-clustering, one filling)
     int device = 0;
     int num_sms = 0;
     // Stores of all layers, [L][U][...].
@@ -140,6 +144,7 @@ struct DecodeArgs {
     int32_t budget;
     int32_t B, Hkv, G;
     int32_t n_sink, pending, C;
+    int32_t pstart, pring;  // pending token j is in ring row n_sink + (pstart + j) % pring
     int64_t m;
     const uint16_t* kp;
     const uint16_t* vp;
@@ -183,6 +188,7 @@ int launch_append(const uint16_t* k, const uint16_t* v, int32_t U, uint16_t* spk
 struct ReclusterArgs {
     int32_t U;
     int32_t n_sink, window, C_new, iters;
+    int32_t win_row0;  // row of the window's first token in a unit's sink / pending rows
     int32_t C_old;
     int64_t m_old;
     uint64_t seed;

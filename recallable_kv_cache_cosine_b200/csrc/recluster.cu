@@ -35,8 +35,8 @@ __global__ void __launch_bounds__(kRT) recluster_kernel(const ReclusterArgs a) {
 
     const int u = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = kRT / 32;
-    const uint16_t* wk = a.spk + ((int64_t)u * a.sp_ustride + a.n_sink) * kD;
-    const uint16_t* wv = a.spv + ((int64_t)u * a.sp_ustride + a.n_sink) * kD;
+    const uint16_t* wk = a.spk + ((int64_t)u * a.sp_ustride + a.win_row0) * kD;
+    const uint16_t* wv = a.spv + ((int64_t)u * a.sp_ustride + a.win_row0) * kD;
     // window keys into shared memory
     for (int i = tid; i < W * kD / 8; i += kRT)
         reinterpret_cast<uint4*>(skey)[i] = reinterpret_cast<const uint4*>(wk)[i];

@@ -324,10 +324,15 @@ __global__ void __launch_bounds__(kNT, 2)
         fence_mbar_init();
     }
     if (tid * 32 <= C) prefetch_l2(off + tid * 32);  // the boundaries, one 128-byte line each
-    if (rank == 0 && tid == 0 && a.n_sink + a.pending > 0) {  // sinks and pending rows
-        const uint32_t bytes = (uint32_t)(a.n_sink + a.pending) * kD * 2;
-        prefetch_l2_bulk(a.spk + sp_base * kD, bytes);
-        prefetch_l2_bulk(a.spv + sp_base * kD, bytes);
+    if (rank == 0 && tid == 0) {  // sinks, then the pending rows (up to two runs of the ring)
+        const int32_t run1 = min(a.pending, a.pring - a.pstart);
+        const int64_t r0[3] = {0, a.n_sink + a.pstart, a.n_sink};
+        const int32_t nr[3] = {a.n_sink, run1, a.pending - run1};
+        for (int k = 0; k < 3; ++k)
+            if (nr[k] > 0) {
+                prefetch_l2_bulk(a.spk + (sp_base + r0[k]) * kD, (uint32_t)nr[k] * kD * 2);
+                prefetch_l2_bulk(a.spv + (sp_base + r0[k]) * kD, (uint32_t)nr[k] * kD * 2);
+            }
     }
     cluster_arrive_relaxed();
     pdl_wait();
@@ -597,8 +602,8 @@ __global__ void __launch_bounds__(kNT, 2)
     auto fill_rsrc = [&](int32_t c0, int32_t c1, int p0) {
         for (int32_t idx = c0 + tid; idx < c1; idx += kNT) {
             int32_t r;
-            if (idx < base_w) {
-                r = -1 - idx;
+            if (idx < base_w) {  // a sink, or pending token idx - n_sink of the ring
+                r = -1 - (idx < a.n_sink ? idx : a.n_sink + (a.pstart + idx - a.n_sink) % a.pring);
             } else if (idx < base_p) {
                 const int32_t x = idx - base_w;
                 int k0 = 0, khi = n_whole - 1;  // last k with spre[k] <= x

@@ -130,3 +130,80 @@ def test_window_full_and_order_errors():
     assert e.value.code == ckv.CKV_EINVAL
     torch.cuda.synchronize()
     ctx.check_device_error()
+
+
+def _exports_equal(a, b):
+    for key in ("mu", "offsets", "ids", "kp", "vp", "sp_k", "sp_v"):
+        x, y = a[key], b[key]
+        assert x.shape == y.shape, key
+        assert torch.equal(x.view(torch.int16) if x.dtype == torch.bfloat16 else x,
+                           y.view(torch.int16) if y.dtype == torch.bfloat16 else y), key
+
+
+def test_async_recluster_overlaps_decode():
+    """recluster_begin on a second stream while appends and decode continue on the first
+    (ClusterKV explainer, section 4.1: clustering runs asynchronously with decoding). During
+    the overlap the layer attends its old clusters plus every pending token (the window being
+    clustered and the tokens appended since); after recluster_finish the store equals the one
+    the synchronous recluster_increment builds at the same position. Two windows are run, so
+    the second overlap wraps around the pending ring."""
+    import recallable_kv_cache_cosine_b200 as ckv
+    seed, G, W = 9, 4, 320
+    B, Hkv, n, C, n_centers = 1, 2, 2048, 32, 32
+    extra = (50, 77)  # tokens appended during each overlap
+    K = np.empty((B, Hkv, n, 128), np.uint16)
+    V = np.empty_like(K)
+    AK = np.empty((B, Hkv, 3 * W, 128), np.uint16)
+    AV = np.empty_like(AK)
+    for b in range(B):
+        for h in range(Hkv):
+            u = si.unit_id(0, b, h, B, Hkv)
+            K[b, h], V[b, h] = si.keys_values(seed, u, n, n_centers)
+            AK[b, h], AV[b, h] = si.appended_tokens(seed, u, 3 * W, n_centers)
+    make = lambda: ckv.ClusterKV(1, B, Hkv, Hkv * G, capacity=n + 3 * W, max_clusters=C + 8, seed=seed)
+    actx, sctx = make(), make()
+    actx.cluster_prefill(0, to_dev(K), to_dev(V), C)
+    sctx.cluster_prefill(0, to_dev(K), to_dev(V), C)
+    # every appended token as its own device tensor, ready before any stream uses it
+    tk = [to_dev(np.ascontiguousarray(AK[:, :, i])) for i in range(3 * W)]
+    tv = [to_dev(np.ascontiguousarray(AV[:, :, i])) for i in range(3 * W)]
+    tok = lambda a, i: tk[i] if a is AK else tv[i]
+    qs = np.stack([si.queries(seed, 0, b, 8, Hkv * G) for b in range(B)], axis=1)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    stats = {}
+    j = 0
+    for window in range(2):
+        C_old, m_old = C + 4 * window, n - 16 + window * W
+        # fill the window (both contexts)
+        while actx.layer_info(0).pending < W:
+            actx.append_kv(0, tok(AK, j), tok(AV, j), stream=s1)
+            sctx.append_kv(0, tok(AK, j), tok(AV, j))
+            j += 1
+        s2.wait_stream(s1)
+        actx.recluster_begin(0, stream=s2)
+        with pytest.raises(ckv.CkvError):
+            actx.recluster_increment(0, stream=s1)
+        sctx.recluster_increment(0)
+        for t in range(extra[window]):
+            actx.append_kv(0, tok(AK, j), tok(AV, j), stream=s1)
+            sctx.append_kv(0, tok(AK, j), tok(AV, j))
+            j += 1
+            if t in (0, extra[window] - 1):
+                info = actx.layer_info(0)
+                assert (info.C, info.m, info.pending) == (C_old, m_old, W + t + 1)
+                with torch.cuda.stream(s1):
+                    _decode_check(actx, qs[t % 8], 512, B, Hkv, G, stats, window)
+        actx.recluster_finish(0, stream=s1)
+        info = actx.layer_info(0)
+        assert (info.C, info.m, info.pending, info.windows) == (C_old + 4, m_old + W, extra[window], window + 1)
+        with torch.cuda.stream(s1):
+            _decode_check(actx, qs[window], 512, B, Hkv, G, stats, window + 1)
+        torch.cuda.synchronize()
+        actx.check_device_error()
+        for b in range(B):
+            for h in range(Hkv):
+                _exports_equal(actx.export_unit(0, b, h), sctx.export_unit(0, b, h))
+    with pytest.raises(ckv.CkvError):
+        actx.recluster_finish(0)
+    assert stats["near_tie"] <= 1
