@@ -177,6 +177,16 @@ def oracle_time_layer_steps(st, q, n_layer_steps):
     return (time.perf_counter() - t0) / n_layer_steps
 
 
+def workload_config(L, D, world):
+    """The workload both arms report (the reference arm times a sample of it)."""
+    return {"workload": "llama3.1-8b-shaped layer (32 q / 8 kv heads, d=128), n=32768, "
+                        "batch 1, C=400, budget=1024, held as 32 distinct layer stores",
+            "layer_stores": L, "decode_steps": D, "n": N_CTX, "batch": B, "kv_heads": HKV,
+            "q_heads": HQ, "C": C_CLUSTERS, "budget": BUDGET, "iters": ITERS,
+            "window": WINDOW, "parallelism": f"replicas x{world} (units independent)",
+            "l2": "inputs larger than L2: 32 layer stores, ~193 MB selected per decode pass"}
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return
@@ -194,8 +204,7 @@ def run_reference(args, world, rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": us * per_step / 1e3,
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": "llama3.1-8b-shaped layer, n=32768, B=1, 8 kv / 32 q heads, "
-                                   "C=400, budget=1024 (CPU oracle sample)"},
+            "config": workload_config(args.layers, args.decode_steps, args.gpus),
             "cpu_baseline": {"value": us, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": us, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -482,12 +491,7 @@ def run_gpu(args, world, rank, local):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K_steps,
             "warmup": args.warmup, "ms_per_step": t_step / K_steps * 1e3, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "llama3.1-8b-shaped layer (32 q / 8 kv heads, d=128), n=32768, "
-                                   "batch 1, C=400, budget=1024, held as 32 distinct layer stores",
-                       "layer_stores": L, "decode_steps": D, "n": N_CTX, "batch": B, "kv_heads": HKV,
-                       "q_heads": HQ, "C": C_CLUSTERS, "budget": BUDGET, "iters": ITERS,
-                       "window": W, "parallelism": f"replicas x{world} (units independent)",
-                       "l2": "inputs larger than L2: 32 layer stores, ~193 MB selected per decode pass"},
+            "config": workload_config(L, D, world),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
                          "frac": achieved / hbm_gbs, "traffic": SELECT_ATTEND_TRAFFIC,
                          "kernel": "select_attend_kernel<4>", "bytes_per_launch": bytes_launch,
