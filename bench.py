@@ -494,7 +494,7 @@ def run_gpu(args, world, rank, local):
             "config": workload_config(L, D, world),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
                          "frac": achieved / hbm_gbs, "traffic": SELECT_ATTEND_TRAFFIC,
-                         "kernel": "select_attend_kernel<4>", "bytes_per_launch": bytes_launch,
+                         "kernel": "select_attend_kernel<4, false>", "bytes_per_launch": bytes_launch,
                          "us_per_launch": launch_us, "peak_kind": peak_kind},
             "kmeans": {"keys_per_s": keys_per_s, "roofline_keys_per_s": keys_roof,
                        "frac": keys_per_s / keys_roof, "prefill_ms_per_layer": tA / (K_steps * L) * 1e3,

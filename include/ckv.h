@@ -118,6 +118,17 @@ CKV_API int cluster_prefill(ckv_ctx* ctx, int32_t layer, const void* K, const vo
 CKV_API int select_and_attend(ckv_ctx* ctx, int32_t layer, const void* q, int32_t budget, float* out,
                       int32_t* sel_idx, int32_t* sel_count, void* stream);
 
+/* The same decode step with one selection per query head: query head j scores the clusters
+ * of its KV head j / group by q_j . mu_c (instead of the group's qbar), fills its own
+ * partial cluster by q_j . k and attends its own `budget` rows. This is the alternative
+ * reading of the explainer's single-query select_clusters for grouped heads.
+ *   q, out, budget : as for select_and_attend.
+ *   sel_idx   : optional device int32 [batch, n_q_heads, budget], per query head.
+ *   sel_count : optional device int32 [batch, n_q_heads].
+ * Same errors as select_and_attend. */
+CKV_API int select_and_attend_per_head(ckv_ctx* ctx, int32_t layer, const void* q, int32_t budget,
+                               float* out, int32_t* sel_idx, int32_t* sel_count, void* stream);
+
 /* Appends one generated token's K/V per unit to the layer's pending rows (the tokens a
  * later re-clustering will cluster). The pending rows form a ring of 2 x window rows per
  * unit: one window can be re-clustering (recluster_begin) while the next one fills.

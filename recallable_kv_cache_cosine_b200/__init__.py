@@ -56,6 +56,7 @@ SIGNATURES = {
     "ckv_device_bytes": (C.c_int64, [P]),
     "cluster_prefill": (C.c_int, [P, I32, P, P, I64, I32, P]),
     "select_and_attend": (C.c_int, [P, I32, P, I32, P, P, P, P]),
+    "select_and_attend_per_head": (C.c_int, [P, I32, P, I32, P, P, P, P]),
     "ckv_append_kv": (C.c_int, [P, I32, P, P, P]),
     "recluster_increment": (C.c_int, [P, I32, P]),
     "recluster_increment_traced": (C.c_int, [P, I32, P, P, P]),
@@ -169,6 +170,16 @@ class ClusterKV:
         _check(lib().select_and_attend(self._ctx, layer, _bf16(q, "q"), budget, _ptr(out),
                                        _ptr(sel_idx), _ptr(sel_count), _stream(stream)),
                "select_and_attend")
+
+    def select_and_attend_per_head(self, layer: int, q: torch.Tensor, budget: int, out: torch.Tensor,
+                                   sel_idx: torch.Tensor | None = None,
+                                   sel_count: torch.Tensor | None = None, stream=None):
+        """One selection per query head; sel_idx [batch, n_q_heads, budget], sel_count [batch, n_q_heads]."""
+        if out.dtype != torch.float32 or not out.is_cuda:
+            raise TypeError("out must be a CUDA float32 tensor")
+        _check(lib().select_and_attend_per_head(self._ctx, layer, _bf16(q, "q"), budget, _ptr(out),
+                                                _ptr(sel_idx), _ptr(sel_count), _stream(stream)),
+               "select_and_attend_per_head")
 
     def append_kv(self, layer: int, k: torch.Tensor, v: torch.Tensor, stream=None):
         """k, v: [batch, n_kv_heads, 128] bf16."""

@@ -191,6 +191,57 @@ void commit_window(Ctx* c, LayerState& L) {
     L.pstart = (L.pstart + c->cfg.window) % c->ring;
     L.windows += 1;
 }
+int decode_call(ckv_ctx* ctx, int32_t layer, const void* q, int32_t budget, float* out,
+                int32_t* sel_idx, int32_t* sel_count, void* stream, bool per_head) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    Ctx* c = C_(ctx);
+    if ((rc = check_layer(c, layer))) return rc;
+    const LayerState& L = c->layers[(size_t)layer];
+    if (!L.prefilled) {
+        set_error("select_and_attend before cluster_prefill for this layer");
+        return CKV_ESTATE;
+    }
+    if (!aligned16(q) || !aligned16(out)) return einval("q and out must be non-null and 16-byte aligned");
+    if ((sel_idx && ((uintptr_t)sel_idx & 3u)) || (sel_count && ((uintptr_t)sel_count & 3u)))
+        return einval("sel_idx / sel_count must be 4-byte aligned");
+    if (budget < 1 || (int64_t)budget < (int64_t)c->cfg.n_sink + L.pending)
+        return einval("budget must be >= n_sink + pending and >= 1");
+    DecodeArgs a{};
+    a.q = (const uint16_t*)q;
+    a.out = out;
+    a.sel_idx = sel_idx;
+    a.sel_count = sel_count;
+    a.budget = budget;
+    a.B = c->cfg.batch;
+    // per head: G = 1 over (b, query head) virtual units, each reading its KV head's store
+    a.Hkv = per_head ? c->cfg.n_q_heads : c->cfg.n_kv_heads;
+    a.G = per_head ? 1 : c->group;
+    a.qsplit = per_head ? c->group : 1;
+    a.n_sink = c->cfg.n_sink;
+    a.pending = L.pending;
+    a.pstart = L.pstart;
+    a.pring = c->ring;
+    a.C = L.C;
+    a.m = L.m;
+    a.kp = c->kp + c->rows_kp(layer, 0) * kD;
+    a.vp = c->vp + c->rows_kp(layer, 0) * kD;
+    a.spk = c->spk + c->rows_sp(layer, 0) * kD;
+    a.spv = c->spv + c->rows_sp(layer, 0) * kD;
+    a.ids = c->ids + c->rows_kp(layer, 0);
+    a.offsets = c->offsets + c->off_base(layer, 0);
+    a.mu = c->mu + c->mu_rows(layer, 0) * kD;
+    a.kp_ustride = c->cap_c;
+    a.sp_ustride = c->sp_rows;
+    a.off_ustride = c->cfg.max_clusters + 1;
+    a.mu_ustride = c->cfg.max_clusters;
+    a.part_scratch = c->ws.part;
+    a.part_ustride = c->cap_c;
+    a.err = c->err;
+    return per_head ? launch_select_attend_per_head(a, c->num_sms, (cudaStream_t)stream)
+                    : launch_select_attend(a, c->num_sms, (cudaStream_t)stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -271,7 +322,7 @@ int ckv_create(const ckv_config* cfg, ckv_ctx** out) {
     rc = rc ? rc : dev_alloc(&c->ws.best, (size_t)(U * c->cap_c), c);
     rc = rc ? rc : dev_alloc(&c->ws.perm, (size_t)(U * c->cap_c), c);
     rc = rc ? rc : dev_alloc(&c->ws.chunk, (size_t)(U * n_chunks(c->cap_c) * cmax), c);
-    rc = rc ? rc : dev_alloc(&c->ws.part, (size_t)(U * c->cap_c), c);
+    rc = rc ? rc : dev_alloc(&c->ws.part, (size_t)(U * c->group * c->cap_c), c);  // per query head
     rc = rc ? rc : dev_alloc(&c->err, 4, c);
     if (rc == CKV_OK) {
         cudaError_t e = cudaMemset(c->err, 0, 16);
@@ -373,50 +424,12 @@ int cluster_prefill(ckv_ctx* ctx, int32_t layer, const void* K, const void* V, i
 
 int select_and_attend(ckv_ctx* ctx, int32_t layer, const void* q, int32_t budget, float* out,
                       int32_t* sel_idx, int32_t* sel_count, void* stream) {
-    int rc = check_ctx(ctx);
-    if (rc) return rc;
-    Ctx* c = C_(ctx);
-    if ((rc = check_layer(c, layer))) return rc;
-    const LayerState& L = c->layers[(size_t)layer];
-    if (!L.prefilled) {
-        set_error("select_and_attend before cluster_prefill for this layer");
-        return CKV_ESTATE;
-    }
-    if (!aligned16(q) || !aligned16(out)) return einval("q and out must be non-null and 16-byte aligned");
-    if ((sel_idx && ((uintptr_t)sel_idx & 3u)) || (sel_count && ((uintptr_t)sel_count & 3u)))
-        return einval("sel_idx / sel_count must be 4-byte aligned");
-    if (budget < 1 || (int64_t)budget < (int64_t)c->cfg.n_sink + L.pending)
-        return einval("budget must be >= n_sink + pending and >= 1");
-    DecodeArgs a{};
-    a.q = (const uint16_t*)q;
-    a.out = out;
-    a.sel_idx = sel_idx;
-    a.sel_count = sel_count;
-    a.budget = budget;
-    a.B = c->cfg.batch;
-    a.Hkv = c->cfg.n_kv_heads;
-    a.G = c->group;
-    a.n_sink = c->cfg.n_sink;
-    a.pending = L.pending;
-    a.pstart = L.pstart;
-    a.pring = c->ring;
-    a.C = L.C;
-    a.m = L.m;
-    a.kp = c->kp + c->rows_kp(layer, 0) * kD;
-    a.vp = c->vp + c->rows_kp(layer, 0) * kD;
-    a.spk = c->spk + c->rows_sp(layer, 0) * kD;
-    a.spv = c->spv + c->rows_sp(layer, 0) * kD;
-    a.ids = c->ids + c->rows_kp(layer, 0);
-    a.offsets = c->offsets + c->off_base(layer, 0);
-    a.mu = c->mu + c->mu_rows(layer, 0) * kD;
-    a.kp_ustride = c->cap_c;
-    a.sp_ustride = c->sp_rows;
-    a.off_ustride = c->cfg.max_clusters + 1;
-    a.mu_ustride = c->cfg.max_clusters;
-    a.part_scratch = c->ws.part;
-    a.part_ustride = c->cap_c;
-    a.err = c->err;
-    return launch_select_attend(a, c->num_sms, (cudaStream_t)stream);
+    return decode_call(ctx, layer, q, budget, out, sel_idx, sel_count, stream, false);
+}
+
+int select_and_attend_per_head(ckv_ctx* ctx, int32_t layer, const void* q, int32_t budget,
+                               float* out, int32_t* sel_idx, int32_t* sel_count, void* stream) {
+    return decode_call(ctx, layer, q, budget, out, sel_idx, sel_count, stream, true);
 }
 
 int ckv_append_kv(ckv_ctx* ctx, int32_t layer, const void* k, const void* v, void* stream) {

@@ -145,6 +145,7 @@ struct DecodeArgs {
     int32_t B, Hkv, G;
     int32_t n_sink, pending, C;
     int32_t pstart, pring;  // pending token j is in ring row n_sink + (pstart + j) % pring
+    int32_t qsplit;         // per-head selection: virtual units per KV unit (query heads)
     int64_t m;
     const uint16_t* kp;
     const uint16_t* vp;
@@ -181,6 +182,7 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 }
 
 int launch_select_attend(const DecodeArgs& a, int num_sms, cudaStream_t s);
+int launch_select_attend_per_head(const DecodeArgs& a, int num_sms, cudaStream_t s);
 
 int launch_append(const uint16_t* k, const uint16_t* v, int32_t U, uint16_t* spk, uint16_t* spv,
                   int64_t sp_ustride_rows, int32_t row, cudaStream_t s);

@@ -263,13 +263,17 @@ CKV_DEV size_t ring_bytes_of(int G, int RB) {
     return r;
 }
 
-template <int G>
+// kPerHead: one selection per query head. The kernel then runs with G = 1 over virtual
+// units (b, query head): virtual unit v reads the store of KV unit v / a.qsplit and its own
+// query, output and selection rows.
+template <int G, bool kPerHead>
 __global__ void __launch_bounds__(kNT, 2)
     select_attend_kernel(const DecodeArgs a, int32_t S, int32_t prow_cap, int32_t RB) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const int C = a.C;
     const uint32_t rank = cluster_ctarank();
     const int unit = blockIdx.x / S;
+    const int su = kPerHead ? unit / a.qsplit : unit;  // the store's unit
     const int b = unit / a.Hkv, h = unit % a.Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -307,10 +311,10 @@ __global__ void __launch_bounds__(kNT, 2)
         sm.full = (uint64_t*)take(sizeof(uint64_t));
     }
 
-    const int64_t kp_base = (int64_t)unit * a.kp_ustride;
-    const int64_t sp_base = (int64_t)unit * a.sp_ustride;
-    const int32_t* off = a.offsets + (int64_t)unit * a.off_ustride;
-    const float* mu = a.mu + (int64_t)unit * a.mu_ustride * kD;
+    const int64_t kp_base = (int64_t)su * a.kp_ustride;
+    const int64_t sp_base = (int64_t)su * a.sp_ustride;
+    const int32_t* off = a.offsets + (int64_t)su * a.off_ustride;
+    const float* mu = a.mu + (int64_t)su * a.mu_ustride * kD;
     const int c_begin = (int)((int64_t)C * rank / S);
     const int c_end = (int)((int64_t)C * (rank + 1) / S);
 
@@ -1102,7 +1106,7 @@ int max_active_clusters(void (*kern)(DecodeArgs, int32_t, int32_t, int32_t), int
 // One launch plan per (device, group size, units, C, budget), found once. The cluster size S
 // is the largest power of two <= 16 whose clusters for all units are resident at once (one
 // wave), with U * S <= 2 * SMs; otherwise the smallest S that fits in shared memory.
-template <int G>
+template <int G, bool kPerHead>
 int plan_for(const DecodeArgs& a, int num_sms, Plan* out) {
     static std::mutex mtx;
     static std::map<std::tuple<int, int, int, int>, Plan> cache;
@@ -1118,7 +1122,7 @@ int plan_for(const DecodeArgs& a, int num_sms, Plan* out) {
         *out = it->second;
         return CKV_OK;
     }
-    auto kern = select_attend_kernel<G>;
+    auto kern = select_attend_kernel<G, kPerHead>;
     Plan best{};
     // Few units: one CTA per SM (a 256-row ring makes two CTAs too large for one SM) and at
     // most half of the SMs per launch, so that the next launch's CTAs, started early by
@@ -1154,10 +1158,10 @@ int plan_for(const DecodeArgs& a, int num_sms, Plan* out) {
     return CKV_OK;
 }
 
-template <int G>
+template <int G, bool kPerHead = false>
 int launch_g(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     Plan plan;
-    int rc = plan_for<G>(a, num_sms, &plan);
+    int rc = plan_for<G, kPerHead>(a, num_sms, &plan);
     if (rc != CKV_OK) return rc;
     const int U = a.B * a.Hkv;
     const int S = plan.S;
@@ -1176,12 +1180,21 @@ int launch_g(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     attrs[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attrs;
     cfg.numAttrs = 2;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, select_attend_kernel<G>, a, (int32_t)S, pc, (int32_t)plan.RB);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, select_attend_kernel<G, kPerHead>, a, (int32_t)S, pc,
+                                       (int32_t)plan.RB);
     if (e != cudaSuccess) return cuda_fail(e, "select_attend: launch");
     return CKV_OK;
 }
 
 }  // namespace
+
+int launch_select_attend_per_head(const DecodeArgs& a, int num_sms, cudaStream_t s) {
+    if (a.G != 1) {
+        set_error("select_and_attend_per_head: internal group size must be 1");
+        return CKV_EINVAL;
+    }
+    return launch_g<1, true>(a, num_sms, s);
+}
 
 int launch_select_attend(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     switch (a.G) {

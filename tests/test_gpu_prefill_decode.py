@@ -172,3 +172,37 @@ def test_decode_exact_prefix_budgets_take_no_partial():
     stats = {}
     for bud in budgets:
         _decode_and_check(ctx, 0, q, bud, stats, 1, 1, 4)
+
+
+@pytest.mark.parametrize("B,Hkv,G,n,C,n_centers,budget", [(2, 2, 4, 3000, 40, 30, 256),
+                                                          (1, 8, 4, 32768, 400, 400, 1024)])
+def test_per_query_head_selection(B, Hkv, G, n, C, n_centers, budget):
+    """select_and_attend_per_head: every query head selects and attends on its own. Each head
+    is the oracle's decode of its KV head's store with a one-head group (qbar = q_j)."""
+    ckv = _ckv()
+    seed = 13
+    K, V = _layer_data(seed, 0, B, Hkv, n, n_centers)
+    ctx = ckv.ClusterKV(1, B, Hkv, Hkv * G, capacity=n, max_clusters=C, seed=seed)
+    ctx.cluster_prefill(0, to_dev(K), to_dev(V), C)
+    Hq = Hkv * G
+    q = np.stack([si.queries(seed, 0, b, 1, Hq)[0] for b in range(B)])  # [B, Hq, 128]
+    out = torch.empty(B, Hq, 128, device="cuda", dtype=torch.float32)
+    sel = torch.empty(B, Hq, budget, device="cuda", dtype=torch.int32)
+    cnt = torch.empty(B, Hq, device="cuda", dtype=torch.int32)
+    ctx.select_and_attend_per_head(0, to_dev(q), budget, out, sel, cnt)
+    torch.cuda.synchronize()
+    ctx.check_device_error()
+    outs, sels, cnts = out.cpu().numpy(), sel.cpu().numpy(), cnt.cpu().numpy()
+    stats = {}
+    heads = range(Hq) if n <= 4096 else (0, 5, 18, 31)
+    for b in range(B):
+        stores = {}
+        for j in heads:
+            h = j // G
+            if h not in stores:
+                stores[h] = store_from_export(ctx.export_unit(0, b, h), n_sink=ctx.cfg.n_sink)
+            check_decode_unit(stores[h], q[b, j:j + 1], budget, outs[b, j:j + 1], sels[b, j],
+                              int(cnts[b, j]), stats)
+    assert stats["near_tie"] <= 1
+    # the grouped call still uses one selection per KV head
+    _decode_and_check(ctx, 0, q, budget, {}, B, Hkv, G)
