@@ -8,9 +8,9 @@
 //    scatter), and the mean is a segmented reduction that reads the keys in that order.
 //    The last iteration also writes the permuted K and V rows into the cluster store.
 //
-// Determinism: integer counts only (no float atomics). Each centroid is summed by one
-// warp in a fixed order (ascending key index within the cluster), so runs are
-// bit-reproducible.
+// Determinism: integer counts only (no float atomics). Each centroid is summed in a fixed
+// order (every dimension by one thread over the members in ascending key index, in four
+// interleaved partial sums added in a fixed order), so runs are bit-reproducible.
 #include "ckv_common.cuh"
 #include "ckv_internal.h"
 

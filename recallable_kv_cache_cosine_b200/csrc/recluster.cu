@@ -6,6 +6,9 @@
 // prefill rule, keyed by (seed, unit, window number). The new clusters are appended after the
 // existing ones, which are left unchanged.
 //
+// The window is read from the pending ring (two windows of rows after the sinks: the one being
+// clustered and the one still filling) at the row the host passes.
+//
 // The window is small (320 x 128 bf16 = 80 KB), so one CTA per unit runs the whole clustering
 // in shared memory: init, 10 x (normalise, assign, stable counting sort, mean), then it writes
 // the permuted K/V rows, their token ids, the new offsets and the new centroids into the

@@ -20,15 +20,16 @@
 //   2. every CTA then computes the whole selection on its own, without a second exchange:
 //      the walk in descending score order stops at the first cluster whose inclusive token
 //      count exceeds the remaining budget, so that cluster (the cut) is the weighted
-//      quantile of the scores with the cluster sizes as weights. A 4-pass radix select over
-//      the order-preserving score bits, with size-weighted histograms, finds its score; ties
-//      at that score are walked in index order. The whole clusters (score above the cut) are
-//      few; they are compacted and ranked among themselves for their prefix sums;
-//   3. the selected rows form one index space: sinks, pending, whole clusters by rank, then
-//      the partial tokens of the cut cluster. With a partial fill and S > 1, CTA S-1 takes
-//      exactly the partial tokens: it copies the cut cluster's K and V rows into shared
-//      memory, ranks the tokens by qbar . k there and attends the top ones in place. The
-//      other CTAs split the rest;
+//      quantile of the scores with the cluster sizes as weights. The scores are mapped
+//      monotonically onto 256 linear buckets; a size-weighted histogram gives the bucket that
+//      holds the cut, and the clusters of that bucket and above (a dozen or so) are compacted
+//      and ranked exactly among themselves for their prefix sums;
+//   3. the selected rows form one index space: sinks, pending (in append order, from the
+//      two-window pending ring), whole clusters by rank, then the partial tokens of the cut
+//      cluster. With a partial fill and S > 1, CTA S-1 takes exactly the partial tokens: it
+//      copies the cut cluster's K and V rows into shared memory (started during the
+//      selection when the histogram isolates the cut), ranks the tokens by qbar . k there
+//      and attends the top ones in place. The other CTAs split the rest;
 //   4. rows reach a two-slot shared-memory ring through cp.async (16 bytes per thread,
 //      coalesced rows, XOR-swizzled 16-byte chunks); all of a CTA's rows are in flight at
 //      once when they fit the ring. Each warp runs flash-decode on 16-row tiles with
@@ -38,7 +39,8 @@
 //   5. the warp partials (max, sum, accumulator) are merged per CTA, and the CTA partials in
 //      CTA 0 through distributed shared memory, which writes the fp32 output.
 // The kernel triggers programmatic dependent launch at entry and prefetches its centroid
-// slice into L2 before waiting on the previous grid.
+// slice into L2 before waiting on the previous grid. A compile-time flag instantiates it for
+// one selection per query head (G = 1 over (sequence, query head) units).
 #include <float.h>
 
 #include <map>
