@@ -48,6 +48,10 @@ def lib():
             "orc_kmeans": (None, [P, i64, i32, i32, P, P, P, P, P]),
             "orc_prefill_unit": (None, [P, P, i64, i32, i32, i32, u64, P, P, P, P, P, P]),
             "orc_recluster_window": (None, [P, P, i64, i32, i32, u64, i64, P, P, P, P, P, P]),
+            "orc_cluster_drift": (None, [P, P, P, i32, P]),
+            "orc_split_key": (u64, [u64, i64, u64, i32]),
+            "orc_split_drifted": (i32, [P, P, P, P, P, i32, C.c_double, i32, i32, u64, i64,
+                                        u64, P, P, P, P, P, P]),
             "orc_group_query": (None, [P, i32, P]),
             "orc_select": (i32, [P, P, i32, P, P, P, P]),
             "orc_attend": (None, [P, P, i32, P, i32, P]),
@@ -249,6 +253,51 @@ def recluster(st: Store, seed: int, unit: int, C_new: int = NEW_CLUSTERS,
                 np.concatenate([st.offsets, st.m + offs[1:]]).astype(np.int32),
                 np.concatenate([st.mu, mu]), st.n_sink, st.windows + 1)
     return new, a
+
+
+def cluster_drift(st: Store) -> np.ndarray:
+    """Mean cosine distance of each cluster's members to its centroid (explainer section
+    3.2, drift detection). Returns [C] float64."""
+    s = st._c()
+    out = np.empty(max(st.C, 1), np.float64)
+    lib().orc_cluster_drift(s.kp, s.offsets, s.mu, st.C, _p(out))
+    return out[: st.C].copy()
+
+
+def split_key(seed: int, unit: int, window: int, c: int) -> int:
+    return lib().orc_split_key(seed, unit, window, c)
+
+
+def split_drifted(st: Store, threshold: float, seed: int, unit: int, room: int,
+                  iters: int = ITERS):
+    """One split pass (explainer section 3.2, decode phase): every cluster with drift above
+    ``threshold`` and at least two members is split by 2-cluster cosine K-means, at most
+    ``room`` of them (lowest index first). Returns (new Store, split flags [C])."""
+    st._c()
+    C_, m = st.C, st.m
+    kp2 = np.empty_like(st.kp)
+    vp2 = np.empty_like(st.vp)
+    ids2 = np.empty_like(st.ids)
+    offs2 = np.empty(C_ + max(room, 0) + 1, np.int32)
+    mu2 = np.empty((C_ + max(room, 0), D), np.float64)
+    flags = np.empty(max(C_, 1), np.int32)
+    n = lib().orc_split_drifted(_p(st.kp), _p(st.vp), _p(st.ids), _p(st.offsets), _p(st.mu), C_,
+                                float(threshold), room, iters, seed, unit, st.windows,
+                                _p(kp2), _p(vp2), _p(ids2), _p(offs2), _p(mu2), _p(flags))
+    assert offs2[n] == m
+    new = dataclasses.replace(st, kp=kp2, vp=vp2, ids=ids2, offsets=offs2[: n + 1].copy(),
+                              mu=mu2[:n].copy())
+    return new, flags[:C_].copy()
+
+
+def pad_clusters(st: Store, C_total: int) -> Store:
+    """Appends empty clusters (zero centroid, no rows) up to ``C_total``. An empty cluster
+    never adds a row to a selection."""
+    extra = C_total - st.C
+    assert extra >= 0
+    return dataclasses.replace(
+        st, offsets=np.concatenate([st.offsets, np.full(extra, st.m, np.int32)]).astype(np.int32),
+        mu=np.concatenate([st.mu, np.zeros((extra, D))]))
 
 
 @dataclasses.dataclass

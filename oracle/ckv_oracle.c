@@ -10,7 +10,8 @@
  *   [EXPL] "大模型KV Cache压缩技术：ClusterKV的语义空间优化" (ClusterKV explainer),
  *          section 3.1 (attention formula, centroid mean, cluster-importance relation),
  *          section 3.2 (16 sinks, cosine K-means at prefill, incremental clustering
- *          every 320 tokens), section 3.3 (select_clusters listing), section 4.1
+ *          every 320 tokens, splitting of drifted clusters), section 3.3
+ *          (select_clusters listing), section 4.1
  *          (half-precision distance matmul, cluster-contiguous KV layout).
  *   [ABS]  "ClusterKV: Manipulating LLM KV Cache in Semantic Space for Recallable
  *          Compression" (arXiv 2412.03213 listing), abstract.
@@ -270,6 +271,109 @@ void orc_recluster_window(const uint16_t* wk, const uint16_t* wv, int64_t w, int
     }
     free(init);
     free(perm);
+}
+
+/* --------------------------------------------------- drift check and split ---------- */
+/* [EXPL] 3.2, decode phase: centroid drift is detected and a cluster whose mean
+ * intra-cluster distance is above a threshold is split. The page gives neither the
+ * distance, the threshold nor the way of splitting. Readings:
+ *   - the distance of a member is its cosine distance to the cluster's centroid,
+ *     1 - cos(k_i, mu_c), the same distance the clustering uses; a cosine with a zero
+ *     vector counts as 0. An empty cluster has drift 0;
+ *   - the threshold is a caller parameter;
+ *   - a split is cosine K-means with 2 clusters on the cluster's own rows, the prefill's
+ *     rule on a smaller set (same init rule, same iterations), and its two halves replace
+ *     the cluster. */
+
+/* drift[c] = (1/|c|) sum over the members of c of (1 - cos(k_i, mu_c)). */
+void orc_cluster_drift(const uint16_t* kp, const int32_t* offsets, const double* mu, int32_t C,
+                       double* drift) {
+    for (int32_t c = 0; c < C; c++) {
+        int32_t lo = offsets[c], hi = offsets[c + 1];
+        if (hi == lo) {
+            drift[c] = 0.0;
+            continue;
+        }
+        const double* mc = mu + (int64_t)c * ORC_D;
+        double mm = 0.0;
+        for (int d = 0; d < ORC_D; d++) mm += mc[d] * mc[d];
+        double acc = 0.0;
+        for (int32_t j = lo; j < hi; j++) {
+            double dot = 0.0, kk = 0.0;
+            for (int d = 0; d < ORC_D; d++) {
+                double x = orc_bf16_to_double(kp[(int64_t)j * ORC_D + d]);
+                dot += x * mc[d];
+                kk += x * x;
+            }
+            double cosv = (kk > 0.0 && mm > 0.0) ? dot / (sqrt(kk) * sqrt(mm)) : 0.0;
+            acc += 1.0 - cosv;
+        }
+        drift[c] = acc / (double)(hi - lo);
+    }
+}
+
+/* Init stream of the split of cluster c: the unit's stream key for the current window
+ * number, mixed with (c + 1) times the 64-bit golden-ratio constant (the Weyl increment of
+ * SplitMix64), so that every cluster of a split pass draws its own init. */
+uint64_t orc_split_key(uint64_t seed, int64_t unit, uint64_t window, int32_t c) {
+    return orc_stream_key(seed, unit, window) ^ ((uint64_t)(c + 1) * 0x9E3779B97F4A7C15ULL);
+}
+
+/* One split pass over a unit's store (offsets [C + 1], m = offsets[C]). Cluster c is split
+ * when drift[c] > threshold and it has at least two members, for at most `room` clusters
+ * (the lowest indices first). A split runs orc_kmeans with 2 clusters and `iters`
+ * iterations on the cluster's rows in store order, from orc_init_indices(|c|, 2,
+ * orc_split_key(seed, unit, window, c)). The rows are reordered inside the cluster's segment:
+ * the first child's rows, then the second's, each in their previous order. The children
+ * take indices c' and c' + 1, with c' = c + (number of split clusters below c), and their
+ * centroids are the means of their rows. Any other cluster keeps its rows and centroid
+ * and moves to index c + (number of split clusters below c).
+ * Outputs: kp2, vp2 [m, 128], ids2 [m], offsets2 [C + room + 1], mu2 [C + room, 128] (only
+ * the first (return value) clusters are written), split [C] (1 where c was split).
+ * Returns the new cluster count. */
+int32_t orc_split_drifted(const uint16_t* kp, const uint16_t* vp, const int32_t* ids,
+                          const int32_t* offsets, const double* mu, int32_t C, double threshold,
+                          int32_t room, int32_t iters, uint64_t seed, int64_t unit,
+                          uint64_t window, uint16_t* kp2, uint16_t* vp2, int32_t* ids2,
+                          int32_t* offsets2, double* mu2, int32_t* split) {
+    double* drift = (double*)malloc(sizeof(double) * (size_t)(C > 0 ? C : 1));
+    orc_cluster_drift(kp, offsets, mu, C, drift);
+    int32_t n_split = 0, out = 0;
+    for (int32_t c = 0; c < C; c++) {
+        int32_t lo = offsets[c], hi = offsets[c + 1], size = hi - lo;
+        split[c] = drift[c] > threshold && size >= 2 && n_split < room;
+        if (!split[c]) {
+            offsets2[out] = lo;
+            memcpy(mu2 + (int64_t)out * ORC_D, mu + (int64_t)c * ORC_D, sizeof(double) * ORC_D);
+            memcpy(kp2 + (int64_t)lo * ORC_D, kp + (int64_t)lo * ORC_D, sizeof(uint16_t) * (size_t)size * ORC_D);
+            memcpy(vp2 + (int64_t)lo * ORC_D, vp + (int64_t)lo * ORC_D, sizeof(uint16_t) * (size_t)size * ORC_D);
+            memcpy(ids2 + lo, ids + lo, sizeof(int32_t) * (size_t)size);
+            out += 1;
+            continue;
+        }
+        int32_t init[2], coff[3];
+        double cmu[2 * ORC_D];
+        int32_t* cperm = (int32_t*)malloc(sizeof(int32_t) * (size_t)size);
+        int32_t* casg = (int32_t*)malloc(sizeof(int32_t) * (size_t)size);
+        orc_init_indices(size, 2, orc_split_key(seed, unit, window, c), init);
+        orc_kmeans(kp + (int64_t)lo * ORC_D, size, 2, iters, init, cmu, coff, cperm, casg);
+        offsets2[out] = lo;
+        offsets2[out + 1] = lo + coff[1];
+        memcpy(mu2 + (int64_t)out * ORC_D, cmu, sizeof(double) * 2 * ORC_D);
+        for (int32_t j = 0; j < size; j++) {
+            int64_t src = (int64_t)lo + cperm[j], dst = (int64_t)lo + j;
+            memcpy(kp2 + dst * ORC_D, kp + src * ORC_D, sizeof(uint16_t) * ORC_D);
+            memcpy(vp2 + dst * ORC_D, vp + src * ORC_D, sizeof(uint16_t) * ORC_D);
+            ids2[dst] = ids[src];
+        }
+        free(cperm);
+        free(casg);
+        out += 2;
+        n_split++;
+    }
+    offsets2[out] = C > 0 ? offsets[C] : 0;
+    free(drift);
+    return out;
 }
 
 /* ------------------------------------------------------------- selection ---------- */
