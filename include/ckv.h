@@ -17,7 +17,8 @@
  *     elements, 16-byte aligned base). fp32 and int32 tensors are 16-byte aligned too.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Work is enqueued
  *     asynchronously on it. No call synchronises the host, except ckv_create,
- *     ckv_destroy, ckv_check_device_error, ckv_export_unit and ckv_import_unit.
+ *     ckv_destroy, ckv_check_device_error, ckv_export_unit, ckv_import_unit and
+ *     split_drifted_clusters.
  *   - Return 0 (CKV_OK) on success or a negative CKV_E* code. All arguments are checked on
  *     the host before anything is enqueued. A call that fails its checks leaves the
  *     cluster store unchanged. ckv_last_error() gives a one-line reason (per thread).
@@ -169,6 +170,34 @@ CKV_API int recluster_increment_traced(ckv_ctx* ctx, int32_t layer, float* mu_tr
  * ckv_import_unit of the layer return CKV_ESTATE. */
 CKV_API int recluster_begin(ckv_ctx* ctx, int32_t layer, void* stream);
 CKV_API int recluster_finish(ckv_ctx* ctx, int32_t layer, void* stream);
+
+/* Drift check and split of one layer's clusters ([EXPL] 3.2, decode phase: a cluster whose
+ * mean intra-cluster distance passes a threshold is split). Readings of the page, which
+ * gives no formula: a cluster's drift is the mean over its members of 1 - cos(k_i, mu_c)
+ * (a cosine with a zero vector counts as 0, an empty cluster has drift 0), computed in
+ * fp32. A cluster with drift > threshold and at least two members is split by cosine
+ * K-means with 2 clusters and `iters` iterations on its own rows (rows in store order;
+ * init: the first two entries of the SplitMix64 Fisher-Yates shuffle keyed by
+ * seed ^ (unit << 32) ^ windows ^ ((c + 1) * 0x9E3779B97F4A7C15), windows = the layer's
+ * incremental clusterings so far), at most max_clusters - C clusters per unit, lowest
+ * index first. The halves take indices c' and c' + 1, with c' = c + (splits below c), and
+ * later clusters move up. A split cluster's rows are reordered inside its own segment
+ * (first half, then second half, each in store order), so ids stay ascending in every
+ * cluster. The layer's cluster count becomes C + the largest split count of its units;
+ * units that split fewer clusters get empty clusters (no rows, zero centroid) at the end,
+ * which never add a selected row.
+ *   threshold : split when drift > threshold (+inf: never, -inf: every cluster of 2+ rows);
+ *               NaN is CKV_EINVAL.
+ *   drift     : optional device fp32 [batch * n_kv_heads, C] (C before the call), every
+ *               cluster's drift.
+ *   splits    : optional HOST int32 [batch * n_kv_heads], clusters split per unit.
+ * Synchronises `stream` (the new cluster count is read back), so it cannot be captured in
+ * a CUDA graph. The first call allocates a scratch of about 520 bytes per token of
+ * capacity per unit of one layer (CKV_ENOMEM if that fails). It shares no workspace with
+ * cluster_prefill. CKV_ESTATE before cluster_prefill or while a re-clustering of the layer
+ * is in flight. */
+CKV_API int split_drifted_clusters(ckv_ctx* ctx, int32_t layer, float threshold, float* drift,
+                                   int32_t* splits, void* stream);
 
 typedef struct ckv_layer_info {
     int64_t n_total;   /* tokens per unit: n_sink + m + pending */

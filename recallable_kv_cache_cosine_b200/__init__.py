@@ -62,6 +62,7 @@ SIGNATURES = {
     "recluster_increment_traced": (C.c_int, [P, I32, P, P, P]),
     "recluster_begin": (C.c_int, [P, I32, P]),
     "recluster_finish": (C.c_int, [P, I32, P]),
+    "split_drifted_clusters": (C.c_int, [P, I32, C.c_float, P, P, P]),
     "ckv_get_layer_info": (C.c_int, [P, I32, P]),
     "ckv_export_unit": (C.c_int, [P, I32, I32, I32, P, P]),
     "ckv_import_unit": (C.c_int, [P, I32, I32, I32, I64, I32, I32, P, P]),
@@ -197,6 +198,21 @@ class ClusterKV:
     def recluster_finish(self, layer: int, stream=None):
         """Makes `stream` wait for that re-clustering and switches the layer to its clusters."""
         _check(lib().recluster_finish(self._ctx, layer, _stream(stream)), "recluster_finish")
+
+    def split_drifted_clusters(self, layer: int, threshold: float, drift: torch.Tensor | None = None,
+                               stream=None) -> list[int]:
+        """Splits the layer's clusters whose drift (mean cosine distance of the members to
+        the centroid) is above `threshold`. drift: optional CUDA float32 [units, C] that
+        receives every cluster's drift. Returns the clusters split per unit. Synchronises
+        the stream."""
+        if drift is not None and (drift.dtype != torch.float32 or not drift.is_cuda):
+            raise TypeError("drift must be a CUDA float32 tensor")
+        U = self.cfg.batch * self.cfg.n_kv_heads
+        splits = (C.c_int32 * U)()
+        _check(lib().split_drifted_clusters(self._ctx, layer, float(threshold), _ptr(drift),
+                                            C.cast(splits, C.c_void_p), _stream(stream)),
+               "split_drifted_clusters")
+        return list(splits)
 
     # -- inspection
     def layer_info(self, layer: int) -> LayerInfo:

@@ -134,7 +134,9 @@ int dev_alloc(T** p, size_t count, Ctx* c) {
 
 void free_all(Ctx* c) {
     void* ptrs[] = {c->kp, c->vp, c->spk, c->spv, c->ids, c->offsets, c->mu, c->ws.mu_hat,
-                    c->ws.assign, c->ws.best, c->ws.perm, c->ws.chunk, c->ws.part, c->err};
+                    c->ws.assign, c->ws.best, c->ws.perm, c->ws.chunk, c->ws.part, c->err,
+                    c->split.drift, c->split.plan, c->split.count, c->split.cmu, c->split.n0,
+                    c->split.lab, c->split.rk, c->split.rv, c->split.rid};
     for (void* p : ptrs)
         if (p) cudaFree(p);
 }
@@ -191,6 +193,23 @@ void commit_window(Ctx* c, LayerState& L) {
     L.pstart = (L.pstart + c->cfg.window) % c->ring;
     L.windows += 1;
 }
+// Allocates the split scratch on first use (each buffer once; a failed call can be retried).
+int ensure_split_scratch(Ctx* c) {
+    SplitScratch& sp = c->split;
+    const size_t U = (size_t)c->units, cmax = (size_t)c->cfg.max_clusters, cap = (size_t)c->cap_c;
+    int rc = CKV_OK;
+    if (!sp.drift) rc = dev_alloc(&sp.drift, U * cmax, c);
+    if (!rc && !sp.plan) rc = dev_alloc(&sp.plan, U * cmax, c);
+    if (!rc && !sp.count) rc = dev_alloc(&sp.count, U, c);
+    if (!rc && !sp.cmu) rc = dev_alloc(&sp.cmu, U * cmax * 2 * kD, c);
+    if (!rc && !sp.n0) rc = dev_alloc(&sp.n0, U * cmax, c);
+    if (!rc && !sp.lab) rc = dev_alloc(&sp.lab, U * cap, c);
+    if (!rc && !sp.rk) rc = dev_alloc(&sp.rk, U * cap * kD, c);
+    if (!rc && !sp.rv) rc = dev_alloc(&sp.rv, U * cap * kD, c);
+    if (!rc && !sp.rid) rc = dev_alloc(&sp.rid, U * cap, c);
+    return rc;
+}
+
 int decode_call(ckv_ctx* ctx, int32_t layer, const void* q, int32_t budget, float* out,
                 int32_t* sel_idx, int32_t* sel_count, void* stream, bool per_head) {
     int rc = check_ctx(ctx);
@@ -512,6 +531,66 @@ int recluster_finish(ckv_ctx* ctx, int32_t layer, void* stream) {
     if (e != cudaSuccess) return cuda_fail(e, "recluster_finish: wait");
     L.in_flight = 0;
     commit_window(c, L);
+    return CKV_OK;
+}
+
+int split_drifted_clusters(ckv_ctx* ctx, int32_t layer, float threshold, float* drift,
+                           int32_t* splits, void* stream) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    Ctx* c = C_(ctx);
+    if ((rc = check_layer(c, layer))) return rc;
+    LayerState& L = c->layers[(size_t)layer];
+    if (!L.prefilled || L.in_flight) {
+        set_error(L.in_flight ? "a re-clustering of this layer is in flight; call recluster_finish"
+                              : "split before cluster_prefill for this layer");
+        return CKV_ESTATE;
+    }
+    if (threshold != threshold) return einval("threshold is NaN");
+    if (drift && ((uintptr_t)drift & 3u)) return einval("drift must be 4-byte aligned");
+    if (c->units > 65535) return einval("more than 65535 units per layer");
+    if ((rc = ensure_split_scratch(c))) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    SplitArgs a{};
+    a.U = c->units;
+    a.C = L.C;
+    a.Cmax = c->cfg.max_clusters;
+    a.room = c->cfg.max_clusters - L.C;
+    a.iters = c->cfg.iters;
+    a.m = L.m;
+    a.tau = threshold;
+    a.seed = c->cfg.seed;
+    a.unit_base = (int64_t)layer * c->units;
+    a.window_no = (uint64_t)L.windows;
+    a.kp = c->kp + c->rows_kp(layer, 0) * kD;
+    a.vp = c->vp + c->rows_kp(layer, 0) * kD;
+    a.ids = c->ids + c->rows_kp(layer, 0);
+    a.kp_ustride = c->cap_c;
+    a.offsets = c->offsets + c->off_base(layer, 0);
+    a.off_ustride = c->cfg.max_clusters + 1;
+    a.mu = c->mu + c->mu_rows(layer, 0) * kD;
+    a.mu_ustride = c->cfg.max_clusters;
+    a.drift = c->split.drift;
+    a.drift_out = drift;
+    a.plan = c->split.plan;
+    a.count = c->split.count;
+    a.cmu = c->split.cmu;
+    a.n0 = c->split.n0;
+    a.lab = c->split.lab;
+    a.rk = c->split.rk;
+    a.rv = c->split.rv;
+    a.rid = c->split.rid;
+    a.err = c->err;
+    if ((rc = launch_split(a, s))) return rc;
+    std::vector<int32_t> cnt((size_t)c->units);
+    cudaError_t e = cudaMemcpyAsync(cnt.data(), c->split.count, sizeof(int32_t) * cnt.size(),
+                                    cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "split: read split counts");
+    int32_t mx = 0;
+    for (int32_t v : cnt) mx = std::max(mx, v);
+    L.C += mx;
+    if (splits) std::copy(cnt.begin(), cnt.end(), splits);
     return CKV_OK;
 }
 

@@ -48,6 +48,19 @@ struct Workspace {
     int32_t cmax = 0;
 };
 
+// Scratch of split_drifted_clusters, allocated by its first call.
+struct SplitScratch {
+    float* drift = nullptr;   // [U][Cmax] drift of every cluster
+    int32_t* plan = nullptr;  // [U][Cmax] 2 * new index + split flag
+    int32_t* count = nullptr; // [U] splits per unit
+    float* cmu = nullptr;     // [U][Cmax][2][128] centroids of the two halves
+    int32_t* n0 = nullptr;    // [U][Cmax] rows of the first half
+    int32_t* lab = nullptr;   // [U][cap_c] half of every row (segments above the staging size)
+    uint16_t* rk = nullptr;   // [U][cap_c][128] row scratch of the stable partition
+    uint16_t* rv = nullptr;
+    int32_t* rid = nullptr;   // [U][cap_c]
+};
+
 struct Ctx {
     ckv_config cfg{};
     int32_t units = 0;   // batch * n_kv_heads
@@ -66,6 +79,7 @@ struct Ctx {
     int32_t* offsets = nullptr;
     float* mu = nullptr;
     Workspace ws;
+    SplitScratch split;
     uint32_t* err = nullptr;  // device error word
     std::vector<LayerState> layers;
     int64_t bytes = 0;
@@ -211,5 +225,36 @@ struct ReclusterArgs {
     int32_t* assign_trace;
 };
 int launch_recluster(const ReclusterArgs& a, cudaStream_t s);
+
+struct SplitArgs {
+    int32_t U, C, Cmax, room, iters;
+    int64_t m;
+    float tau;  // split when drift > tau
+    uint64_t seed;
+    int64_t unit_base;
+    uint64_t window_no;
+    uint16_t* kp;
+    uint16_t* vp;
+    int32_t* ids;
+    int64_t kp_ustride;   // rows (also of lab, rk, rv, rid)
+    int32_t* offsets;
+    int64_t off_ustride;  // ints
+    float* mu;
+    int64_t mu_ustride;   // rows of 128
+    float* drift;         // [U][Cmax]
+    float* drift_out;     // optional [U][C]
+    int32_t* plan;
+    int32_t* count;
+    float* cmu;
+    int32_t* n0;
+    int32_t* lab;
+    uint16_t* rk;
+    uint16_t* rv;
+    int32_t* rid;
+    uint32_t* err;
+};
+// Drift, plan, 2-means split and renumbering of one layer (four launches on `s`). The new
+// cluster count is C + max over units of count[u].
+int launch_split(const SplitArgs& a, cudaStream_t s);
 
 }  // namespace ckv

@@ -1,0 +1,310 @@
+// Drift check and split of drifted clusters for ClusterKV decode (sm_100a).
+//
+// Page: "大模型KV Cache压缩技术：ClusterKV的语义空间优化" (ClusterKV explainer), section 3.2,
+// decode phase: centroid drift is detected, and a cluster whose mean intra-cluster distance
+// is above a threshold is split. The page fixes neither the distance, nor the threshold, nor
+// the split. Readings:
+//   - drift_c = mean over the members of c of (1 - cos(k_i, mu_c)), the clustering's cosine
+//     distance to the stored centroid (a cosine with a zero vector counts as 0, an empty
+//     cluster has drift 0);
+//   - the threshold is a parameter;
+//   - a cluster with drift above the threshold and at least two members is split by cosine
+//     K-means with 2 clusters on its own rows (the prefill's init rule and iteration count),
+//     at most `room` clusters per unit, lowest index first.
+// The two halves take indices c' and c' + 1 (c' = c + splits below c); later clusters shift
+// up. Rows move only inside the cluster's own segment (first half, then second half, each in
+// its previous order), so the token ids stay ascending inside every cluster.
+//
+// Four launches, one pass each:
+//   drift    one warp per (unit, cluster): the mean cosine distance, fp32;
+//   plan     one CTA per unit: flags, the cap, the new index of every cluster (a block scan);
+//   kmeans   one CTA per (cluster, unit), idle unless the cluster splits: 2-means on the
+//            segment (staged in shared memory up to 384 rows, else read from global memory),
+//            then the stable partition of its K/V rows and ids through a row scratch;
+//   renumber one CTA per unit: centroids and offsets move to their new indices, highest
+//            first, so the move can run in place; units with fewer splits than the layer's
+//            maximum get empty clusters (no rows, zero centroid) so that every unit of the
+//            layer has the same cluster count. An empty cluster never adds a selected row.
+#include "ckv_common.cuh"
+#include "ckv_internal.h"
+
+namespace ckv {
+namespace {
+
+constexpr int kDriftWarps = 8;
+constexpr int kPlanThreads = 256;
+constexpr int kSplitThreads = 256;
+constexpr int kStageRows = 384;  // segments up to this size are staged in shared memory
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;  // the xor butterfly leaves the same value in every lane
+}
+
+__device__ __forceinline__ bool segment_ok(int32_t lo, int32_t hi, int64_t m) {
+    return lo >= 0 && hi >= lo && (int64_t)hi <= m;
+}
+
+__global__ void __launch_bounds__(kDriftWarps * 32) drift_kernel(const SplitArgs a) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int u = blockIdx.y, c = blockIdx.x * kDriftWarps + warp;
+    if (c >= a.C) return;
+    const int32_t* off = a.offsets + (int64_t)u * a.off_ustride;
+    int32_t lo = off[c], hi = off[c + 1];
+    if (!segment_ok(lo, hi, a.m)) {
+        if (lane == 0) atomicOr(a.err, kErrBadState);
+        lo = hi = 0;
+    }
+    const float4 mu = reinterpret_cast<const float4*>(a.mu + ((int64_t)u * a.mu_ustride + c) * kD)[lane];
+    const float mm = warp_sum(mu.x * mu.x + mu.y * mu.y + mu.z * mu.z + mu.w * mu.w);
+    const float nm = __fsqrt_rn(mm);
+    const uint16_t* base = a.kp + (int64_t)u * a.kp_ustride * kD + lane * 4;
+    float acc = 0.f;
+    for (int32_t j = lo; j < hi; j += 4) {
+        uint2 w[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+            if (j + r < hi) w[r] = *reinterpret_cast<const uint2*>(base + (int64_t)(j + r) * kD);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            if (j + r >= hi) break;  // warp-uniform
+            const float k0 = bf16_lo(w[r].x), k1 = bf16_hi(w[r].x), k2 = bf16_lo(w[r].y),
+                        k3 = bf16_hi(w[r].y);
+            const float dot = warp_sum(k0 * mu.x + k1 * mu.y + k2 * mu.z + k3 * mu.w);
+            const float kk = warp_sum(k0 * k0 + k1 * k1 + k2 * k2 + k3 * k3);
+            const float cs = (kk > 0.f && mm > 0.f) ? __fdiv_rn(dot, __fmul_rn(__fsqrt_rn(kk), nm)) : 0.f;
+            acc += 1.f - cs;
+        }
+    }
+    const float drift = hi > lo ? __fdiv_rn(acc, (float)(hi - lo)) : 0.f;
+    if (lane == 0) {
+        a.drift[(int64_t)u * a.Cmax + c] = drift;
+        if (a.drift_out) a.drift_out[(int64_t)u * a.C + c] = drift;
+    }
+}
+
+// plan[u][c] = 2 * (new index of c) + (1 if c splits). count[u] = splits of unit u.
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const SplitArgs a) {
+    pdl_launch_dependents();
+    pdl_wait();
+    __shared__ int wsum[kPlanThreads / 32];
+    __shared__ int carry;
+    const int u = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int32_t* off = a.offsets + (int64_t)u * a.off_ustride;
+    if (tid == 0) carry = 0;
+    __syncthreads();
+    for (int base = 0; base < a.C; base += kPlanThreads) {
+        const int c = base + tid;
+        bool f = false;
+        if (c < a.C) {
+            const int32_t lo = off[c], hi = off[c + 1];
+            f = segment_ok(lo, hi, a.m) && hi - lo >= 2 && a.drift[(int64_t)u * a.Cmax + c] > a.tau;
+        }
+        const uint32_t bal = __ballot_sync(0xffffffffu, f);
+        if (lane == 0) wsum[warp] = __popc(bal);
+        __syncthreads();
+        int before = carry + __popc(bal & ((1u << lane) - 1u)), total = 0;
+        for (int w = 0; w < kPlanThreads / 32; ++w) {
+            if (w < warp) before += wsum[w];
+            total += wsum[w];
+        }
+        if (c < a.C) {
+            const bool kept = f && before < a.room;
+            const int ni = c + min(before, a.room);
+            a.plan[(int64_t)u * a.Cmax + c] = 2 * ni + (kept ? 1 : 0);
+        }
+        __syncthreads();
+        if (tid == 0) carry += total;
+        __syncthreads();
+    }
+    if (tid == 0) a.count[u] = min(carry, a.room);
+}
+
+__global__ void __launch_bounds__(kSplitThreads) split_kmeans_kernel(const SplitArgs a) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int c = blockIdx.x, u = blockIdx.y;
+    if (!(a.plan[(int64_t)u * a.Cmax + c] & 1)) return;  // whole CTA: this cluster stays
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    uint16_t* skey = (uint16_t*)smem_raw;                     // [kStageRows][128] bf16
+    int32_t* slab = (int32_t*)(skey + (size_t)kStageRows * kD);  // [kStageRows]
+    float* smu = (float*)(slab + kStageRows);                 // [2][128]
+    float* smh = smu + 2 * kD;                                // [2][128] bf16 values as fp32
+    int32_t* sidx = (int32_t*)(smh + 2 * kD);                 // [2] init rows
+    int32_t* scnt = sidx + 2;                                 // [1] rows in the second half
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int32_t* off = a.offsets + (int64_t)u * a.off_ustride;
+    const int32_t lo = off[c], hi = off[c + 1], s = hi - lo;
+    if (!segment_ok(lo, hi, a.m) || s < 2) {  // the plan only marks segments of 2+ rows
+        if (tid == 0) atomicOr(a.err, kErrBadState);
+        return;
+    }
+    const int64_t row0 = (int64_t)u * a.kp_ustride + lo;  // first row of the segment
+    const uint16_t* gk = a.kp + row0 * kD;
+    const bool staged = s <= kStageRows;
+    if (staged)
+        for (int t = tid; t < s * (kD / 8); t += kSplitThreads)
+            reinterpret_cast<uint4*>(skey)[t] = reinterpret_cast<const uint4*>(gk)[t];
+    const uint16_t* rows = staged ? skey : gk;
+    int32_t* lab = staged ? slab : a.lab + row0;
+    if (tid == 0) {
+        // first two entries of a Fisher-Yates shuffle of 0..s-1 (SplitMix64 draws mapped by
+        // Lemire's multiply-shift): the first draw j0 is taken as is; the second j1 >= 1 lands
+        // on j1 itself unless the first swap moved entry 0 there.
+        uint64_t state = a.seed ^ ((uint64_t)(a.unit_base + u) << 32) ^ a.window_no;
+        state ^= (uint64_t)(c + 1) * 0x9E3779B97F4A7C15ull;
+        const int j0 = (int)bounded_draw(splitmix64_next(state), (uint32_t)s);
+        const int j1 = 1 + (int)bounded_draw(splitmix64_next(state), (uint32_t)(s - 1));
+        sidx[0] = j0;
+        sidx[1] = j1 == j0 ? 0 : j1;
+    }
+    __syncthreads();
+    {
+        const int ch = tid >> 7, d = tid & (kD - 1);
+        smu[ch * kD + d] = __uint_as_float((uint32_t)rows[(int64_t)sidx[ch] * kD + d] << 16);
+    }
+    __syncthreads();
+    for (int it = 0; it < a.iters; ++it) {
+        if (warp < 2) {  // normalise: mu_hat = bf16_rn(mu / |mu|), zero for a zero centroid
+            const float4 v = reinterpret_cast<const float4*>(smu + warp * kD)[lane];
+            const float nrm = __fsqrt_rn(warp_sum(v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w));
+            float4 h4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (nrm > 0.f) {
+                h4.x = __bfloat162float(__float2bfloat16_rn(__fdiv_rn(v.x, nrm)));
+                h4.y = __bfloat162float(__float2bfloat16_rn(__fdiv_rn(v.y, nrm)));
+                h4.z = __bfloat162float(__float2bfloat16_rn(__fdiv_rn(v.z, nrm)));
+                h4.w = __bfloat162float(__float2bfloat16_rn(__fdiv_rn(v.w, nrm)));
+            }
+            reinterpret_cast<float4*>(smh + warp * kD)[lane] = h4;
+        }
+        if (tid == 0) scnt[0] = 0;
+        __syncthreads();
+        // assign, one warp per row: the second half wins only on a strictly larger dot
+        const float4 h0 = reinterpret_cast<const float4*>(smh)[lane];
+        const float4 h1 = reinterpret_cast<const float4*>(smh + kD)[lane];
+        for (int i = warp; i < s; i += kSplitThreads / 32) {
+            const uint2 w = *reinterpret_cast<const uint2*>(rows + (int64_t)i * kD + lane * 4);
+            const float k0 = bf16_lo(w.x), k1 = bf16_hi(w.x), k2 = bf16_lo(w.y), k3 = bf16_hi(w.y);
+            const float d0 = warp_sum(fmaf(k3, h0.w, fmaf(k2, h0.z, fmaf(k1, h0.y, k0 * h0.x))));
+            const float d1 = warp_sum(fmaf(k3, h1.w, fmaf(k2, h1.z, fmaf(k1, h1.y, k0 * h1.x))));
+            if (lane == 0) {
+                const int l = d1 > d0 ? 1 : 0;
+                lab[i] = l;
+                if (l) atomicAdd(scnt, 1);
+            }
+        }
+        __syncthreads();
+        {  // update: thread (half, d) sums dimension d over the half's rows in segment order
+            const int ch = tid >> 7, d = tid & (kD - 1);
+            float acc = 0.f;
+            int cnt = 0;
+            for (int j = 0; j < s; ++j)
+                if (lab[j] == ch) {
+                    acc += __uint_as_float((uint32_t)rows[(int64_t)j * kD + d] << 16);
+                    ++cnt;
+                }
+            if (cnt > 0) smu[ch * kD + d] = __fdiv_rn(acc, (float)cnt);  // an empty half keeps mu
+        }
+        __syncthreads();
+    }
+    const int n0 = s - scnt[0];
+    // destination of every row: a stable partition (first half, then second half)
+    if (warp == 0) {
+        int c0 = 0, c1 = 0;
+        const uint32_t lt = (1u << lane) - 1u;
+        for (int b = 0; b < s; b += 32) {
+            const int i = b + lane;
+            const int l = i < s ? lab[i] : 2;
+            const uint32_t m0 = __ballot_sync(0xffffffffu, l == 0);
+            const uint32_t m1 = __ballot_sync(0xffffffffu, l == 1);
+            if (i < s) lab[i] = l == 0 ? c0 + __popc(m0 & lt) : n0 + c1 + __popc(m1 & lt);
+            c0 += __popc(m0);
+            c1 += __popc(m1);
+        }
+    }
+    // the segment's rows and ids into the row scratch (same rows), then back permuted
+    uint16_t* rk = a.rk + row0 * kD;
+    uint16_t* rv = a.rv + row0 * kD;
+    int32_t* rid = a.rid + row0;
+    uint16_t* kp = a.kp + row0 * kD;
+    uint16_t* vp = a.vp + row0 * kD;
+    int32_t* ids = a.ids + row0;
+    for (int t = tid; t < s * (kD / 8); t += kSplitThreads) {
+        reinterpret_cast<uint4*>(rk)[t] = reinterpret_cast<const uint4*>(kp)[t];
+        reinterpret_cast<uint4*>(rv)[t] = reinterpret_cast<const uint4*>(vp)[t];
+    }
+    for (int i = tid; i < s; i += kSplitThreads) rid[i] = ids[i];
+    __syncthreads();
+    for (int t = tid; t < s * (kD / 8); t += kSplitThreads) {
+        const int i = t / (kD / 8), w = t % (kD / 8);
+        const int64_t dst = (int64_t)lab[i] * (kD / 8) + w;
+        reinterpret_cast<uint4*>(kp)[dst] = reinterpret_cast<const uint4*>(rk)[t];
+        reinterpret_cast<uint4*>(vp)[dst] = reinterpret_cast<const uint4*>(rv)[t];
+    }
+    for (int i = tid; i < s; i += kSplitThreads) ids[lab[i]] = rid[i];
+    float* cmu = a.cmu + ((int64_t)u * a.Cmax + c) * 2 * kD;
+    cmu[tid] = smu[tid];  // 256 threads = 2 halves x 128
+    if (tid == 0) a.n0[(int64_t)u * a.Cmax + c] = n0;
+}
+
+// Thread d moves column d of every centroid (thread 0 also moves the offsets), from the
+// highest cluster down: a cluster's new index is never below its old one, so every entry is
+// read before any write can reach it.
+__global__ void __launch_bounds__(kD) renumber_kernel(const SplitArgs a) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int u = blockIdx.x, d = threadIdx.x;
+    int mx = 0;
+    for (int i = 0; i < a.U; ++i) mx = max(mx, a.count[i]);
+    const int Cu = a.C + a.count[u], Cn = a.C + mx;
+    int32_t* off = a.offsets + (int64_t)u * a.off_ustride;
+    float* mu = a.mu + (int64_t)u * a.mu_ustride * kD;
+    for (int c2 = Cu; c2 < Cn; ++c2) mu[(int64_t)c2 * kD + d] = 0.f;
+    if (d == 0)
+        for (int k = Cu; k <= Cn; ++k) off[k] = (int32_t)a.m;
+    for (int c = a.C - 1; c >= 0; --c) {
+        const int p = a.plan[(int64_t)u * a.Cmax + c];
+        const int ni = p >> 1;
+        if (p & 1) {
+            const float* cm = a.cmu + ((int64_t)u * a.Cmax + c) * 2 * kD;
+            mu[(int64_t)ni * kD + d] = cm[d];
+            mu[(int64_t)(ni + 1) * kD + d] = cm[kD + d];
+            if (d == 0) {
+                const int32_t lo = off[c];
+                off[ni] = lo;
+                off[ni + 1] = lo + a.n0[(int64_t)u * a.Cmax + c];
+            }
+        } else {
+            const float v = mu[(int64_t)c * kD + d];
+            mu[(int64_t)ni * kD + d] = v;
+            if (d == 0) off[ni] = off[c];
+        }
+    }
+}
+
+}  // namespace
+
+int launch_split(const SplitArgs& a, cudaStream_t s) {
+    if (a.C < 1 || a.U < 1 || a.iters < 1 || a.room < 0) {
+        set_error("split: bad sizes");
+        return CKV_EINVAL;
+    }
+    cudaError_t e = launch_pdl(drift_kernel, dim3((a.C + kDriftWarps - 1) / kDriftWarps, a.U),
+                               dim3(kDriftWarps * 32), 0, s, a);
+    if (e != cudaSuccess) return cuda_fail(e, "split: drift launch");
+    e = launch_pdl(plan_kernel, dim3(a.U), dim3(kPlanThreads), 0, s, a);
+    if (e != cudaSuccess) return cuda_fail(e, "split: plan launch");
+    const size_t smem = (size_t)kStageRows * kD * 2 + (size_t)kStageRows * 4 + 4 * kD * 4 + 16;
+    const int rc = ensure_smem((const void*)split_kmeans_kernel, smem, "split: set smem");
+    if (rc != CKV_OK) return rc;
+    e = launch_pdl(split_kmeans_kernel, dim3(a.C, a.U), dim3(kSplitThreads), smem, s, a);
+    if (e != cudaSuccess) return cuda_fail(e, "split: kmeans launch");
+    e = launch_pdl(renumber_kernel, dim3(a.U), dim3(kD), 0, s, a);
+    return e == cudaSuccess ? CKV_OK : cuda_fail(e, "split: renumber launch");
+}
+
+}  // namespace ckv
