@@ -136,7 +136,8 @@ void free_all(Ctx* c) {
     void* ptrs[] = {c->kp, c->vp, c->spk, c->spv, c->ids, c->offsets, c->mu, c->ws.mu_hat,
                     c->ws.assign, c->ws.best, c->ws.perm, c->ws.chunk, c->ws.part, c->err,
                     c->split.drift, c->split.plan, c->split.count, c->split.cmu, c->split.n0,
-                    c->split.lab, c->split.rk, c->split.rv, c->split.rid};
+                    c->split.mu2, c->split.off2, c->split.lab, c->split.rk, c->split.rv,
+                    c->split.rid};
     for (void* p : ptrs)
         if (p) cudaFree(p);
 }
@@ -203,6 +204,8 @@ int ensure_split_scratch(Ctx* c) {
     if (!rc && !sp.count) rc = dev_alloc(&sp.count, U, c);
     if (!rc && !sp.cmu) rc = dev_alloc(&sp.cmu, U * cmax * 2 * kD, c);
     if (!rc && !sp.n0) rc = dev_alloc(&sp.n0, U * cmax, c);
+    if (!rc && !sp.mu2) rc = dev_alloc(&sp.mu2, U * cmax * kD, c);
+    if (!rc && !sp.off2) rc = dev_alloc(&sp.off2, U * (cmax + 1), c);
     if (!rc && !sp.lab) rc = dev_alloc(&sp.lab, U * cap, c);
     if (!rc && !sp.rk) rc = dev_alloc(&sp.rk, U * cap * kD, c);
     if (!rc && !sp.rv) rc = dev_alloc(&sp.rv, U * cap * kD, c);
@@ -576,6 +579,8 @@ int split_drifted_clusters(ckv_ctx* ctx, int32_t layer, float threshold, float* 
     a.count = c->split.count;
     a.cmu = c->split.cmu;
     a.n0 = c->split.n0;
+    a.mu2 = c->split.mu2;
+    a.off2 = c->split.off2;
     a.lab = c->split.lab;
     a.rk = c->split.rk;
     a.rv = c->split.rv;

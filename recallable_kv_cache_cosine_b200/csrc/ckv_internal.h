@@ -55,6 +55,8 @@ struct SplitScratch {
     int32_t* count = nullptr; // [U] splits per unit
     float* cmu = nullptr;     // [U][Cmax][2][128] centroids of the two halves
     int32_t* n0 = nullptr;    // [U][Cmax] rows of the first half
+    float* mu2 = nullptr;     // [U][Cmax][128] centroids at their new indices
+    int32_t* off2 = nullptr;  // [U][Cmax + 1] offsets at their new indices
     int32_t* lab = nullptr;   // [U][cap_c] half of every row (segments above the staging size)
     uint16_t* rk = nullptr;   // [U][cap_c][128] row scratch of the stable partition
     uint16_t* rv = nullptr;
@@ -247,13 +249,15 @@ struct SplitArgs {
     int32_t* count;
     float* cmu;
     int32_t* n0;
+    float* mu2;
+    int32_t* off2;
     int32_t* lab;
     uint16_t* rk;
     uint16_t* rv;
     int32_t* rid;
     uint32_t* err;
 };
-// Drift, plan, 2-means split and renumbering of one layer (four launches on `s`). The new
+// Drift, plan, 2-means split and renumbering of one layer (five launches on `s`). The new
 // cluster count is C + max over units of count[u].
 int launch_split(const SplitArgs& a, cudaStream_t s);
 

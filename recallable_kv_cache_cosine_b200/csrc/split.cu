@@ -15,16 +15,18 @@
 // up. Rows move only inside the cluster's own segment (first half, then second half, each in
 // its previous order), so the token ids stay ascending inside every cluster.
 //
-// Four launches, one pass each:
+// Five launches, one pass each:
 //   drift    one warp per (unit, cluster): the mean cosine distance, fp32;
 //   plan     one CTA per unit: flags, the cap, the new index of every cluster (a block scan);
 //   kmeans   one CTA per (cluster, unit), idle unless the cluster splits: 2-means on the
-//            segment (staged in shared memory up to 384 rows, else read from global memory),
+//            segment (staged in shared memory up to 192 rows, else read from global memory),
 //            then the stable partition of its K/V rows and ids through a row scratch;
-//   renumber one CTA per unit: centroids and offsets move to their new indices, highest
-//            first, so the move can run in place; units with fewer splits than the layer's
+//   scatter  one warp per (cluster, unit): the cluster's centroid(s) and offset(s) go to
+//            their new indices in a scratch copy; units with fewer splits than the layer's
 //            maximum get empty clusters (no rows, zero centroid) so that every unit of the
-//            layer has the same cluster count. An empty cluster never adds a selected row.
+//            layer has the same cluster count. An empty cluster never adds a selected row;
+//   copy     the scratch copy back into the store (a move in place would have to run
+//            serially, highest index first).
 #include "ckv_common.cuh"
 #include "ckv_internal.h"
 
@@ -34,7 +36,7 @@ namespace {
 constexpr int kDriftWarps = 8;
 constexpr int kPlanThreads = 256;
 constexpr int kSplitThreads = 256;
-constexpr int kStageRows = 384;  // segments up to this size are staged in shared memory
+constexpr int kStageRows = 192;  // segments up to this size are staged in shared memory
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -133,7 +135,8 @@ __global__ void __launch_bounds__(kSplitThreads) split_kmeans_kernel(const Split
     int32_t* slab = (int32_t*)(skey + (size_t)kStageRows * kD);  // [kStageRows]
     float* smu = (float*)(slab + kStageRows);                 // [2][128]
     float* smh = smu + 2 * kD;                                // [2][128] bf16 values as fp32
-    int32_t* sidx = (int32_t*)(smh + 2 * kD);                 // [2] init rows
+    float* sred = smh + 2 * kD;                               // [2 parts][2 halves][128]
+    int32_t* sidx = (int32_t*)(sred + 4 * kD);                // [2] init rows
     int32_t* scnt = sidx + 2;                                 // [1] rows in the second half
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -183,31 +186,65 @@ __global__ void __launch_bounds__(kSplitThreads) split_kmeans_kernel(const Split
         }
         if (tid == 0) scnt[0] = 0;
         __syncthreads();
-        // assign, one warp per row: the second half wins only on a strictly larger dot
+        // assign, one warp per row, four rows in flight: the second half wins only on a
+        // strictly larger dot
         const float4 h0 = reinterpret_cast<const float4*>(smh)[lane];
         const float4 h1 = reinterpret_cast<const float4*>(smh + kD)[lane];
-        for (int i = warp; i < s; i += kSplitThreads / 32) {
-            const uint2 w = *reinterpret_cast<const uint2*>(rows + (int64_t)i * kD + lane * 4);
-            const float k0 = bf16_lo(w.x), k1 = bf16_hi(w.x), k2 = bf16_lo(w.y), k3 = bf16_hi(w.y);
-            const float d0 = warp_sum(fmaf(k3, h0.w, fmaf(k2, h0.z, fmaf(k1, h0.y, k0 * h0.x))));
-            const float d1 = warp_sum(fmaf(k3, h1.w, fmaf(k2, h1.z, fmaf(k1, h1.y, k0 * h1.x))));
+        constexpr int kNW = kSplitThreads / 32;
+        for (int i0 = warp; i0 < s; i0 += 4 * kNW) {
+            float p0[4], p1[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int i = i0 + r * kNW;
+                p0[r] = p1[r] = 0.f;
+                if (i < s) {
+                    const uint2 w = *reinterpret_cast<const uint2*>(rows + (int64_t)i * kD + lane * 4);
+                    const float k0 = bf16_lo(w.x), k1 = bf16_hi(w.x), k2 = bf16_lo(w.y),
+                                k3 = bf16_hi(w.y);
+                    p0[r] = fmaf(k3, h0.w, fmaf(k2, h0.z, fmaf(k1, h0.y, k0 * h0.x)));
+                    p1[r] = fmaf(k3, h1.w, fmaf(k2, h1.z, fmaf(k1, h1.y, k0 * h1.x)));
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    p0[r] += __shfl_xor_sync(0xffffffffu, p0[r], o);
+                    p1[r] += __shfl_xor_sync(0xffffffffu, p1[r], o);
+                }
             if (lane == 0) {
-                const int l = d1 > d0 ? 1 : 0;
-                lab[i] = l;
-                if (l) atomicAdd(scnt, 1);
+                int ones = 0;
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int i = i0 + r * kNW;
+                    if (i < s) {
+                        const int l = p1[r] > p0[r] ? 1 : 0;
+                        lab[i] = l;
+                        ones += l;
+                    }
+                }
+                if (ones) atomicAdd(scnt, ones);
             }
         }
         __syncthreads();
-        {  // update: thread (half, d) sums dimension d over the half's rows in segment order
+        {  // update: thread (part, d) sums dimension d of both halves over the rows of its
+           // parity (part 0: even rows, part 1: odd rows) in segment order; part 0 + part 1
+            const int part = tid >> 7, d = tid & (kD - 1);
+            float a0 = 0.f, a1 = 0.f;
+            for (int j = part; j < s; j += 2) {
+                const float v = __uint_as_float((uint32_t)rows[(int64_t)j * kD + d] << 16);
+                if (lab[j]) a1 += v;
+                else a0 += v;
+            }
+            sred[(part * 2 + 0) * kD + d] = a0;
+            sred[(part * 2 + 1) * kD + d] = a1;
+        }
+        __syncthreads();
+        {
             const int ch = tid >> 7, d = tid & (kD - 1);
-            float acc = 0.f;
-            int cnt = 0;
-            for (int j = 0; j < s; ++j)
-                if (lab[j] == ch) {
-                    acc += __uint_as_float((uint32_t)rows[(int64_t)j * kD + d] << 16);
-                    ++cnt;
-                }
-            if (cnt > 0) smu[ch * kD + d] = __fdiv_rn(acc, (float)cnt);  // an empty half keeps mu
+            const int cnt = ch ? scnt[0] : s - scnt[0];
+            if (cnt > 0)  // an empty half keeps mu
+                smu[ch * kD + d] = __fdiv_rn(sred[ch * kD + d] + sred[(2 + ch) * kD + d], (float)cnt);
         }
         __syncthreads();
     }
@@ -251,39 +288,58 @@ __global__ void __launch_bounds__(kSplitThreads) split_kmeans_kernel(const Split
     if (tid == 0) a.n0[(int64_t)u * a.Cmax + c] = n0;
 }
 
-// Thread d moves column d of every centroid (thread 0 also moves the offsets), from the
-// highest cluster down: a cluster's new index is never below its old one, so every entry is
-// read before any write can reach it.
-__global__ void __launch_bounds__(kD) renumber_kernel(const SplitArgs a) {
+// One warp per (cluster, unit): the cluster's centroid(s) and offset(s) into the scratch copy
+// at the new index. The warps past the unit's last cluster write its empty padding clusters
+// and the closing offset.
+__global__ void __launch_bounds__(kDriftWarps * 32) scatter_kernel(const SplitArgs a) {
     pdl_launch_dependents();
     pdl_wait();
-    const int u = blockIdx.x, d = threadIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int u = blockIdx.y, c = blockIdx.x * kDriftWarps + warp;
     int mx = 0;
     for (int i = 0; i < a.U; ++i) mx = max(mx, a.count[i]);
     const int Cu = a.C + a.count[u], Cn = a.C + mx;
-    int32_t* off = a.offsets + (int64_t)u * a.off_ustride;
-    float* mu = a.mu + (int64_t)u * a.mu_ustride * kD;
-    for (int c2 = Cu; c2 < Cn; ++c2) mu[(int64_t)c2 * kD + d] = 0.f;
-    if (d == 0)
-        for (int k = Cu; k <= Cn; ++k) off[k] = (int32_t)a.m;
-    for (int c = a.C - 1; c >= 0; --c) {
+    const int32_t* off = a.offsets + (int64_t)u * a.off_ustride;
+    float4* mu2 = reinterpret_cast<float4*>(a.mu2 + (int64_t)u * a.Cmax * kD);
+    int32_t* off2 = a.off2 + (int64_t)u * (a.Cmax + 1);
+    if (c < a.C) {
         const int p = a.plan[(int64_t)u * a.Cmax + c];
         const int ni = p >> 1;
         if (p & 1) {
-            const float* cm = a.cmu + ((int64_t)u * a.Cmax + c) * 2 * kD;
-            mu[(int64_t)ni * kD + d] = cm[d];
-            mu[(int64_t)(ni + 1) * kD + d] = cm[kD + d];
-            if (d == 0) {
-                const int32_t lo = off[c];
-                off[ni] = lo;
-                off[ni + 1] = lo + a.n0[(int64_t)u * a.Cmax + c];
+            const float4* cm = reinterpret_cast<const float4*>(a.cmu + ((int64_t)u * a.Cmax + c) * 2 * kD);
+            mu2[(int64_t)ni * (kD / 4) + lane] = cm[lane];
+            mu2[(int64_t)(ni + 1) * (kD / 4) + lane] = cm[kD / 4 + lane];
+            if (lane == 0) {
+                off2[ni] = off[c];
+                off2[ni + 1] = off[c] + a.n0[(int64_t)u * a.Cmax + c];
             }
         } else {
-            const float v = mu[(int64_t)c * kD + d];
-            mu[(int64_t)ni * kD + d] = v;
-            if (d == 0) off[ni] = off[c];
+            mu2[(int64_t)ni * (kD / 4) + lane] =
+                reinterpret_cast<const float4*>(a.mu + ((int64_t)u * a.mu_ustride + c) * kD)[lane];
+            if (lane == 0) off2[ni] = off[c];
         }
+    } else {
+        const int c2 = Cu + (c - a.C);  // padding cluster c2, or the closing offset at Cn
+        if (c2 < Cn) mu2[(int64_t)c2 * (kD / 4) + lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c2 <= Cn && lane == 0) off2[c2] = (int32_t)a.m;
     }
+}
+
+// The scratch copy back into the store: clusters [0, Cn) and offsets [0, Cn].
+__global__ void __launch_bounds__(kDriftWarps * 32) copy_back_kernel(const SplitArgs a) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int u = blockIdx.y, c = blockIdx.x * kDriftWarps + warp;
+    int mx = 0;
+    for (int i = 0; i < a.U; ++i) mx = max(mx, a.count[i]);
+    const int Cn = a.C + mx;
+    if (c > Cn) return;
+    if (c < Cn)
+        reinterpret_cast<float4*>(a.mu + ((int64_t)u * a.mu_ustride + c) * kD)[lane] =
+            reinterpret_cast<const float4*>(a.mu2 + ((int64_t)u * a.Cmax + c) * kD)[lane];
+    if (lane == 0)
+        a.offsets[(int64_t)u * a.off_ustride + c] = a.off2[(int64_t)u * (a.Cmax + 1) + c];
 }
 
 }  // namespace
@@ -298,13 +354,17 @@ int launch_split(const SplitArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return cuda_fail(e, "split: drift launch");
     e = launch_pdl(plan_kernel, dim3(a.U), dim3(kPlanThreads), 0, s, a);
     if (e != cudaSuccess) return cuda_fail(e, "split: plan launch");
-    const size_t smem = (size_t)kStageRows * kD * 2 + (size_t)kStageRows * 4 + 4 * kD * 4 + 16;
+    const size_t smem = (size_t)kStageRows * kD * 2 + (size_t)kStageRows * 4 + 8 * kD * 4 + 16;
     const int rc = ensure_smem((const void*)split_kmeans_kernel, smem, "split: set smem");
     if (rc != CKV_OK) return rc;
     e = launch_pdl(split_kmeans_kernel, dim3(a.C, a.U), dim3(kSplitThreads), smem, s, a);
     if (e != cudaSuccess) return cuda_fail(e, "split: kmeans launch");
-    e = launch_pdl(renumber_kernel, dim3(a.U), dim3(kD), 0, s, a);
-    return e == cudaSuccess ? CKV_OK : cuda_fail(e, "split: renumber launch");
+    // grids cover every cluster a unit can end with (Cmax) plus the closing offset
+    const dim3 gw((a.Cmax + 1 + kDriftWarps - 1) / kDriftWarps, a.U);
+    e = launch_pdl(scatter_kernel, gw, dim3(kDriftWarps * 32), 0, s, a);
+    if (e != cudaSuccess) return cuda_fail(e, "split: scatter launch");
+    e = launch_pdl(copy_back_kernel, gw, dim3(kDriftWarps * 32), 0, s, a);
+    return e == cudaSuccess ? CKV_OK : cuda_fail(e, "split: copy launch");
 }
 
 }  // namespace ckv
