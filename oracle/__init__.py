@@ -52,6 +52,11 @@ def lib():
             "orc_split_key": (u64, [u64, i64, u64, i32]),
             "orc_split_drifted": (i32, [P, P, P, P, P, i32, C.c_double, i32, i32, u64, i64,
                                         u64, P, P, P, P, P, P]),
+            "orc_e4m3_from_float": (C.c_uint8, [C.c_float]),
+            "orc_e4m3_from_float_array": (None, [P, i64, P]),
+            "orc_e4m3_to_double": (C.c_double, [C.c_uint8]),
+            "orc_quantize_rows_e4m3": (None, [P, i64, P, P]),
+            "orc_attend_mixed": (None, [P, P, i32, P, P, i32, i32, P, P, P, P, P]),
             "orc_group_query": (None, [P, i32, P]),
             "orc_select": (i32, [P, P, i32, P, P, P, P]),
             "orc_attend": (None, [P, P, i32, P, i32, P]),
@@ -350,6 +355,56 @@ def attend(st: Store, q, sel: Selection) -> np.ndarray:
 def select_and_attend(st: Store, q, budget: int):
     sel = select(st, q, budget)
     return attend(st, q, sel), sel
+
+
+# ------------------------------------------------------------------ far clusters in fp8
+
+def e4m3_from_f32(x) -> np.ndarray:
+    """fp8 e4m3 codes of float32 values (ties to even, saturating at 448)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, np.uint8)
+    lib().orc_e4m3_from_float_array(_p(x), x.size, _p(out))
+    return out
+
+
+def e4m3_to_f64(codes) -> np.ndarray:
+    table = np.array([lib().orc_e4m3_to_double(b) for b in range(256)])
+    return table[np.asarray(codes, dtype=np.uint8)]
+
+
+def quantize_rows_e4m3(rows) -> tuple[np.ndarray, np.ndarray]:
+    """Per-row fp8 copy of bf16 rows [n, 128]: (codes uint8 [n, 128], scales float32 [n])."""
+    rows = _u16(rows)
+    n = rows.shape[0]
+    codes = np.empty((n, D), np.uint8)
+    scales = np.empty(max(n, 1), np.float32)
+    lib().orc_quantize_rows_e4m3(_p(rows), n, _p(codes), _p(scales))
+    return codes, scales[:n].copy()
+
+
+def walk_rank(st: Store, sel: "Selection") -> np.ndarray:
+    """Walk rank (0 = highest score, ties to the lower index) of every cluster."""
+    order = sorted(range(st.C), key=lambda c: (-sel.scores[c], c))
+    rank = np.empty(st.C, np.int32)
+    rank[order] = np.arange(st.C, dtype=np.int32)
+    return rank
+
+
+def attend_mixed(st: Store, q, sel: "Selection", n_near: int, k8, ks, v8, vs) -> np.ndarray:
+    """Attention like ``attend``, reading the selected rows of clusters at walk rank >= n_near
+    from the fp8 copy (explainer section 7, mixed precision for far clusters)."""
+    q = _u16(q)
+    s = st._c()
+    rows = _i32(sel.rows)
+    rank = walk_rank(st, sel)
+    clus = np.searchsorted(st.offsets, np.maximum(rows, 0), side="right") - 1
+    row_rank = _i32(np.where(rows >= 0, rank[np.clip(clus, 0, max(st.C - 1, 0))], -1))
+    k8, v8 = np.ascontiguousarray(k8, np.uint8), np.ascontiguousarray(v8, np.uint8)
+    ks, vs = np.ascontiguousarray(ks, np.float32), np.ascontiguousarray(vs, np.float32)
+    out = np.empty((q.shape[0], D), np.float64)
+    lib().orc_attend_mixed(C.byref(s), _p(q), q.shape[0], _p(rows), _p(row_rank), rows.shape[0],
+                           n_near, _p(k8), _p(ks), _p(v8), _p(vs), _p(out))
+    return out
 
 
 def dense_attention(K, V, q) -> np.ndarray:

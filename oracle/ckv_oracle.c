@@ -11,7 +11,8 @@
  *          section 3.1 (attention formula, centroid mean, cluster-importance relation),
  *          section 3.2 (16 sinks, cosine K-means at prefill, incremental clustering
  *          every 320 tokens, splitting of drifted clusters), section 3.3
- *          (select_clusters listing), section 4.1
+ *          (select_clusters listing), section 7 (lower precision for far clusters),
+ *          section 4.1
  *          (half-precision distance matmul, cluster-contiguous KV layout).
  *   [ABS]  "ClusterKV: Manipulating LLM KV Cache in Semantic Space for Recallable
  *          Compression" (arXiv 2412.03213 listing), abstract.
@@ -534,6 +535,117 @@ void orc_dense_attention(const uint16_t* K, const uint16_t* V, int64_t n, const 
             double p = exp(z[i] - zmax);
             den += p;
             for (int d = 0; d < ORC_D; d++) acc[d] += p * orc_bf16_to_double(V[i * ORC_D + d]);
+        }
+        for (int d = 0; d < ORC_D; d++) out[(int64_t)g * ORC_D + d] = acc[d] / den;
+    }
+    free(z);
+}
+
+/* ------------------------------------------- far clusters in fp8 (e4m3) ---------- */
+/* [EXPL] 7 (outlook) lists mixed precision: a lower-precision KV cache for the clusters far
+ * from the current query. The page gives no format, scale or distance rule. Readings:
+ *   - the low-precision copy is fp8 e4m3 (1 sign, 4 exponent bits with bias 7, 3 mantissa
+ *     bits, no infinities, largest finite 448), one fp32 scale per row:
+ *     scale = max_d |x_d| / 448 and code_d = e4m3(x_d / scale), both steps in fp32, the
+ *     rounding to nearest with ties to even; a zero row has scale 0 and zero codes;
+ *   - "far" is the walk order of the selection: whole clusters taken at rank >= n_near
+ *     (rank 0 = highest score), and the cut cluster when its rank is >= n_near, are read
+ *     from the fp8 copy; sinks, pending rows and the nearer clusters stay bf16. The
+ *     selection itself is unchanged (it scores with the fp32 centroids and bf16 keys). */
+
+/* e4m3 code of x, ties to even. Magnitudes above 448 saturate to 448 (the copy's scale keeps
+ * every input at or below 448, so this rule only guards the format); NaN gives 0x7F. */
+uint8_t orc_e4m3_from_float(float x) {
+    if (isnan(x)) return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0;
+    double ax = fabs((double)x);
+    if (ax == 0.0) return sign;
+    int e;
+    frexp(ax, &e);            /* ax in [2^(e-1), 2^e) */
+    int ex = e - 1;
+    if (ex < -6) ex = -6;     /* subnormals: fixed quantum 2^-9 */
+    double quantum = ldexp(1.0, ex - 3);
+    double r = nearbyint(ax / quantum) * quantum;
+    if (r > 448.0) r = 448.0;
+    if (r == 0.0) return sign;
+    frexp(r, &e);
+    int rex = e - 1;
+    uint8_t code;
+    if (rex < -6) {           /* subnormal: r = mant * 2^-9, mant in 1..7 */
+        code = (uint8_t)(r / ldexp(1.0, -9));
+    } else {                  /* normal: r = (1 + mant/8) * 2^rex */
+        int mant = (int)(r / ldexp(1.0, rex - 3)) - 8;
+        code = (uint8_t)(((rex + 7) << 3) | mant);
+    }
+    return sign | code;
+}
+
+void orc_e4m3_from_float_array(const float* x, int64_t n, uint8_t* out) {
+    for (int64_t i = 0; i < n; i++) out[i] = orc_e4m3_from_float(x[i]);
+}
+
+double orc_e4m3_to_double(uint8_t b) {
+    int sign = b >> 7, ex = (b >> 3) & 15, mant = b & 7;
+    if (ex == 15 && mant == 7) return NAN;
+    double v = ex == 0 ? ldexp((double)mant, -9) : ldexp(1.0 + mant / 8.0, ex - 7);
+    return sign ? -v : v;
+}
+
+/* Per-row fp8 copy of n rows of 128 bf16 values: codes [n, 128], scales [n]. */
+void orc_quantize_rows_e4m3(const uint16_t* rows, int64_t n, uint8_t* codes, float* scales) {
+    for (int64_t i = 0; i < n; i++) {
+        float mx = 0.0f;
+        for (int d = 0; d < ORC_D; d++) {
+            float a = (float)fabs(orc_bf16_to_double(rows[i * ORC_D + d]));
+            if (a > mx) mx = a;
+        }
+        float scale = mx / 448.0f;
+        scales[i] = scale;
+        for (int d = 0; d < ORC_D; d++) {
+            float x = (float)orc_bf16_to_double(rows[i * ORC_D + d]);
+            codes[i * ORC_D + d] = scale > 0.0f ? orc_e4m3_from_float(x / scale) : 0;
+        }
+    }
+}
+
+/* Attention over the selected rows like orc_attend, except that a clustered row whose
+ * cluster has walk rank >= n_near (row_rank[i], -1 for sinks and pending) is read from the
+ * fp8 copy: x = e4m3(code) * scale, in double. k8/v8 [m, 128], ks/vs [m]. */
+void orc_attend_mixed(const orc_store* s, const uint16_t* q, int32_t G, const int32_t* sel_rows,
+                      const int32_t* row_rank, int32_t count, int32_t n_near, const uint8_t* k8,
+                      const float* ks, const uint8_t* v8, const float* vs, double* out) {
+    double* z = (double*)malloc(sizeof(double) * (size_t)(count > 0 ? count : 1));
+    const double scale = 1.0 / sqrt((double)ORC_D);
+    for (int32_t g = 0; g < G; g++) {
+        const uint16_t* qg = q + (int64_t)g * ORC_D;
+        double zmax = -INFINITY;
+        for (int32_t i = 0; i < count; i++) {
+            int32_t r = sel_rows[i];
+            double dot = 0.0;
+            if (r >= 0 && row_rank[i] >= n_near) {
+                for (int d = 0; d < ORC_D; d++)
+                    dot += orc_bf16_to_double(qg[d]) *
+                           (orc_e4m3_to_double(k8[(int64_t)r * ORC_D + d]) * (double)ks[r]);
+            } else {
+                const uint16_t* k = r >= 0 ? s->kp + (int64_t)r * ORC_D : s->sp_k + (int64_t)(-r - 1) * ORC_D;
+                dot = dot_bf16_bf16(qg, k);
+            }
+            z[i] = dot * scale;
+            if (z[i] > zmax) zmax = z[i];
+        }
+        double den = 0.0;
+        double acc[ORC_D] = {0};
+        for (int32_t i = 0; i < count; i++) {
+            int32_t r = sel_rows[i];
+            double p = exp(z[i] - zmax);
+            den += p;
+            if (r >= 0 && row_rank[i] >= n_near) {
+                for (int d = 0; d < ORC_D; d++)
+                    acc[d] += p * (orc_e4m3_to_double(v8[(int64_t)r * ORC_D + d]) * (double)vs[r]);
+            } else {
+                const uint16_t* v = r >= 0 ? s->vp + (int64_t)r * ORC_D : s->sp_v + (int64_t)(-r - 1) * ORC_D;
+                for (int d = 0; d < ORC_D; d++) acc[d] += p * orc_bf16_to_double(v[d]);
+            }
         }
         for (int d = 0; d < ORC_D; d++) out[(int64_t)g * ORC_D + d] = acc[d] / den;
     }
