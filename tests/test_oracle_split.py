@@ -211,3 +211,32 @@ def test_split_children_match_two_cluster_kmeans_on_the_rows(iters):
     np.testing.assert_array_equal(new.offsets[c2:c2 + 3], lo + offs)
     np.testing.assert_array_equal(new.ids[lo:hi], st.ids[lo + perm])
     np.testing.assert_array_equal(new.mu[c2:c2 + 2], mu)
+
+
+def test_split_then_window_keeps_the_store_consistent():
+    seed, unit, n, n_centers = 8, 1, 1200, 10
+    K, V = si.keys_values(seed, unit, n, n_centers)
+    st, _ = oracle.prefill_unit(K, V, 10, oracle.stream_key(seed, unit, 0), iters=5)
+    st, flags = oracle.split_drifted(st, float(np.median(oracle.cluster_drift(st))), seed, unit, room=10)
+    C1 = st.C
+    assert C1 == 10 + int(flags.sum())
+    ka, va = si.appended_tokens(seed, unit, oracle.WINDOW, n_centers)
+    for j in range(oracle.WINDOW):
+        st = oracle.append(st, ka[j], va[j])
+    new, _ = oracle.recluster(st, seed, unit)
+    assert new.C == C1 + 4 and new.windows == 1
+    np.testing.assert_array_equal(new.offsets[:C1 + 1], st.offsets)
+    np.testing.assert_array_equal(np.sort(np.concatenate([np.arange(16), new.ids])), np.arange(new.n_total))
+    for c in range(new.C):  # ids ascend inside every cluster, the decode's tie rule
+        seg = new.ids[new.offsets[c]:new.offsets[c + 1]]
+        assert np.all(np.diff(seg) > 0)
+    q = si.queries(seed, 0, 0, 1, 4)[0]
+    for budget in (100, 600, new.n_total):
+        assert len(oracle.select(new, q, budget).ids) == min(budget, new.n_total)
+    # a second split pass draws its inits from the new window number
+    again, flags2 = oracle.split_drifted(new, -1.0, seed, unit, room=2)
+    c = int(np.flatnonzero(flags2)[0])
+    lo, hi = new.offsets[c], new.offsets[c + 1]
+    init = oracle.init_indices(hi - lo, 2, oracle.split_key(seed, unit, 1, c))
+    mu, offs, perm, _ = oracle.kmeans(new.kp[lo:hi], 2, oracle.ITERS, init)
+    np.testing.assert_array_equal(again.ids[lo:hi], new.ids[lo + perm])
