@@ -115,10 +115,14 @@ def test_mixed_attention_reads_only_far_clusters_from_the_copy():
     k8b[near_rows] = 0x7E
     v8b[near_rows] = 0x7E
     np.testing.assert_array_equal(oracle.attend_mixed(st, q, sel, n_near, k8b, ks, v8b, vs), mixed)
-    # a far selected cluster's copy is read
+    # the first far cluster (rank == n_near) is selected, and both its K and its V copy are read
     far = [c for c in range(st.C) if rank[c] == n_near][0]
-    v8c = v8.copy()
-    v8c[st.offsets[far]:st.offsets[far + 1]] = 0
+    lo, hi = st.offsets[far], st.offsets[far + 1]
+    assert np.isin(st.ids[lo:hi], sel.ids).any()
+    k8c, v8c = k8.copy(), v8.copy()
+    k8c[lo:hi] = 0
+    v8c[lo:hi] = 0
+    assert np.abs(oracle.attend_mixed(st, q, sel, n_near, k8c, ks, v8, vs) - mixed).max() > 1e-6
     assert np.abs(oracle.attend_mixed(st, q, sel, n_near, k8, ks, v8c, vs) - mixed).max() > 1e-6
 
 

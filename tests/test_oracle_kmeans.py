@@ -123,3 +123,30 @@ def test_prefill_unit_store_invariants_tiny_config():
     # the run starts from the seeded init: C distinct non-sink tokens
     init = oracle.init_indices(n - 16, C, oracle.stream_key(0, 0, 0))
     assert len(set(init.tolist())) == C
+
+
+def test_assign_gap_closed_forms_and_brute_force():
+    """The cosine gap that the GPU parity tests use to accept near-tie disagreements:
+    (k . mu_hat_best - k . mu_hat_other) / |k|, zero for the argmax itself, positive for
+    a worse cluster, infinite for an index outside [0, C)."""
+    e = np.zeros((3, 128), np.float32)
+    e[0, 0], e[1, 1], e[2, 0] = 1.0, 1.0, 2.0
+    mu_hat = si.to_bf16_bits(e[:2])                 # unit vectors along dims 0 and 1
+    keys = si.to_bf16_bits(np.stack([e[0], 3.0 * e[1], e[2]]))
+    gap = oracle.assign_gap(keys, mu_hat, np.array([1, 0, 1], np.int32))
+    np.testing.assert_allclose(gap, [1.0, 1.0, 1.0], rtol=0, atol=1e-15)
+    gap0 = oracle.assign_gap(keys, mu_hat, oracle.assign(keys, mu_hat))
+    np.testing.assert_array_equal(gap0, [0.0, 0.0, 0.0])
+    assert np.isinf(oracle.assign_gap(keys[:1], mu_hat, np.array([5], np.int32))[0])
+    # brute force on a random case, every (key, other cluster) pair
+    K, _ = si.keys_values(6, 0, 300, 7)
+    mu = oracle.bf16_to_f64(K[:9])
+    mh = oracle.normalize(mu)
+    k = oracle.bf16_to_f64(K)
+    s = k @ oracle.bf16_to_f64(mh).T
+    for c in range(9):
+        other = np.full(300, c, np.int32)
+        want = (s.max(axis=1) - s[:, c]) / np.linalg.norm(k, axis=1)
+        got = oracle.assign_gap(K, mh, other)
+        np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+        assert np.all(got >= 0)
