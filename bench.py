@@ -315,6 +315,84 @@ def extra_measurements(ckv, ctx, q, out, s, L, dev, hbm_gbs, bf16_tflops):
         cs.close()
         del Ks, Vs
     res["prefill_sweep"] = sweep
+    for key, fn in (("per_head", per_head_decode), ("split", split_pass)):
+        try:
+            res[key] = fn(ckv, ctx, q, s, L, dev, hbm_gbs)
+        except Exception as exc:  # a failed extra never hides the headline line
+            res[key] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+    return res
+
+
+def per_head_decode(ckv, ctx, q, s, L, dev, hbm_gbs):
+    """One selection per query head (select_and_attend_per_head) against the grouped
+    selection, both as eager calls over the 32 layer stores, 8 decode steps."""
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    steps = 8
+    out = torch.empty(L, B, HQ, 128, dtype=torch.float32, device=dev)
+    res = {}
+    for name in ("select_and_attend", "select_and_attend_per_head"):
+        call = getattr(ctx, name)
+        with torch.cuda.stream(s):
+            for l in range(L):
+                call(l, q[0, l], BUDGET, out[l], stream=s)
+        s.synchronize()
+        e0, e1 = ev(), ev()
+        with torch.cuda.stream(s):
+            e0.record(s)
+            for d in range(steps):
+                for l in range(L):
+                    call(l, q[d, l], BUDGET, out[l], stream=s)
+            e1.record(s)
+        s.synchronize()
+        res[name] = e0.elapsed_time(e1) * 1e3 / (steps * L)
+    ctx.check_device_error(stream=s)
+    by = select_attend_bytes(B * HQ, BUDGET, C_CLUSTERS, N_CTX - N_SINK, 1)
+    us = res["select_and_attend_per_head"]
+    return {"us_per_layer_step": us, "grouped_us_per_layer_step": res["select_and_attend"],
+            "bytes_per_launch": by, "achieved_gbs": by / (us * 1e-6) / 1e9,
+            "frac": by / (us * 1e-6) / 1e9 / hbm_gbs,
+            "what": "32 query heads each select their own budget-1024 rows; eager calls over "
+                    "32 layer stores x 8 steps, next to the grouped selection timed the same way"}
+
+
+def split_pass(ckv, ctx, q, s, L, dev, hbm_gbs):
+    """split_drifted_clusters on one 32k layer (8 KV heads, C=400): the drift check alone
+    (threshold +inf) and a pass at the median drift, each on a freshly prefilled store."""
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    Ks = torch.empty(1, HKV, N_CTX, 128, dtype=torch.bfloat16, device=dev)
+    Vs = torch.empty_like(Ks)
+    for h in range(HKV):
+        Ks[0, h], Vs[0, h] = si.keys_values_torch(SEED + 13, h, N_CTX, N_CENTERS, dev)
+    cs = ckv.ClusterKV(n_layers=1, batch=1, n_kv_heads=HKV, n_q_heads=HQ, capacity=N_CTX,
+                       max_clusters=1024, seed=SEED)
+    drift = torch.empty(HKV, C_CLUSTERS, dtype=torch.float32, device=dev)
+    res = {}
+    try:
+        for label, tau in (("detect_only", float("inf")), ("median", None)):
+            ts, n_split = [], 0
+            for rep in range(4):
+                with torch.cuda.stream(s):
+                    cs.cluster_prefill(0, Ks, Vs, C_CLUSTERS, stream=s)
+                    if tau is None:
+                        cs.split_drifted_clusters(0, float("inf"), drift, stream=s)
+                        t = float(drift.median())
+                        cs.cluster_prefill(0, Ks, Vs, C_CLUSTERS, stream=s)
+                    else:
+                        t = tau
+                    e0, e1 = ev(), ev()
+                    e0.record(s)
+                    n_split = sum(cs.split_drifted_clusters(0, t, drift, stream=s))
+                    e1.record(s)
+                s.synchronize()
+                if rep > 0:  # the first call allocates the scratch
+                    ts.append(e0.elapsed_time(e1) * 1e3)
+            res[label] = {"us": statistics.median(ts), "clusters_split": n_split}
+        cs.check_device_error(stream=s)
+    finally:
+        cs.close()
+    res["drift_read_bytes"] = HKV * (N_CTX - N_SINK) * 256
+    res["what"] = ("one layer, 8 KV heads x 32752 keys, C=400; CUDA events around the call, "
+                   "which includes its read-back of the split counts")
     return res
 
 
