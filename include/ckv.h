@@ -194,8 +194,9 @@ CKV_API int recluster_finish(ckv_ctx* ctx, int32_t layer, void* stream);
  * Synchronises `stream` (the new cluster count is read back), so it cannot be captured in
  * a CUDA graph. The first call allocates a scratch of about 520 bytes per token of
  * capacity per unit of one layer (CKV_ENOMEM if that fails). It shares no workspace with
- * cluster_prefill. CKV_ESTATE before cluster_prefill or while a re-clustering of the layer
- * is in flight. */
+ * cluster_prefill, but all split calls of a context share that scratch: calls from
+ * several host threads must not overlap in time. CKV_ESTATE before cluster_prefill or
+ * while a re-clustering of the layer is in flight. */
 CKV_API int split_drifted_clusters(ckv_ctx* ctx, int32_t layer, float threshold, float* drift,
                                    int32_t* splits, void* stream);
 
