@@ -83,6 +83,24 @@ def test_calls_on_null_context_fail_cleanly(built):
     assert built.ckv_destroy(None) == 0
 
 
+def test_every_context_call_rejects_a_null_context(built):
+    """Each entry point that takes a context checks it on the host first: a null context is
+    CKV_EINVAL, with no device call."""
+    no_ctx = {"ckv_config_default", "ckv_create", "ckv_destroy", "ckv_strerror",
+              "ckv_last_error", "ckv_device_bytes", "ckv_kmeans_update_noalloc"}
+    checked = []
+    for name, (_, argtypes) in ckv.SIGNATURES.items():
+        if name in no_ctx:
+            continue
+        args = [None] + [0.0 if t is C.c_float else (None if t is C.c_void_p else 0)
+                         for t in argtypes[1:]]
+        assert getattr(built, name)(*args) == ckv.CKV_EINVAL, name
+        assert built.ckv_last_error(), name
+        checked.append(name)
+    assert "split_drifted_clusters" in checked and "select_and_attend_per_head" in checked
+    assert built.ckv_device_bytes(None) == 0
+
+
 def test_product_path_does_not_reference_the_oracle():
     pkg = os.path.join(ROOT, "recallable_kv_cache_cosine_b200")
     for dirpath, _, files in os.walk(pkg):
