@@ -562,6 +562,16 @@ def run_gpu(args, world, rank, local):
                "sample": (f"{n_ls} layer-steps of select+attend over one 32k-token layer (8 KV heads, "
                           f"G=4, C=400, budget 1024); clusters = the generator's mixture components "
                           f"with one oracle mean update; OpenMP over the 8 units")}
+        try:  # the same sample on one thread
+            prev = oracle.set_threads(1)
+            n1 = max(8, n_ls // 16)
+            try:
+                cpu["single_thread"] = {"value": oracle_time_layer_steps(st, qo, n1) * 1e6,
+                                        "unit": UNIT, "layer_steps": n1}
+            finally:
+                oracle.set_threads(prev)
+        except Exception as exc:
+            cpu["single_thread"] = {"error": f"{type(exc).__name__}: {exc}"[:200]}
 
     if rank == 0:
         clocks = clk.summary()

@@ -61,6 +61,7 @@ def lib():
             "orc_select": (i32, [P, P, i32, P, P, P, P]),
             "orc_attend": (None, [P, P, i32, P, i32, P]),
             "orc_dense_attention": (None, [P, P, i64, P, i32, P]),
+            "orc_set_threads": (i32, [i32]),
             "orc_prefill_batch": (None, [i32, P, P, i64, i32, i32, i32, P, P, P, P, P, P, P]),
             "orc_select_attend_batch": (None, [i32, i32, i32, i64, i32, P, P, P, P, P, P, P, P,
                                                i32, i32, P, P, P]),
@@ -449,3 +450,8 @@ def select_attend_batch(sp_k, sp_v, kp, vp, ids, offsets, mu, q, budget: int, n_
 
 def omp_threads() -> int:
     return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def set_threads(n: int) -> int:
+    """Threads of the batched (timing) calls; returns the previous setting."""
+    return int(lib().orc_set_threads(n))

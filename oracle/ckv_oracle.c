@@ -656,6 +656,23 @@ void orc_attend_mixed(const orc_store* s, const uint16_t* q, int32_t G, const in
 /* Independent units run in parallel (OpenMP, when compiled with it). Each unit's
  * arithmetic is exactly the single-unit function above. */
 
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Sets the number of threads of the batched calls; returns the previous setting (1 without
+ * OpenMP). */
+int32_t orc_set_threads(int32_t n) {
+#ifdef _OPENMP
+    int32_t prev = (int32_t)omp_get_max_threads();
+    if (n > 0) omp_set_num_threads(n);
+    return prev;
+#else
+    (void)n;
+    return 1;
+#endif
+}
+
 void orc_prefill_batch(int32_t U, const uint16_t* K, const uint16_t* V, int64_t n,
                        int32_t n_sink, int32_t C, int32_t iters, const uint64_t* keys,
                        uint16_t* kp, uint16_t* vp, int32_t* ids, int32_t* offsets,

@@ -24,3 +24,11 @@ def test_reference_arm_prints_one_json_line():
     assert d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["cpu_baseline"]["value"] == d["value"] and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_oracle_thread_setting_round_trips():
+    import oracle
+    prev = oracle.set_threads(1)
+    assert prev >= 1
+    assert oracle.set_threads(prev) == 1
+    assert oracle.set_threads(0) == prev  # 0 reads the setting without changing it
