@@ -1112,13 +1112,16 @@ template <int G, bool kPerHead>
 int plan_for(const DecodeArgs& a, int num_sms, Plan* out) {
     static std::mutex mtx;
     static std::map<std::tuple<int, int, int, int>, Plan> cache;
-    static size_t smem_set = 0;
-    static bool nonportable_set = false;
+    // kernel attributes are set per device: what has been set, by device
+    static std::map<int, size_t> smem_set_by_dev;
+    static std::map<int, bool> nonportable_set_by_dev;
     int dev = 0;
     cudaGetDevice(&dev);
     const int U = a.B * a.Hkv;
     const auto key = std::make_tuple(dev, U, a.C, a.budget);
     std::lock_guard<std::mutex> lock(mtx);
+    size_t& smem_set = smem_set_by_dev[dev];
+    bool& nonportable_set = nonportable_set_by_dev[dev];
     auto it = cache.find(key);
     if (it != cache.end()) {
         *out = it->second;
