@@ -346,13 +346,18 @@ def per_head_decode(ckv, ctx, q, s, L, dev, hbm_gbs):
         s.synchronize()
         res[name] = e0.elapsed_time(e1) * 1e3 / (steps * L)
     ctx.check_device_error(stream=s)
-    by = select_attend_bytes(B * HQ, BUDGET, C_CLUSTERS, N_CTX - N_SINK, 1)
+    # rows, cut-cluster keys, q and o per query head (the rows as if the heads' selections were
+    # disjoint: an upper bound of their union); centroids and offsets once per KV head
+    m = N_CTX - N_SINK
+    by = (B * HQ * (BUDGET * 512 + (m / C_CLUSTERS) * 256 + 128 * 2 + 128 * 4)
+          + B * HKV * (C_CLUSTERS * 512 + (C_CLUSTERS + 1) * 4))
     us = res["select_and_attend_per_head"]
     return {"us_per_layer_step": us, "grouped_us_per_layer_step": res["select_and_attend"],
             "bytes_per_launch": by, "achieved_gbs": by / (us * 1e-6) / 1e9,
             "frac": by / (us * 1e-6) / 1e9 / hbm_gbs,
             "what": "32 query heads each select their own budget-1024 rows; eager calls over "
-                    "32 layer stores x 8 steps, next to the grouped selection timed the same way"}
+                    "32 layer stores x 8 steps, next to the grouped selection timed the same way; "
+                    "bytes count each head's rows and each KV head's centroids once"}
 
 
 def split_pass(ckv, ctx, q, s, L, dev, hbm_gbs):
