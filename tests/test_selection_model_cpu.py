@@ -1,0 +1,106 @@
+"""The decode kernel's way of finding the cut, restated in Python, agrees with the oracle's
+sorted walk (ClusterKV explainer, section 3.3) on adversarial cases.
+
+The kernel does not sort the clusters. Each CTA:
+1. maps the fp32 scores monotonically onto 256 linear buckets between the smallest and the
+   largest score;
+2. builds a histogram of cluster sizes per bucket and finds the bucket b* holding the cut
+   (the first cluster, in descending (score, -index) order, whose inclusive size exceeds the
+   remaining budget);
+3. ranks exactly, by the key (orderable score, -index), only the clusters in buckets >= b*;
+   the orderable score maps -0 and +0 to one key, so they tie like equal doubles.
+   A cluster whose exclusive prefix plus its size fits is whole; the one whose prefix fits
+   but whose size does not is the cut.
+
+This model is checked against the oracle's `select` on stores whose scores are exactly the
+chosen fp32 values (centroid c = s_c * e_0, query e_0): many ties, all-equal scores, a tiny
+score range, and zero-size clusters. It is a check of the algorithm; the GPU parity tests
+check the kernel.
+"""
+import numpy as np
+
+import oracle
+
+D = 128
+
+
+def _orderable(x: np.float32) -> int:
+    """Unsigned key with the order of the float; -0 and +0 give the same key (they tie)."""
+    u = int((np.array([x], np.float32) + np.float32(0)).view(np.uint32)[0])
+    return (~u) & 0xFFFFFFFF if u & 0x80000000 else u | 0x80000000
+
+
+def bucket_cut(sc: np.ndarray, sz: np.ndarray, R: int):
+    """Whole clusters (set), cut cluster and its exclusive prefix, or None if all fit."""
+    sc = sc.astype(np.float32)
+    if sz.sum() <= R:
+        return None
+    mn, mx = sc.min(), sc.max()
+    span = np.float32(mx - mn)
+    inv = np.float32(255.99) / span if span > 1e-30 else np.float32(0)
+    b = np.clip(np.nan_to_num((sc - mn).astype(np.float32) * inv, nan=0.0), 0, 255).astype(np.int64)
+    hist = np.zeros(256, np.int64)
+    np.add.at(hist, b[sz > 0], sz[sz > 0])
+    above, bstar = 0, 0
+    for d in range(255, -1, -1):
+        if above <= R < above + hist[d]:
+            bstar = d
+            break
+        above += hist[d]
+    cand = [c for c in range(len(sc)) if b[c] >= bstar]
+    key = {c: (_orderable(sc[c]) << 32) | (0xFFFFFFFF - c) for c in cand}
+    whole, cut = set(), None
+    for c in cand:
+        pre = sum(int(sz[j]) for j in cand if key[j] > key[c])
+        if pre + sz[c] <= R:
+            whole.add(c)
+        elif pre <= R:
+            cut = (c, pre)
+    return whole, cut[0], cut[1]
+
+
+def _store(sc, sz):
+    m = int(sz.sum())
+    offs = np.concatenate([[0], np.cumsum(sz)]).astype(np.int32)
+    mu = np.zeros((len(sc), D))
+    mu[:, 0] = sc.astype(np.float64)
+    kp = np.zeros((m, D), np.uint16)
+    kp[:, 1] = 0x3F80  # 1.0: every token scores 0 on e_0, the partial fill is by id
+    sink = np.zeros((16, D), np.uint16)
+    return oracle.Store(sink, sink.copy(), kp, kp.copy(), np.arange(16, 16 + m, dtype=np.int32),
+                        offs, mu)
+
+
+def test_bucket_histogram_cut_equals_the_sorted_walk():
+    rng = np.random.default_rng(0)
+    qbar = np.zeros(D)
+    qbar[0] = 1.0
+    checked = 0
+    for trial in range(800):
+        C = int(rng.integers(1, 80))
+        kind = trial % 4
+        sc = rng.normal(0, 30, C).astype(np.float32)
+        if kind == 1:
+            sc = (np.round(sc / 10) * 10).astype(np.float32)       # many ties
+        elif kind == 2:
+            sc[:] = np.float32(5.0)                                  # all equal
+        elif kind == 3:
+            sc = (rng.normal(0, 1e-6, C) + 100).astype(np.float32)  # a tiny range
+        sz = rng.integers(0, 60, C)
+        if trial % 5 == 0:
+            sz[rng.integers(0, C, max(1, C // 3))] = 0
+        R = int(rng.integers(0, max(1, int(sz.sum()) + 10)))
+        st = _store(sc, sz)
+        sel = oracle.select_qbar(st, qbar, R + 16)
+        got = bucket_cut(sc, sz, R)
+        if got is None:
+            assert sel.cut == -1
+            continue
+        whole, cut, pre = got
+        assert cut == sel.cut, (trial, cut, sel.cut)
+        assert R - pre == sel.r, (trial, R - pre, sel.r)
+        taken = {int(c) for c in np.searchsorted(st.offsets, sel.rows[sel.rows >= 0], side="right") - 1}
+        nonempty_whole = {c for c in whole if sz[c] > 0}
+        assert nonempty_whole == taken - {cut}, trial
+        checked += 1
+    assert checked > 600
