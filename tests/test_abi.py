@@ -109,3 +109,20 @@ def test_product_path_does_not_reference_the_oracle():
                 txt = open(os.path.join(dirpath, f), encoding="utf-8").read()
                 assert "import oracle" not in txt and "from oracle" not in txt, f
                 assert "ckv_oracle" not in txt and "libckv_oracle" not in txt, f
+
+
+def test_binding_constants_and_structs_match_the_header():
+    src = open(HEADER).read()
+    codes = dict(re.findall(r"#define (CKV_E\w+|CKV_OK)\s+\(?(-?\d+)\)?", src))
+    assert codes and all(getattr(ckv, k) == int(v) for k, v in codes.items()), codes
+    # field order and types of the structs the binding mirrors
+    for cname, pyt in (("ckv_config", ckv.Config), ("ckv_layer_info", ckv.LayerInfo),
+                       ("ckv_unit_buffers", ckv.UnitBuffers)):
+        body = re.search(r"typedef struct %s \{(.*?)\} %s;" % (cname, cname), src, re.S).group(1)
+        body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+        decls = re.findall(r"([\w ]+?)\s*(\*?)\s*(\w+)\s*;", body)
+        assert [d[2] for d in decls] == [f for f, _ in pyt._fields_], (cname, decls)
+        ctype = {"int32_t": C.c_int32, "int64_t": C.c_int64, "uint64_t": C.c_uint64}
+        for (typ, star, name), (_, pt) in zip(decls, pyt._fields_):
+            want = C.c_void_p if star else ctype[typ.strip()]
+            assert pt is want, (cname, name, typ, star, pt)
