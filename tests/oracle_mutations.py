@@ -64,6 +64,11 @@ M = [
  ("split rows unpermuted", "int64_t src = (int64_t)lo + cperm[j],", "int64_t src = (int64_t)lo + j,", 0),
  ("e4m3 decode subnormal", "ldexp((double)mant, -9)", "ldexp((double)mant, -10)", 0),
  ("e4m3 decode bias", "ldexp(1.0 + mant / 8.0, ex - 7)", "ldexp(1.0 + mant / 8.0, ex - 8)", 0),
+ ("batch sp no pending", "int64_t sp = (int64_t)n_sink + pending;", "int64_t sp = (int64_t)n_sink;", 0),
+ ("batch offsets stride C", "s.offsets = offsets + (int64_t)u * (C + 1);", "s.offsets = offsets + (int64_t)u * C;", 0),
+ ("prefill batch offsets stride C", "offsets + (int64_t)u * (C + 1),\n                         mu", "offsets + (int64_t)u * C,\n                         mu", 0),
+ ("batch qbar stride", "orc_group_query(q + (int64_t)u * G * ORC_D, G, qbar);", "orc_group_query(q + (int64_t)u * ORC_D, G, qbar);", 0),
+ ("batch attend q stride", "orc_attend(&s, q + (int64_t)u * G * ORC_D", "orc_attend(&s, q + (int64_t)u * ORC_D", 0),
  ("mixed v path bf16 from k", "const uint16_t* v = r >= 0 ? s->vp + (int64_t)r * ORC_D", "const uint16_t* v = r >= 0 ? s->kp + (int64_t)r * ORC_D", 1),
 ]
 
