@@ -263,7 +263,10 @@ CKV_API int ckv_kmeans_assign(ckv_ctx* ctx, const void* keys, int64_t n_rows, in
 /* Centroid update ([EXPL] 3.1 mean, 4.1 contiguous layout): stable counting sort by
  * cluster (offsets int32 [U, C + 1], perm int32 [U, m] = member indices in ascending
  * order per cluster), then mu[u, c] = mean of its members (fp32, summed in perm order),
- * empty clusters keep mu, and mu_hat = bf16(mu / |mu|). mu: fp32 [U, C, 128], in/out. */
+ * empty clusters keep mu, and mu_hat = bf16(mu / |mu|). mu: fp32 [U, C, 128], in/out.
+ * An assignment outside [0, C) is skipped: that key joins no cluster, offsets[u][C]
+ * counts only the keys placed (below m), perm entries from there on are left unwritten,
+ * and the device error word makes ckv_check_device_error return CKV_EINVAL. */
 CKV_API int ckv_kmeans_update(ckv_ctx* ctx, const void* keys, int64_t n_rows, int64_t row0, int64_t m,
                       int32_t U, const int32_t* assign, int32_t C, float* mu, void* mu_hat,
                       int32_t* offsets, int32_t* perm, void* stream);
@@ -275,7 +278,10 @@ CKV_API int ckv_kmeans_update(ckv_ctx* ctx, const void* keys, int64_t n_rows, in
  * application owns the device memory. It needs no context. The inputs and outputs are the
  * caller's, exactly as for ckv_kmeans_update (keys bf16 [U, n_rows, 128]; assign int32
  * [U, m]; mu fp32 [U, C, 128] in/out; mu_hat bf16 [U, C, 128]; offsets int32 [U, C + 1];
- * perm int32 [U, m]), and so are the results.
+ * perm int32 [U, m]), and so are the results, bit for bit.
+ * Having no context, it has no device error word: an assignment outside [0, C) is skipped
+ * without a report. The key joins no cluster, and offsets[u][C] then counts only the keys
+ * placed, so a caller detects bad input by comparing offsets[u][C] with m.
  * The kernels' scratch, the per-chunk cluster counts of the counting sort, is a fixed
  * array of 2^21 int32 (8 MiB) compiled into the library. Every GPU that loads the library
  * holds it until the process exits. A call needs U * ceil(m / 1024) * C counts. Larger

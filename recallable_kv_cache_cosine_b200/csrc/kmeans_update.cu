@@ -147,7 +147,9 @@ __global__ void __launch_bounds__(256) kmeans_count_kernel(const int32_t* assign
 }
 
 // ---------------------------------------------------------------------- scan
-// Per unit: sizes[c] = sum over chunks; offsets = exclusive scan of sizes (offsets[C] = m);
+// Per unit: sizes[c] = sum over chunks; offsets = exclusive scan of sizes, and offsets[C] =
+// the keys counted (m, unless the count kernel skipped out-of-range assignments; the mean
+// kernel then never reaches perm entries that the scatter did not write);
 // chunk[u][ch][c] becomes the number of keys of cluster c in chunks before ch.
 __global__ void __launch_bounds__(1024) kmeans_scan_kernel(int32_t* chunk, int32_t nch, int32_t C,
                                                            int64_t m, int32_t* offsets,
@@ -206,7 +208,7 @@ __global__ void __launch_bounds__(1024) kmeans_scan_kernel(int32_t* chunk, int32
             off[c0 + j] = run;
             run += sz[c0 + j];
         }
-    if (threadIdx.x == 0) off[C] = (int32_t)m;
+    if (threadIdx.x == 0) off[C] = wsum[31];  // total over the warps: the keys counted
 }
 
 // ---------------------------------------------------------------------- scatter
