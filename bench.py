@@ -213,6 +213,71 @@ def run_reference(args, world, rank):
 
 # ---------------------------------------------------------------------- GPU leg
 
+def decode_shape(ckv, s, dev, hbm_gbs, B, L, D, budget, n, C, what, mixed_n_near=None):
+    """µs per select+attend launch at one shape: L layer stores of B sequences x 8 KV heads,
+    D decode steps x L layers as one CUDA graph of back-to-back launches, and the fraction of
+    the HBM peak by the algorithmic bytes per launch."""
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    G = HQ // HKV
+    try:
+        cx = ckv.ClusterKV(n_layers=L, batch=B, n_kv_heads=HKV, n_q_heads=HQ, capacity=n,
+                           max_clusters=C, seed=SEED)
+    except Exception as exc:
+        return {"error": f"{type(exc).__name__}: {exc}"[:300]}
+    try:
+        K = torch.empty(B, HKV, n, 128, dtype=torch.bfloat16, device=dev)
+        V = torch.empty_like(K)
+        qs = torch.empty(D, L, B, HQ, 128, dtype=torch.bfloat16, device=dev)
+        os_ = torch.empty(D, L, B, HQ, 128, dtype=torch.float32, device=dev)
+        for l in range(L):
+            for b in range(B):
+                for h in range(HKV):
+                    K[b, h], V[b, h] = si.keys_values_torch(SEED + 7, si.unit_id(l, b, h, B, HKV), n,
+                                                            C, dev)
+                qs[:, l, b] = si.queries_torch(SEED + 7, l, b, D, HQ, dev)
+            with torch.cuda.stream(s):
+                cx.cluster_prefill(l, K, V, C, stream=s)
+        if mixed_n_near is not None:
+            cx.enable_fp8(stream=s)
+        s.synchronize()
+        del K, V
+
+        def dec():
+            for d in range(D):
+                for l in range(L):
+                    if mixed_n_near is None:
+                        cx.select_and_attend(l, qs[d, l], budget, os_[d, l], stream=s)
+                    else:
+                        cx.select_and_attend_mixed(l, qs[d, l], budget, mixed_n_near, os_[d, l], stream=s)
+        with torch.cuda.stream(s):
+            dec()
+        s.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s, capture_error_mode="thread_local"):
+            dec()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = ev(), ev()
+        with torch.cuda.stream(s):
+            e0.record(s)
+            for _ in range(5):
+                g.replay()
+            e1.record(s)
+        torch.cuda.synchronize()
+        cx.check_device_error(stream=s)
+        us = e0.elapsed_time(e1) * 1e3 / (5 * D * L)
+        by = select_attend_bytes(B * HKV, budget, C, n - N_SINK, G)
+        del g
+        return {"us_per_layer_step": us, "units": B * HKV, "bytes_per_launch": by,
+                "achieved_gbs": by / (us * 1e-6) / 1e9, "frac": by / (us * 1e-6) / 1e9 / hbm_gbs,
+                "what": what + ", CUDA graph of %d launches" % (D * L)}
+    except Exception as exc:
+        return {"error": f"{type(exc).__name__}: {exc}"[:300]}
+    finally:
+        cx.close()
+
+
 def extra_measurements(ckv, ctx, q, out, s, L, dev, hbm_gbs, bf16_tflops):
     """Single-launch latency with L2 flushed, the batch-8 / budget-2048 shape, and the prefill
     keys/s sweep over n in {8k, 32k, 128k}."""
@@ -234,56 +299,31 @@ def extra_measurements(ckv, ctx, q, out, s, L, dev, hbm_gbs, bf16_tflops):
     res["single_launch_us_l2_flushed"] = statistics.median(single[1:])
     del flush
 
-    # batch 8, budget 2048: 64 units per launch, 4 layer stores (320 MB per decode pass)
-    B8, L8, D8, BUD8 = 8, 4, 8, 2048
-    c8 = ckv.ClusterKV(n_layers=L8, batch=B8, n_kv_heads=HKV, n_q_heads=HQ, capacity=N_CTX,
-                       max_clusters=C_CLUSTERS, seed=SEED)
-    K8 = torch.empty(B8, HKV, N_CTX, 128, dtype=torch.bfloat16, device=dev)
-    V8 = torch.empty_like(K8)
-    q8 = torch.empty(D8, L8, B8, HQ, 128, dtype=torch.bfloat16, device=dev)
-    o8 = torch.empty(D8, L8, B8, HQ, 128, dtype=torch.float32, device=dev)
-    for l in range(L8):
-        for b in range(B8):
-            for h in range(HKV):
-                K8[b, h], V8[b, h] = si.keys_values_torch(SEED + 7, si.unit_id(l, b, h, B8, HKV), N_CTX,
-                                                          N_CENTERS, dev)
-            q8[:, l, b] = si.queries_torch(SEED + 7, l, b, D8, HQ, dev)
-        with torch.cuda.stream(s):
-            c8.cluster_prefill(l, K8, V8, C_CLUSTERS, stream=s)
-    s.synchronize()
-    del K8, V8
-
-    def dec8():
-        for d in range(D8):
-            for l in range(L8):
-                c8.select_and_attend(l, q8[d, l], BUD8, o8[d, l], stream=s)
-    with torch.cuda.stream(s):
-        dec8()
-    s.synchronize()
-    g8 = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g8, stream=s, capture_error_mode="thread_local"):
-        dec8()
-    for _ in range(3):
-        g8.replay()
-    torch.cuda.synchronize()
-    e0, e1 = ev(), ev()
-    with torch.cuda.stream(s):
-        e0.record(s)
-        for _ in range(5):
-            g8.replay()
-        e1.record(s)
-    torch.cuda.synchronize()
-    c8.check_device_error(stream=s)
-    us8 = e0.elapsed_time(e1) * 1e3 / (5 * D8 * L8)
-    by8 = select_attend_bytes(B8 * HKV, BUD8, C_CLUSTERS, N_CTX - N_SINK, G)
-    res["batch8_budget2k"] = {"us_per_layer_step": us8, "units": B8 * HKV, "bytes_per_launch": by8,
-                              "achieved_gbs": by8 / (us8 * 1e-6) / 1e9,
-                              "frac": by8 / (us8 * 1e-6) / 1e9 / hbm_gbs,
-                              "what": "batch 8 x 8 KV heads, n=32768, C=400, budget 2048, 4 layer "
-                                      "stores (320 MB per decode pass), CUDA graph of 32 launches"}
-    del g8
-    c8.close()
-    del q8, o8
+    # the other decode shapes of the workload family, each as back-to-back launches over
+    # distinct layer stores in one CUDA graph (inputs larger than L2)
+    res["batch8_budget2k"] = decode_shape(ckv, s, dev, hbm_gbs, B=8, L=4, D=8, budget=2048, n=N_CTX,
+                                          C=C_CLUSTERS, what="batch 8 x 8 KV heads, n=32768, C=400, "
+                                          "budget 2048, 4 layer stores (320 MB per decode pass)")
+    res["batch4_budget1k"] = decode_shape(ckv, s, dev, hbm_gbs, B=4, L=8, D=8, budget=1024, n=N_CTX,
+                                          C=C_CLUSTERS, what="batch 4 x 8 KV heads, n=32768, C=400, "
+                                          "budget 1024, 8 layer stores (189 MB per decode pass)")
+    mix = decode_shape(ckv, s, dev, hbm_gbs, B=1, L=32, D=8, budget=BUDGET, n=N_CTX, C=C_CLUSTERS,
+                       mixed_n_near=0, what="select_and_attend_mixed with n_near = 0 (every selected "
+                       "cluster attended from the fp8 copy) at the headline shape, 32 layer stores")
+    if "us_per_layer_step" in mix:
+        # far rows move codes and scales (2 x 132 B) instead of 2 x 256 B
+        by = mix["bytes_per_launch"] - B * HKV * (BUDGET - N_SINK) * (512 - 264)
+        mix["bytes_per_launch"] = by
+        mix["achieved_gbs"] = by / (mix["us_per_layer_step"] * 1e-6) / 1e9
+        mix["frac"] = mix["achieved_gbs"] / hbm_gbs
+    res["mixed_fp8"] = mix
+    res["mixed_fp8_near6"] = decode_shape(ckv, s, dev, hbm_gbs, B=1, L=32, D=8, budget=BUDGET, n=N_CTX,
+                                          C=C_CLUSTERS, mixed_n_near=6,
+                                          what="select_and_attend_mixed with n_near = 6 at the "
+                                          "headline shape (bytes counted as bf16 rows)")
+    res["long_128k"] = decode_shape(ckv, s, dev, hbm_gbs, B=1, L=16, D=8, budget=2048, n=131072,
+                                    C=1600, what="batch 1 x 8 KV heads, n=131072, C=1600, budget "
+                                    "2048, 16 layer stores (242 MB per decode pass)")
 
     # prefill keys/s sweep, one layer of 8 KV heads each
     sweep = []
@@ -362,42 +402,48 @@ def per_head_decode(ckv, ctx, q, s, L, dev, hbm_gbs):
 
 def split_pass(ckv, ctx, q, s, L, dev, hbm_gbs):
     """split_drifted_clusters on one 32k layer (8 KV heads, C=400): the drift check alone
-    (threshold +inf) and a pass at the median drift, each on a freshly prefilled store."""
+    (threshold +inf, max_splits 0) and a pass at the median drift (max_splits = the room left,
+    624), each on a freshly prefilled store, timed with CUDA events around the call (which
+    reads nothing back)."""
     ev = lambda: torch.cuda.Event(enable_timing=True)
     Ks = torch.empty(1, HKV, N_CTX, 128, dtype=torch.bfloat16, device=dev)
     Vs = torch.empty_like(Ks)
     for h in range(HKV):
         Ks[0, h], Vs[0, h] = si.keys_values_torch(SEED + 13, h, N_CTX, N_CENTERS, dev)
+    cmax = 1024
     cs = ckv.ClusterKV(n_layers=1, batch=1, n_kv_heads=HKV, n_q_heads=HQ, capacity=N_CTX,
-                       max_clusters=1024, seed=SEED)
+                       max_clusters=cmax, seed=SEED)
     drift = torch.empty(HKV, C_CLUSTERS, dtype=torch.float32, device=dev)
+    cnt = torch.empty(HKV, dtype=torch.int32, device=dev)
     res = {}
     try:
-        for label, tau in (("detect_only", float("inf")), ("median", None)):
+        for label, tau, mx in (("detect_only", float("inf"), 0), ("median", None, cmax - C_CLUSTERS)):
             ts, n_split = [], 0
             for rep in range(4):
                 with torch.cuda.stream(s):
                     cs.cluster_prefill(0, Ks, Vs, C_CLUSTERS, stream=s)
                     if tau is None:
-                        cs.split_drifted_clusters(0, float("inf"), drift, stream=s)
+                        cs.split_drifted_clusters(0, float("inf"), 0, drift, stream=s)
+                        s.synchronize()
                         t = float(drift.median())
-                        cs.cluster_prefill(0, Ks, Vs, C_CLUSTERS, stream=s)
                     else:
                         t = tau
                     e0, e1 = ev(), ev()
                     e0.record(s)
-                    n_split = sum(cs.split_drifted_clusters(0, t, drift, stream=s))
+                    cs.split_drifted_clusters(0, t, mx, drift, cnt, stream=s)
                     e1.record(s)
                 s.synchronize()
+                n_split = int(cnt.sum())
                 if rep > 0:  # the first call allocates the scratch
                     ts.append(e0.elapsed_time(e1) * 1e3)
-            res[label] = {"us": statistics.median(ts), "clusters_split": n_split}
+            res[label] = {"us": statistics.median(ts), "clusters_split": n_split, "max_splits": mx}
         cs.check_device_error(stream=s)
     finally:
         cs.close()
     res["drift_read_bytes"] = HKV * (N_CTX - N_SINK) * 256
-    res["what"] = ("one layer, 8 KV heads x 32752 keys, C=400; CUDA events around the call, "
-                   "which includes its read-back of the split counts")
+    res["drift_floor_us"] = res["drift_read_bytes"] / (hbm_gbs * 1e3)
+    res["what"] = ("one layer, 8 KV heads x 32752 keys, C=400; CUDA events around the call; "
+                   "the call reads nothing back and can be captured in a CUDA graph")
     return res
 
 

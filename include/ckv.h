@@ -17,8 +17,8 @@
  *     elements, 16-byte aligned base). fp32 and int32 tensors are 16-byte aligned too.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Work is enqueued
  *     asynchronously on it. No call synchronises the host, except ckv_create,
- *     ckv_destroy, ckv_check_device_error, ckv_export_unit, ckv_import_unit and
- *     split_drifted_clusters.
+ *     ckv_destroy, ckv_check_device_error, ckv_export_unit, ckv_export_unit_fp8 and
+ *     ckv_import_unit (and the first ckv_enable_fp8, which allocates).
  *   - Return 0 (CKV_OK) on success or a negative CKV_E* code. All arguments are checked on
  *     the host before anything is enqueued. A call that fails its checks leaves the
  *     cluster store unchanged. ckv_last_error() gives a one-line reason (per thread).
@@ -110,12 +110,16 @@ CKV_API int cluster_prefill(ckv_ctx* ctx, int32_t layer, const void* K, const vo
  *   budget    : tokens attended per unit (sinks and pending included), >= n_sink + pending.
  *   out       : device fp32 [batch, n_q_heads, 128].
  *   sel_idx   : optional device int32 [batch, n_kv_heads, budget]. Original token ids of
- *               the selected rows in selection order: sinks, pending, whole clusters by
- *               descending score (each in store order), then the partial tokens (in store
- *               order). Entries past the count are -1.
+ *               the selected rows in the kernel's order: sinks, pending, the whole clusters
+ *               in cluster-index order (each in store order), then the partial tokens (in
+ *               store order). Entries past the count are -1.
  *   sel_count : optional device int32 [batch, n_kv_heads] = min(budget, n_total).
  * Reads the store only, so it can be captured in a CUDA graph. The token counts are read
- * at call time and baked into a captured launch. */
+ * at call time and baked into a captured launch. The kernel uses programmatic dependent
+ * launch: it may start while the previous kernel of `stream` still runs and read the
+ * layer's cluster store then (only this library writes the store, and its calls that do
+ * let a following kernel start only once the store is complete); it waits for the previous
+ * work before it reads q or the pending rows and before it writes any output. */
 CKV_API int select_and_attend(ckv_ctx* ctx, int32_t layer, const void* q, int32_t budget, float* out,
                       int32_t* sel_idx, int32_t* sel_count, void* stream);
 
@@ -179,26 +183,29 @@ CKV_API int recluster_finish(ckv_ctx* ctx, int32_t layer, void* stream);
  * K-means with 2 clusters and `iters` iterations on its own rows (rows in store order;
  * init: the first two entries of the SplitMix64 Fisher-Yates shuffle keyed by
  * seed ^ (unit << 32) ^ windows ^ ((c + 1) * 0x9E3779B97F4A7C15), windows = the layer's
- * incremental clusterings so far), at most max_clusters - C clusters per unit, lowest
- * index first. The halves take indices c' and c' + 1, with c' = c + (splits below c), and
- * later clusters move up. A split cluster's rows are reordered inside its own segment
- * (first half, then second half, each in store order), so ids stay ascending in every
- * cluster. The layer's cluster count becomes C + the largest split count of its units;
- * units that split fewer clusters get empty clusters (no rows, zero centroid) at the end,
- * which never add a selected row.
- *   threshold : split when drift > threshold (+inf: never, -inf: every cluster of 2+ rows);
- *               NaN is CKV_EINVAL.
- *   drift     : optional device fp32 [batch * n_kv_heads, C] (C before the call), every
- *               cluster's drift.
- *   splits    : optional HOST int32 [batch * n_kv_heads], clusters split per unit.
- * Synchronises `stream` (the new cluster count is read back), so it cannot be captured in
- * a CUDA graph. The first call allocates a scratch of about 520 bytes per token of
- * capacity per unit of one layer (CKV_ENOMEM if that fails). It shares no workspace with
- * cluster_prefill, but all split calls of a context share that scratch: calls from
- * several host threads must not overlap in time. CKV_ESTATE before cluster_prefill or
- * while a re-clustering of the layer is in flight. */
-CKV_API int split_drifted_clusters(ckv_ctx* ctx, int32_t layer, float threshold, float* drift,
-                                   int32_t* splits, void* stream);
+ * incremental clusterings so far), at most room = min(max_splits, max_clusters - C)
+ * clusters per unit, lowest index first. The halves take indices c' and c' + 1, with
+ * c' = c + (splits below c), and later clusters move up. A split cluster's rows are
+ * reordered inside its own segment (first half, then second half, each in store order), so
+ * ids stay ascending in every cluster. The layer's cluster count becomes exactly C + room:
+ * a unit that split fewer than room clusters gets empty clusters (no rows, zero centroid) at
+ * the end, which never add a selected row. The new count is therefore known on the host
+ * without reading anything back: the call never synchronises and can be captured in a
+ * CUDA graph. Pick max_splits near the number of splits expected; every padding cluster is
+ * scored by later decode steps.
+ *   threshold  : split when drift > threshold (+inf: never, -inf: every cluster of 2+ rows);
+ *                NaN is CKV_EINVAL.
+ *   max_splits : >= 0 (CKV_EINVAL otherwise); 0 only measures the drift.
+ *   drift      : optional device fp32 [batch * n_kv_heads, C] (C before the call), every
+ *                cluster's drift.
+ *   splits     : optional device int32 [batch * n_kv_heads], clusters split per unit.
+ * The first call allocates a scratch of about 520 bytes per token of capacity per unit of
+ * one layer (CKV_ENOMEM if that fails). It shares no workspace with cluster_prefill, but all
+ * split calls of a context share that scratch: calls whose work overlaps on the GPU must not
+ * be issued. CKV_ESTATE before cluster_prefill or while a re-clustering of the layer is in
+ * flight. */
+CKV_API int split_drifted_clusters(ckv_ctx* ctx, int32_t layer, float threshold, int32_t max_splits,
+                                   float* drift, int32_t* splits, void* stream);
 
 typedef struct ckv_layer_info {
     int64_t n_total;   /* tokens per unit: n_sink + m + pending */
@@ -240,6 +247,50 @@ CKV_API int ckv_import_unit(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h, i
  * CKV_ETIMEOUT if a kernel's bounded wait gave up, or CKV_EINVAL if a kernel skipped an
  * out-of-range input (a caller-supplied assignment outside [0, C)). */
 CKV_API int ckv_check_device_error(ckv_ctx* ctx, void* stream);
+
+/* Lower precision for far clusters ([EXPL] section 7, outlook: a lower-precision KV cache for
+ * clusters far from the current query). The page fixes no format; the reading: every
+ * clustered row also keeps an fp8 e4m3 copy with one fp32 scale per row, scale = max|x| / 448,
+ * code = e4m3(x / scale) (round to nearest, ties to even, saturating at 448; fp32
+ * arithmetic; a zero row has scale 0). The dequantised value is e4m3(code) * scale.
+ * ckv_enable_fp8 allocates the copy for every layer (about 264 bytes per clustered row of
+ * capacity; CKV_ENOMEM if that fails), fills it for the layers already clustered, and from
+ * then on every call that writes the store (cluster_prefill, recluster_increment,
+ * recluster_begin, split_drifted_clusters, ckv_import_unit) refreshes the rows it wrote, on
+ * the same stream. Calling it again only refreshes. Asynchronous on `stream` apart from the
+ * first call's allocation. */
+CKV_API int ckv_enable_fp8(ckv_ctx* ctx, void* stream);
+
+/* select_and_attend with the far clusters attended from the fp8 copy ([EXPL] section 7).
+ * The selection is exactly select_and_attend's. Then a selected cluster whose walk rank
+ * (its position in the descending-score walk over all C clusters, ties to the lower index,
+ * rank 0 first) is >= n_near is attended from its fp8 rows, x = e4m3(code) * scale; this
+ * includes the partial rows of the cut cluster when its rank is >= n_near. Sinks, pending
+ * rows and clusters of rank < n_near are attended in bf16 as usual. n_near >= C attends
+ * everything in bf16 (the result then equals select_and_attend's); n_near = 0 attends every
+ * clustered row from the copy. A far row moves 264 bytes (codes and scales of K and V)
+ * instead of 512.
+ *   n_near : >= 0 (CKV_EINVAL otherwise). Other arguments as for select_and_attend.
+ * CKV_ESTATE without ckv_enable_fp8. */
+CKV_API int select_and_attend_mixed(ckv_ctx* ctx, int32_t layer, const void* q, int32_t budget,
+                                    int32_t n_near, float* out, int32_t* sel_idx,
+                                    int32_t* sel_count, void* stream);
+
+/* Copy of one unit's fp8 rows (layouts: k8, v8 uint8 [m, 128]; ks, vs fp32 [m]); any NULL
+ * pointer is skipped, host or device buffers. Synchronises `stream`. CKV_ESTATE without
+ * ckv_enable_fp8 or before the layer is clustered. */
+CKV_API int ckv_export_unit_fp8(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h, void* k8,
+                                float* ks, void* v8, float* vs, void* stream);
+
+/* Test hook for failure detection (the pages have no counterpart). Every wait inside the
+ * library's kernels is bounded: when it runs out, the kernel sets the context's device error
+ * word and unwinds, and ckv_check_device_error returns CKV_ETIMEOUT. This call makes one such
+ * wait run out on purpose, with no fault: a one-thread kernel waits with the given limit on
+ * an mbarrier that nothing completes, then sets the error word and returns.
+ *   limit_ns  : the wait's limit, 1 us .. 1 s (CKV_EINVAL outside).
+ *   waited_ns : optional device uint32 [1], the time the wait took (ns, saturating).
+ * Asynchronous on `stream`; the context stays usable afterwards. */
+CKV_API int ckv_debug_expire_wait(ckv_ctx* ctx, uint64_t limit_ns, uint32_t* waited_ns, void* stream);
 
 /* ---- Stage-level K-means calls: the same kernels cluster_prefill runs, exposed so that
  * each stage can be checked on its own. They run on U units whose keys are rows

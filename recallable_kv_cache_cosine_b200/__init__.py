@@ -62,11 +62,15 @@ SIGNATURES = {
     "recluster_increment_traced": (C.c_int, [P, I32, P, P, P]),
     "recluster_begin": (C.c_int, [P, I32, P]),
     "recluster_finish": (C.c_int, [P, I32, P]),
-    "split_drifted_clusters": (C.c_int, [P, I32, C.c_float, P, P, P]),
+    "split_drifted_clusters": (C.c_int, [P, I32, C.c_float, I32, P, P, P]),
     "ckv_get_layer_info": (C.c_int, [P, I32, P]),
     "ckv_export_unit": (C.c_int, [P, I32, I32, I32, P, P]),
     "ckv_import_unit": (C.c_int, [P, I32, I32, I32, I64, I32, I32, P, P]),
     "ckv_check_device_error": (C.c_int, [P, P]),
+    "ckv_debug_expire_wait": (C.c_int, [P, U64, P, P]),
+    "ckv_enable_fp8": (C.c_int, [P, P]),
+    "select_and_attend_mixed": (C.c_int, [P, I32, P, I32, I32, P, P, P, P]),
+    "ckv_export_unit_fp8": (C.c_int, [P, I32, I32, I32, P, P, P, P, P]),
     "ckv_kmeans_init": (C.c_int, [P, P, I64, I64, I64, I32, I32, U64, I64, U64, P, P, P, P]),
     "ckv_kmeans_assign": (C.c_int, [P, P, I64, I64, I64, I32, P, I32, P, P]),
     "ckv_kmeans_update": (C.c_int, [P, P, I64, I64, I64, I32, P, I32, P, P, P, P, P]),
@@ -199,20 +203,23 @@ class ClusterKV:
         """Makes `stream` wait for that re-clustering and switches the layer to its clusters."""
         _check(lib().recluster_finish(self._ctx, layer, _stream(stream)), "recluster_finish")
 
-    def split_drifted_clusters(self, layer: int, threshold: float, drift: torch.Tensor | None = None,
-                               stream=None) -> list[int]:
+    def split_drifted_clusters(self, layer: int, threshold: float, max_splits: int,
+                               drift: torch.Tensor | None = None, splits: torch.Tensor | None = None,
+                               stream=None) -> torch.Tensor:
         """Splits the layer's clusters whose drift (mean cosine distance of the members to
-        the centroid) is above `threshold`. drift: optional CUDA float32 [units, C] that
-        receives every cluster's drift. Returns the clusters split per unit. Synchronises
-        the stream."""
+        the centroid) is above `threshold`, at most `max_splits` per unit; the layer's
+        cluster count grows by exactly min(max_splits, room left). drift: optional CUDA
+        float32 [units, C] receiving every cluster's drift; splits: optional CUDA int32
+        [units] receiving the clusters split per unit (both filled asynchronously). Returns
+        `splits`."""
         if drift is not None and (drift.dtype != torch.float32 or not drift.is_cuda):
             raise TypeError("drift must be a CUDA float32 tensor")
-        U = self.cfg.batch * self.cfg.n_kv_heads
-        splits = (C.c_int32 * U)()
-        _check(lib().split_drifted_clusters(self._ctx, layer, float(threshold), _ptr(drift),
-                                            C.cast(splits, C.c_void_p), _stream(stream)),
+        if splits is not None and (splits.dtype != torch.int32 or not splits.is_cuda):
+            raise TypeError("splits must be a CUDA int32 tensor")
+        _check(lib().split_drifted_clusters(self._ctx, layer, float(threshold), int(max_splits),
+                                            _ptr(drift), _ptr(splits), _stream(stream)),
                "split_drifted_clusters")
-        return list(splits)
+        return splits
 
     # -- inspection
     def layer_info(self, layer: int) -> LayerInfo:
@@ -251,6 +258,35 @@ class ClusterKV:
 
     def check_device_error(self, stream=None):
         _check(lib().ckv_check_device_error(self._ctx, _stream(stream)), "ckv_check_device_error")
+
+    def enable_fp8(self, stream=None):
+        """Keep an fp8 (e4m3, per-row scale) copy of every layer's clustered rows."""
+        _check(lib().ckv_enable_fp8(self._ctx, _stream(stream)), "ckv_enable_fp8")
+
+    def select_and_attend_mixed(self, layer: int, q, budget: int, n_near: int, out, sel_idx=None,
+                                sel_count=None, stream=None):
+        """select_and_attend with clusters at walk rank >= n_near attended from the fp8 copy."""
+        _check(lib().select_and_attend_mixed(self._ctx, layer, _bf16(q, "q"), budget, n_near, _ptr(out),
+                                             _ptr(sel_idx), _ptr(sel_count), _stream(stream)),
+               "select_and_attend_mixed")
+        return out
+
+    def export_unit_fp8(self, layer: int, b: int, h: int, stream=None):
+        """One unit's fp8 copy as CPU tensors: k8, v8 uint8 [m, 128]; ks, vs float32 [m]."""
+        m = self.layer_info(layer).m
+        k8 = torch.empty(m, 128, dtype=torch.uint8)
+        v8 = torch.empty_like(k8)
+        ks = torch.empty(m, dtype=torch.float32)
+        vs = torch.empty_like(ks)
+        _check(lib().ckv_export_unit_fp8(self._ctx, layer, b, h, _ptr(k8), _ptr(ks), _ptr(v8), _ptr(vs),
+                                         _stream(stream)), "ckv_export_unit_fp8")
+        return {"k8": k8, "ks": ks, "v8": v8, "vs": vs}
+
+    def debug_expire_wait(self, limit_ns: int, waited_ns=None, stream=None):
+        """Test hook: one bounded device wait that nothing completes runs out after
+        ``limit_ns``; the error word is then set (see ``check_device_error``)."""
+        _check(lib().ckv_debug_expire_wait(self._ctx, int(limit_ns), _ptr(waited_ns), _stream(stream)),
+               "ckv_debug_expire_wait")
 
     # -- stage-level K-means calls (same kernels as cluster_prefill)
     def kmeans_init(self, keys, row0, m, C_, seed, unit_base=0, window=0, init_idx=None, mu=None,

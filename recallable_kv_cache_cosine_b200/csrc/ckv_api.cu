@@ -135,11 +135,20 @@ int dev_alloc(T** p, size_t count, Ctx* c) {
 void free_all(Ctx* c) {
     void* ptrs[] = {c->kp, c->vp, c->spk, c->spv, c->ids, c->offsets, c->mu, c->ws.mu_hat,
                     c->ws.assign, c->ws.best, c->ws.perm, c->ws.chunk, c->ws.part, c->err,
-                    c->split.drift, c->split.plan, c->split.count, c->split.cmu, c->split.n0,
+                    c->split.drift, c->split.plan, c->split.count, c->split.tasks, c->split.cmu, c->split.n0,
                     c->split.mu2, c->split.off2, c->split.lab, c->split.rk, c->split.rv,
-                    c->split.rid};
+                    c->split.rid, c->kp8, c->vp8, c->ks8, c->vs8};
     for (void* p : ptrs)
         if (p) cudaFree(p);
+}
+
+// Refreshes the fp8 copy of rows [r0, r0 + nrows) of every unit of a layer, when the copy is
+// kept (ckv_enable_fp8). Launched last by every call that writes those rows.
+int refresh_fp8(Ctx* c, int32_t layer, int64_t r0, int64_t nrows, cudaStream_t s) {
+    if (!c->kp8 || nrows <= 0) return CKV_OK;
+    const int64_t o = c->rows_kp(layer, 0);
+    return launch_quantize_rows(c->kp + o * kD, c->vp + o * kD, c->kp8 + o * kD, c->vp8 + o * kD,
+                                c->ks8 + o, c->vs8 + o, c->cap_c, r0, nrows, c->units, s);
 }
 
 // Checks and launches the re-clustering of layer's full window (the `window` oldest pending
@@ -183,7 +192,9 @@ int launch_window_recluster(Ctx* c, int32_t layer, float* mu_trace, int32_t* ass
     a.mu_ustride = c->cfg.max_clusters;
     a.mu_trace = mu_trace;
     a.assign_trace = assign_trace;
-    return launch_recluster(a, stream);
+    int rc = launch_recluster(a, stream);
+    if (rc) return rc;
+    return refresh_fp8(c, layer, L.m, c->cfg.window, stream);
 }
 
 // The window's tokens join the cluster store: the layer's host state after a re-clustering.
@@ -202,6 +213,7 @@ int ensure_split_scratch(Ctx* c) {
     if (!sp.drift) rc = dev_alloc(&sp.drift, U * cmax, c);
     if (!rc && !sp.plan) rc = dev_alloc(&sp.plan, U * cmax, c);
     if (!rc && !sp.count) rc = dev_alloc(&sp.count, U, c);
+    if (!rc && !sp.tasks) rc = dev_alloc(&sp.tasks, U * cmax, c);
     if (!rc && !sp.cmu) rc = dev_alloc(&sp.cmu, U * cmax * 2 * kD, c);
     if (!rc && !sp.n0) rc = dev_alloc(&sp.n0, U * cmax, c);
     if (!rc && !sp.mu2) rc = dev_alloc(&sp.mu2, U * cmax * kD, c);
@@ -214,7 +226,8 @@ int ensure_split_scratch(Ctx* c) {
 }
 
 int decode_call(ckv_ctx* ctx, int32_t layer, const void* q, int32_t budget, float* out,
-                int32_t* sel_idx, int32_t* sel_count, void* stream, bool per_head) {
+                int32_t* sel_idx, int32_t* sel_count, void* stream, bool per_head,
+                int32_t n_near = -1) {
     int rc = check_ctx(ctx);
     if (rc) return rc;
     Ctx* c = C_(ctx);
@@ -260,6 +273,19 @@ int decode_call(ckv_ctx* ctx, int32_t layer, const void* q, int32_t budget, floa
     a.part_scratch = c->ws.part;
     a.part_ustride = c->cap_c;
     a.err = c->err;
+    if (n_near >= 0) {  // mixed precision: far clusters from the fp8 copy
+        if (!c->kp8) {
+            set_error("select_and_attend_mixed needs the fp8 copy: call ckv_enable_fp8 first");
+            return CKV_ESTATE;
+        }
+        const int64_t o = c->rows_kp(layer, 0);
+        a.kp8 = c->kp8 + o * kD;
+        a.vp8 = c->vp8 + o * kD;
+        a.ks8 = c->ks8 + o;
+        a.vs8 = c->vs8 + o;
+        a.n_near = n_near;
+        return launch_select_attend_mixed(a, c->num_sms, (cudaStream_t)stream);
+    }
     return per_head ? launch_select_attend_per_head(a, c->num_sms, (cudaStream_t)stream)
                     : launch_select_attend(a, c->num_sms, (cudaStream_t)stream);
 }
@@ -434,6 +460,7 @@ int cluster_prefill(ckv_ctx* ctx, int32_t layer, const void* K, const void* V, i
                                c->spv + c->rows_sp(layer, 0) * kD, c->sp_rows, s);
         if (rc) return rc;
     }
+    if ((rc = refresh_fp8(c, layer, 0, n - ns, s))) return rc;
     LayerState& L = c->layers[(size_t)layer];
     L.prefilled = 1;
     L.m = n - ns;
@@ -452,6 +479,13 @@ int select_and_attend(ckv_ctx* ctx, int32_t layer, const void* q, int32_t budget
 int select_and_attend_per_head(ckv_ctx* ctx, int32_t layer, const void* q, int32_t budget,
                                float* out, int32_t* sel_idx, int32_t* sel_count, void* stream) {
     return decode_call(ctx, layer, q, budget, out, sel_idx, sel_count, stream, true);
+}
+
+int select_and_attend_mixed(ckv_ctx* ctx, int32_t layer, const void* q, int32_t budget,
+                            int32_t n_near, float* out, int32_t* sel_idx, int32_t* sel_count,
+                            void* stream) {
+    if (n_near < 0) return einval("n_near must be >= 0");
+    return decode_call(ctx, layer, q, budget, out, sel_idx, sel_count, stream, false, n_near);
 }
 
 int ckv_append_kv(ckv_ctx* ctx, int32_t layer, const void* k, const void* v, void* stream) {
@@ -537,8 +571,8 @@ int recluster_finish(ckv_ctx* ctx, int32_t layer, void* stream) {
     return CKV_OK;
 }
 
-int split_drifted_clusters(ckv_ctx* ctx, int32_t layer, float threshold, float* drift,
-                           int32_t* splits, void* stream) {
+int split_drifted_clusters(ckv_ctx* ctx, int32_t layer, float threshold, int32_t max_splits,
+                           float* drift, int32_t* splits, void* stream) {
     int rc = check_ctx(ctx);
     if (rc) return rc;
     Ctx* c = C_(ctx);
@@ -550,7 +584,9 @@ int split_drifted_clusters(ckv_ctx* ctx, int32_t layer, float threshold, float* 
         return CKV_ESTATE;
     }
     if (threshold != threshold) return einval("threshold is NaN");
+    if (max_splits < 0) return einval("max_splits must be >= 0");
     if (drift && ((uintptr_t)drift & 3u)) return einval("drift must be 4-byte aligned");
+    if (splits && ((uintptr_t)splits & 3u)) return einval("splits must be 4-byte aligned");
     if (c->units > 65535) return einval("more than 65535 units per layer");
     if ((rc = ensure_split_scratch(c))) return rc;
     cudaStream_t s = (cudaStream_t)stream;
@@ -558,7 +594,7 @@ int split_drifted_clusters(ckv_ctx* ctx, int32_t layer, float threshold, float* 
     a.U = c->units;
     a.C = L.C;
     a.Cmax = c->cfg.max_clusters;
-    a.room = c->cfg.max_clusters - L.C;
+    a.room = std::min(max_splits, c->cfg.max_clusters - L.C);
     a.iters = c->cfg.iters;
     a.m = L.m;
     a.tau = threshold;
@@ -577,6 +613,7 @@ int split_drifted_clusters(ckv_ctx* ctx, int32_t layer, float threshold, float* 
     a.drift_out = drift;
     a.plan = c->split.plan;
     a.count = c->split.count;
+    a.tasks = c->split.tasks;
     a.cmu = c->split.cmu;
     a.n0 = c->split.n0;
     a.mu2 = c->split.mu2;
@@ -587,15 +624,13 @@ int split_drifted_clusters(ckv_ctx* ctx, int32_t layer, float threshold, float* 
     a.rid = c->split.rid;
     a.err = c->err;
     if ((rc = launch_split(a, s))) return rc;
-    std::vector<int32_t> cnt((size_t)c->units);
-    cudaError_t e = cudaMemcpyAsync(cnt.data(), c->split.count, sizeof(int32_t) * cnt.size(),
-                                    cudaMemcpyDeviceToHost, s);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-    if (e != cudaSuccess) return cuda_fail(e, "split: read split counts");
-    int32_t mx = 0;
-    for (int32_t v : cnt) mx = std::max(mx, v);
-    L.C += mx;
-    if (splits) std::copy(cnt.begin(), cnt.end(), splits);
+    if ((rc = refresh_fp8(c, layer, 0, L.m, s))) return rc;
+    if (splits) {  // the per-unit split counts, left on the device
+        cudaError_t e = cudaMemcpyAsync(splits, c->split.count, sizeof(int32_t) * (size_t)c->units,
+                                        cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) return cuda_fail(e, "split: copy split counts");
+    }
+    L.C += a.room;
     return CKV_OK;
 }
 
@@ -715,6 +750,12 @@ int ckv_import_unit(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h, int64_t m
         e = cudaMemcpyAsync(it.d, it.s, it.n, cudaMemcpyDefault, s);
         if (e != cudaSuccess) return cuda_fail(e, "import: copy");
     }
+    if (c->kp8 && m > 0) {  // the unit's fp8 copy
+        const int64_t o = c->rows_kp(layer, u);
+        rc = launch_quantize_rows(c->kp + o * kD, c->vp + o * kD, c->kp8 + o * kD, c->vp8 + o * kD,
+                                  c->ks8 + o, c->vs8 + o, c->cap_c, 0, m, 1, s);
+        if (rc) return rc;
+    }
     e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e, "import: sync");
     if (first) {
@@ -749,6 +790,74 @@ int ckv_check_device_error(ckv_ctx* ctx, void* stream) {
         return CKV_EINVAL;
     }
     return CKV_OK;
+}
+
+int ckv_enable_fp8(ckv_ctx* ctx, void* stream) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    Ctx* c = C_(ctx);
+    if (!c->kp8) {
+        const size_t rows = (size_t)c->cfg.n_layers * c->units * c->cap_c;
+        uint8_t *k8 = nullptr, *v8 = nullptr;
+        float *ks = nullptr, *vs = nullptr;
+        rc = dev_alloc(&k8, rows * kD, c);
+        if (!rc) rc = dev_alloc(&v8, rows * kD, c);
+        if (!rc) rc = dev_alloc(&ks, rows, c);
+        if (!rc) rc = dev_alloc(&vs, rows, c);
+        if (rc) {
+            for (void* p : {(void*)k8, (void*)v8, (void*)ks, (void*)vs})
+                if (p) cudaFree(p);
+            return rc;
+        }
+        c->kp8 = k8;
+        c->vp8 = v8;
+        c->ks8 = ks;
+        c->vs8 = vs;
+    }
+    for (int32_t l = 0; l < c->cfg.n_layers; ++l) {
+        const LayerState& L = c->layers[(size_t)l];
+        if (L.prefilled && (rc = refresh_fp8(c, l, 0, L.m, (cudaStream_t)stream))) return rc;
+    }
+    return CKV_OK;
+}
+
+int ckv_export_unit_fp8(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h, void* k8, float* ks,
+                        void* v8, float* vs, void* stream) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    Ctx* c = C_(ctx);
+    if ((rc = check_layer(c, layer))) return rc;
+    if (b < 0 || b >= c->cfg.batch || h < 0 || h >= c->cfg.n_kv_heads) return einval("unit out of range");
+    if (!c->kp8) {
+        set_error("no fp8 copy: call ckv_enable_fp8 first");
+        return CKV_ESTATE;
+    }
+    const LayerState& L = c->layers[(size_t)layer];
+    if (!L.prefilled) {
+        set_error("layer not prefilled");
+        return CKV_ESTATE;
+    }
+    const int64_t o = c->rows_kp(layer, b * c->cfg.n_kv_heads + h);
+    cudaStream_t s = (cudaStream_t)stream;
+    struct Item { void* d; const void* s; size_t n; } items[] = {
+        {k8, c->kp8 + o * kD, (size_t)L.m * kD}, {v8, c->vp8 + o * kD, (size_t)L.m * kD},
+        {ks, c->ks8 + o, sizeof(float) * (size_t)L.m}, {vs, c->vs8 + o, sizeof(float) * (size_t)L.m}};
+    for (auto& it : items) {
+        if (!it.d || it.n == 0) continue;
+        cudaError_t e = cudaMemcpyAsync(it.d, it.s, it.n, cudaMemcpyDefault, s);
+        if (e != cudaSuccess) return cuda_fail(e, "export fp8: copy");
+    }
+    cudaError_t e = cudaStreamSynchronize(s);
+    return e == cudaSuccess ? CKV_OK : cuda_fail(e, "export fp8: sync");
+}
+
+int ckv_debug_expire_wait(ckv_ctx* ctx, uint64_t limit_ns, uint32_t* waited_ns, void* stream) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    if (limit_ns < 1000 || limit_ns > 1000000000ull)
+        return einval("limit_ns must be in [1 us, 1 s]");
+    if (waited_ns && ((uintptr_t)waited_ns & 3u)) return einval("waited_ns must be 4-byte aligned");
+    return launch_expire_wait(C_(ctx)->err, limit_ns, waited_ns, (cudaStream_t)stream);
 }
 
 static int check_stage(const Ctx* c, const void* keys, int64_t n_rows, int64_t row0, int64_t m,

@@ -55,17 +55,21 @@ CKV_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait on the phase with the given parity. Returns false (and sets *err) on timeout.
-CKV_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+// Bounded wait on the phase with the given parity, giving up after `limit_ns`. Returns false
+// (and sets *err) on timeout.
+CKV_DEV bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint32_t* err, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 255u && globaltimer() - t0 > kWaitNs) {
+        if ((it & 255u) == 255u && globaltimer() - t0 > limit_ns) {
             if (err) atomicOr(err, kErrTimeout);
             return false;
         }
     }
+}
+CKV_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+    return mbar_wait_for(bar, parity, err, kWaitNs);
 }
 
 // ------------------------------------------------------------------ TMA

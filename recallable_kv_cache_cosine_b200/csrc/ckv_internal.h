@@ -53,6 +53,7 @@ struct SplitScratch {
     float* drift = nullptr;   // [U][Cmax] drift of every cluster
     int32_t* plan = nullptr;  // [U][Cmax] 2 * new index + split flag
     int32_t* count = nullptr; // [U] splits per unit
+    int32_t* tasks = nullptr; // [U][Cmax] clusters to split, in index order
     float* cmu = nullptr;     // [U][Cmax][2][128] centroids of the two halves
     int32_t* n0 = nullptr;    // [U][Cmax] rows of the first half
     float* mu2 = nullptr;     // [U][Cmax][128] centroids at their new indices
@@ -80,6 +81,12 @@ struct Ctx {
     int32_t* ids = nullptr;
     int32_t* offsets = nullptr;
     float* mu = nullptr;
+    // fp8 (e4m3) copy of the clustered rows with per-row scales, [L][U][cap_c] rows; allocated
+    // by ckv_enable_fp8 and kept current by every call that writes the store afterwards.
+    uint8_t* kp8 = nullptr;
+    uint8_t* vp8 = nullptr;
+    float* ks8 = nullptr;
+    float* vs8 = nullptr;
     Workspace ws;
     SplitScratch split;
     uint32_t* err = nullptr;  // device error word
@@ -177,10 +184,20 @@ struct DecodeArgs {
     float* part_scratch;  // [U][cap]
     int64_t part_ustride;
     uint32_t* err;
+    // mixed precision (select_and_attend_mixed): clusters at walk rank >= n_near are attended
+    // from the fp8 copy (same row layout as kp / vp)
+    const uint8_t* kp8;
+    const uint8_t* vp8;
+    const float* ks8;
+    const float* vs8;
+    int32_t n_near;
 };
 // Launch with programmatic dependent launch allowed: the kernel may be scheduled while the
 // previous kernel in the stream is still running. Every kernel launched this way calls
-// pdl_wait() before it touches memory that earlier work writes, so stream order holds.
+// pdl_wait() before it touches memory that earlier work writes, so stream order holds. The
+// one exception is the decode kernel, which reads the cluster store before its wait: the last
+// kernel of every call that writes the store therefore does not trigger its dependents early
+// (they start when it ends).
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
                               cudaStream_t s, Args&&... args) {
@@ -197,8 +214,17 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// fp8 copy of rows [r0, r0 + nrows) of U units (stride ustride rows); no early trigger.
+int launch_quantize_rows(const uint16_t* kp, const uint16_t* vp, uint8_t* kp8, uint8_t* vp8,
+                         float* ks, float* vs, int64_t ustride, int64_t r0, int64_t nrows,
+                         int32_t U, cudaStream_t s);
+
+// One bounded mbarrier wait that nothing completes, with the given limit (test hook).
+int launch_expire_wait(uint32_t* err, uint64_t limit_ns, uint32_t* waited_ns, cudaStream_t s);
+
 int launch_select_attend(const DecodeArgs& a, int num_sms, cudaStream_t s);
 int launch_select_attend_per_head(const DecodeArgs& a, int num_sms, cudaStream_t s);
+int launch_select_attend_mixed(const DecodeArgs& a, int num_sms, cudaStream_t s);
 
 int launch_append(const uint16_t* k, const uint16_t* v, int32_t U, uint16_t* spk, uint16_t* spv,
                   int64_t sp_ustride_rows, int32_t row, cudaStream_t s);
@@ -247,6 +273,7 @@ struct SplitArgs {
     float* drift_out;     // optional [U][C]
     int32_t* plan;
     int32_t* count;
+    int32_t* tasks;
     float* cmu;
     int32_t* n0;
     float* mu2;
@@ -257,8 +284,8 @@ struct SplitArgs {
     int32_t* rid;
     uint32_t* err;
 };
-// Drift, plan, 2-means split and renumbering of one layer (five launches on `s`). The new
-// cluster count is C + max over units of count[u].
+// Drift, plan, 2-means split and renumbering of one layer (five launches on `s`). Every unit
+// ends with C + room clusters (padding with empty clusters where it split fewer).
 int launch_split(const SplitArgs& a, cudaStream_t s);
 
 }  // namespace ckv

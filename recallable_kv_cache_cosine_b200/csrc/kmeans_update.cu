@@ -46,72 +46,58 @@ CKV_DEV float4 load_row4_bf16(const uint16_t* row) {
 // ---------------------------------------------------------------------- init
 // Seeded init: the first C entries of a Fisher-Yates shuffle of 0..m-1, driven by SplitMix64
 // with key seed ^ (unit << 32) ^ window, each draw mapped into [0, m-i) by Lemire's
-// multiply-shift. SplitMix64 is counter-based (draw i mixes key + (i+1) * gamma), so the C
-// swap targets are computed in parallel. Only the swaps run in order, on a dense
-// shared-memory copy of the index array when it fits (`dense`, chosen by the host from the
-// shared-memory size), otherwise on an open-addressing table of the <= C displaced positions.
-constexpr size_t kInitSmemLimit = 200 * 1024;
-
+// multiply-shift. The sequential shuffle is: for i < C, j_i = i + draw_i; chosen[i] = a[j_i];
+// a[j_i] = a[i] (position i is never read again). SplitMix64 is counter-based, so every j_i
+// is computed at once, and every chosen[i] is resolved without the loop: a position p >= i
+// changed before step i only as the target of an earlier step, so a[p] before step i is the
+// value position s held just before step s, s being the last step < i with j_s = p (prev[i]),
+// or p itself if there is none; and the value position s held before step s is, by the same
+// rule, found by following the last step < s with j = s (link[s]) until a step whose own
+// position was never a target: that step's index is the value. Each thread scans the earlier
+// targets for its steps (C^2 / 2 shared-memory compares per unit) and follows the short chains.
 __global__ void __launch_bounds__(256) kmeans_init_kernel(KeysView k, int32_t C, uint64_t seed,
                                                           int64_t unit_base, uint64_t window,
                                                           int32_t* init_idx, float* mu,
                                                           int64_t mu_ustride, uint16_t* mu_hat,
-                                                          int64_t muhat_ustride, int32_t tbits,
-                                                          int32_t dense) {
+                                                          int64_t muhat_ustride) {
     pdl_launch_dependents();  // let the next kernel in the stream be scheduled early
     pdl_wait();               // the previous kernel's writes are visible from here on
     extern __shared__ int32_t sm[];
     const int u = blockIdx.x;
     const int32_t m = (int32_t)k.m;
-    int32_t* target = sm;          // [C] swap target of step i
-    int32_t* chosen = sm + C;      // [C]
-    int32_t* work = sm + 2 * C;    // dense [m] array, or table keys [2^tbits] + values [2^tbits]
+    int32_t* target = sm;        // [C] j_i
+    int32_t* prev = sm + C;      // [C] last earlier step with the same target, or -1
+    int32_t* link = sm + 2 * C;  // [C] last earlier step whose target is this step, or -1
     const uint64_t key = seed ^ ((uint64_t)(unit_base + u) << 32) ^ window;
     for (int i = threadIdx.x; i < C; i += blockDim.x) {
         uint64_t st = key + (uint64_t)i * 0x9E3779B97F4A7C15ull;  // state before draw i
         const uint64_t x = splitmix64_next(st);
         target[i] = i + (int32_t)bounded_draw(x, (uint32_t)(m - i));
     }
-    const int32_t tsize = 1 << tbits;
-    if (dense) {
-        for (int i = threadIdx.x; i < m; i += blockDim.x) work[i] = i;
-    } else {
-        for (int i = threadIdx.x; i < tsize; i += blockDim.x) work[i] = -1;
-    }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        if (dense) {
-            for (int32_t i = 0; i < C; ++i) {
-                const int32_t j = target[i];
-                const int32_t vj = work[j];
-                work[j] = work[i];  // position i is never read again
-                chosen[i] = vj;
-            }
-        } else {
-            int32_t* tkey = work;
-            int32_t* tval = work + tsize;
-            auto slot = [&](int32_t pos) -> int32_t {
-                uint32_t hsh = ((uint32_t)pos * 2654435761u) >> (32 - tbits);
-                while (tkey[hsh] != -1 && tkey[hsh] != pos) hsh = (hsh + 1) & (uint32_t)(tsize - 1);
-                return (int32_t)hsh;
-            };
-            for (int32_t i = 0; i < C; ++i) {
-                const int32_t j = target[i];
-                const int32_t si = slot(i);
-                const int32_t vi = tkey[si] == i ? tval[si] : i;
-                const int32_t sj = slot(j);
-                const int32_t vj = tkey[sj] == j ? tval[sj] : j;
-                tkey[sj] = j;  // a[j] <- old a[i]; position i is never read again
-                tval[sj] = vi;
-                chosen[i] = vj;
-            }
+    for (int t = threadIdx.x; t < C; t += blockDim.x) {
+        const int32_t p = target[t];
+        int32_t pv = -1, lv = -1;
+        for (int s = t - 1; s >= 0 && (pv < 0 || lv < 0); --s) {
+            const int32_t ts = target[s];
+            if (pv < 0 && ts == p) pv = s;
+            if (lv < 0 && ts == t) lv = s;
         }
+        prev[t] = pv;
+        link[t] = lv;
     }
     __syncthreads();
     const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     const uint16_t* keys = k.base + ((int64_t)u * k.n_rows + k.row0) * kD;
     for (int c = warp; c < C; c += nw) {
-        const int32_t idx = chosen[c];
+        int32_t x = prev[c];
+        int32_t idx;
+        if (x < 0) {
+            idx = target[c];
+        } else {
+            while (link[x] >= 0) x = link[x];  // every step strictly lowers x
+            idx = x;
+        }
         const float4 v = load_row4_bf16(keys + (int64_t)idx * kD);
         store_centroid(v, mu + ((int64_t)u * mu_ustride + c) * kD,
                        mu_hat + ((int64_t)u * muhat_ustride + c) * kD);
@@ -212,63 +198,65 @@ __global__ void __launch_bounds__(1024) kmeans_scan_kernel(int32_t* chunk, int32
 }
 
 // ---------------------------------------------------------------------- scatter
-// One warp per chunk, keys in index order, 32 at a time: lanes with equal clusters are
-// grouped with match.any and ranked by lane. This gives a stable counting sort.
-__global__ void __launch_bounds__(32) kmeans_scatter_kernel(const int32_t* assign, int64_t a_ustride,
-                                                            int64_t m, int32_t C, int32_t nch,
-                                                            const int32_t* chunk,
-                                                            const int32_t* offsets,
-                                                            int64_t off_ustride, int32_t* perm,
-                                                            int64_t perm_ustride) {
+// One CTA of 8 warps per chunk of 1024 keys. Warp w takes keys [128 w, 128 w + 128) of the
+// chunk, 32 at a time in index order: lanes with equal clusters are grouped with match.any and
+// ranked by lane on top of the warp's running count of that cluster. Then, per cluster, a scan
+// over the 8 warps starting at the cluster's offset plus the chunk's prefix gives each warp's
+// first position, and every key lands at that position plus its rank. Keys of one cluster
+// therefore keep their index order: a stable counting sort.
+constexpr int kScatterWarps = 8;
+constexpr int kScatterKeysPerWarp = kChunk / kScatterWarps;  // 128
+
+__global__ void __launch_bounds__(kScatterWarps * 32) kmeans_scatter_kernel(
+    const int32_t* assign, int64_t a_ustride, int64_t m, int32_t C, int32_t nch,
+    const int32_t* chunk, const int32_t* offsets, int64_t off_ustride, int32_t* perm,
+    int64_t perm_ustride) {
     pdl_launch_dependents();  // let the next kernel in the stream be scheduled early
     pdl_wait();               // the previous kernel's writes are visible from here on
-    extern __shared__ int32_t cnt[];  // [C] counters, then [kChunk] assignments
-    int32_t* sa = cnt + C;
+    extern __shared__ int32_t cntw[];  // [kScatterWarps][C] counts, then first positions
+    int32_t* sa = cntw + kScatterWarps * C;  // [kChunk] assignments (-1: none / out of range)
+    int32_t* srank = sa + kChunk;            // [kChunk] rank among the warp's keys of its cluster
     const int ch = blockIdx.x, u = blockIdx.y;
-    const int lane = threadIdx.x;
-    const int32_t* base = chunk + ((int64_t)u * nch + ch) * C;
-    const int32_t* off = offsets + (int64_t)u * off_ustride;
-    const int32_t* a = assign + (int64_t)u * a_ustride;
-    int32_t* pm = perm + (int64_t)u * perm_ustride;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t lo = (int64_t)ch * kChunk;
     const int64_t hi = lo + kChunk < m ? lo + kChunk : m;
-    // Stage the counters and the chunk's assignments in shared memory with all loads in
-    // flight, so the sequential loop below touches shared memory only.
-    static_assert(kChunk == 1024, "the staging below loads 32 assignments per lane");
-    int32_t av[32];
-#pragma unroll
-    for (int t = 0; t < 32; ++t) {
-        const int64_t i = lo + t * 32 + lane;
-        av[t] = i < hi ? a[i] : -1;
-    }
-    for (int c0 = 0; c0 < C; c0 += 32 * 16) {
-        int32_t o[16], bb[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            const int c = c0 + t * 32 + lane;
-            o[t] = c < C ? off[c] : 0;
-            bb[t] = c < C ? base[c] : 0;
-        }
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            const int c = c0 + t * 32 + lane;
-            if (c < C) cnt[c] = o[t] + bb[t];
-        }
-    }
-#pragma unroll
-    for (int t = 0; t < 32; ++t) sa[t * 32 + lane] = av[t];
-    __syncwarp();
-    const uint32_t lt = (1u << lane) - 1u;
-    for (int64_t i0 = lo; i0 < hi; i0 += 32) {
-        const int64_t i = i0 + lane;
-        int32_t c = sa[i - lo];
+    const int32_t* a = assign + (int64_t)u * a_ustride;
+    for (int i = tid; i < kChunk; i += kScatterWarps * 32) {
+        int32_t c = lo + i < hi ? a[lo + i] : -1;
         if ((uint32_t)c >= (uint32_t)C) c = -1;  // out of range (flagged by the count kernel)
+        sa[i] = c;
+    }
+    for (int i = tid; i < kScatterWarps * C; i += kScatterWarps * 32) cntw[i] = 0;
+    __syncthreads();
+    int32_t* mine = cntw + warp * C;
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int r = 0; r < kScatterKeysPerWarp / 32; ++r) {  // warp-uniform trip count
+        const int i = warp * kScatterKeysPerWarp + r * 32 + lane;
+        const int32_t c = sa[i];
         const uint32_t same = __match_any_sync(0xffffffffu, c);
-        const int32_t pos = c >= 0 ? cnt[c] + __popc(same & lt) : 0;
+        const int32_t before = c >= 0 ? mine[c] : 0;
         __syncwarp();
-        if (c >= 0 && (same & lt) == 0) cnt[c] += __popc(same);
+        if (c >= 0 && (same & lt) == 0) mine[c] = before + __popc(same);
+        srank[i] = before + __popc(same & lt);
         __syncwarp();
-        if (c >= 0) pm[pos] = (int32_t)i;
+    }
+    __syncthreads();
+    const int32_t* off = offsets + (int64_t)u * off_ustride;
+    const int32_t* base = chunk + ((int64_t)u * nch + ch) * C;
+    for (int c = tid; c < C; c += kScatterWarps * 32) {
+        int32_t run = off[c] + base[c];
+#pragma unroll
+        for (int w = 0; w < kScatterWarps; ++w) {
+            const int32_t t = cntw[w * C + c];
+            cntw[w * C + c] = run;
+            run += t;
+        }
+    }
+    __syncthreads();
+    int32_t* pm = perm + (int64_t)u * perm_ustride;
+    for (int i = tid; i < kChunk; i += kScatterWarps * 32) {
+        const int32_t c = sa[i];
+        if (c >= 0) pm[cntw[(i / kScatterKeysPerWarp) * C + c] + srank[i]] = (int32_t)(lo + i);
     }
 }
 
@@ -295,8 +283,10 @@ __global__ void __launch_bounds__(kMeanThreads) kmeans_mean_kernel(KeysView k, c
                                                                    uint16_t* mu_hat,
                                                                    int64_t muhat_ustride,
                                                                    Relayout rl) {
-    pdl_launch_dependents();  // let the next kernel in the stream be scheduled early
-    pdl_wait();               // the previous kernel's writes are visible from here on
+    // The relayout pass ends a prefill: it writes the cluster store, which the decode kernel
+    // reads before its own dependency wait, so it lets its dependents start only when it ends.
+    if (rl.kp == nullptr) pdl_launch_dependents();
+    pdl_wait();  // the previous kernel's writes are visible from here on
     static_assert(kMeanThreads == kD, "one thread per dimension");
     __shared__ __align__(16) uint16_t srow[kMeanRows * kD];
     __shared__ int32_t sidx[kMeanRows];
@@ -369,8 +359,9 @@ __global__ void __launch_bounds__(kMeanThreads) kmeans_mean_kernel(KeysView k, c
 
 __global__ void copy_sinks_kernel(const uint16_t* K, const uint16_t* V, int64_t n, int32_t n_sink,
                                   uint16_t* spk, uint16_t* spv, int64_t sp_ustride) {
-    pdl_launch_dependents();  // let the next kernel in the stream be scheduled early
-    pdl_wait();               // the previous kernel's writes are visible from here on
+    // The last kernel of a prefill: no early trigger, so a following decode kernel, which
+    // reads the cluster store before its dependency wait, starts once the store is complete.
+    pdl_wait();  // the previous kernel's writes are visible from here on
     const int u = blockIdx.x;
     const int64_t words = (int64_t)n_sink * kD / 8;  // 16-byte words
     const uint4* ks = reinterpret_cast<const uint4*>(K + (int64_t)u * n * kD);
@@ -389,16 +380,12 @@ int launch_kmeans_init(const KeysView& k, int32_t C, uint64_t seed, int64_t unit
                        uint64_t window, int32_t* init_idx, float* mu, int64_t mu_ustride,
                        uint16_t* mu_hat, int64_t muhat_ustride, uint32_t* err, cudaStream_t s) {
     (void)err;
-    int tbits = 6;
-    while ((1 << tbits) < 2 * C) ++tbits;
-    const bool dense = (2 * (size_t)C + (size_t)k.m) * sizeof(int32_t) <= kInitSmemLimit;
-    const size_t work = dense ? (size_t)k.m : (size_t)2 * (1 << tbits);
-    const size_t smem = (2 * (size_t)C + work) * sizeof(int32_t);
+    const size_t smem = 3 * (size_t)C * sizeof(int32_t);  // C <= 4096: at most 48 KB
     int rc = ensure_smem((const void*)kmeans_init_kernel, smem, "init: set smem");
     if (rc != CKV_OK) return rc;
     cudaError_t e;
     e = launch_pdl(kmeans_init_kernel, dim3(k.U), dim3(256), smem, s, k, C, seed, unit_base, window,
-                   init_idx, mu, mu_ustride, mu_hat, muhat_ustride, tbits, dense ? 1 : 0);
+                   init_idx, mu, mu_ustride, mu_hat, muhat_ustride);
     return e == cudaSuccess ? CKV_OK : cuda_fail(e, "init: launch");
 }
 
@@ -410,7 +397,7 @@ int launch_kmeans_update(const KeysView& k, const int32_t* assign, int64_t assig
     const int32_t nch = (int32_t)n_chunks(k.m);
     cudaError_t e;
     const size_t hsmem = (size_t)C * sizeof(int32_t);
-    const size_t scsmem = (size_t)(C + kChunk) * sizeof(int32_t);
+    const size_t scsmem = ((size_t)kScatterWarps * C + 2 * kChunk) * sizeof(int32_t);
     const size_t ssmem = (size_t)(C + 32) * sizeof(int32_t);
     int rc = ensure_smem((const void*)kmeans_count_kernel, hsmem, "count: set smem");
     if (rc == CKV_OK) rc = ensure_smem((const void*)kmeans_scatter_kernel, scsmem, "scatter: set smem");
@@ -425,7 +412,7 @@ int launch_kmeans_update(const KeysView& k, const int32_t* assign, int64_t assig
                    offsets, off_ustride);
     if (e != cudaSuccess) return cuda_fail(e, "update: scan launch");
     if (nch > 0) {
-        e = launch_pdl(kmeans_scatter_kernel, dim3(nch, k.U), dim3(32), scsmem, s, assign,
+        e = launch_pdl(kmeans_scatter_kernel, dim3(nch, k.U), dim3(kScatterWarps * 32), scsmem, s, assign,
                        assign_ustride, k.m, C, nch, chunk_ws, offsets, off_ustride, perm,
                        perm_ustride);
         if (e != cudaSuccess) return cuda_fail(e, "update: scatter launch");

@@ -23,7 +23,8 @@ namespace {
 constexpr int kRT = 512;
 
 __global__ void __launch_bounds__(kRT) recluster_kernel(const ReclusterArgs a) {
-    pdl_launch_dependents();  // let the next kernel in the stream be scheduled early
+    // No early trigger: this kernel writes the cluster store (new rows, offsets and
+    // centroids), which the decode kernel reads before its dependency wait.
     pdl_wait();               // the previous kernel's writes are visible from here on
     extern __shared__ __align__(16) uint8_t smem_raw[];
     const int W = a.window, Cn = a.C_new;

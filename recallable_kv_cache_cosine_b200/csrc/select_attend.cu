@@ -12,35 +12,52 @@
 // lower cluster index and the lower token id; the 16 sinks and the pending tokens are always
 // attended and counted against the budget.
 //
-// One unit (sequence b, KV head h) is served by a thread-block cluster of S CTAs:
-//   1. each CTA scores a slice of the C centroids (fp32; a quarter-warp per centroid, the
-//      next round's loads in flight during the current one) and broadcasts the scores to
-//      every CTA of the cluster through distributed shared memory. Every CTA loads the
-//      cluster boundaries itself;
-//   2. every CTA then computes the whole selection on its own, without a second exchange:
-//      the walk in descending score order stops at the first cluster whose inclusive token
-//      count exceeds the remaining budget, so that cluster (the cut) is the weighted
-//      quantile of the scores with the cluster sizes as weights. The scores are mapped
-//      monotonically onto 256 linear buckets; a size-weighted histogram gives the bucket that
-//      holds the cut, and the clusters of that bucket and above (a dozen or so) are compacted
-//      and ranked exactly among themselves for their prefix sums;
+// One unit (sequence b, KV head h) is served by a thread-block cluster of S CTAs. The launch
+// is split around the programmatic-dependent-launch wait:
+//   0. before the wait, while the previous kernel of the stream may still run, each CTA
+//      bulk-copies its slice of the fp32 centroids into shared memory, loads the cluster
+//      boundaries and prefetches the queries and the sink / pending rows into L2. The store
+//      is only written by this library's own kernels, and the last kernel of every call that
+//      writes it signals its dependents only when it ends, so these reads see the finished
+//      store. The queries, the sink / pending rows and every output are touched only after
+//      the wait;
+//   1. qbar = sum of the group's queries; each CTA scores its slice (a warp per centroid,
+//      four in flight) and writes the scores into every CTA of the cluster through
+//      distributed shared memory;
+//   2. every CTA computes the same selection on its own. The walk in descending
+//      (score, -index) order stops at the first cluster whose inclusive token count exceeds
+//      the remaining budget R: the cut, a size-weighted quantile of the scores. The scores are
+//      mapped monotonically onto 256 linear buckets between the smallest and the largest;
+//      a size-weighted histogram gives the cut's bucket b*. Every cluster of a higher bucket
+//      is taken whole; only the few clusters of bucket b* are ranked exactly, which gives the
+//      cut and the whole clusters of b* (those ranked before the cut). Whole clusters are laid
+//      out in cluster-index order (attention over a set does not depend on row order), by one
+//      block scan of their sizes;
 //   3. the selected rows form one index space: sinks, pending (in append order, from the
-//      two-window pending ring), whole clusters by rank, then the partial tokens of the cut
-//      cluster. With a partial fill and S > 1, CTA S-1 takes exactly the partial tokens: it
-//      copies the cut cluster's K and V rows into shared memory (started during the
-//      selection when the histogram isolates the cut), ranks the tokens by qbar . k there
-//      and attends the top ones in place. The other CTAs split the rest;
-//   4. rows reach a two-slot shared-memory ring through cp.async (16 bytes per thread,
-//      coalesced rows, XOR-swizzled 16-byte chunks); all of a CTA's rows are in flight at
-//      once when they fit the ring. Each warp runs flash-decode on 16-row tiles with
+//      two-window pending ring), whole clusters by index, then the partial tokens of the cut
+//      cluster in store order. With a partial fill and S > 1, CTA S-1 takes exactly the
+//      partial tokens: it bulk-copies the cut cluster's K and V rows (started during the
+//      selection when the histogram isolates the cut), ranks the tokens by qbar . k there and
+//      attends the top ones in place. The other CTAs split the rest evenly;
+//   4. rows reach a shared-memory ring through cp.async (16 bytes per thread, coalesced
+//      rows, XOR-swizzled 16-byte chunks). Each warp runs flash-decode on 16-row tiles with
 //      tensor-core MMAs (mma.sync m16n8k16, bf16 in, fp32 accumulate): S^T = K Q^T with the
 //      rows as M and the G query heads as N, an online softmax per head, then O^T += V^T P
 //      with P split into bf16 high and low parts;
 //   5. the warp partials (max, sum, accumulator) are merged per CTA, and the CTA partials in
 //      CTA 0 through distributed shared memory, which writes the fp32 output.
-// The kernel triggers programmatic dependent launch at entry and prefetches its centroid
-// slice into L2 before waiting on the previous grid. A compile-time flag instantiates it for
-// one selection per query head (G = 1 over (sequence, query head) units).
+// Every loop that holds a warp-synchronous operation (shuffle, ballot, reduce) starts at a
+// warp- or CTA-uniform value and steps by a uniform stride, so all 32 lanes run every
+// iteration. Bounded waits that give up set the device error word; the CTA then skips its
+// arithmetic but still takes part in every cluster barrier, so no CTA of the cluster hangs.
+// A compile-time flag instantiates the kernel for one selection per query head (G = 1 over
+// (sequence, query head) units). Another instantiates the mixed-precision decode of the
+// explainer's outlook (section 7, lower precision for far clusters): the selection is the
+// same, but the rows of clusters at walk rank >= n_near arrive as fp8 e4m3 codes with one fp32
+// scale per row. Their codes are staged in the upper half of their ring row, converted
+// exactly to bf16 (e4m3 values are bf16 values) by one warp per row, and the row's scales
+// multiply its scores (K) and its softmax weights in the P V product (V).
+#include <cuda_fp8.h>
 #include <float.h>
 
 #include <map>
@@ -58,11 +75,29 @@ constexpr int kWarps = kNT / 32;
 constexpr int kPartCap = 4096;    // cut-cluster tokens ranked in shared memory (outside the ring path)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kRowBytes = 2 * kD * 2;  // one K row and one V row, bf16
+constexpr int kCombStride = 130;       // accumulator[128], max, sum
+
+// wbuf slots
+constexpr int kWCnt = 40;     // candidates found in the cut's bucket
+constexpr int kWCut = 41;     // the cut cluster
+constexpr int kWPre = 42;     // tokens of bucket b* ranked before the cut
+constexpr int kWCopy = 45;    // the cut cluster's bulk copies were issued
+constexpr int kWBad = 46;     // a bounded wait of this CTA gave up
+constexpr int kWCnt2 = 47;    // candidates found in the bucket of walk rank n_near - 1
+constexpr int kWNear = 64;    // [2] the walk key of rank n_near - 1 (two halves)
+constexpr int32_t kFarBit = 0x40000000;  // rsrc flag: a store row read from the fp8 copy
 
 CKV_DEV uint32_t orderable(float f) {
     f = f + 0.0f;  // -0 -> +0
     const uint32_t u = __float_as_uint(f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+CKV_DEV float from_orderable(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+// Walk order key of cluster c: larger = visited earlier (score descending, index ascending).
+CKV_DEV uint64_t walk_key(float score, int c) {
+    return ((uint64_t)orderable(score) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)c);
 }
 
 // 16-byte chunk j of ring row p, XOR-swizzled by the row's low 3 bits.
@@ -72,7 +107,41 @@ CKV_DEV uint32_t swz_addr(uint32_t base, int p, int j) {
 CKV_DEV void cp_async16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
+CKV_DEV void cp_async4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
 CKV_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+CKV_DEV void sts_v4(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
+// Two e4m3 codes (low byte first) -> two bf16 in one word, exactly (every e4m3 value,
+// subnormals included, is a bf16 value).
+CKV_DEV uint32_t e4m3x2_to_bf16x2(uint32_t two) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
+    const float lo = __half2float(__half(__half_raw{h.x}));
+    const float hi = __half2float(__half(__half_raw{h.y}));
+    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+           ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+}
+// The fp8 copy's value of four bf16 elements held by each lane of a warp (one 128-element
+// row): scale = max|x| / 448, code = e4m3(x / scale) (ties to even, saturating), returned
+// as the codes' bf16 values; *scale_out = scale. The same arithmetic as the stored copy.
+CKV_DEV uint2 fp8_row_values(uint2 w, float* scale_out) {
+    const float x0 = bf16_lo(w.x), x1 = bf16_hi(w.x), x2 = bf16_lo(w.y), x3 = bf16_hi(w.y);
+    float mx = fmaxf(fmaxf(fabsf(x0), fabsf(x1)), fmaxf(fabsf(x2), fabsf(x3)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float scale = __fdiv_rn(mx, 448.0f);
+    *scale_out = scale;
+    if (!(scale > 0.f)) return make_uint2(0u, 0u);
+    const __nv_fp8x2_storage_t c01 = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fdiv_rn(x0, scale), __fdiv_rn(x1, scale)), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t c23 = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fdiv_rn(x2, scale), __fdiv_rn(x3, scale)), __NV_SATFINITE, __NV_E4M3);
+    return make_uint2(e4m3x2_to_bf16x2(c01), e4m3x2_to_bf16x2(c23));
+}
 template <int N>
 CKV_DEV void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
@@ -135,7 +204,7 @@ CKV_DEV float half_row_dot(const uint16_t* row, int half, const float* qbar) {
 }
 
 // Exclusive block scan of one int per thread. `tot` receives the block total.
-CKV_DEV int32_t block_excl_scan(int32_t v, int32_t* wbuf, int32_t* tot) {
+CKV_DEV int32_t block_excl_scan(int32_t v, int32_t* wscan, int32_t* tot) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int32_t incl = v;
 #pragma unroll
@@ -143,55 +212,18 @@ CKV_DEV int32_t block_excl_scan(int32_t v, int32_t* wbuf, int32_t* tot) {
         const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
     }
-    if (lane == 31) wbuf[warp] = incl;
+    if (lane == 31) wscan[warp] = incl;
     __syncthreads();
     int32_t before = 0, total = 0;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
-        const int32_t x = wbuf[w];
+        const int32_t x = wscan[w];
         if (w < warp) before += x;
         total += x;
     }
     __syncthreads();
     *tot = total;
     return before + incl - v;
-}
-
-CKV_DEV float from_orderable(uint32_t k) {
-    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
-}
-
-// The bin (of 256, scanned from the top) whose inclusive cumulative weight first exceeds
-// `need`, computed by a whole warp; every lane returns it.
-CKV_DEV int radix_bin_warp(const int32_t* hist, int32_t need) {
-    const int lane = threadIdx.x & 31;
-    int32_t cnt[8], tot = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        cnt[e] = hist[255 - 8 * lane - e];
-        tot += cnt[e];
-    }
-    int32_t incl = tot;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    int32_t above = incl - tot;
-    int bin = 255;
-    const bool mine = above <= need && need < incl;
-    if (mine) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            if (need < above + cnt[e]) {
-                bin = 255 - 8 * lane - e;
-                break;
-            }
-            above += cnt[e];
-        }
-    }
-    const uint32_t who = __ballot_sync(0xffffffffu, mine);
-    return __shfl_sync(0xffffffffu, bin, who ? __ffs(who) - 1 : 0);
 }
 
 // Warp 0 of a radix pass: bins hold weights in descending digit order; find the digit whose
@@ -227,110 +259,169 @@ CKV_DEV void radix_pick_bin(const int32_t* hist, int32_t need, bool first_exceed
     }
 }
 
-struct Smem {
-    uint16_t* ringK;  // [RB][128] K rows of the current chunk(s)
-    uint16_t* ringV;  // [RB][128] V rows
-    float* wcomb;     // [kWarps][G][130]  (aliases the ring, after the last chunk)
-    uint32_t* pkey;   // [kPartCap + 4]    (aliases the ring, before the first chunk)
-    float* qg;        // [G][128], scaled by log2(e)/sqrt(128)
-    float* qbar;      // [128]
-    float* score;     // [C] every cluster's score (written through distributed shared memory)
-    int32_t* off;     // [C + 1] cluster boundaries
-    int32_t* spre;    // [C + 1] prefix of the whole cluster of rank k
-    int32_t* srow;    // [C + 1] first store row of the whole cluster of rank k
-    uint64_t* word;   // [cand_slots(C)] candidates: order key (score bits, inverted index)
-    int32_t* wsz;     // [cand_slots(C)] candidates: sizes
-    int32_t* hist;    // [256] histogram weights
-    int32_t* hcnt;    // [256] histogram counts (clusters with tokens)
-    uint32_t* rkey;   // [RB + 4] keys of a cut cluster held in the ring
-    int32_t* prow;    // [prow_cap] partial rows of this CTA's share (ring positions or rows)
-    int32_t* wbuf;    // [96] scan / misc scratch
-    float* scl;       // [(kWarps + S) * G] merge scales, then [2 * G] sums
-    float* ccomb;     // [S][G][130] (filled in CTA 0)
-    int32_t* rsrc;    // [RB] source row of every ring row
-    uint16_t* qh;     // [G][128] the queries, bf16 as given
-    uint16_t* pbuf;   // [kWarps][2][8][16] softmax weights of a tile (bf16 high, low)
-    uint64_t* full;   // mbarrier of the cut cluster's bulk copies
+// The bucket (of 256, scanned from the top) whose inclusive cumulative weight first exceeds
+// `need`, and the weight of the buckets above it, computed by a whole warp; every lane
+// returns both. The caller guarantees that the total weight exceeds `need`.
+CKV_DEV int cut_bucket_warp(const int32_t* hist, int32_t need, int32_t* above_out) {
+    const int lane = threadIdx.x & 31;
+    int32_t cnt[8], tot = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        cnt[e] = hist[255 - 8 * lane - e];
+        tot += cnt[e];
+    }
+    int32_t incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    int32_t above = incl - tot;
+    int bin = 255;
+    int32_t ab = 0;
+    const bool mine = above <= need && need < incl;
+    if (mine) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            if (need < above + cnt[e]) {
+                bin = 255 - 8 * lane - e;
+                ab = above;
+                break;
+            }
+            above += cnt[e];
+        }
+    }
+    const uint32_t who = __ballot_sync(0xffffffffu, mine);
+    const int src = who ? __ffs(who) - 1 : 0;
+    *above_out = __shfl_sync(0xffffffffu, ab, src);
+    return __shfl_sync(0xffffffffu, bin, src);
+}
+
+// Shared-memory layout, computed identically on the host (launch size) and the device.
+struct Layout {
+    uint32_t ring, qbar, qh, score, off, spre, cand, hist, hcnt, hnear, rkey, prow, rsrc, rks, rvs,
+        wbuf, scl, ccomb, pbuf, bars, total;
 };
-
-// Candidate list slots: kWarps lists of 32 * ceil(C / kNT) entries.
-__host__ __device__ inline int cand_slots(int C) { return kNT * ((C + kNT - 1) / kNT); }
-
-CKV_DEV size_t ring_bytes_of(int G, int RB) {
-    size_t r = (size_t)RB * kRowBytes;
-    const size_t w = sizeof(float) * kWarps * G * 130;
-    const size_t k = sizeof(uint32_t) * (kPartCap + 4);
+// The ring also holds, before any row arrives, the centroid slice (up to ring / 512 rows of
+// fp32 centroids per chunk) and the cut cluster's keys; after the last row, the warp partials.
+__host__ __device__ inline uint32_t ring_bytes(int G, int RB) {
+    uint32_t r = (uint32_t)RB * kRowBytes;
+    const uint32_t w = 4u * kWarps * G * kCombStride;
+    const uint32_t k = 4u * (kPartCap + 4);
     if (w > r) r = w;
     if (k > r) r = k;
     return r;
 }
+__host__ __device__ inline Layout make_layout(int G, int S, int C, int RB, int prow_cap) {
+    Layout L{};
+    uint32_t p = 0;
+    auto take = [&](uint32_t bytes) {
+        const uint32_t r = p;
+        p += (bytes + 127u) & ~127u;
+        return r;
+    };
+    L.ring = take(ring_bytes(G, RB));
+    L.qbar = take(4u * kD);
+    L.qh = take(2u * G * kD);
+    L.score = take(4u * C);
+    L.off = take(4u * (C + 1));
+    L.spre = take(4u * (C + 1));
+    L.cand = take(4u * C);
+    L.hist = take(4u * 256);
+    L.hcnt = take(4u * 256);
+    L.hnear = take(4u * 256);
+    L.rkey = take(4u * (RB + 4));
+    L.prow = take(4u * prow_cap);
+    L.rsrc = take(4u * RB);
+    L.rks = take(4u * RB);
+    L.rvs = take(4u * RB);
+    L.wbuf = take(4u * 128);
+    L.scl = take(4u * ((kWarps + S) * G + 2 * G));
+    L.ccomb = take(4u * S * G * kCombStride);
+    L.pbuf = take(2u * kWarps * 256);
+    L.bars = take(8u * 2);
+    L.total = p;
+    return L;
+}
+
+struct Params {
+    int32_t S;         // CTAs per unit (thread-block cluster size)
+    int32_t RB;        // ring rows
+    int32_t prow_cap;  // partial rows one CTA may own
+};
 
 // kPerHead: one selection per query head. The kernel then runs with G = 1 over virtual
 // units (b, query head): virtual unit v reads the store of KV unit v / a.qsplit and its own
-// query, output and selection rows.
-template <int G, bool kPerHead>
-__global__ void __launch_bounds__(kNT, 2)
-    select_attend_kernel(const DecodeArgs a, int32_t S, int32_t prow_cap, int32_t RB) {
+// query, output and selection rows. kMixed: rows of clusters at walk rank >= a.n_near are
+// read from the fp8 copy.
+template <int G, bool kPerHead, bool kMixed>
+__global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs a, const Params P) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const int C = a.C;
+    const int S = P.S, RB = P.RB;
     const uint32_t rank = cluster_ctarank();
     const int unit = blockIdx.x / S;
     const int su = kPerHead ? unit / a.qsplit : unit;  // the store's unit
     const int b = unit / a.Hkv, h = unit % a.Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    Smem sm;
-    {
-        uint8_t* p = smem_raw;
-        auto take = [&](size_t bytes) {
-            uint8_t* r = p;
-            p += (bytes + 127) & ~(size_t)127;
-            return r;
-        };
-        uint8_t* ring = take(ring_bytes_of(G, RB));
-        sm.ringK = (uint16_t*)ring;
-        sm.ringV = sm.ringK + (size_t)RB * kD;
-        sm.wcomb = (float*)ring;
-        sm.pkey = (uint32_t*)ring;
-        sm.qg = (float*)take(sizeof(float) * G * kD);
-        sm.qbar = (float*)take(sizeof(float) * kD);
-        sm.score = (float*)take(sizeof(float) * C);
-        sm.off = (int32_t*)take(sizeof(int32_t) * (C + 1));
-        sm.spre = (int32_t*)take(sizeof(int32_t) * (C + 1));
-        sm.srow = (int32_t*)take(sizeof(int32_t) * (C + 1));
-        sm.word = (uint64_t*)take(sizeof(uint64_t) * cand_slots(C));
-        sm.wsz = (int32_t*)take(sizeof(int32_t) * cand_slots(C));
-        sm.hist = (int32_t*)take(sizeof(int32_t) * 256);
-        sm.hcnt = (int32_t*)take(sizeof(int32_t) * 256);
-        sm.rkey = (uint32_t*)take(sizeof(uint32_t) * (RB + 4));
-        sm.prow = (int32_t*)take(sizeof(int32_t) * prow_cap);
-        sm.wbuf = (int32_t*)take(sizeof(int32_t) * 96);
-        sm.scl = (float*)take(sizeof(float) * ((kWarps + S) * G + 2 * G));
-        sm.ccomb = (float*)take(sizeof(float) * S * G * 130);
-        sm.rsrc = (int32_t*)take(sizeof(int32_t) * RB);
-        sm.qh = (uint16_t*)take(sizeof(uint16_t) * G * kD);
-        sm.pbuf = (uint16_t*)take(sizeof(uint16_t) * kWarps * 256);
-        sm.full = (uint64_t*)take(sizeof(uint64_t));
-    }
+    const Layout Ly = make_layout(G, S, C, RB, P.prow_cap);
+    const int cch = (int)(ring_bytes(G, RB) / (kD * 4));  // centroid rows per slice chunk
+    uint8_t* const base = smem_raw;
+    float* const s_qbar = (float*)(base + Ly.qbar);
+    uint16_t* const s_qh = (uint16_t*)(base + Ly.qh);
+    float* const s_score = (float*)(base + Ly.score);
+    int32_t* const s_off = (int32_t*)(base + Ly.off);
+    int32_t* const s_spre = (int32_t*)(base + Ly.spre);
+    int32_t* const s_cand = (int32_t*)(base + Ly.cand);
+    int32_t* const s_hist = (int32_t*)(base + Ly.hist);
+    int32_t* const s_hcnt = (int32_t*)(base + Ly.hcnt);
+    int32_t* const s_hnear = (int32_t*)(base + Ly.hnear);
+    float* const s_rks = (float*)(base + Ly.rks);  // per ring row: K scale (1 for bf16 rows)
+    float* const s_rvs = (float*)(base + Ly.rvs);  // per ring row: V scale
+    uint32_t* const s_rkey = (uint32_t*)(base + Ly.rkey);
+    int32_t* const s_prow = (int32_t*)(base + Ly.prow);
+    int32_t* const s_rsrc = (int32_t*)(base + Ly.rsrc);
+    int32_t* const s_wbuf = (int32_t*)(base + Ly.wbuf);
+    float* const s_scl = (float*)(base + Ly.scl);
+    float* const s_ccomb = (float*)(base + Ly.ccomb);
+    uint16_t* const s_pbuf = (uint16_t*)(base + Ly.pbuf);
+    uint64_t* const cbar = (uint64_t*)(base + Ly.bars);      // centroid slice
+    uint64_t* const fbar = cbar + 1;                         // cut cluster rows
+    float* const s_cent = (float*)(base + Ly.ring);          // centroid slice (aliases the ring)
+    float* const s_wcomb = (float*)(base + Ly.ring);         // warp partials (after the rows)
+    uint32_t* const s_pkey = (uint32_t*)(base + Ly.ring);    // cut keys (before the rows)
+    const uint32_t ringK = smem_u32(base + Ly.ring);
+    const uint32_t ringV = ringK + (uint32_t)RB * 256u;
 
     const int64_t kp_base = (int64_t)su * a.kp_ustride;
     const int64_t sp_base = (int64_t)su * a.sp_ustride;
-    const int32_t* off = a.offsets + (int64_t)su * a.off_ustride;
+    const int32_t* off_g = a.offsets + (int64_t)su * a.off_ustride;
     const float* mu = a.mu + (int64_t)su * a.mu_ustride * kD;
     const int c_begin = (int)((int64_t)C * rank / S);
     const int c_end = (int)((int64_t)C * (rank + 1) / S);
+    const int nc = c_end - c_begin;
+    const uint16_t* qsrc = a.q + ((int64_t)b * a.Hkv * G + (int64_t)h * G) * kD;
 
-    // ---------------------------------------------------------------- phase 0
+    // ---------------------------------------------------------------- phase 0: the store
+    // (before the dependency wait; see the header comment for why the store may be read here)
     pdl_launch_dependents();
     if (tid == 0) {
-        if (c_end > c_begin)
-            prefetch_l2_bulk(mu + (int64_t)c_begin * kD, (uint32_t)(c_end - c_begin) * kD * 4);
-        sm.wbuf[45] = 0;  // cut cluster copies issued
-        mbar_init(sm.full, 1);
+        mbar_init(cbar, 1);
+        mbar_init(fbar, 1);
         fence_mbar_init();
+        s_wbuf[kWCnt] = 0;
+        s_wbuf[kWCopy] = 0;
+        s_wbuf[kWBad] = 0;
     }
-    if (tid * 32 <= C) prefetch_l2(off + tid * 32);  // the boundaries, one 128-byte line each
-    if (rank == 0 && tid == 0) {  // sinks, then the pending rows (up to two runs of the ring)
+    __syncthreads();
+    if (tid == 0 && nc > 0) {  // the slice's first chunk
+        const uint32_t bytes = (uint32_t)min(nc, cch) * kD * 4;
+        mbar_arrive_expect_tx(cbar, bytes);
+        bulk_load(s_cent, mu + (int64_t)c_begin * kD, bytes, cbar);
+    }
+    if (tid < 2 * G) prefetch_l2(qsrc + tid * 64);  // the queries, one 128-byte line each
+    if (rank == 0 && tid == 32) {  // sinks, then the pending rows (up to two runs of the ring)
         const int32_t run1 = min(a.pending, a.pring - a.pstart);
         const int64_t r0[3] = {0, a.n_sink + a.pstart, a.n_sink};
         const int32_t nr[3] = {a.n_sink, run1, a.pending - run1};
@@ -340,109 +431,112 @@ __global__ void __launch_bounds__(kNT, 2)
                 prefetch_l2_bulk(a.spv + (sp_base + r0[k]) * kD, (uint32_t)nr[k] * kD * 2);
             }
     }
+    for (int i = tid; i <= C; i += kNT) s_off[i] = off_g[i];
+    s_hist[tid] = 0;
+    s_hcnt[tid] = 0;
+    s_hnear[tid] = 0;
+    if (tid == 0) s_wbuf[kWCnt2] = 0;
     cluster_arrive_relaxed();
     pdl_wait();
 
     // ---------------------------------------------------------------- phase 1: scores
-    // A quarter-warp (8 lanes) per centroid, 16 dimensions per lane: 32 centroids per CTA
-    // per round. The first round's centroid loads and the boundary loads are issued before
-    // the query loads, so they share one memory round trip; later rounds are loaded one
-    // round ahead.
     const int32_t pend = a.pending;
     const int32_t R = a.budget - a.n_sink - pend;  // >= 0 (host-checked)
-    const int q8 = lane >> 3, l8 = lane & 7;
-    constexpr int kPerRound = kWarps * 4;
-    auto load_centroid = [&](int c, float4* mv) {
-        if (c < c_end) {
-            const float4* row = reinterpret_cast<const float4*>(mu + (int64_t)c * kD) + l8 * 4;
-#pragma unroll
-            for (int t = 0; t < 4; ++t) mv[t] = row[t];
-        } else {
-#pragma unroll
-            for (int t = 0; t < 4; ++t) mv[t] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-    };
-    float4 mv[4];
-    load_centroid(c_begin + warp * 4 + q8, mv);
-    for (int i = tid; i <= C; i += kNT) sm.off[i] = off[i];
-    {
-        const uint16_t* q = a.q + ((int64_t)b * a.Hkv * G + (int64_t)h * G) * kD;
-        const float scale = kLog2e * rsqrtf((float)kD);
-        for (int i = tid; i < kD; i += kNT) {
-            float s = 0.f;
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const uint16_t raw = q[g * kD + i];
-                const float x = __uint_as_float((uint32_t)raw << 16);
-                s += x;
-                sm.qg[g * kD + i] = x * scale;
-                sm.qh[g * kD + i] = raw;
-            }
-            sm.qbar[i] = s;
-        }
-    }
-    __syncthreads();
-    cluster_wait_acquire();  // every CTA of the cluster is running
-    for (int r0 = 0; r0 < c_end - c_begin; r0 += kPerRound) {
-        const int c = c_begin + r0 + warp * 4 + q8;
-        const bool more = r0 + kPerRound < c_end - c_begin;  // CTA-uniform
-        float4 mn[4];
-        if (more) load_centroid(c + kPerRound, mn);
-        const float4* qb4 = reinterpret_cast<const float4*>(sm.qbar) + l8 * 4;
+    if (tid < kD) {
         float s = 0.f;
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            const float4 qv4 = qb4[t];
-            s += qv4.x * mv[t].x + qv4.y * mv[t].y + qv4.z * mv[t].z + qv4.w * mv[t].w;
+        for (int g = 0; g < G; ++g) {
+            const uint16_t raw = qsrc[g * kD + tid];
+            s += __uint_as_float((uint32_t)raw << 16);
+            s_qh[g * kD + tid] = raw;
         }
-        s += __shfl_xor_sync(0xffffffffu, s, 4);
-        s += __shfl_xor_sync(0xffffffffu, s, 2);
-        s += __shfl_xor_sync(0xffffffffu, s, 1);
-        if (c < c_end) {
-            for (int r = l8; r < S; r += 8) st_cluster_f32(map_shared_rank(smem_u32(&sm.score[c]), r), s);
-        }
-        if (more) {
+        s_qbar[tid] = s;
+    }
+    __syncthreads();
+    bool ok = true;
+    cluster_wait_acquire();  // every CTA of the cluster is running: remote stores are safe
+    {
+        const float4 qv = reinterpret_cast<const float4*>(s_qbar)[lane];
+        // The slice in chunks of at most cch centroids (one chunk unless C / S exceeds the
+        // ring); a warp per centroid (lane: dims 4 lane .. 4 lane + 3, a conflict-free 512-byte
+        // row), four centroids per warp in flight.
+        for (int done = 0, chunk_no = 0; done < nc; ++chunk_no) {
+            const int n1 = min(nc - done, cch);
+            ok = ok && mbar_wait(cbar, (uint32_t)(chunk_no & 1), a.err);
+            for (int j0 = warp; j0 < n1; j0 += 4 * kWarps) {
+                float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+                float* sk[4] = {&s0, &s1, &s2, &s3};
 #pragma unroll
-            for (int t = 0; t < 4; ++t) mv[t] = mn[t];
+                for (int k = 0; k < 4; ++k) {
+                    const int j = j0 + k * kWarps;
+                    if (ok && j < n1) {
+                        const float4 mv = reinterpret_cast<const float4*>(s_cent + (size_t)j * kD)[lane];
+                        *sk[k] = fmaf(qv.w, mv.w, fmaf(qv.z, mv.z, fmaf(qv.y, mv.y, qv.x * mv.x)));
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+                    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+                    s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+                    s3 += __shfl_xor_sync(0xffffffffu, s3, o);
+                }
+                for (int t = lane; t < 4 * S; t += 32) {
+                    const int k = t / S, r = t - k * S;
+                    const int j = j0 + k * kWarps;
+                    const float v = k == 0 ? s0 : (k == 1 ? s1 : (k == 2 ? s2 : s3));
+                    if (j < n1)
+                        st_cluster_f32(map_shared_rank(smem_u32(&s_score[c_begin + done + j]), (uint32_t)r), v);
+                }
+            }
+            done += n1;
+            if (done < nc) {  // the next chunk, once every warp is done with this one
+                __syncthreads();
+                if (tid == 0) {
+                    fence_proxy_async();
+                    const uint32_t bytes = (uint32_t)min(nc - done, cch) * kD * 4;
+                    mbar_arrive_expect_tx(cbar, bytes);
+                    bulk_load(s_cent, mu + (int64_t)(c_begin + done) * kD, bytes, cbar);
+                }
+            }
         }
     }
     cluster_arrive_release();
     cluster_wait_acquire();
 
     // ---------------------------------------------------------------- phase 2: selection
-    // Every CTA holds all C scores and sizes and computes the same selection. The walk in
-    // descending (score, -index) order stops at the first cluster whose inclusive token count
-    // exceeds R: the cut. Scores are bucketed by a monotone map onto 256 linear buckets
-    // between the smallest and the largest score, so bucket order never contradicts score
-    // order. A size-weighted histogram gives the bucket that holds the cut; the clusters of
-    // that bucket and above (the candidates) are compacted and ranked exactly among
-    // themselves. A candidate is whole when its prefix plus its size fits R; the cut is the
-    // candidate whose prefix fits and whose prefix plus size does not.
-    const int32_t m_tot = sm.off[C] - sm.off[0];
+    const int32_t m_tot = s_off[C] - s_off[0];
     const bool has_cut = m_tot > R;  // otherwise every cluster is whole
     float smin = 0.f, inv = 0.f;
-    int32_t bstar = 0;
+    int bstar = 0;
+    int32_t w_above = 0;
     auto bucket = [&](float sc) {
         const float t = (sc + 0.0f - smin) * inv;
         return (int)fminf(fmaxf(t, 0.f), 255.f);
     };
-    if (has_cut) {
-        // smallest and largest score (order keys; one warp reduction each)
+    auto size_of = [&](int c) { return s_off[c + 1] - s_off[c]; };
+    int32_t cut_c = -1, w_cut = 0;  // w_cut: tokens of bucket b* ranked before the cut
+    uint64_t kcut = 0;
+    // mixed precision: the walk key of rank n_near - 1 separates near from far clusters
+    const bool mid_near = kMixed && a.n_near > 0 && a.n_near < C;
+    if (has_cut || mid_near) {
+        // smallest and largest score of the clusters with tokens (of every cluster for the
+        // mixed-precision rank, which counts empty clusters too), as order keys
         uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
         for (int c = tid; c < C; c += kNT) {
-            const uint32_t k = orderable(sm.score[c]);
-            kmn = min(kmn, k);
-            kmx = max(kmx, k);
+            if (kMixed || size_of(c) > 0) {
+                const uint32_t k = orderable(s_score[c]);
+                kmn = min(kmn, k);
+                kmx = max(kmx, k);
+            }
         }
         kmn = __reduce_min_sync(0xffffffffu, kmn);
         kmx = __reduce_max_sync(0xffffffffu, kmx);
-        uint32_t* kb = reinterpret_cast<uint32_t*>(sm.wbuf + 48);  // [8] minima, [8] maxima
+        uint32_t* kb = reinterpret_cast<uint32_t*>(s_wbuf + 48);  // [8] minima, [8] maxima
         if (lane == 0) {
             kb[warp] = kmn;
             kb[8 + warp] = kmx;
         }
-        sm.hist[tid] = 0;
-        sm.hcnt[tid] = 0;
         __syncthreads();
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) {
@@ -453,116 +547,152 @@ __global__ void __launch_bounds__(kNT, 2)
         const float range = mx - mn;
         smin = mn;
         inv = range > 1e-30f ? 255.99f / range : 0.f;  // finite; 0 puts every score in bucket 0
+    }
+    if (has_cut) {
         for (int c = tid; c < C; c += kNT) {
-            const int32_t w = sm.off[c + 1] - sm.off[c];
+            const int32_t w = size_of(c);
             if (w > 0) {
-                const int bk = bucket(sm.score[c]);
-                atomicAdd(&sm.hist[bk], w);
-                atomicAdd(&sm.hcnt[bk], 1);
+                const int bk = bucket(s_score[c]);
+                atomicAdd(&s_hist[bk], w);
+                atomicAdd(&s_hcnt[bk], 1);
             }
         }
         __syncthreads();
         // every warp finds the cut's bucket itself (no extra block barrier)
-        bstar = radix_bin_warp(sm.hist, R);
-        // When bstar holds a single cluster with tokens, that cluster is the cut: CTA S-1,
-        // which fills the partial tokens, starts copying its K and V rows now, while the
-        // whole clusters are still being ranked.
-        if ((int)rank == S - 1 && S > 1 && sm.hcnt[bstar] == 1) {
+        bstar = cut_bucket_warp(s_hist, R, &w_above);
+        // When b* holds a single cluster with tokens, that cluster is the cut: CTA S-1, which
+        // fills the partial tokens, starts copying its K and V rows now.
+        if ((int)rank == S - 1 && S > 1 && s_hcnt[bstar] == 1) {
             for (int c = tid; c < C; c += kNT) {
-                const int32_t w = sm.off[c + 1] - sm.off[c];
-                if (w > 0 && w <= RB && w <= kNT && bucket(sm.score[c]) == bstar) {
-                    const int64_t row = kp_base + sm.off[c];
+                const int32_t w = size_of(c);
+                if (w > 0 && w <= RB && w <= kNT && bucket(s_score[c]) == bstar) {
+                    fence_proxy_async();  // the ring's centroid reads come before the copies
+                    const int64_t row = kp_base + s_off[c];
                     const uint32_t bytes = (uint32_t)w * kD * 2;
-                    mbar_arrive_expect_tx(sm.full, 2 * bytes);
-                    bulk_load(sm.ringK, a.kp + row * kD, bytes, sm.full);
-                    bulk_load(sm.ringV, a.vp + row * kD, bytes, sm.full);
-                    sm.wbuf[45] = 1;
+                    mbar_arrive_expect_tx(fbar, 2 * bytes);
+                    bulk_load(base + Ly.ring, a.kp + row * kD, bytes, fbar);
+                    bulk_load(base + Ly.ring + (size_t)RB * 256, a.vp + row * kD, bytes, fbar);
+                    s_wbuf[kWCopy] = 1;
                 }
             }
         }
-    }
-    // Candidates: every cluster without a cut, else the buckets >= bstar. Each warp compacts
-    // the clusters it visits into its own list (kWarps lists of cap entries, any order).
-    const int cap = 32 * ((C + kNT - 1) / kNT);
-    int32_t n_mine = 0;
-    for (int c0 = 0; c0 < C; c0 += kNT) {
-        const int c = c0 + tid;
-        bool cand = false;
-        uint32_t k = 0;
-        if (c < C) {
-            const float sc = sm.score[c];
-            k = orderable(sc);
-            cand = !has_cut || bucket(sc) >= bstar;
+        // the clusters of bucket b* (any order)
+        for (int c0 = 0; c0 < C; c0 += kNT) {
+            const int c = c0 + tid;
+            const bool in_b = c < C && size_of(c) > 0 && bucket(s_score[c]) == bstar;
+            const uint32_t bal = __ballot_sync(0xffffffffu, in_b);
+            int32_t pos0 = 0;
+            if (lane == 0 && bal) pos0 = atomicAdd(&s_wbuf[kWCnt], __popc(bal));
+            pos0 = __shfl_sync(0xffffffffu, pos0, 0);
+            if (in_b) s_cand[pos0 + __popc(bal & ((1u << lane) - 1u))] = c;
         }
-        const uint32_t bal = __ballot_sync(0xffffffffu, cand);
-        if (cand) {
-            const int pos = warp * cap + n_mine + __popc(bal & ((1u << lane) - 1u));
-            sm.word[pos] = ((uint64_t)k << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)c);
-            sm.wsz[pos] = sm.off[c + 1] - sm.off[c];
-        }
-        n_mine += __popc(bal);
-    }
-    if (lane == 0) sm.wbuf[64 + warp] = n_mine;
-    __syncthreads();
-    int32_t pref[kWarps + 1];  // list starts in the flat candidate order
-    pref[0] = 0;
+        __syncthreads();
+        const int32_t n_b = s_wbuf[kWCnt];
+        // exact rank of each candidate among them: 8 threads per candidate
+        for (int i0 = 0; i0 < n_b; i0 += kNT / 8) {
+            const int i = i0 + (tid >> 3), sub = tid & 7;
+            const int ci = i < n_b ? s_cand[i] : 0;
+            const uint64_t ki = i < n_b ? walk_key(s_score[ci], ci) : ~0ull;
+            int32_t pre = 0;
+            for (int j = sub; j < n_b; j += 8) {
+                const int cj = s_cand[j];
+                if (walk_key(s_score[cj], cj) > ki) pre += size_of(cj);
+            }
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) pref[w + 1] = pref[w] + sm.wbuf[64 + w];
-    const int32_t n_cand = pref[kWarps];
-    // flat candidate index f -> slot in the warp lists
-    auto slot_of = [&](int f) {
-        int slot = f;
-#pragma unroll
-        for (int v = 1; v < kWarps; ++v)
-            if (f >= pref[v]) slot = f - pref[v] + v * cap;
-        return slot;
-    };
-    // rank and prefix of every candidate: 8 threads per candidate
-    for (int i0 = 0; i0 < n_cand; i0 += kNT / 8) {
-        const int i = i0 + (tid >> 3), sub = tid & 7;
-        const int si = i < n_cand ? slot_of(i) : 0;
-        const uint64_t ki = i < n_cand ? sm.word[si] : ~0ull;
-        int32_t rk = 0, pre = 0;
-#pragma unroll 4
-        for (int j = sub; j < n_cand; j += 8) {
-            const int sj = slot_of(j);
-            const bool before = sm.word[sj] > ki;
-            rk += before ? 1 : 0;
-            pre += before ? sm.wsz[sj] : 0;
-        }
-#pragma unroll
-        for (int o = 4; o > 0; o >>= 1) {
-            rk += __shfl_xor_sync(0xffffffffu, rk, o);
-            pre += __shfl_xor_sync(0xffffffffu, pre, o);
-        }
-        if (i < n_cand && sub == 0) {
-            const int c = (int)(0xFFFFFFFFu - (uint32_t)(ki & 0xFFFFFFFFull));
-            const int32_t sz = sm.wsz[si];
-            if (pre + sz <= R || !has_cut) {  // whole
-                sm.spre[rk] = pre;
-                sm.srow[rk] = sm.off[c];
-            } else if (pre <= R) {  // the cut
-                sm.wbuf[36] = c;
-                sm.wbuf[37] = pre;
-                sm.wbuf[38] = rk;
+            for (int o = 4; o > 0; o >>= 1) pre += __shfl_xor_sync(0xffffffffu, pre, o);
+            if (i < n_b && sub == 0) {
+                const int32_t before = w_above + pre;
+                if (before <= R && R < before + size_of(ci)) {  // the cut (exactly one)
+                    s_wbuf[kWCut] = ci;
+                    s_wbuf[kWPre] = pre;
+                }
             }
         }
+        __syncthreads();
+        cut_c = s_wbuf[kWCut];
+        w_cut = s_wbuf[kWPre];
+        kcut = walk_key(s_score[cut_c], cut_c);
+    }
+    // near(c): walk rank < n_near, i.e. walk key >= the key of rank n_near - 1. The count
+    // histogram over the same buckets gives the bucket of that rank; its clusters are ranked
+    // exactly among themselves.
+    uint64_t k_near = 0;
+    if (mid_near) {
+        for (int c = tid; c < C; c += kNT) atomicAdd(&s_hnear[bucket(s_score[c])], 1);
+        __syncthreads();
+        int32_t n_above = 0;
+        const int bn = cut_bucket_warp(s_hnear, a.n_near - 1, &n_above);
+        int32_t* cand2 = s_spre;  // free until the whole-size scan below
+        for (int c0 = 0; c0 < C; c0 += kNT) {
+            const int c = c0 + tid;
+            const bool in_b = c < C && bucket(s_score[c]) == bn;
+            const uint32_t bal = __ballot_sync(0xffffffffu, in_b);
+            int32_t pos0 = 0;
+            if (lane == 0 && bal) pos0 = atomicAdd(&s_wbuf[kWCnt2], __popc(bal));
+            pos0 = __shfl_sync(0xffffffffu, pos0, 0);
+            if (in_b) cand2[pos0 + __popc(bal & ((1u << lane) - 1u))] = c;
+        }
+        __syncthreads();
+        const int32_t n_bn = s_wbuf[kWCnt2];
+        for (int i = tid; i < n_bn; i += kNT) {
+            const int ci = cand2[i];
+            const uint64_t ki = walk_key(s_score[ci], ci);
+            int32_t rk = n_above;
+            for (int j = 0; j < n_bn; ++j) {
+                const int cj = cand2[j];
+                rk += walk_key(s_score[cj], cj) > ki ? 1 : 0;
+            }
+            if (rk == a.n_near - 1) {  // exactly one cluster has this rank
+                s_wbuf[kWNear] = (int32_t)(uint32_t)(ki >> 32);
+                s_wbuf[kWNear + 1] = (int32_t)(uint32_t)ki;
+            }
+        }
+        __syncthreads();
+        k_near = ((uint64_t)(uint32_t)s_wbuf[kWNear] << 32) | (uint64_t)(uint32_t)s_wbuf[kWNear + 1];
+    }
+    auto is_far = [&](int c) -> bool {
+        if (!kMixed || a.n_near >= C) return false;
+        if (a.n_near <= 0) return true;
+        return walk_key(s_score[c], c) < k_near;
+    };
+    // whole clusters: every cluster without a cut; else buckets above b*, and the clusters of
+    // b* ranked before the cut. Their rows are laid out in cluster-index order: spre[c] is the
+    // exclusive prefix of the whole sizes (one block scan, a contiguous run per thread).
+    auto whole_size = [&](int c) -> int32_t {
+        const int32_t w = size_of(c);
+        if (w == 0 || !has_cut) return w;
+        const float sc = s_score[c];
+        const int bk = bucket(sc);
+        return (bk > bstar || (bk == bstar && walk_key(sc, c) > kcut)) ? w : 0;
+    };
+    {
+        const int per = (C + kNT - 1) / kNT;
+        const int c0 = tid * per;
+        int32_t local = 0;
+        for (int j = 0; j < per; ++j)
+            if (c0 + j < C) local += whole_size(c0 + j);
+        int32_t tot;
+        int32_t run = block_excl_scan(local, s_wbuf, &tot);
+        for (int j = 0; j < per; ++j)
+            if (c0 + j < C) {
+                s_spre[c0 + j] = run;
+                run += whole_size(c0 + j);
+            }
+        if (tid == 0) s_spre[C] = tot;
     }
     __syncthreads();
-    const int32_t cut_c = has_cut ? sm.wbuf[36] : -1;
-    const int32_t n_whole = has_cut ? sm.wbuf[38] : C;
 
     // Index-space quantities are below the budget (int32).
-    const int32_t W = has_cut ? sm.wbuf[37] : m_tot;  // tokens in whole clusters
+    const int32_t W = has_cut ? w_above + w_cut : m_tot;  // tokens in whole clusters
     const int32_t r_part = has_cut ? R - W : 0;
-    const int32_t csz = has_cut ? sm.off[cut_c + 1] - sm.off[cut_c] : 0;
-    const int32_t crow = has_cut ? sm.off[cut_c] : 0;
+    const int32_t csz = has_cut ? size_of(cut_c) : 0;
+    const int32_t crow = has_cut ? s_off[cut_c] : 0;
     const int32_t base_w = a.n_sink + pend;
     const int32_t base_p = base_w + W;
     const int32_t T = base_p + r_part;
     // Work split of the selection index space [0, T). With a partial fill, CTA S-1 takes
     // exactly the partial tokens (it also ranks them) and the other CTAs split the rest.
-    const bool dedicated = r_part > 0 && S > 1 && r_part <= prow_cap;
+    const bool dedicated = r_part > 0 && S > 1 && r_part <= P.prow_cap;
     int32_t lo, hi;
     if (dedicated) {
         if ((int)rank == S - 1) {
@@ -580,28 +710,59 @@ __global__ void __launch_bounds__(kNT, 2)
     const int32_t p_hi = hi > base_p ? hi - base_p : 0;
     const bool big_cut = csz > kPartCap;
     const bool resident = dedicated && (int)rank == S - 1 && csz <= RB && csz <= kNT;
+    const bool cut_far = kMixed && has_cut && is_far(cut_c);
     int32_t* sel_out = a.sel_idx ? a.sel_idx + (int64_t)unit * a.budget : nullptr;
     const int32_t* ids = a.ids + kp_base;
 
     // ---------------------------------------------------------------- phase 3/4: rows
-    // Rows reach shared memory through cp.async (16 bytes per thread; 16 threads per 256-byte
-    // row) into an XOR-swizzled ring: the 16-byte chunk j of ring row p sits at chunk
-    // j ^ (p & 7), so the 8 rows of an ldmatrix tile fall in 8 different bank groups.
     // rsrc[p] names the source of ring row p: a store row (>= 0) or a sink / pending row
     // (-1 - index).
-    const uint32_t ringK = smem_u32(sm.ringK), ringV = smem_u32(sm.ringV);
     // parts: 1 = K rows, 2 = V rows, 3 = both (one commit group)
+    // A far row (kMixed) arrives as its 128 fp8 codes, staged unswizzled in the upper half of
+    // its ring row, plus its two scales; convert_far turns the codes into the bf16 row.
     auto copy_rows = [&](int p0, int n, int parts) {
         const int per_row = parts == 3 ? 32 : 16;
         for (int i = tid; i < n * per_row; i += kNT) {
             const int p = p0 + i / per_row, j = i & 15;
             const int part = parts == 3 ? (i >> 4) & 1 : parts - 1;
-            const int32_t r = sm.rsrc[p];
+            const int32_t r = s_rsrc[p];
+            if (kMixed && r >= 0 && (r & kFarBit) != 0) {
+                const int64_t row = kp_base + (r & ~kFarBit);
+                if (j < 8)
+                    cp_async16((part ? ringV : ringK) + (uint32_t)p * 256u + 128u + (uint32_t)j * 16u,
+                               (part ? a.vp8 : a.kp8) + row * kD + j * 16);
+                else if (j == 8)
+                    cp_async4(smem_u32(part ? &s_rvs[p] : &s_rks[p]), (part ? a.vs8 : a.ks8) + row);
+                continue;
+            }
             const uint16_t* src = r >= 0 ? (part ? a.vp : a.kp) + (kp_base + r) * kD
                                          : (part ? a.spv : a.spk) + (sp_base + (-1 - r)) * kD;
             cp_async16(swz_addr(part ? ringV : ringK, p, j), src + j * 8);
+            if (kMixed && j == 0) (part ? s_rvs : s_rks)[p] = 1.f;
         }
         cp_async_commit();
+    };
+    // Far rows of ring rows [p0, p0 + n): one warp per row; lanes 0-7 hold the K code chunks,
+    // lanes 8-15 the V code chunks (16 codes each), all read before any bf16 chunk is written.
+    auto convert_far = [&](int p0, int n) {
+        for (int p = p0 + warp; p < p0 + n; p += kWarps) {  // warp-uniform trip count
+            const int32_t r = s_rsrc[p];
+            if (r < 0 || (r & kFarBit) == 0) continue;  // uniform across the warp
+            const int jj = lane & 7;
+            const uint32_t rb = (lane < 8 ? ringK : ringV) + (uint32_t)p * 256u;
+            uint4 c = make_uint4(0u, 0u, 0u, 0u);
+            if (lane < 16) c = lds_v4(rb + 128u + (uint32_t)jj * 16u);
+            __syncwarp();
+            if (lane < 16) {
+                const uint4 lo = make_uint4(e4m3x2_to_bf16x2(c.x & 0xFFFFu), e4m3x2_to_bf16x2(c.x >> 16),
+                                            e4m3x2_to_bf16x2(c.y & 0xFFFFu), e4m3x2_to_bf16x2(c.y >> 16));
+                const uint4 hi = make_uint4(e4m3x2_to_bf16x2(c.z & 0xFFFFu), e4m3x2_to_bf16x2(c.z >> 16),
+                                            e4m3x2_to_bf16x2(c.w & 0xFFFFu), e4m3x2_to_bf16x2(c.w >> 16));
+                sts_v4(swz_addr(rb - (uint32_t)p * 256u, p, 2 * jj), lo);
+                sts_v4(swz_addr(rb - (uint32_t)p * 256u, p, 2 * jj + 1), hi);
+            }
+            __syncwarp();
+        }
     };
     // Sources (and, when asked for, original token ids) of the selection positions [c0, c1),
     // written to ring rows p0 ...
@@ -612,17 +773,20 @@ __global__ void __launch_bounds__(kNT, 2)
                 r = -1 - (idx < a.n_sink ? idx : a.n_sink + (a.pstart + idx - a.n_sink) % a.pring);
             } else if (idx < base_p) {
                 const int32_t x = idx - base_w;
-                int k0 = 0, khi = n_whole - 1;  // last k with spre[k] <= x
+                int k0 = 0, khi = C - 1;  // last cluster with spre[k] <= x: a whole one holding x
                 while (k0 < khi) {
                     const int mid = (k0 + khi + 1) >> 1;
-                    if (sm.spre[mid] <= x) k0 = mid; else khi = mid - 1;
+                    if (s_spre[mid] <= x) k0 = mid; else khi = mid - 1;
                 }
-                r = sm.srow[k0] + (x - sm.spre[k0]);
+                r = s_off[k0] + (x - s_spre[k0]);
+                if (kMixed && is_far(k0)) r |= kFarBit;
             } else {
-                r = sm.prow[idx - base_p - p_lo];
+                r = s_prow[idx - base_p - p_lo];
+                if (kMixed && cut_far) r |= kFarBit;
             }
-            sm.rsrc[p0 + (idx - c0)] = r;
-            if (sel_out) sel_out[idx] = r >= 0 ? ids[r] : (idx < a.n_sink ? idx : (int32_t)(a.m + idx));
+            s_rsrc[p0 + (idx - c0)] = r;
+            if (sel_out)
+                sel_out[idx] = r >= 0 ? ids[r & ~kFarBit] : (idx < a.n_sink ? idx : (int32_t)(a.m + idx));
         }
     };
 
@@ -634,20 +798,20 @@ __global__ void __launch_bounds__(kNT, 2)
     uint32_t qb[8][2];  // Q^T fragments: Q[head g8][16 s + 2 t4 ...], unscaled bf16
 #pragma unroll
     for (int s8 = 0; s8 < 8; ++s8) {
-        qb[s8][0] = g8 < G ? *reinterpret_cast<const uint32_t*>(sm.qh + g8 * kD + 16 * s8 + 2 * t4) : 0u;
-        qb[s8][1] = g8 < G ? *reinterpret_cast<const uint32_t*>(sm.qh + g8 * kD + 16 * s8 + 2 * t4 + 8) : 0u;
+        qb[s8][0] = g8 < G ? *reinterpret_cast<const uint32_t*>(s_qh + g8 * kD + 16 * s8 + 2 * t4) : 0u;
+        qb[s8][1] = g8 < G ? *reinterpret_cast<const uint32_t*>(s_qh + g8 * kD + 16 * s8 + 2 * t4 + 8) : 0u;
     }
     float oacc[8][4];
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) oacc[mt][0] = oacc[mt][1] = oacc[mt][2] = oacc[mt][3] = 0.f;
     float m2[2] = {-INFINITY, -INFINITY}, l2[2] = {0.f, 0.f};  // heads 2 t4, 2 t4 + 1
-    uint16_t* pw = sm.pbuf + warp * 256;  // [2][8 heads][16 rows] bf16 (high, low)
+    uint16_t* pw = s_pbuf + warp * 256;  // [2][8 heads][16 rows] bf16 (high, low)
     const float qscale = kLog2e * rsqrtf((float)kD);
     // rows: ring row of tile row t is pos[t] (pos != nullptr) or p0 + t;
     // swz: rows XOR-swizzled (cp.async ring) or plain (bulk copies of the cut cluster)
     auto attend = [&](int p0, int n, const int32_t* pos, bool swz) {
-        auto addr = [&](uint32_t base, int p, int j) {
-            return base + (uint32_t)p * 256u + ((uint32_t)(j ^ (swz ? (p & 7) : 0)) << 4);
+        auto addr = [&](uint32_t rbase, int p, int j) {
+            return rbase + (uint32_t)p * 256u + ((uint32_t)(j ^ (swz ? (p & 7) : 0)) << 4);
         };
         const int n_tiles = (n + 15) >> 4;
         for (int tile = warp; tile < n_tiles; tile += kWarps) {
@@ -667,11 +831,21 @@ __global__ void __launch_bounds__(kNT, 2)
             }
             // S^T: [0], [1] = row g8, heads 2 t4, 2 t4 + 1; [2], [3] = row g8 + 8
             const bool v0 = r0 + g8 < n, v1 = r0 + g8 + 8 < n;
+            // per-row scales of the fp8 copy (1 for bf16 rows)
+            float ksa = 1.f, ksb = 1.f, vsa = 1.f, vsb = 1.f;
+            if (kMixed) {
+                const int ta = v0 ? r0 + g8 : r0, tb = v1 ? r0 + g8 + 8 : r0;
+                const int pa = pos ? pos[ta] : p0 + ta, pb = pos ? pos[tb] : p0 + tb;
+                ksa = s_rks[pa];
+                ksb = s_rks[pb];
+                vsa = s_rvs[pa];
+                vsb = s_rvs[pb];
+            }
             float pr[4];
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                const float z0 = v0 ? (sa[hh] + sb[hh]) * qscale : -INFINITY;
-                const float z1 = v1 ? (sa[2 + hh] + sb[2 + hh]) * qscale : -INFINITY;
+                const float z0 = v0 ? ((sa[hh] + sb[hh]) * ksa) * qscale : -INFINITY;
+                const float z1 = v1 ? ((sa[2 + hh] + sb[2 + hh]) * ksb) * qscale : -INFINITY;
                 float mx = fmaxf(z0, z1);
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
@@ -691,10 +865,11 @@ __global__ void __launch_bounds__(kNT, 2)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int hd = 2 * t4 + (e & 1), rr = g8 + (e >> 1) * 8;
-                const __nv_bfloat16 hi = __float2bfloat16_rn(pr[e]);
-                const __nv_bfloat16 lo = __float2bfloat16_rn(pr[e] - __bfloat162float(hi));
-                pw[hd * 16 + rr] = __bfloat16_as_ushort(hi);
-                pw[128 + hd * 16 + rr] = __bfloat16_as_ushort(lo);
+                const float pv_ = kMixed ? pr[e] * ((e & 2) ? vsb : vsa) : pr[e];  // weight of V
+                const __nv_bfloat16 hi_ = __float2bfloat16_rn(pv_);
+                const __nv_bfloat16 lo_ = __float2bfloat16_rn(pv_ - __bfloat162float(hi_));
+                pw[hd * 16 + rr] = __bfloat16_as_ushort(hi_);
+                pw[128 + hd * 16 + rr] = __bfloat16_as_ushort(lo_);
             }
             __syncwarp();
             // P fragments (k = tile rows, n = heads): [r = 2 t4 (+8) ...][h = g8]
@@ -713,6 +888,7 @@ __global__ void __launch_bounds__(kNT, 2)
         }
     };
 
+    if (!ok) s_wbuf[kWBad] = 1;
     const int32_t n_rows = resident ? csz : hi - lo;
     const int chunk = (resident || n_rows <= RB) ? RB : RB / 2;
     const int n_chunks = resident ? 1 : (n_rows + chunk - 1) / chunk;
@@ -728,25 +904,27 @@ __global__ void __launch_bounds__(kNT, 2)
     if (resident) {
         // ---- the cut cluster in shared memory (plain 256-byte rows): two bulk copies, issued
         // during the selection when the histogram isolated the cut, else now
-        if (tid == 0 && sm.wbuf[45] == 0) {
+        if (tid == 0 && s_wbuf[kWCopy] == 0) {
+            fence_proxy_async();  // the ring's centroid reads come before the copies
             const uint32_t bytes = (uint32_t)csz * kD * 2;
-            mbar_arrive_expect_tx(sm.full, 2 * bytes);
-            bulk_load(sm.ringK, a.kp + (kp_base + crow) * kD, bytes, sm.full);
-            bulk_load(sm.ringV, a.vp + (kp_base + crow) * kD, bytes, sm.full);
+            mbar_arrive_expect_tx(fbar, 2 * bytes);
+            bulk_load(base + Ly.ring, a.kp + (kp_base + crow) * kD, bytes, fbar);
+            bulk_load(base + Ly.ring + (size_t)RB * 256, a.vp + (kp_base + crow) * kD, bytes, fbar);
         }
-        mbar_wait(sm.full, 0, a.err);
+        const bool got = __syncthreads_and(mbar_wait(fbar, 0, a.err) ? 1 : 0) != 0;
+        if (!got) s_wbuf[kWBad] = 1;
         // qbar . k, a half-warp per row (16-byte reads covering one 256-byte row), 8 rows
         // per half-warp in flight
         const int hw = tid >> 4, l16 = tid & 15;
-        const float4 qa = reinterpret_cast<const float4*>(sm.qbar)[l16 * 2];
-        const float4 qb4 = reinterpret_cast<const float4*>(sm.qbar)[l16 * 2 + 1];
+        const float4 qa = reinterpret_cast<const float4*>(s_qbar)[l16 * 2];
+        const float4 qb4 = reinterpret_cast<const float4*>(s_qbar)[l16 * 2 + 1];
         for (int r0 = 0; r0 < csz; r0 += 8 * (kNT / 16)) {
             float s[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 const int e = r0 + hw + k * (kNT / 16);
                 s[k] = 0.f;
-                if (e < csz) {
+                if (got && e < csz) {
                     const uint4 w = lds_v4(ringK + (uint32_t)e * 256u + l16 * 16);
                     float t = qa.x * bf16_lo(w.x);
                     t = fmaf(qa.y, bf16_hi(w.x), t);
@@ -766,18 +944,18 @@ __global__ void __launch_bounds__(kNT, 2)
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 const int e = r0 + hw + k * (kNT / 16);
-                if (e < csz && l16 == 0) sm.rkey[e] = orderable(s[k]);
+                if (e < csz && l16 == 0) s_rkey[e] = orderable(s[k]);
             }
         }
-        if (tid < 4) sm.rkey[csz + tid] = 0u;  // pad: never outranks a key
+        if (tid < 4) s_rkey[csz + tid] = 0u;  // pad: never outranks a key
         __syncthreads();
         // comparison rank (ties: lower index), tpe threads per token, 4 keys per load
         const int tpe = csz <= 32 ? 8 : (csz <= 64 ? 4 : (csz <= 128 ? 2 : 1));
         const int e = tid / tpe, sub = tid % tpe;
         int32_t rk = 0;
         if (e < csz) {
-            const uint32_t ke = sm.rkey[e];
-            const uint4* k4 = reinterpret_cast<const uint4*>(sm.rkey);
+            const uint32_t ke = s_rkey[e];
+            const uint4* k4 = reinterpret_cast<const uint4*>(s_rkey);
             const int n4 = (csz + 3) >> 2;
 #pragma unroll 4
             for (int j4 = sub; j4 < n4; j4 += tpe) {
@@ -796,15 +974,44 @@ __global__ void __launch_bounds__(kNT, 2)
         }
         const int32_t sel = (e < csz && sub == 0 && rk < r_part) ? 1 : 0;
         int32_t tot;
-        const int32_t pos = block_excl_scan(sel, sm.wbuf, &tot);
+        const int32_t pos = block_excl_scan(sel, s_wbuf, &tot);
         if (sel) {
-            sm.prow[pos] = e;
+            s_prow[pos] = e;
             if (sel_out) sel_out[base_p + pos] = ids[crow + e];
         }
         __syncthreads();
-        attend(0, r_part, sm.prow, false);
+        if (kMixed) {
+            // the selected rows of a far cut cluster take their fp8 copy's values in place;
+            // a near one keeps its bf16 rows (scale 1)
+            for (int t = warp; t < r_part; t += kWarps) {  // warp-uniform trip count
+                const int er = s_prow[t];
+                if (cut_far) {
+#pragma unroll
+                    for (int part = 0; part < 2; ++part) {
+                        uint2* row = reinterpret_cast<uint2*>(base + Ly.ring + (size_t)part * RB * 256 +
+                                                              (size_t)er * 256);
+                        float sc;
+                        const uint2 v = fp8_row_values(row[lane], &sc);
+                        __syncwarp();
+                        row[lane] = v;
+                        if (lane == 0) (part ? s_rvs : s_rks)[er] = sc;
+                    }
+                } else if (lane == 0) {
+                    s_rks[er] = 1.f;
+                    s_rvs[er] = 1.f;
+                }
+            }
+            __syncthreads();
+        }
+        if (got) attend(0, r_part, s_prow, false);
     } else {
-        if (sm.wbuf[45] != 0) mbar_wait(sm.full, 0, a.err);  // cut copies land before the ring is reused
+        if (s_wbuf[kWCopy] != 0) {  // cut copies land before the ring is reused
+            const bool got = __syncthreads_and(mbar_wait(fbar, 0, a.err) ? 1 : 0) != 0;
+            if (!got) {
+                s_wbuf[kWBad] = 1;
+                mbar_wait(fbar, 0, a.err);  // one more bounded wait for the copies in flight
+            }
+        }
         // ---- partial tokens of this CTA's share outside the ring path: rows into prow
         uint32_t* gkeys = a.part_scratch ? reinterpret_cast<uint32_t*>(a.part_scratch) +
                                                (int64_t)unit * a.part_ustride
@@ -815,7 +1022,7 @@ __global__ void __launch_bounds__(kNT, 2)
                 const int64_t i = i0 + (tid >> 1);
                 const int half = tid & 1;
                 float s = 0.f;
-                if (i < k1) s = half_row_dot(a.kp + (kp_base + crow + i) * kD, half, sm.qbar);
+                if (i < k1) s = half_row_dot(a.kp + (kp_base + crow + i) * kD, half, s_qbar);
                 s += __shfl_xor_sync(0xffffffffu, s, 1);
                 if (i < k1 && half == 0) dst[i] = orderable(s);
             }
@@ -828,10 +1035,10 @@ __global__ void __launch_bounds__(kNT, 2)
             cluster_wait_acquire();
         }
         if (r_part > 0 && p_hi > p_lo) {
-            auto key_at = [&](int i) -> uint32_t { return big_cut ? __ldcg(gkeys + i) : sm.pkey[i]; };
+            auto key_at = [&](int i) -> uint32_t { return big_cut ? __ldcg(gkeys + i) : s_pkey[i]; };
             if (!big_cut) {
-                score_keys(0, csz, sm.pkey);
-                if (tid < 4) sm.pkey[csz + tid] = 0u;  // pad: never outranks a key
+                score_keys(0, csz, s_pkey);
+                if (tid < 4) s_pkey[csz + tid] = 0u;  // pad: never outranks a key
             }
             __syncthreads();
             if (!big_cut && csz <= kNT) {
@@ -839,8 +1046,8 @@ __global__ void __launch_bounds__(kNT, 2)
                 const int e = tid / tpe, sub = tid % tpe;
                 int32_t rk = 0;
                 if (e < csz) {
-                    const uint32_t ke = sm.pkey[e];
-                    const uint4* k4 = reinterpret_cast<const uint4*>(sm.pkey);
+                    const uint32_t ke = s_pkey[e];
+                    const uint4* k4 = reinterpret_cast<const uint4*>(s_pkey);
                     const int n4 = (csz + 3) >> 2;
 #pragma unroll 4
                     for (int j4 = sub; j4 < n4; j4 += tpe) {
@@ -859,8 +1066,8 @@ __global__ void __launch_bounds__(kNT, 2)
                 }
                 const int32_t sel = (e < csz && sub == 0 && rk < r_part) ? 1 : 0;
                 int32_t tot;
-                const int32_t pos = block_excl_scan(sel, sm.wbuf, &tot);
-                if (sel && pos >= p_lo && pos < p_hi) sm.prow[pos - p_lo] = crow + e;
+                const int32_t pos = block_excl_scan(sel, s_wbuf, &tot);
+                if (sel && pos >= p_lo && pos < p_hi) s_prow[pos - p_lo] = crow + e;
             } else {
                 // radix select over 4 digits of 8 bits, most significant first: the threshold
                 // key theta and `pneed` = how many keys equal to theta are taken (the
@@ -869,31 +1076,31 @@ __global__ void __launch_bounds__(kNT, 2)
                 int32_t pneed = r_part;
                 for (int pass = 0; pass < 4; ++pass) {
                     const int shift = 24 - 8 * pass;
-                    sm.hist[tid] = 0;
+                    s_hist[tid] = 0;
                     __syncthreads();
                     for (int i = tid; i < csz; i += kNT) {
                         const uint32_t k = key_at(i);
-                        if ((k & mask) == prefix) atomicAdd(&sm.hist[(k >> shift) & 255u], 1);
+                        if ((k & mask) == prefix) atomicAdd(&s_hist[(k >> shift) & 255u], 1);
                     }
                     __syncthreads();
-                    if (warp == 0) radix_pick_bin(sm.hist, pneed, false, sm.wbuf + 32);
+                    if (warp == 0) radix_pick_bin(s_hist, pneed, false, s_wbuf + 32);
                     __syncthreads();
-                    pneed -= sm.wbuf[33];
-                    prefix |= (uint32_t)sm.wbuf[32] << shift;
+                    pneed -= s_wbuf[33];
+                    prefix |= (uint32_t)s_wbuf[32] << shift;
                     mask |= 255u << shift;
                 }
                 const uint32_t theta = prefix;
                 int32_t eq_run = 0, sel_run = 0;
-                for (int base = 0; base < csz; base += kNT) {
-                    const int i = base + tid;
+                for (int bse = 0; bse < csz; bse += kNT) {
+                    const int i = bse + tid;
                     const uint32_t k = i < csz ? key_at(i) : 0u;
                     const int32_t eq = (i < csz && k == theta) ? 1 : 0;
                     int32_t eq_tot;
-                    const int32_t eq_before = eq_run + block_excl_scan(eq, sm.wbuf, &eq_tot);
+                    const int32_t eq_before = eq_run + block_excl_scan(eq, s_wbuf, &eq_tot);
                     const int32_t sel = (i < csz) && (k > theta || (eq && eq_before < pneed));
                     int32_t sel_tot;
-                    const int32_t pos = sel_run + block_excl_scan(sel, sm.wbuf, &sel_tot);
-                    if (sel && pos >= p_lo && pos < p_hi) sm.prow[pos - p_lo] = crow + i;
+                    const int32_t pos = sel_run + block_excl_scan(sel, s_wbuf, &sel_tot);
+                    if (sel && pos >= p_lo && pos < p_hi) s_prow[pos - p_lo] = crow + i;
                     eq_run += eq_tot;
                     sel_run += sel_tot;
                 }
@@ -907,7 +1114,12 @@ __global__ void __launch_bounds__(kNT, 2)
             __syncthreads();
             const int32_t c0 = lo + ch * chunk;
             const int n = (hi - c0) < chunk ? (hi - c0) : chunk;
-            attend(n_chunks == 1 ? 0 : (ch & 1) * chunk, n, nullptr, true);
+            const int pb0 = n_chunks == 1 ? 0 : (ch & 1) * chunk;
+            if (kMixed) {
+                convert_far(pb0, n);
+                __syncthreads();
+            }
+            if (s_wbuf[kWBad] == 0) attend(pb0, n, nullptr, true);
             if (ch + 2 < n_chunks) {
                 __syncthreads();  // every warp is done with this slot
                 issue(ch + 2);
@@ -928,7 +1140,7 @@ __global__ void __launch_bounds__(kNT, 2)
     for (int hh = 0; hh < 2; ++hh) {
         const int hd = 2 * t4 + hh;
         if (hd < G) {
-            float* w = sm.wcomb + (warp * G + hd) * 130;
+            float* w = s_wcomb + (warp * G + hd) * kCombStride;
             if (g8 == 0) {
                 w[128] = m2[hh];
                 w[129] = l2[hh];
@@ -942,9 +1154,9 @@ __global__ void __launch_bounds__(kNT, 2)
     }
     __syncthreads();
     // per-head merge scales of the 8 warps, computed once
-    float* wsc = sm.scl;                     // [kWarps][G]
-    float* rsc = sm.scl + kWarps * G;        // [S][G]
-    float* sums = sm.scl + (kWarps + S) * G; // [G] max, [G] sum
+    float* wsc = s_scl;                     // [kWarps][G]
+    float* rsc = s_scl + kWarps * G;        // [S][G]
+    float* sums = s_scl + (kWarps + S) * G; // [G] max, [G] sum
     // thread (g, w) in groups of 8 lanes: warp w's state for head g
     static_assert(kWarps == 8, "the merge below maps one lane per warp in groups of 8");
     if (tid < 8 * G) {
@@ -952,13 +1164,13 @@ __global__ void __launch_bounds__(kNT, 2)
         const int active = min(32, 8 * G - 32 * warp);
         const uint32_t gmask = active >= 32 ? 0xffffffffu : ((1u << active) - 1u);
         const int g = tid >> 3, w = tid & 7;
-        const float mw = sm.wcomb[(w * G + g) * 130 + 128];
+        const float mw = s_wcomb[(w * G + g) * kCombStride + 128];
         float mx = mw;
 #pragma unroll
         for (int o = 4; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(gmask, mx, o));
         const float sc = mw == -INFINITY ? 0.f : exp2f(mw - mx);
         wsc[w * G + g] = sc;
-        float l = sm.wcomb[(w * G + g) * 130 + 129] * sc;
+        float l = s_wcomb[(w * G + g) * kCombStride + 129] * sc;
 #pragma unroll
         for (int o = 4; o > 0; o >>= 1) l += __shfl_xor_sync(gmask, l, o);
         if (w == 0) {
@@ -969,9 +1181,9 @@ __global__ void __launch_bounds__(kNT, 2)
     __syncthreads();
     // warps -> CTA partial, written into CTA 0's combine buffer
     {
-        const uint32_t dst0 = map_shared_rank(smem_u32(sm.ccomb), 0);
-        for (int t = tid; t < G * 130; t += kNT) {
-            const int g = t / 130, e = t % 130;
+        const uint32_t dst0 = map_shared_rank(smem_u32(s_ccomb), 0);
+        for (int t = tid; t < G * kCombStride; t += kNT) {
+            const int g = t / kCombStride, e = t % kCombStride;
             float v;
             if (e == 128) {
                 v = sums[g];
@@ -980,9 +1192,10 @@ __global__ void __launch_bounds__(kNT, 2)
             } else {
                 v = 0.f;
 #pragma unroll
-                for (int w = 0; w < kWarps; ++w) v = fmaf(sm.wcomb[(w * G + g) * 130 + e], wsc[w * G + g], v);
+                for (int w = 0; w < kWarps; ++w)
+                    v = fmaf(s_wcomb[(w * G + g) * kCombStride + e], wsc[w * G + g], v);
             }
-            st_cluster_f32(dst0 + (uint32_t)(((rank * G + g) * 130 + e) * 4), v);
+            st_cluster_f32(dst0 + (uint32_t)(((rank * G + g) * kCombStride + e) * 4), v);
         }
     }
     cluster_arrive_release();
@@ -993,12 +1206,12 @@ __global__ void __launch_bounds__(kNT, 2)
             const int active = min(32, S * G - 32 * warp);
             const uint32_t gmask = active >= 32 ? 0xffffffffu : ((1u << active) - 1u);
             const int g = tid / S, r = tid % S;
-            const float mr = sm.ccomb[(r * G + g) * 130 + 128];
+            const float mr = s_ccomb[(r * G + g) * kCombStride + 128];
             float mx = mr;
             for (int o = S >> 1; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(gmask, mx, o));
             const float sc = mr == -INFINITY ? 0.f : exp2f(mr - mx);
             rsc[r * G + g] = sc;
-            float l = sm.ccomb[(r * G + g) * 130 + 129] * sc;
+            float l = s_ccomb[(r * G + g) * kCombStride + 129] * sc;
             for (int o = S >> 1; o > 0; o >>= 1) l += __shfl_xor_sync(gmask, l, o);
             if (r == 0) sums[G + g] = 1.f / l;
         }
@@ -1009,7 +1222,7 @@ __global__ void __launch_bounds__(kNT, 2)
             float num = 0.f;
 #pragma unroll
             for (int r = 0; r < 16; ++r)
-                if (r < S) num = fmaf(sm.ccomb[(r * G + g) * 130 + d], rsc[r * G + g], num);
+                if (r < S) num = fmaf(s_ccomb[(r * G + g) * kCombStride + d], rsc[r * G + g], num);
             o[t] = num * sums[G + g];
         }
         if (a.sel_count && tid == 0) a.sel_count[unit] = (int32_t)T;
@@ -1024,57 +1237,15 @@ __global__ void __launch_bounds__(kNT, 2)
 // whose share is at most budget / S + 1.
 int32_t prow_capacity(int budget, int S) { return (int32_t)(2 * ((int64_t)budget / S) + 2); }
 
-size_t smem_bytes(int G, int S, int C, int budget, int RB) {
-    const int32_t pc = prow_capacity(budget, S);
-    size_t b = 0;
-    auto add = [&](size_t x) { b += (x + 127) & ~(size_t)127; };
-    size_t ring = (size_t)RB * kRowBytes;
-    ring = ring > sizeof(float) * kWarps * G * 130 ? ring : sizeof(float) * kWarps * G * 130;
-    ring = ring > sizeof(uint32_t) * (kPartCap + 4) ? ring : sizeof(uint32_t) * (kPartCap + 4);
-    add(ring);
-    add(sizeof(float) * G * kD);
-    add(sizeof(float) * kD);
-    add(sizeof(float) * C);
-    add(sizeof(int32_t) * (C + 1));
-    add(sizeof(int32_t) * (C + 1));
-    add(sizeof(int32_t) * (C + 1));
-    add(sizeof(uint64_t) * cand_slots(C));
-    add(sizeof(int32_t) * cand_slots(C));
-    add(sizeof(int32_t) * 256);
-    add(sizeof(int32_t) * 256);
-    add(sizeof(uint32_t) * (RB + 4));
-    add(sizeof(int32_t) * pc);
-    add(sizeof(int32_t) * 96);
-    add(sizeof(float) * ((kWarps + S) * G + 2 * G));
-    add(sizeof(float) * S * G * 130);
-    add(sizeof(int32_t) * RB);
-    add(sizeof(uint16_t) * G * kD);
-    add(sizeof(uint16_t) * kWarps * 256);
-    add(sizeof(uint64_t));
-    return b;
-}
-
-// Ring rows for a cluster size S: enough for one CTA's even share of the budget in one
-// chunk (128 to 256 rows), reduced while two CTAs would not fit one SM's shared memory.
-int ring_rows(int G, int S, int C, int budget) {
-    const int64_t share = (int64_t)budget / (S > 1 ? S - 1 : 1) + 2;
-    int rb = (int)(share > 256 ? 256 : ((share + 31) / 32) * 32);
-    if (rb < 128) rb = 128;  // also holds most cut clusters whole
-    const size_t two_per_sm = 113 * 1024;
-    while (rb > 64 && smem_bytes(G, S, C, budget, rb) > two_per_sm) rb -= 32;
-    return rb;
-}
-
 struct Plan {
-    int S = 0;
-    int RB = 0;
+    Params p{};
     size_t smem = 0;
 };
 
 // Clusters of S CTAs with `smem` bytes each that can be resident at once (0 when none). Raises
 // the kernel's shared-memory limit and allows 16-CTA clusters as needed.
-int max_active_clusters(void (*kern)(DecodeArgs, int32_t, int32_t, int32_t), int S, size_t smem,
-                        size_t* smem_set, bool* nonportable_set, int* nclusters) {
+int max_active_clusters(void (*kern)(DecodeArgs, Params), int S, size_t smem, size_t* smem_set,
+                        bool* nonportable_set, int* nclusters) {
     *nclusters = 0;
     if (smem > *smem_set) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -1105,10 +1276,21 @@ int max_active_clusters(void (*kern)(DecodeArgs, int32_t, int32_t, int32_t), int
     return CKV_OK;
 }
 
-// One launch plan per (device, group size, units, C, budget), found once. The cluster size S
-// is the largest power of two <= 16 whose clusters for all units are resident at once (one
-// wave), with U * S <= 2 * SMs; otherwise the smallest S that fits in shared memory.
-template <int G, bool kPerHead>
+// Ring rows for a cluster of S CTAs: one CTA's even share of the budget (plus the cut
+// cluster's usual size) in one chunk, at least 128 and at most 256 rows, in steps of 16.
+int ring_rows(int S, int budget) {
+    const int64_t share = (int64_t)budget / (S > 1 ? S - 1 : 1) + 2;
+    int64_t rb = ((share + 15) / 16) * 16;
+    if (rb < 128) rb = 128;  // also holds most cut clusters whole
+    if (rb > 256) rb = 256;
+    return (int)rb;
+}
+
+// One launch plan per (device, units, C, budget), found once. The cluster size S is the
+// largest power of two <= 16 (and <= 64 / G, which bounds CTA 0's combine buffer) with all
+// U * S CTAs on distinct SMs; with more units than SMs, S = 1. The ring takes one CTA's share
+// of the budget, reduced in steps of 16 rows while the launch does not fit.
+template <int G, bool kPerHead, bool kMixed>
 int plan_for(const DecodeArgs& a, int num_sms, Plan* out) {
     static std::mutex mtx;
     static std::map<std::tuple<int, int, int, int>, Plan> cache;
@@ -1127,34 +1309,23 @@ int plan_for(const DecodeArgs& a, int num_sms, Plan* out) {
         *out = it->second;
         return CKV_OK;
     }
-    auto kern = select_attend_kernel<G, kPerHead>;
+    auto kern = select_attend_kernel<G, kPerHead, kMixed>;
     Plan best{};
-    // Few units: one CTA per SM (a 256-row ring makes two CTAs too large for one SM) and at
-    // most half of the SMs per launch, so that the next launch's CTAs, started early by
-    // programmatic dependent launch, wait on other SMs instead of sharing these.
-    for (int S = 16; S >= 2 && best.S == 0; S /= 2) {
-        if ((int64_t)U * S * 2 > num_sms) continue;
-        const int RB = 256;
-        const size_t smem = smem_bytes(G, S, a.C, a.budget, RB);
-        if (smem > 227 * 1024 || smem < 116 * 1024) continue;
-        int nclusters = 0;
-        const int rc = max_active_clusters(kern, S, smem, &smem_set, &nonportable_set, &nclusters);
-        if (rc != CKV_OK) return rc;
-        if (nclusters >= U) best = Plan{S, RB, smem};
+    for (int S = 16; S >= 1 && best.p.S == 0; S /= 2) {
+        if (S > 1 && (S * G > 64 || (int64_t)U * S > num_sms)) continue;
+        for (int RB = ring_rows(S, a.budget); RB >= 64 && best.p.S == 0; RB -= 16) {
+            const int pc = prow_capacity(a.budget, S);
+            const Layout L = make_layout(G, S, a.C, RB, pc);
+            if (L.total > 227 * 1024) continue;
+            int nclusters = 0;
+            const int rc = max_active_clusters(kern, S, L.total, &smem_set, &nonportable_set, &nclusters);
+            if (rc != CKV_OK) return rc;
+            if (nclusters <= 0) continue;
+            best.p = Params{S, RB, pc};
+            best.smem = L.total;
+        }
     }
-    for (int S = 16; S >= 1 && best.S == 0; S /= 2) {
-        const int RB = ring_rows(G, S, a.C, a.budget);
-        const size_t smem = smem_bytes(G, S, a.C, a.budget, RB);
-        if (smem > 227 * 1024) continue;
-        if ((int64_t)U * S > 2 * (int64_t)num_sms && S > 1) continue;
-        int nclusters = 0;
-        const int rc = max_active_clusters(kern, S, smem, &smem_set, &nonportable_set, &nclusters);
-        if (rc != CKV_OK) return rc;
-        if (nclusters <= 0) continue;
-        best = Plan{S, RB, smem};
-        if (nclusters >= U) break;
-    }
-    if (best.S == 0) {
+    if (best.p.S == 0) {
         set_error("select_and_attend: no launch shape fits (budget or C too large for shared memory)");
         return CKV_ECAPACITY;
     }
@@ -1163,14 +1334,13 @@ int plan_for(const DecodeArgs& a, int num_sms, Plan* out) {
     return CKV_OK;
 }
 
-template <int G, bool kPerHead = false>
+template <int G, bool kPerHead = false, bool kMixed = false>
 int launch_g(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     Plan plan;
-    int rc = plan_for<G, kPerHead>(a, num_sms, &plan);
+    int rc = plan_for<G, kPerHead, kMixed>(a, num_sms, &plan);
     if (rc != CKV_OK) return rc;
     const int U = a.B * a.Hkv;
-    const int S = plan.S;
-    const int32_t pc = prow_capacity(a.budget, S);
+    const int S = plan.p.S;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)(U * S));
     cfg.blockDim = dim3(kNT);
@@ -1185,8 +1355,7 @@ int launch_g(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     attrs[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attrs;
     cfg.numAttrs = 2;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, select_attend_kernel<G, kPerHead>, a, (int32_t)S, pc,
-                                       (int32_t)plan.RB);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, select_attend_kernel<G, kPerHead, kMixed>, a, plan.p);
     if (e != cudaSuccess) return cuda_fail(e, "select_attend: launch");
     return CKV_OK;
 }
@@ -1199,6 +1368,20 @@ int launch_select_attend_per_head(const DecodeArgs& a, int num_sms, cudaStream_t
         return CKV_EINVAL;
     }
     return launch_g<1, true>(a, num_sms, s);
+}
+
+int launch_select_attend_mixed(const DecodeArgs& a, int num_sms, cudaStream_t s) {
+    switch (a.G) {
+        case 1: return launch_g<1, false, true>(a, num_sms, s);
+        case 2: return launch_g<2, false, true>(a, num_sms, s);
+        case 3: return launch_g<3, false, true>(a, num_sms, s);
+        case 4: return launch_g<4, false, true>(a, num_sms, s);
+        case 5: return launch_g<5, false, true>(a, num_sms, s);
+        case 6: return launch_g<6, false, true>(a, num_sms, s);
+        case 7: return launch_g<7, false, true>(a, num_sms, s);
+        case 8: return launch_g<8, false, true>(a, num_sms, s);
+        default: set_error("select_and_attend_mixed: group size must be 1..8"); return CKV_EINVAL;
+    }
 }
 
 int launch_select_attend(const DecodeArgs& a, int num_sms, cudaStream_t s) {

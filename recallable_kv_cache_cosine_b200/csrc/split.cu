@@ -10,15 +10,19 @@
 //   - the threshold is a parameter;
 //   - a cluster with drift above the threshold and at least two members is split by cosine
 //     K-means with 2 clusters on its own rows (the prefill's init rule and iteration count),
-//     at most `room` clusters per unit, lowest index first.
+//     at most `room` clusters per unit, lowest index first; `room` is the caller's maximum
+//     clamped to the clusters left, and every unit ends with exactly C + room clusters
+//     (units that split fewer pad with empty clusters), so the host knows the new count
+//     without reading anything back.
 // The two halves take indices c' and c' + 1 (c' = c + splits below c); later clusters shift
 // up. Rows move only inside the cluster's own segment (first half, then second half, each in
 // its previous order), so the token ids stay ascending inside every cluster.
 //
 // Five launches, one pass each:
-//   drift    one warp per (unit, cluster): the mean cosine distance, fp32;
-//   plan     one CTA per unit: flags, the cap, the new index of every cluster (a block scan);
-//   kmeans   one CTA per (cluster, unit), idle unless the cluster splits: 2-means on the
+//   drift    one warp per (unit, cluster), 16 rows in flight: the mean cosine distance, fp32;
+//   plan     one CTA per unit: flags, the cap, the new index of every cluster (a block scan),
+//            and the unit's list of clusters to split;
+//   kmeans   one CTA per (list entry, unit) for at most `room` entries: 2-means on the
 //            segment (staged in shared memory up to 192 rows, else read from global memory),
 //            then the stable partition of its K/V rows and ids through a row scratch;
 //   scatter  one warp per (cluster, unit): the cluster's centroid(s) and offset(s) go to
@@ -65,13 +69,14 @@ __global__ void __launch_bounds__(kDriftWarps * 32) drift_kernel(const SplitArgs
     const float nm = __fsqrt_rn(mm);
     const uint16_t* base = a.kp + (int64_t)u * a.kp_ustride * kD + lane * 4;
     float acc = 0.f;
-    for (int32_t j = lo; j < hi; j += 4) {
-        uint2 w[4];
+    constexpr int kInFlight = 16;
+    for (int32_t j = lo; j < hi; j += kInFlight) {  // warp-uniform trip count
+        uint2 w[kInFlight];
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int r = 0; r < kInFlight; ++r)
             if (j + r < hi) w[r] = *reinterpret_cast<const uint2*>(base + (int64_t)(j + r) * kD);
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
+        for (int r = 0; r < kInFlight; ++r) {
             if (j + r >= hi) break;  // warp-uniform
             const float k0 = bf16_lo(w[r].x), k1 = bf16_hi(w[r].x), k2 = bf16_lo(w[r].y),
                         k3 = bf16_hi(w[r].y);
@@ -117,6 +122,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const SplitArgs a) {
             const bool kept = f && before < a.room;
             const int ni = c + min(before, a.room);
             a.plan[(int64_t)u * a.Cmax + c] = 2 * ni + (kept ? 1 : 0);
+            if (kept) a.tasks[(int64_t)u * a.Cmax + before] = c;  // the unit's split list
         }
         __syncthreads();
         if (tid == 0) carry += total;
@@ -128,8 +134,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const SplitArgs a) {
 __global__ void __launch_bounds__(kSplitThreads) split_kmeans_kernel(const SplitArgs a) {
     pdl_launch_dependents();
     pdl_wait();
-    const int c = blockIdx.x, u = blockIdx.y;
-    if (!(a.plan[(int64_t)u * a.Cmax + c] & 1)) return;  // whole CTA: this cluster stays
+    const int k = blockIdx.x, u = blockIdx.y;
+    if (k >= a.count[u]) return;  // whole CTA: fewer splits in this unit
+    const int c = a.tasks[(int64_t)u * a.Cmax + k];
     extern __shared__ __align__(16) uint8_t smem_raw[];
     uint16_t* skey = (uint16_t*)smem_raw;                     // [kStageRows][128] bf16
     int32_t* slab = (int32_t*)(skey + (size_t)kStageRows * kD);  // [kStageRows]
@@ -296,9 +303,7 @@ __global__ void __launch_bounds__(kDriftWarps * 32) scatter_kernel(const SplitAr
     pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u = blockIdx.y, c = blockIdx.x * kDriftWarps + warp;
-    int mx = 0;
-    for (int i = 0; i < a.U; ++i) mx = max(mx, a.count[i]);
-    const int Cu = a.C + a.count[u], Cn = a.C + mx;
+    const int Cu = a.C + a.count[u], Cn = a.C + a.room;
     const int32_t* off = a.offsets + (int64_t)u * a.off_ustride;
     float4* mu2 = reinterpret_cast<float4*>(a.mu2 + (int64_t)u * a.Cmax * kD);
     int32_t* off2 = a.off2 + (int64_t)u * (a.Cmax + 1);
@@ -327,13 +332,12 @@ __global__ void __launch_bounds__(kDriftWarps * 32) scatter_kernel(const SplitAr
 
 // The scratch copy back into the store: clusters [0, Cn) and offsets [0, Cn].
 __global__ void __launch_bounds__(kDriftWarps * 32) copy_back_kernel(const SplitArgs a) {
-    pdl_launch_dependents();
+    // The last kernel of a split: no early trigger, so a following decode kernel, which reads
+    // the cluster store before its dependency wait, starts once the store is complete.
     pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u = blockIdx.y, c = blockIdx.x * kDriftWarps + warp;
-    int mx = 0;
-    for (int i = 0; i < a.U; ++i) mx = max(mx, a.count[i]);
-    const int Cn = a.C + mx;
+    const int Cn = a.C + a.room;
     if (c > Cn) return;
     if (c < Cn)
         reinterpret_cast<float4*>(a.mu + ((int64_t)u * a.mu_ustride + c) * kD)[lane] =
@@ -357,10 +361,12 @@ int launch_split(const SplitArgs& a, cudaStream_t s) {
     const size_t smem = (size_t)kStageRows * kD * 2 + (size_t)kStageRows * 4 + 8 * kD * 4 + 16;
     const int rc = ensure_smem((const void*)split_kmeans_kernel, smem, "split: set smem");
     if (rc != CKV_OK) return rc;
-    e = launch_pdl(split_kmeans_kernel, dim3(a.C, a.U), dim3(kSplitThreads), smem, s, a);
-    if (e != cudaSuccess) return cuda_fail(e, "split: kmeans launch");
-    // grids cover every cluster a unit can end with (Cmax) plus the closing offset
-    const dim3 gw((a.Cmax + 1 + kDriftWarps - 1) / kDriftWarps, a.U);
+    if (a.room > 0) {
+        e = launch_pdl(split_kmeans_kernel, dim3(a.room, a.U), dim3(kSplitThreads), smem, s, a);
+        if (e != cudaSuccess) return cuda_fail(e, "split: kmeans launch");
+    }
+    // grids cover every cluster a unit ends with (C + room) plus the closing offset
+    const dim3 gw((a.C + a.room + 1 + kDriftWarps - 1) / kDriftWarps, a.U);
     e = launch_pdl(scatter_kernel, gw, dim3(kDriftWarps * 32), 0, s, a);
     if (e != cudaSuccess) return cuda_fail(e, "split: scatter launch");
     e = launch_pdl(copy_back_kernel, gw, dim3(kDriftWarps * 32), 0, s, a);

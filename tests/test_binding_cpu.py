@@ -43,7 +43,7 @@ def test_host_or_mistyped_tensors_are_refused_before_the_library():
     with pytest.raises(TypeError):
         obj.cluster_prefill(0, torch.zeros(1, 8, 64, 128), torch.zeros(1, 8, 64, 128), 4)
     with pytest.raises(TypeError):
-        obj.split_drifted_clusters(0, 0.5, drift=torch.zeros(8, 4))
+        obj.split_drifted_clusters(0, 0.5, 4, drift=torch.zeros(8, 4))
 
 
 def test_null_context_calls_raise_with_the_reason():
@@ -52,6 +52,6 @@ def test_null_context_calls_raise_with_the_reason():
         obj.recluster_increment(0, stream=0)  # an explicit (null) stream handle
     assert e.value.code == ckv.CKV_EINVAL and "context" in str(e.value)
     with pytest.raises(ckv.CkvError):
-        obj.split_drifted_clusters(0, 0.5, stream=0)
+        obj.split_drifted_clusters(0, 0.5, 4, stream=0)
     with pytest.raises(ckv.CkvError):
         obj.layer_info(0)

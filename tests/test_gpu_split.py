@@ -11,7 +11,9 @@ so both sides start from identical inputs.
   centroids are the means of their rows; the halves' centroids within 1e-3;
 * every other cluster: rows and centroid unchanged, at its shifted index; padding clusters
   empty with a zero centroid;
-* decode on the split store matches the oracle.
+* decode on the split store matches the oracle;
+* the layer's cluster count grows by exactly min(max_splits, room), with no read-back, so the
+  call can be captured in a CUDA graph (checked by capturing one and replaying it).
 """
 import math
 
@@ -40,6 +42,14 @@ def _ctx(B, Hkv, n, C, n_centers, seed, max_clusters, G=4, window=320):
     ctx.cluster_prefill(0, to_dev(K), to_dev(V), C)
     torch.cuda.synchronize()
     return ctx, K, V
+
+
+def _split(ctx, layer, tau, max_splits, drift=None):
+    """split_drifted_clusters with its per-unit split counts read back as a list."""
+    U = ctx.cfg.batch * ctx.cfg.n_kv_heads
+    cnt = torch.full((U,), -1, device="cuda", dtype=torch.int32)
+    ctx.split_drifted_clusters(layer, tau, max_splits, drift, cnt)
+    return cnt.tolist()
 
 
 def _stores(ctx, B, Hkv, windows=0):
@@ -144,13 +154,14 @@ def test_split_matches_oracle(B, Hkv, n, C, n_centers, q):
     drifts = [oracle.cluster_drift(st) for st in pre]
     tau = _threshold_in_gap(drifts, q)
     drift_gpu = torch.full((U, C), -7.0, device="cuda", dtype=torch.float32)
-    splits = ctx.split_drifted_clusters(0, tau, drift_gpu)
+    room = (2 * C + 8) - C
+    splits = _split(ctx, 0, tau, room, drift_gpu)
     ctx.check_device_error()
     d = drift_gpu.cpu().numpy()
     for u in range(U):
         assert np.abs(d[u] - drifts[u]).max() <= DRIFT_TOL
     info = ctx.layer_info(0)
-    assert info.C == C + max(splits) and info.m == n - 16
+    assert info.C == C + room and info.m == n - 16
     post = _stores(ctx, B, Hkv)
     stats = {}
     for u in range(U):
@@ -170,29 +181,30 @@ def test_split_large_clusters_through_global_memory():
     ctx, _, _ = _ctx(B, Hkv, n, C, 8, seed, max_clusters=8)
     pre = _stores(ctx, B, Hkv)
     assert all(np.diff(st.offsets).max() > 384 for st in pre)
-    splits = ctx.split_drifted_clusters(0, -math.inf)
+    splits = _split(ctx, 0, -math.inf, 6)
     ctx.check_device_error()
-    assert splits == [2, 2] and ctx.layer_info(0).C == 4
+    assert splits == [2, 2] and ctx.layer_info(0).C == 8  # 2 + 6: two splits, two padding
     post = _stores(ctx, B, Hkv)
     stats = {}
     for u in range(B * Hkv):
         want, flags = oracle.split_drifted(pre[u], -math.inf, seed, u, room=6, iters=iters)
-        _check_split_unit(pre[u], post[u], want, flags, seed, u, iters, stats)
+        _check_split_unit(pre[u], post[u], oracle.pad_clusters(want, 8), flags, seed, u, iters, stats)
     _decode_all(ctx, B, Hkv, 4, 700, seed, 0, {})
 
 
 def test_split_room_cap_padding_and_no_op():
     B, Hkv, n, C, seed = 1, 2, 2048, 16, 3
-    ctx, _, _ = _ctx(B, Hkv, n, C, 20, seed, max_clusters=C + 3)
+    ctx, _, _ = _ctx(B, Hkv, n, C, 20, seed, max_clusters=C + 5)
     pre = _stores(ctx, B, Hkv)
-    # +inf splits nothing and leaves every byte of the store as it was
-    assert ctx.split_drifted_clusters(0, math.inf) == [0, 0]
+    # +inf with max_splits 0 only measures: every byte of the store stays as it was
+    assert _split(ctx, 0, math.inf, 0) == [0, 0]
+    assert ctx.layer_info(0).C == C
     same = _stores(ctx, B, Hkv)
     for a, b in zip(pre, same):
         for name in ("kp", "vp", "ids", "offsets", "mu"):
             np.testing.assert_array_equal(getattr(a, name), getattr(b, name))
-    # -inf: every cluster of 2+ rows qualifies; the room of 3 keeps the lowest three
-    splits = ctx.split_drifted_clusters(0, -math.inf)
+    # -inf: every cluster of 2+ rows qualifies; max_splits 3 keeps the lowest three
+    splits = _split(ctx, 0, -math.inf, 3)
     assert splits == [3, 3] and ctx.layer_info(0).C == C + 3
     post = _stores(ctx, B, Hkv)
     stats = {}
@@ -200,10 +212,55 @@ def test_split_room_cap_padding_and_no_op():
         want, flags = oracle.split_drifted(pre[u], -math.inf, seed, u, room=3)
         np.testing.assert_array_equal(np.flatnonzero(flags), np.flatnonzero(np.diff(pre[u].offsets) >= 2)[:3])
         _check_split_unit(pre[u], post[u], want, flags, seed, u, 10, stats)
-    # no room left: nothing splits
-    assert ctx.split_drifted_clusters(0, -math.inf) == [0, 0]
-    assert ctx.layer_info(0).C == C + 3
+    # +inf with max_splits 2: nothing splits, the count still grows by 2 (empty padding)
+    assert _split(ctx, 0, math.inf, 2) == [0, 0]
+    assert ctx.layer_info(0).C == C + 5
+    padded = _stores(ctx, B, Hkv)
+    for a, b in zip(post, padded):
+        np.testing.assert_array_equal(b.offsets[: a.C + 1], a.offsets)
+        np.testing.assert_array_equal(b.mu[: a.C], a.mu)
+        assert np.all(b.offsets[a.C:] == b.m) and not b.mu[a.C:].any()
+    # no room left: nothing splits and the count stays
+    assert _split(ctx, 0, -math.inf, 4) == [0, 0]
+    assert ctx.layer_info(0).C == C + 5
     ctx.check_device_error()
+    _decode_all(ctx, B, Hkv, 4, 500, seed, 0, {})
+
+
+def test_split_is_captured_in_a_cuda_graph():
+    """The split needs no read-back, so it can be recorded in a CUDA graph with a decode step
+    after it; one replay gives the oracle's split and decode."""
+    B, Hkv, n, C, seed, G = 1, 2, 3000, 12, 8, 4
+    ctx, _, _ = _ctx(B, Hkv, n, C, 30, seed, max_clusters=C + 16)
+    ctx.split_drifted_clusters(0, math.inf, 0)  # first call: allocates the scratch
+    torch.cuda.synchronize()
+    pre = _stores(ctx, B, Hkv)
+    tau = _threshold_in_gap([oracle.cluster_drift(st) for st in pre], 0.5)
+    budget = 400
+    q = np.stack([si.queries(seed, 0, b, 1, Hkv * G)[0] for b in range(B)])
+    qd = to_dev(q)
+    out = torch.empty(B, Hkv * G, 128, device="cuda", dtype=torch.float32)
+    sel = torch.empty(B, Hkv, budget, device="cuda", dtype=torch.int32)
+    cnt = torch.empty(B, Hkv, device="cuda", dtype=torch.int32)
+    splits = torch.zeros(B * Hkv, device="cuda", dtype=torch.int32)
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s, capture_error_mode="thread_local"):
+        ctx.split_drifted_clusters(0, tau, 8, splits=splits, stream=s)
+        ctx.select_and_attend(0, qd, budget, out, sel, cnt, stream=s)
+    assert ctx.layer_info(0).C == C + 8  # the host count moved at capture
+    g.replay()
+    torch.cuda.synchronize()
+    ctx.check_device_error()
+    post = _stores(ctx, B, Hkv)
+    stats = {}
+    for u in range(B * Hkv):
+        want, flags = oracle.split_drifted(pre[u], tau, seed, u, room=8)
+        assert int(splits[u]) == int(flags.sum())
+        _check_split_unit(pre[u], post[u], oracle.pad_clusters(want, C + 8), flags, seed, u, 10, stats)
+        check_decode_unit(post[u], q[0, u * G:(u + 1) * G], budget, out[0, u * G:(u + 1) * G].cpu().numpy(),
+                          sel[0, u].cpu().numpy(), int(cnt[0, u]), stats)
+    del g
 
 
 def test_split_then_window_recluster_and_decode():
@@ -211,8 +268,8 @@ def test_split_then_window_recluster_and_decode():
     ctx, _, _ = _ctx(B, Hkv, n, C, 20, seed, max_clusters=48)
     pre = _stores(ctx, B, Hkv)
     tau = _threshold_in_gap([oracle.cluster_drift(st) for st in pre], 0.6)
-    splits = ctx.split_drifted_clusters(0, tau)
-    C1 = C + max(splits)
+    ctx.split_drifted_clusters(0, tau, 8)
+    C1 = C + 8
     AK = np.empty((B, Hkv, W, 128), np.uint16)
     AV = np.empty_like(AK)
     for h in range(Hkv):
@@ -236,11 +293,13 @@ def test_split_then_window_recluster_and_decode():
     # a second split pass uses the window number in its init key
     pre2 = _stores(ctx, B, Hkv, windows=1)
     tau2 = _threshold_in_gap([oracle.cluster_drift(st) for st in pre2], 0.5)
-    splits2 = ctx.split_drifted_clusters(0, tau2)
+    room2 = 48 - pre2[0].C
+    splits2 = _split(ctx, 0, tau2, room2)
     post2 = _stores(ctx, B, Hkv, windows=1)
+    assert post2[0].C == 48
     stats = {}
     for u in range(2):
-        want, flags = oracle.split_drifted(pre2[u], tau2, seed, u, room=48 - pre2[u].C)
+        want, flags = oracle.split_drifted(pre2[u], tau2, seed, u, room=room2)
         assert splits2[u] == int(flags.sum())
         want = oracle.pad_clusters(want, post2[u].C)
         _check_split_unit(pre2[u], post2[u], want, flags, seed, u, 10, stats)
@@ -251,15 +310,18 @@ def test_split_argument_and_state_errors():
     import recallable_kv_cache_cosine_b200 as ckv
     ctx = ckv.ClusterKV(2, 1, 2, 8, capacity=2048 + 640, max_clusters=24, seed=1)
     with pytest.raises(ckv.CkvError) as e:
-        ctx.split_drifted_clusters(0, 0.5)   # layer not prefilled
+        ctx.split_drifted_clusters(0, 0.5, 4)   # layer not prefilled
     assert e.value.code == ckv.CKV_ESTATE
     K = to_dev(np.stack([np.stack([si.keys_values(1, h, 2048, 10)[0] for h in range(2)])]))
     ctx.cluster_prefill(0, K, K, 12)
     with pytest.raises(ckv.CkvError) as e:
-        ctx.split_drifted_clusters(0, float("nan"))
+        ctx.split_drifted_clusters(0, float("nan"), 4)
     assert e.value.code == ckv.CKV_EINVAL
     with pytest.raises(ckv.CkvError) as e:
-        ctx.split_drifted_clusters(5, 0.5)
+        ctx.split_drifted_clusters(0, 0.5, -1)
+    assert e.value.code == ckv.CKV_EINVAL
+    with pytest.raises(ckv.CkvError) as e:
+        ctx.split_drifted_clusters(5, 0.5, 4)
     assert e.value.code == ckv.CKV_EINVAL
     assert ctx.layer_info(0).C == 12
     ctx.check_device_error()

@@ -1,16 +1,21 @@
-"""The decode kernel's way of finding the cut, restated in Python, agrees with the oracle's
-sorted walk (ClusterKV explainer, section 3.3) on adversarial cases.
+"""The decode kernel's way of finding the cut and laying out the selected rows, restated in
+Python, agrees with the oracle's sorted walk (ClusterKV explainer, section 3.3) on
+adversarial cases.
 
 The kernel does not sort the clusters. Each CTA:
 1. maps the fp32 scores monotonically onto 256 linear buckets between the smallest and the
-   largest score;
+   largest score of the clusters with tokens;
 2. builds a histogram of cluster sizes per bucket and finds the bucket b* holding the cut
    (the first cluster, in descending (score, -index) order, whose inclusive size exceeds the
-   remaining budget);
-3. ranks exactly, by the key (orderable score, -index), only the clusters in buckets >= b*;
-   the orderable score maps -0 and +0 to one key, so they tie like equal doubles.
-   A cluster whose exclusive prefix plus its size fits is whole; the one whose prefix fits
-   but whose size does not is the cut.
+   remaining budget) and the tokens in the buckets above it;
+3. ranks exactly, by the key (orderable score, -index), only the clusters of bucket b*; the
+   orderable score maps -0 and +0 to one key, so they tie like equal doubles. The cut is the
+   one whose prefix (tokens above b* plus the b* clusters before it) fits while its size
+   does not; the whole clusters are every cluster of a higher bucket and the b* clusters
+   ranked before the cut;
+4. lays the whole clusters out in cluster-index order: spre is the exclusive prefix of the
+   whole sizes, and selection position x maps to the last cluster c with spre[c] <= x, row
+   offsets[c] + x - spre[c] (a binary search).
 
 This model is checked against the oracle's `select` on stores whose scores are exactly the
 chosen fp32 values (centroid c = s_c * e_0, query e_0): many ties, all-equal scores, a tiny
@@ -31,32 +36,57 @@ def _orderable(x: np.float32) -> int:
 
 
 def bucket_cut(sc: np.ndarray, sz: np.ndarray, R: int):
-    """Whole clusters (set), cut cluster and its exclusive prefix, or None if all fit."""
+    """Whole clusters (set), cut cluster and W (tokens in whole clusters), or None if all fit."""
     sc = sc.astype(np.float32)
     if sz.sum() <= R:
         return None
-    mn, mx = sc.min(), sc.max()
+    live = sz > 0
+    keys = [_orderable(x) for x in sc[live]]
+    mn = np.float32(sc[live][int(np.argmin(keys))])
+    mx = np.float32(sc[live][int(np.argmax(keys))])
     span = np.float32(mx - mn)
     inv = np.float32(255.99) / span if span > 1e-30 else np.float32(0)
     b = np.clip(np.nan_to_num((sc - mn).astype(np.float32) * inv, nan=0.0), 0, 255).astype(np.int64)
     hist = np.zeros(256, np.int64)
-    np.add.at(hist, b[sz > 0], sz[sz > 0])
+    np.add.at(hist, b[live], sz[live])
     above, bstar = 0, 0
     for d in range(255, -1, -1):
         if above <= R < above + hist[d]:
             bstar = d
             break
         above += hist[d]
-    cand = [c for c in range(len(sc)) if b[c] >= bstar]
-    key = {c: (_orderable(sc[c]) << 32) | (0xFFFFFFFF - c) for c in cand}
-    whole, cut = set(), None
+    cand = [c for c in range(len(sc)) if sz[c] > 0 and b[c] == bstar]
+    key = {c: (_orderable(sc[c]) << 32) | (0xFFFFFFFF - c) for c in range(len(sc))}
+    cuts = []
     for c in cand:
         pre = sum(int(sz[j]) for j in cand if key[j] > key[c])
-        if pre + sz[c] <= R:
-            whole.add(c)
-        elif pre <= R:
-            cut = (c, pre)
-    return whole, cut[0], cut[1]
+        if above + pre <= R < above + pre + sz[c]:
+            cuts.append((c, pre))
+    assert len(cuts) == 1
+    cut, pre_cut = cuts[0]
+    whole = {c for c in range(len(sc))
+             if sz[c] > 0 and (b[c] > bstar or (b[c] == bstar and key[c] > key[cut]))}
+    return whole, cut, above + pre_cut
+
+
+def layout_rows(offs: np.ndarray, whole: set, W: int) -> list:
+    """Store rows of selection positions 0..W-1 of the whole clusters (cluster-index order)."""
+    C = len(offs) - 1
+    wsz = [int(offs[c + 1] - offs[c]) if c in whole else 0 for c in range(C)]
+    spre = np.concatenate([[0], np.cumsum(wsz)]).astype(np.int64)
+    assert spre[C] == W
+    rows = []
+    for x in range(W):
+        k0, khi = 0, C - 1  # last cluster with spre[k] <= x
+        while k0 < khi:
+            mid = (k0 + khi + 1) >> 1
+            if spre[mid] <= x:
+                k0 = mid
+            else:
+                khi = mid - 1
+        assert k0 in whole and spre[k0] <= x < spre[k0] + wsz[k0]
+        rows.append(int(offs[k0] + x - spre[k0]))
+    return rows
 
 
 def _store(sc, sz):
@@ -96,11 +126,16 @@ def test_bucket_histogram_cut_equals_the_sorted_walk():
         if got is None:
             assert sel.cut == -1
             continue
-        whole, cut, pre = got
+        whole, cut, W = got
         assert cut == sel.cut, (trial, cut, sel.cut)
-        assert R - pre == sel.r, (trial, R - pre, sel.r)
+        assert R - W == sel.r, (trial, R - W, sel.r)
         taken = {int(c) for c in np.searchsorted(st.offsets, sel.rows[sel.rows >= 0], side="right") - 1}
-        nonempty_whole = {c for c in whole if sz[c] > 0}
-        assert nonempty_whole == taken - {cut}, trial
+        assert whole == taken - {cut}, trial
+        # the whole clusters' rows, laid out by cluster index, are the oracle's whole rows
+        rows = layout_rows(st.offsets, whole, W)
+        assert len(set(rows)) == W
+        want = {int(r) for r in sel.rows[sel.rows >= 0]
+                if not (st.offsets[cut] <= r < st.offsets[cut + 1])}
+        assert set(rows) == want, trial
         checked += 1
     assert checked > 600
