@@ -38,11 +38,6 @@ CKV_DEV void store_centroid(float4 v, float* mu_row, uint16_t* muhat_row) {
     reinterpret_cast<uint2*>(muhat_row)[lane] = h;
 }
 
-CKV_DEV float4 load_row4_bf16(const uint16_t* row) {
-    const uint2 w = reinterpret_cast<const uint2*>(row)[lane_id()];
-    return make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
-}
-
 // ---------------------------------------------------------------------- init
 // Seeded init: the first C entries of a Fisher-Yates shuffle of 0..m-1, driven by SplitMix64
 // with key seed ^ (unit << 32) ^ window, each draw mapped into [0, m-i) by Lemire's
@@ -52,9 +47,12 @@ CKV_DEV float4 load_row4_bf16(const uint16_t* row) {
 // changed before step i only as the target of an earlier step, so a[p] before step i is the
 // value position s held just before step s, s being the last step < i with j_s = p (prev[i]),
 // or p itself if there is none; and the value position s held before step s is, by the same
-// rule, found by following the last step < s with j = s (link[s]) until a step whose own
-// position was never a target: that step's index is the value. Each thread scans the earlier
-// targets for its steps (C^2 / 2 shared-memory compares per unit) and follows the short chains.
+// rule, found by following the last step < s with j = s until a step whose own position was
+// never a target: that step's index is the value. The centroids are split over CTAs of 64;
+// each thread scans the earlier targets for its step and follows the (short) chain, and each
+// warp then loads its 8 chosen key rows with all loads in flight.
+constexpr int kInitPerCta = 64;  // centroids resolved and loaded per CTA (8 per warp)
+
 __global__ void __launch_bounds__(256) kmeans_init_kernel(KeysView k, int32_t C, uint64_t seed,
                                                           int64_t unit_base, uint64_t window,
                                                           int32_t* init_idx, float* mu,
@@ -63,45 +61,64 @@ __global__ void __launch_bounds__(256) kmeans_init_kernel(KeysView k, int32_t C,
     pdl_launch_dependents();  // let the next kernel in the stream be scheduled early
     pdl_wait();               // the previous kernel's writes are visible from here on
     extern __shared__ int32_t sm[];
-    const int u = blockIdx.x;
+    const int u = blockIdx.y;
+    const int c_lo = blockIdx.x * kInitPerCta;           // this CTA's centroids [c_lo, c_hi)
+    const int c_hi = min(C, c_lo + kInitPerCta);
     const int32_t m = (int32_t)k.m;
-    int32_t* target = sm;        // [C] j_i
-    int32_t* prev = sm + C;      // [C] last earlier step with the same target, or -1
-    int32_t* link = sm + 2 * C;  // [C] last earlier step whose target is this step, or -1
+    int32_t* target = sm;                // [c_hi] j_i of every step this CTA's chains can reach
+    int32_t* chosen = sm + c_hi;         // [kInitPerCta]
     const uint64_t key = seed ^ ((uint64_t)(unit_base + u) << 32) ^ window;
-    for (int i = threadIdx.x; i < C; i += blockDim.x) {
+    for (int i = threadIdx.x; i < c_hi; i += blockDim.x) {
         uint64_t st = key + (uint64_t)i * 0x9E3779B97F4A7C15ull;  // state before draw i
         const uint64_t x = splitmix64_next(st);
         target[i] = i + (int32_t)bounded_draw(x, (uint32_t)(m - i));
     }
     __syncthreads();
-    for (int t = threadIdx.x; t < C; t += blockDim.x) {
-        const int32_t p = target[t];
-        int32_t pv = -1, lv = -1;
-        for (int s = t - 1; s >= 0 && (pv < 0 || lv < 0); --s) {
-            const int32_t ts = target[s];
-            if (pv < 0 && ts == p) pv = s;
-            if (lv < 0 && ts == t) lv = s;
+    // chosen[c] for c in [c_lo, c_hi), one warp per 8 centroids: prev = the last step < c with
+    // the same target, then the link chain (the last step < s whose target is s) down to a
+    // step never targeted before. Every search is warp-wide: the lanes stride over the earlier
+    // steps and the largest match wins.
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    auto last_before = [&](int lim, int32_t val) {  // largest s < lim with target[s] == val
+        int32_t best = -1;
+        for (int s0 = 0; s0 < lim; s0 += 32) {  // warp-uniform trip count
+            const int st = s0 + lane;
+            if (st < lim && target[st] == val) best = st;
         }
-        prev[t] = pv;
-        link[t] = lv;
-    }
-    __syncthreads();
-    const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    const uint16_t* keys = k.base + ((int64_t)u * k.n_rows + k.row0) * kD;
-    for (int c = warp; c < C; c += nw) {
-        int32_t x = prev[c];
-        int32_t idx;
-        if (x < 0) {
-            idx = target[c];
-        } else {
-            while (link[x] >= 0) x = link[x];  // every step strictly lowers x
+        return (int32_t)__reduce_max_sync(0xffffffffu, (uint32_t)(best + 1)) - 1;
+    };
+    for (int j = 0; j < 8; ++j) {
+        const int c = c_lo + warp * 8 + j;
+        if (c >= c_hi) break;  // warp-uniform
+        int32_t x = last_before(c, target[c]);
+        int32_t idx = target[c];
+        if (x >= 0) {
+            for (;;) {  // every step strictly lowers x
+                const int32_t lk = last_before(x, x);
+                if (lk < 0) break;
+                x = lk;
+            }
             idx = x;
         }
-        const float4 v = load_row4_bf16(keys + (int64_t)idx * kD);
+        if (lane == 0) chosen[c - c_lo] = idx;
+    }
+    __syncthreads();
+    // one warp per 8 centroids, all 8 key rows in flight at once
+    const uint16_t* keys = k.base + ((int64_t)u * k.n_rows + k.row0) * kD;
+    uint2 w[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int c = c_lo + warp * 8 + j;
+        if (c < c_hi) w[j] = reinterpret_cast<const uint2*>(keys + (int64_t)chosen[c - c_lo] * kD)[lane_id()];
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int c = c_lo + warp * 8 + j;
+        if (c >= c_hi) break;  // warp-uniform
+        const float4 v = make_float4(bf16_lo(w[j].x), bf16_hi(w[j].x), bf16_lo(w[j].y), bf16_hi(w[j].y));
         store_centroid(v, mu + ((int64_t)u * mu_ustride + c) * kD,
                        mu_hat + ((int64_t)u * muhat_ustride + c) * kD);
-        if (init_idx && lane_id() == 0) init_idx[(int64_t)u * C + c] = idx;
+        if (init_idx && lane_id() == 0) init_idx[(int64_t)u * C + c] = chosen[c - c_lo];
     }
 }
 
@@ -380,12 +397,12 @@ int launch_kmeans_init(const KeysView& k, int32_t C, uint64_t seed, int64_t unit
                        uint64_t window, int32_t* init_idx, float* mu, int64_t mu_ustride,
                        uint16_t* mu_hat, int64_t muhat_ustride, uint32_t* err, cudaStream_t s) {
     (void)err;
-    const size_t smem = 3 * (size_t)C * sizeof(int32_t);  // C <= 4096: at most 48 KB
+    const size_t smem = ((size_t)C + kInitPerCta) * sizeof(int32_t);  // C <= 4096: <= 17 KB
     int rc = ensure_smem((const void*)kmeans_init_kernel, smem, "init: set smem");
     if (rc != CKV_OK) return rc;
-    cudaError_t e;
-    e = launch_pdl(kmeans_init_kernel, dim3(k.U), dim3(256), smem, s, k, C, seed, unit_base, window,
-                   init_idx, mu, mu_ustride, mu_hat, muhat_ustride);
+    const dim3 grid((unsigned)((C + kInitPerCta - 1) / kInitPerCta), (unsigned)k.U);
+    cudaError_t e = launch_pdl(kmeans_init_kernel, grid, dim3(256), smem, s, k, C, seed, unit_base,
+                               window, init_idx, mu, mu_ustride, mu_hat, muhat_ustride);
     return e == cudaSuccess ? CKV_OK : cuda_fail(e, "init: launch");
 }
 

@@ -203,8 +203,10 @@ CKV_DEV float half_row_dot(const uint16_t* row, int half, const float* qbar) {
     return s;
 }
 
-// Exclusive block scan of one int per thread. `tot` receives the block total.
-CKV_DEV int32_t block_excl_scan(int32_t v, int32_t* wscan, int32_t* tot) {
+// Exclusive block scan of one int per thread: x = this thread's exclusive prefix, y = the
+// block total. Not inlined: it is called from several places, and one copy of its code
+// keeps the kernel's instruction footprint smaller.
+__device__ __noinline__ int2 block_excl_scan(int32_t v, int32_t* wscan) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int32_t incl = v;
 #pragma unroll
@@ -222,8 +224,52 @@ CKV_DEV int32_t block_excl_scan(int32_t v, int32_t* wscan, int32_t* tot) {
         total += x;
     }
     __syncthreads();
-    *tot = total;
-    return before + incl - v;
+    return make_int2(before + incl - v, total);
+}
+
+// The same scan on two ints at once: x / y = this thread's exclusive prefixes of a / b,
+// z / w = the block totals.
+__device__ __noinline__ int4 block_excl_scan2(int32_t a, int32_t b, int32_t* wscan) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int32_t ia = a, ib = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t ya = __shfl_up_sync(0xffffffffu, ia, o);
+        const int32_t yb = __shfl_up_sync(0xffffffffu, ib, o);
+        if (lane >= o) {
+            ia += ya;
+            ib += yb;
+        }
+    }
+    if (lane == 31) {
+        wscan[warp] = ia;
+        wscan[kWarps + warp] = ib;
+    }
+    __syncthreads();
+    int32_t ba = 0, bb = 0, ta = 0, tb = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+        const int32_t xa = wscan[w], xb = wscan[kWarps + w];
+        if (w < warp) {
+            ba += xa;
+            bb += xb;
+        }
+        ta += xa;
+        tb += xb;
+    }
+    __syncthreads();
+    return make_int4(ba + ia - a, bb + ib - b, ta, tb);
+}
+
+CKV_DEV float ld_cluster_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+CKV_DEV uint32_t ld_cluster_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
 }
 
 // Warp 0 of a radix pass: bins hold weights in descending digit order; find the digit whose
@@ -297,10 +343,120 @@ CKV_DEV int cut_bucket_warp(const int32_t* hist, int32_t need, int32_t* above_ou
     return __shfl_sync(0xffffffffu, bin, src);
 }
 
+// Partial tokens of a cut cluster that is not held in shared memory (a large cluster, or a
+// CTA that is not the dedicated one): this CTA's share [p_lo, p_hi) of the cut's top r_part
+// tokens by qbar . k (ties: lower index, i.e. store order), as store rows in prow. The keys
+// are scored from global memory, into shared memory, or, above kPartCap tokens, into a
+// global scratch written once, split across the cluster's CTAs (every CTA of the cluster
+// calls this function then, for the cluster barrier). Not inlined: a cold path.
+struct PartialArgs {
+    const uint16_t* kp;  // the cut cluster's first K row
+    uint32_t* gkeys;     // global key scratch of the unit (above kPartCap tokens)
+    const float* qbar;   // shared [128]
+    uint32_t* pkey;      // shared [kPartCap + 4]
+    int32_t* hist;       // shared [256]
+    int32_t* wbuf;       // shared scan / pick scratch
+    int32_t* prow;       // shared: this CTA's partial rows
+    int32_t crow, csz, r_part, p_lo, p_hi;
+    int32_t rank, S;
+};
+__device__ __noinline__ void partial_rows(const PartialArgs& P) {
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const bool big_cut = P.csz > kPartCap;
+    auto score_keys = [&](int32_t k0, int32_t k1, uint32_t* dst) {
+        // two threads per row, one memory round trip per pass
+        for (int32_t i0 = k0; i0 < k1; i0 += kNT / 2) {  // CTA-uniform trip count
+            const int32_t i = i0 + (tid >> 1);
+            const int half = tid & 1;
+            float sc = 0.f;
+            if (i < k1) sc = half_row_dot(P.kp + (int64_t)i * kD, half, P.qbar);
+            sc += __shfl_xor_sync(0xffffffffu, sc, 1);
+            if (i < k1 && half == 0) dst[i] = orderable(sc);
+        }
+    };
+    if (big_cut) {
+        const int32_t k0 = (int32_t)((int64_t)P.csz * P.rank / P.S);
+        const int32_t k1 = (int32_t)((int64_t)P.csz * (P.rank + 1) / P.S);
+        score_keys(k0, k1, P.gkeys);
+        cluster_arrive_release();
+        cluster_wait_acquire();
+    }
+    if (P.p_hi <= P.p_lo) return;
+    auto key_at = [&](int i) -> uint32_t { return big_cut ? __ldcg(P.gkeys + i) : P.pkey[i]; };
+    if (!big_cut) {
+        score_keys(0, P.csz, P.pkey);
+        if (tid < 4) P.pkey[P.csz + tid] = 0u;  // pad: never outranks a key
+    }
+    __syncthreads();
+    if (!big_cut && P.csz <= kNT) {
+        // comparison rank (ties: lower index), tpe threads per token, 4 keys per load
+        const int tpe = P.csz <= 32 ? 8 : (P.csz <= 64 ? 4 : (P.csz <= 128 ? 2 : 1));
+        const int e = tid / tpe, sub = tid % tpe;
+        int32_t rk = 0;
+        if (e < P.csz) {
+            const uint32_t ke = P.pkey[e];
+            const uint4* k4 = reinterpret_cast<const uint4*>(P.pkey);
+            const int n4 = (P.csz + 3) >> 2;
+            for (int j4 = sub; j4 < n4; j4 += tpe) {
+                const uint4 v = k4[j4];
+                const int j = 4 * j4;
+                rk += (v.x > ke) || (v.x == ke && j < e);
+                rk += (v.y > ke) || (v.y == ke && j + 1 < e);
+                rk += (v.z > ke) || (v.z == ke && j + 2 < e);
+                rk += (v.w > ke) || (v.w == ke && j + 3 < e);
+            }
+        }
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) {
+            const int32_t y = __shfl_xor_sync(0xffffffffu, rk, o);
+            if (o < tpe) rk += y;
+        }
+        const int32_t sel = (e < P.csz && sub == 0 && rk < P.r_part) ? 1 : 0;
+        const int32_t pos = block_excl_scan(sel, P.wbuf).x;
+        if (sel && pos >= P.p_lo && pos < P.p_hi) P.prow[pos - P.p_lo] = P.crow + e;
+    } else {
+        // radix select over 4 digits of 8 bits, most significant first: the threshold key
+        // theta and `pneed` = how many keys equal to theta are taken (the lowest-index ones),
+        // so that exactly r_part tokens are selected.
+        uint32_t prefix = 0, mask = 0;
+        int32_t pneed = P.r_part;
+        for (int pass = 0; pass < 4; ++pass) {
+            const int shift = 24 - 8 * pass;
+            P.hist[tid] = 0;
+            __syncthreads();
+            for (int i = tid; i < P.csz; i += kNT) {
+                const uint32_t k = key_at(i);
+                if ((k & mask) == prefix) atomicAdd(&P.hist[(k >> shift) & 255u], 1);
+            }
+            __syncthreads();
+            if (warp == 0) radix_pick_bin(P.hist, pneed, false, P.wbuf + 32);
+            __syncthreads();
+            pneed -= P.wbuf[33];
+            prefix |= (uint32_t)P.wbuf[32] << shift;
+            mask |= 255u << shift;
+        }
+        const uint32_t theta = prefix;
+        int32_t eq_run = 0, sel_run = 0;
+        for (int bse = 0; bse < P.csz; bse += kNT) {  // CTA-uniform trip count
+            const int i = bse + tid;
+            const uint32_t k = i < P.csz ? key_at(i) : 0u;
+            const int32_t eq = (i < P.csz && k == theta) ? 1 : 0;
+            const int2 e2 = block_excl_scan(eq, P.wbuf);
+            const int32_t sel = (i < P.csz) && (k > theta || (eq && eq_run + e2.x < pneed));
+            const int2 s2 = block_excl_scan(sel, P.wbuf);
+            const int32_t pos = sel_run + s2.x;
+            if (sel && pos >= P.p_lo && pos < P.p_hi) P.prow[pos - P.p_lo] = P.crow + i;
+            eq_run += e2.y;
+            sel_run += s2.y;
+        }
+    }
+    __syncthreads();
+}
+
 // Shared-memory layout, computed identically on the host (launch size) and the device.
 struct Layout {
-    uint32_t ring, qbar, qh, score, off, spre, cand, hist, hcnt, hnear, rkey, prow, rsrc, rks, rvs,
-        wbuf, scl, ccomb, pbuf, bars, total;
+    uint32_t ring, qbar, qh, score, off, spre, cand, bkt, hist, hcnt, hnear, rkey, prow, rsrc, rks,
+        rvs, wbuf, scl, ccomb, pbuf, bars, total;
 };
 // The ring also holds, before any row arrives, the centroid slice (up to ring / 512 rows of
 // fp32 centroids per chunk) and the cut cluster's keys; after the last row, the warp partials.
@@ -327,6 +483,7 @@ __host__ __device__ inline Layout make_layout(int G, int S, int C, int RB, int p
     L.off = take(4u * (C + 1));
     L.spre = take(4u * (C + 1));
     L.cand = take(4u * C);
+    L.bkt = take((uint32_t)C);
     L.hist = take(4u * 256);
     L.hcnt = take(4u * 256);
     L.hnear = take(4u * 256);
@@ -374,6 +531,7 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     int32_t* const s_off = (int32_t*)(base + Ly.off);
     int32_t* const s_spre = (int32_t*)(base + Ly.spre);
     int32_t* const s_cand = (int32_t*)(base + Ly.cand);
+    uint8_t* const s_bkt = base + Ly.bkt;  // every cluster's score bucket
     int32_t* const s_hist = (int32_t*)(base + Ly.hist);
     int32_t* const s_hcnt = (int32_t*)(base + Ly.hcnt);
     int32_t* const s_hnear = (int32_t*)(base + Ly.hnear);
@@ -398,8 +556,8 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     const int64_t sp_base = (int64_t)su * a.sp_ustride;
     const int32_t* off_g = a.offsets + (int64_t)su * a.off_ustride;
     const float* mu = a.mu + (int64_t)su * a.mu_ustride * kD;
-    const int c_begin = (int)((int64_t)C * rank / S);
-    const int c_end = (int)((int64_t)C * (rank + 1) / S);
+    const int c_begin = C * (int)rank / S;  // C <= 4096, S <= 16: no overflow
+    const int c_end = C * ((int)rank + 1) / S;
     const int nc = c_end - c_begin;
     const uint16_t* qsrc = a.q + ((int64_t)b * a.Hkv * G + (int64_t)h * G) * kD;
 
@@ -436,7 +594,6 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     s_hcnt[tid] = 0;
     s_hnear[tid] = 0;
     if (tid == 0) s_wbuf[kWCnt2] = 0;
-    cluster_arrive_relaxed();
     pdl_wait();
 
     // ---------------------------------------------------------------- phase 1: scores
@@ -454,7 +611,12 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     }
     __syncthreads();
     bool ok = true;
-    cluster_wait_acquire();  // every CTA of the cluster is running: remote stores are safe
+    auto size_of = [&](int c) { return s_off[c + 1] - s_off[c]; };
+    // The slice's scores go to this CTA's own shared memory, with the slice's smallest and
+    // largest order keys (over the clusters with tokens; over every cluster in the mixed-
+    // precision instantiation, whose rank counts empty clusters too). After one cluster
+    // barrier every CTA reads the other slices from the other CTAs.
+    uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
     {
         const float4 qv = reinterpret_cast<const float4*>(s_qbar)[lane];
         // The slice in chunks of at most cch centroids (one chunk unless C / S exceeds the
@@ -481,12 +643,16 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
                     s2 += __shfl_xor_sync(0xffffffffu, s2, o);
                     s3 += __shfl_xor_sync(0xffffffffu, s3, o);
                 }
-                for (int t = lane; t < 4 * S; t += 32) {
-                    const int k = t / S, r = t - k * S;
-                    const int j = j0 + k * kWarps;
-                    const float v = k == 0 ? s0 : (k == 1 ? s1 : (k == 2 ? s2 : s3));
-                    if (j < n1)
-                        st_cluster_f32(map_shared_rank(smem_u32(&s_score[c_begin + done + j]), (uint32_t)r), v);
+                const int j = j0 + lane * kWarps;  // lanes 0..3 store one score each
+                if (lane < 4 && j < n1) {
+                    const float v = lane == 0 ? s0 : (lane == 1 ? s1 : (lane == 2 ? s2 : s3));
+                    const int c = c_begin + done + j;
+                    s_score[c] = v;
+                    if (kMixed || size_of(c) > 0) {
+                        const uint32_t key = orderable(v);
+                        kmn = min(kmn, key);
+                        kmx = max(kmx, key);
+                    }
                 }
             }
             done += n1;
@@ -501,8 +667,36 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
             }
         }
     }
+    {
+        kmn = __reduce_min_sync(0xffffffffu, kmn);
+        kmx = __reduce_max_sync(0xffffffffu, kmx);
+        uint32_t* kb = reinterpret_cast<uint32_t*>(s_wbuf + 48);  // [8] minima, [8] maxima
+        if (lane == 0) {
+            kb[warp] = kmn;
+            kb[8 + warp] = kmx;
+        }
+        __syncthreads();
+        if (tid == 0) {
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) {
+                kmn = min(kmn, kb[w]);
+                kmx = max(kmx, kb[8 + w]);
+            }
+            s_wbuf[80] = (int32_t)kmn;  // this CTA's slice
+            s_wbuf[81] = (int32_t)kmx;
+        }
+    }
     cluster_arrive_release();
-    cluster_wait_acquire();
+    cluster_wait_acquire();  // every slice is written, in every CTA
+    for (int c = tid; c < C; c += kNT) {
+        const int r = (S * (c + 1) - 1) / C;  // the CTA whose slice holds c
+        if (r != (int)rank) s_score[c] = ld_cluster_f32(map_shared_rank(smem_u32(&s_score[c]), (uint32_t)r));
+    }
+    if (tid < S) {
+        s_wbuf[96 + tid] = (int32_t)ld_cluster_u32(map_shared_rank(smem_u32(&s_wbuf[80]), (uint32_t)tid));
+        s_wbuf[112 + tid] = (int32_t)ld_cluster_u32(map_shared_rank(smem_u32(&s_wbuf[81]), (uint32_t)tid));
+    }
+    __syncthreads();
 
     // ---------------------------------------------------------------- phase 2: selection
     const int32_t m_tot = s_off[C] - s_off[0];
@@ -514,50 +708,33 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         const float t = (sc + 0.0f - smin) * inv;
         return (int)fminf(fmaxf(t, 0.f), 255.f);
     };
-    auto size_of = [&](int c) { return s_off[c + 1] - s_off[c]; };
     int32_t cut_c = -1, w_cut = 0;  // w_cut: tokens of bucket b* ranked before the cut
     uint64_t kcut = 0;
     // mixed precision: the walk key of rank n_near - 1 separates near from far clusters
     const bool mid_near = kMixed && a.n_near > 0 && a.n_near < C;
     if (has_cut || mid_near) {
-        // smallest and largest score of the clusters with tokens (of every cluster for the
-        // mixed-precision rank, which counts empty clusters too), as order keys
-        uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
-        for (int c = tid; c < C; c += kNT) {
-            if (kMixed || size_of(c) > 0) {
-                const uint32_t k = orderable(s_score[c]);
-                kmn = min(kmn, k);
-                kmx = max(kmx, k);
-            }
+        // the smallest and largest score over the slices, then every cluster's bucket
+        uint32_t gmn = 0xFFFFFFFFu, gmx = 0u;
+        for (int r = 0; r < S; ++r) {
+            gmn = min(gmn, (uint32_t)s_wbuf[96 + r]);
+            gmx = max(gmx, (uint32_t)s_wbuf[112 + r]);
         }
-        kmn = __reduce_min_sync(0xffffffffu, kmn);
-        kmx = __reduce_max_sync(0xffffffffu, kmx);
-        uint32_t* kb = reinterpret_cast<uint32_t*>(s_wbuf + 48);  // [8] minima, [8] maxima
-        if (lane == 0) {
-            kb[warp] = kmn;
-            kb[8 + warp] = kmx;
-        }
-        __syncthreads();
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            kmn = min(kmn, kb[w]);
-            kmx = max(kmx, kb[8 + w]);
-        }
-        const float mn = from_orderable(kmn), mx = from_orderable(kmx);
+        const float mn = from_orderable(gmn), mx = from_orderable(gmx);
         const float range = mx - mn;
         smin = mn;
         inv = range > 1e-30f ? 255.99f / range : 0.f;  // finite; 0 puts every score in bucket 0
-    }
-    if (has_cut) {
         for (int c = tid; c < C; c += kNT) {
+            const int bk = bucket(s_score[c]);
+            s_bkt[c] = (uint8_t)bk;
             const int32_t w = size_of(c);
-            if (w > 0) {
-                const int bk = bucket(s_score[c]);
+            if (has_cut && w > 0) {
                 atomicAdd(&s_hist[bk], w);
                 atomicAdd(&s_hcnt[bk], 1);
             }
         }
         __syncthreads();
+    }
+    if (has_cut) {
         // every warp finds the cut's bucket itself (no extra block barrier)
         bstar = cut_bucket_warp(s_hist, R, &w_above);
         // When b* holds a single cluster with tokens, that cluster is the cut: CTA S-1, which
@@ -565,7 +742,7 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         if ((int)rank == S - 1 && S > 1 && s_hcnt[bstar] == 1) {
             for (int c = tid; c < C; c += kNT) {
                 const int32_t w = size_of(c);
-                if (w > 0 && w <= RB && w <= kNT && bucket(s_score[c]) == bstar) {
+                if (w > 0 && w <= RB && w <= kNT && s_bkt[c] == bstar) {
                     fence_proxy_async();  // the ring's centroid reads come before the copies
                     const int64_t row = kp_base + s_off[c];
                     const uint32_t bytes = (uint32_t)w * kD * 2;
@@ -579,7 +756,7 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         // the clusters of bucket b* (any order)
         for (int c0 = 0; c0 < C; c0 += kNT) {
             const int c = c0 + tid;
-            const bool in_b = c < C && size_of(c) > 0 && bucket(s_score[c]) == bstar;
+            const bool in_b = c < C && size_of(c) > 0 && s_bkt[c] == bstar;
             const uint32_t bal = __ballot_sync(0xffffffffu, in_b);
             int32_t pos0 = 0;
             if (lane == 0 && bal) pos0 = atomicAdd(&s_wbuf[kWCnt], __popc(bal));
@@ -618,14 +795,14 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     // exactly among themselves.
     uint64_t k_near = 0;
     if (mid_near) {
-        for (int c = tid; c < C; c += kNT) atomicAdd(&s_hnear[bucket(s_score[c])], 1);
+        for (int c = tid; c < C; c += kNT) atomicAdd(&s_hnear[s_bkt[c]], 1);
         __syncthreads();
         int32_t n_above = 0;
         const int bn = cut_bucket_warp(s_hnear, a.n_near - 1, &n_above);
         int32_t* cand2 = s_spre;  // free until the whole-size scan below
         for (int c0 = 0; c0 < C; c0 += kNT) {
             const int c = c0 + tid;
-            const bool in_b = c < C && bucket(s_score[c]) == bn;
+            const bool in_b = c < C && s_bkt[c] == bn;
             const uint32_t bal = __ballot_sync(0xffffffffu, in_b);
             int32_t pos0 = 0;
             if (lane == 0 && bal) pos0 = atomicAdd(&s_wbuf[kWCnt2], __popc(bal));
@@ -656,29 +833,44 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         return walk_key(s_score[c], c) < k_near;
     };
     // whole clusters: every cluster without a cut; else buckets above b*, and the clusters of
-    // b* ranked before the cut. Their rows are laid out in cluster-index order: spre[c] is the
-    // exclusive prefix of the whole sizes (one block scan, a contiguous run per thread).
+    // b* ranked before the cut. Their rows are laid out in cluster-index order. One block scan
+    // (a contiguous run of clusters per thread) of their sizes and counts gives the compact
+    // list of the whole clusters: wl_pre[k] = the selection position of the k-th one's first
+    // row, wl_off[k] = its first store row (kFarBit set when it is attended from the fp8 copy).
     auto whole_size = [&](int c) -> int32_t {
         const int32_t w = size_of(c);
         if (w == 0 || !has_cut) return w;
-        const float sc = s_score[c];
-        const int bk = bucket(sc);
-        return (bk > bstar || (bk == bstar && walk_key(sc, c) > kcut)) ? w : 0;
+        const int bk = s_bkt[c];
+        return (bk > bstar || (bk == bstar && walk_key(s_score[c], c) > kcut)) ? w : 0;
     };
+    int32_t* const wl_pre = s_spre;  // [n_whole + 1]
+    int32_t* const wl_off = s_cand;  // [n_whole]
+    int32_t n_whole;
     {
         const int per = (C + kNT - 1) / kNT;
         const int c0 = tid * per;
-        int32_t local = 0;
-        for (int j = 0; j < per; ++j)
-            if (c0 + j < C) local += whole_size(c0 + j);
-        int32_t tot;
-        int32_t run = block_excl_scan(local, s_wbuf, &tot);
+        int32_t lsz = 0, lcnt = 0;
         for (int j = 0; j < per; ++j)
             if (c0 + j < C) {
-                s_spre[c0 + j] = run;
-                run += whole_size(c0 + j);
+                const int32_t w = whole_size(c0 + j);
+                lsz += w;
+                lcnt += w > 0 ? 1 : 0;
             }
-        if (tid == 0) s_spre[C] = tot;
+        const int4 sc = block_excl_scan2(lsz, lcnt, s_wbuf);
+        int32_t run = sc.x, k = sc.y;
+        for (int j = 0; j < per; ++j)
+            if (c0 + j < C) {
+                const int c = c0 + j;
+                const int32_t w = whole_size(c);
+                if (w > 0) {
+                    wl_pre[k] = run;
+                    wl_off[k] = s_off[c] | ((kMixed && is_far(c)) ? kFarBit : 0);
+                    ++k;
+                    run += w;
+                }
+            }
+        n_whole = sc.w;
+        if (tid == 0) wl_pre[sc.w] = sc.z;
     }
     __syncthreads();
 
@@ -773,13 +965,14 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
                 r = -1 - (idx < a.n_sink ? idx : a.n_sink + (a.pstart + idx - a.n_sink) % a.pring);
             } else if (idx < base_p) {
                 const int32_t x = idx - base_w;
-                int k0 = 0, khi = C - 1;  // last cluster with spre[k] <= x: a whole one holding x
+                int k0 = 0, khi = n_whole - 1;  // the whole cluster holding x: last wl_pre <= x
                 while (k0 < khi) {
                     const int mid = (k0 + khi + 1) >> 1;
-                    if (s_spre[mid] <= x) k0 = mid; else khi = mid - 1;
+                    if (wl_pre[mid] <= x) k0 = mid; else khi = mid - 1;
                 }
-                r = s_off[k0] + (x - s_spre[k0]);
-                if (kMixed && is_far(k0)) r |= kFarBit;
+                const int32_t o = wl_off[k0];
+                r = (o & ~kFarBit) + (x - wl_pre[k0]);
+                if (kMixed && (o & kFarBit)) r |= kFarBit;
             } else {
                 r = s_prow[idx - base_p - p_lo];
                 if (kMixed && cut_far) r |= kFarBit;
@@ -790,6 +983,150 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         }
     };
 
+    if (!ok) s_wbuf[kWBad] = 1;
+    const int32_t n_rows = resident ? csz : hi - lo;
+    const int chunk = (resident || n_rows <= RB) ? RB : RB / 2;
+    const int n_chunks = resident ? 1 : (n_rows + chunk - 1) / chunk;
+    auto issue = [&](int ch) {  // every thread
+        const int32_t c0 = lo + ch * chunk;
+        const int32_t c1 = (c0 + chunk < hi) ? c0 + chunk : hi;
+        const int p0 = n_chunks == 1 ? 0 : (ch & 1) * chunk;
+        fill_rsrc(c0, c1, p0);
+        __syncthreads();
+        copy_rows(p0, c1 - c0, 3);
+    };
+
+    if (resident) {
+        // ---- the cut cluster in shared memory (plain 256-byte rows): two bulk copies, issued
+        // during the selection when the histogram isolated the cut, else now
+        if (tid == 0 && s_wbuf[kWCopy] == 0) {
+            fence_proxy_async();  // the ring's centroid reads come before the copies
+            const uint32_t bytes = (uint32_t)csz * kD * 2;
+            mbar_arrive_expect_tx(fbar, 2 * bytes);
+            bulk_load(base + Ly.ring, a.kp + (kp_base + crow) * kD, bytes, fbar);
+            bulk_load(base + Ly.ring + (size_t)RB * 256, a.vp + (kp_base + crow) * kD, bytes, fbar);
+        }
+        const bool got = __syncthreads_and(mbar_wait(fbar, 0, a.err) ? 1 : 0) != 0;
+        if (!got) s_wbuf[kWBad] = 1;
+        // qbar . k, a half-warp per row (16-byte reads covering one 256-byte row), 8 rows
+        // per half-warp in flight
+        const int hw = tid >> 4, l16 = tid & 15;
+        const float4 qa = reinterpret_cast<const float4*>(s_qbar)[l16 * 2];
+        const float4 qb4 = reinterpret_cast<const float4*>(s_qbar)[l16 * 2 + 1];
+        for (int r0 = 0; r0 < csz; r0 += 8 * (kNT / 16)) {  // CTA-uniform trip count
+            float sk[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int e = r0 + hw + k * (kNT / 16);
+                sk[k] = 0.f;
+                if (got && e < csz) {
+                    const uint4 w = lds_v4(ringK + (uint32_t)e * 256u + l16 * 16);
+                    float t = qa.x * bf16_lo(w.x);
+                    t = fmaf(qa.y, bf16_hi(w.x), t);
+                    t = fmaf(qa.z, bf16_lo(w.y), t);
+                    t = fmaf(qa.w, bf16_hi(w.y), t);
+                    t = fmaf(qb4.x, bf16_lo(w.z), t);
+                    t = fmaf(qb4.y, bf16_hi(w.z), t);
+                    t = fmaf(qb4.z, bf16_lo(w.w), t);
+                    sk[k] = fmaf(qb4.w, bf16_hi(w.w), t);
+                }
+            }
+            __syncwarp();  // all 8 rows' products first, then the reductions
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) sk[k] += __shfl_xor_sync(0xffffffffu, sk[k], o);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int e = r0 + hw + k * (kNT / 16);
+                if (e < csz && l16 == 0) s_rkey[e] = orderable(sk[k]);
+            }
+        }
+        if (tid < 4) s_rkey[csz + tid] = 0u;  // pad: never outranks a key
+        __syncthreads();
+        // comparison rank (ties: lower index), tpe threads per token, 4 keys per load
+        const int tpe = csz <= 32 ? 8 : (csz <= 64 ? 4 : (csz <= 128 ? 2 : 1));
+        const int e = tid / tpe, sub = tid % tpe;
+        int32_t rk = 0;
+        if (e < csz) {
+            const uint32_t ke = s_rkey[e];
+            const uint4* k4 = reinterpret_cast<const uint4*>(s_rkey);
+            const int n4 = (csz + 3) >> 2;
+            for (int j4 = sub; j4 < n4; j4 += tpe) {
+                const uint4 v = k4[j4];
+                const int j = 4 * j4;
+                rk += (v.x > ke) || (v.x == ke && j < e);
+                rk += (v.y > ke) || (v.y == ke && j + 1 < e);
+                rk += (v.z > ke) || (v.z == ke && j + 2 < e);
+                rk += (v.w > ke) || (v.w == ke && j + 3 < e);
+            }
+        }
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) {
+            const int32_t y = __shfl_xor_sync(0xffffffffu, rk, o);
+            if (o < tpe) rk += y;
+        }
+        const int32_t sel = (e < csz && sub == 0 && rk < r_part) ? 1 : 0;
+        const int32_t pos = block_excl_scan(sel, s_wbuf).x;
+        if (sel) {
+            s_prow[pos] = e;
+            if (sel_out) sel_out[base_p + pos] = ids[crow + e];
+        }
+        __syncthreads();
+        if (kMixed) {
+            // the selected rows of a far cut cluster take their fp8 copy's values in place;
+            // a near one keeps its bf16 rows (scale 1)
+            for (int t = warp; t < r_part; t += kWarps) {  // warp-uniform trip count
+                const int er = s_prow[t];
+                if (cut_far) {
+#pragma unroll
+                    for (int part = 0; part < 2; ++part) {
+                        uint2* row = reinterpret_cast<uint2*>(base + Ly.ring + (size_t)part * RB * 256 +
+                                                              (size_t)er * 256);
+                        float sc;
+                        const uint2 v = fp8_row_values(row[lane], &sc);
+                        __syncwarp();
+                        row[lane] = v;
+                        if (lane == 0) (part ? s_rvs : s_rks)[er] = sc;
+                    }
+                } else if (lane == 0) {
+                    s_rks[er] = 1.f;
+                    s_rvs[er] = 1.f;
+                }
+            }
+            __syncthreads();
+        }
+    } else {
+        if (s_wbuf[kWCopy] != 0) {  // cut copies land before the ring is reused
+            const bool got = __syncthreads_and(mbar_wait(fbar, 0, a.err) ? 1 : 0) != 0;
+            if (!got) {
+                s_wbuf[kWBad] = 1;
+                mbar_wait(fbar, 0, a.err);  // one more bounded wait for the copies in flight
+            }
+        }
+        // partial tokens of this CTA's share outside the ring path: rows into prow (every CTA
+        // of the cluster takes part when the keys go through the global scratch)
+        if (r_part > 0 && (big_cut || p_hi > p_lo)) {
+            PartialArgs pa;
+            pa.kp = a.kp + (kp_base + crow) * kD;
+            pa.gkeys = a.part_scratch ? reinterpret_cast<uint32_t*>(a.part_scratch) +
+                                            (int64_t)unit * a.part_ustride
+                                      : nullptr;
+            pa.qbar = s_qbar;
+            pa.pkey = s_pkey;
+            pa.hist = s_hist;
+            pa.wbuf = s_wbuf;
+            pa.prow = s_prow;
+            pa.crow = crow;
+            pa.csz = csz;
+            pa.r_part = r_part;
+            pa.p_lo = p_lo;
+            pa.p_hi = p_hi;
+            pa.rank = (int32_t)rank;
+            pa.S = S;
+            partial_rows(pa);
+        }
+    }
     // Attention on tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate), per warp over
     // 16-row tiles of the ring: S^T = K Q^T with the kv rows as M and the G heads as N (<= 8),
     // then O^T += V^T P with the head dimension as M. P is split into bf16 high and low parts
@@ -888,243 +1225,29 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         }
     };
 
-    if (!ok) s_wbuf[kWBad] = 1;
-    const int32_t n_rows = resident ? csz : hi - lo;
-    const int chunk = (resident || n_rows <= RB) ? RB : RB / 2;
-    const int n_chunks = resident ? 1 : (n_rows + chunk - 1) / chunk;
-    auto issue = [&](int ch) {  // every thread
-        const int32_t c0 = lo + ch * chunk;
-        const int32_t c1 = (c0 + chunk < hi) ? c0 + chunk : hi;
-        const int p0 = n_chunks == 1 ? 0 : (ch & 1) * chunk;
-        fill_rsrc(c0, c1, p0);
-        __syncthreads();
-        copy_rows(p0, c1 - c0, 3);
-    };
-
-    if (resident) {
-        // ---- the cut cluster in shared memory (plain 256-byte rows): two bulk copies, issued
-        // during the selection when the histogram isolated the cut, else now
-        if (tid == 0 && s_wbuf[kWCopy] == 0) {
-            fence_proxy_async();  // the ring's centroid reads come before the copies
-            const uint32_t bytes = (uint32_t)csz * kD * 2;
-            mbar_arrive_expect_tx(fbar, 2 * bytes);
-            bulk_load(base + Ly.ring, a.kp + (kp_base + crow) * kD, bytes, fbar);
-            bulk_load(base + Ly.ring + (size_t)RB * 256, a.vp + (kp_base + crow) * kD, bytes, fbar);
-        }
-        const bool got = __syncthreads_and(mbar_wait(fbar, 0, a.err) ? 1 : 0) != 0;
-        if (!got) s_wbuf[kWBad] = 1;
-        // qbar . k, a half-warp per row (16-byte reads covering one 256-byte row), 8 rows
-        // per half-warp in flight
-        const int hw = tid >> 4, l16 = tid & 15;
-        const float4 qa = reinterpret_cast<const float4*>(s_qbar)[l16 * 2];
-        const float4 qb4 = reinterpret_cast<const float4*>(s_qbar)[l16 * 2 + 1];
-        for (int r0 = 0; r0 < csz; r0 += 8 * (kNT / 16)) {
-            float s[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int e = r0 + hw + k * (kNT / 16);
-                s[k] = 0.f;
-                if (got && e < csz) {
-                    const uint4 w = lds_v4(ringK + (uint32_t)e * 256u + l16 * 16);
-                    float t = qa.x * bf16_lo(w.x);
-                    t = fmaf(qa.y, bf16_hi(w.x), t);
-                    t = fmaf(qa.z, bf16_lo(w.y), t);
-                    t = fmaf(qa.w, bf16_hi(w.y), t);
-                    t = fmaf(qb4.x, bf16_lo(w.z), t);
-                    t = fmaf(qb4.y, bf16_hi(w.z), t);
-                    t = fmaf(qb4.z, bf16_lo(w.w), t);
-                    s[k] = fmaf(qb4.w, bf16_hi(w.w), t);
-                }
+    // ---- attention, chunk by chunk: the resident cut cluster is one chunk (its selected rows
+    // listed in prow, plain rows); otherwise the rows stream through the ring, two chunks in
+    // flight. One call site for each of issue and attend keeps the code small.
+    int next = 0;  // chunks issued
+    for (int ch = 0; ch < n_chunks; ++ch) {  // CTA-uniform trip count
+        int pb0 = 0, n = r_part;
+        if (!resident) {
+            while (next < n_chunks && next <= ch + 1) {
+                if (next >= 2) __syncthreads();  // every warp is done with this slot
+                issue(next);
+                ++next;
             }
-            __syncwarp();  // all 8 rows' products first, then the reductions
-#pragma unroll
-            for (int o = 8; o > 0; o >>= 1)
-#pragma unroll
-                for (int k = 0; k < 8; ++k) s[k] += __shfl_xor_sync(0xffffffffu, s[k], o);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int e = r0 + hw + k * (kNT / 16);
-                if (e < csz && l16 == 0) s_rkey[e] = orderable(s[k]);
-            }
-        }
-        if (tid < 4) s_rkey[csz + tid] = 0u;  // pad: never outranks a key
-        __syncthreads();
-        // comparison rank (ties: lower index), tpe threads per token, 4 keys per load
-        const int tpe = csz <= 32 ? 8 : (csz <= 64 ? 4 : (csz <= 128 ? 2 : 1));
-        const int e = tid / tpe, sub = tid % tpe;
-        int32_t rk = 0;
-        if (e < csz) {
-            const uint32_t ke = s_rkey[e];
-            const uint4* k4 = reinterpret_cast<const uint4*>(s_rkey);
-            const int n4 = (csz + 3) >> 2;
-#pragma unroll 4
-            for (int j4 = sub; j4 < n4; j4 += tpe) {
-                const uint4 v = k4[j4];
-                const int j = 4 * j4;
-                rk += (v.x > ke) || (v.x == ke && j < e);
-                rk += (v.y > ke) || (v.y == ke && j + 1 < e);
-                rk += (v.z > ke) || (v.z == ke && j + 2 < e);
-                rk += (v.w > ke) || (v.w == ke && j + 3 < e);
-            }
-        }
-#pragma unroll
-        for (int o = 4; o > 0; o >>= 1) {
-            const int32_t y = __shfl_xor_sync(0xffffffffu, rk, o);
-            if (o < tpe) rk += y;
-        }
-        const int32_t sel = (e < csz && sub == 0 && rk < r_part) ? 1 : 0;
-        int32_t tot;
-        const int32_t pos = block_excl_scan(sel, s_wbuf, &tot);
-        if (sel) {
-            s_prow[pos] = e;
-            if (sel_out) sel_out[base_p + pos] = ids[crow + e];
-        }
-        __syncthreads();
-        if (kMixed) {
-            // the selected rows of a far cut cluster take their fp8 copy's values in place;
-            // a near one keeps its bf16 rows (scale 1)
-            for (int t = warp; t < r_part; t += kWarps) {  // warp-uniform trip count
-                const int er = s_prow[t];
-                if (cut_far) {
-#pragma unroll
-                    for (int part = 0; part < 2; ++part) {
-                        uint2* row = reinterpret_cast<uint2*>(base + Ly.ring + (size_t)part * RB * 256 +
-                                                              (size_t)er * 256);
-                        float sc;
-                        const uint2 v = fp8_row_values(row[lane], &sc);
-                        __syncwarp();
-                        row[lane] = v;
-                        if (lane == 0) (part ? s_rvs : s_rks)[er] = sc;
-                    }
-                } else if (lane == 0) {
-                    s_rks[er] = 1.f;
-                    s_rvs[er] = 1.f;
-                }
-            }
-            __syncthreads();
-        }
-        if (got) attend(0, r_part, s_prow, false);
-    } else {
-        if (s_wbuf[kWCopy] != 0) {  // cut copies land before the ring is reused
-            const bool got = __syncthreads_and(mbar_wait(fbar, 0, a.err) ? 1 : 0) != 0;
-            if (!got) {
-                s_wbuf[kWBad] = 1;
-                mbar_wait(fbar, 0, a.err);  // one more bounded wait for the copies in flight
-            }
-        }
-        // ---- partial tokens of this CTA's share outside the ring path: rows into prow
-        uint32_t* gkeys = a.part_scratch ? reinterpret_cast<uint32_t*>(a.part_scratch) +
-                                               (int64_t)unit * a.part_ustride
-                                         : nullptr;
-        auto score_keys = [&](int64_t k0, int64_t k1, uint32_t* dst) {
-            // two threads per row, one memory round trip per pass
-            for (int64_t i0 = k0; i0 < k1; i0 += kNT / 2) {
-                const int64_t i = i0 + (tid >> 1);
-                const int half = tid & 1;
-                float s = 0.f;
-                if (i < k1) s = half_row_dot(a.kp + (kp_base + crow + i) * kD, half, s_qbar);
-                s += __shfl_xor_sync(0xffffffffu, s, 1);
-                if (i < k1 && half == 0) dst[i] = orderable(s);
-            }
-        };
-        if (r_part > 0 && big_cut) {
-            // Keys of a large cut cluster are written once, split across the cluster's CTAs.
-            const int64_t k0 = (int64_t)csz * rank / S, k1 = (int64_t)csz * (rank + 1) / S;
-            score_keys(k0, k1, gkeys);
-            cluster_arrive_release();
-            cluster_wait_acquire();
-        }
-        if (r_part > 0 && p_hi > p_lo) {
-            auto key_at = [&](int i) -> uint32_t { return big_cut ? __ldcg(gkeys + i) : s_pkey[i]; };
-            if (!big_cut) {
-                score_keys(0, csz, s_pkey);
-                if (tid < 4) s_pkey[csz + tid] = 0u;  // pad: never outranks a key
-            }
-            __syncthreads();
-            if (!big_cut && csz <= kNT) {
-                const int tpe = csz <= 32 ? 8 : (csz <= 64 ? 4 : (csz <= 128 ? 2 : 1));
-                const int e = tid / tpe, sub = tid % tpe;
-                int32_t rk = 0;
-                if (e < csz) {
-                    const uint32_t ke = s_pkey[e];
-                    const uint4* k4 = reinterpret_cast<const uint4*>(s_pkey);
-                    const int n4 = (csz + 3) >> 2;
-#pragma unroll 4
-                    for (int j4 = sub; j4 < n4; j4 += tpe) {
-                        const uint4 v = k4[j4];
-                        const int j = 4 * j4;
-                        rk += (v.x > ke) || (v.x == ke && j < e);
-                        rk += (v.y > ke) || (v.y == ke && j + 1 < e);
-                        rk += (v.z > ke) || (v.z == ke && j + 2 < e);
-                        rk += (v.w > ke) || (v.w == ke && j + 3 < e);
-                    }
-                }
-#pragma unroll
-                for (int o = 4; o > 0; o >>= 1) {
-                    const int32_t y = __shfl_xor_sync(0xffffffffu, rk, o);
-                    if (o < tpe) rk += y;
-                }
-                const int32_t sel = (e < csz && sub == 0 && rk < r_part) ? 1 : 0;
-                int32_t tot;
-                const int32_t pos = block_excl_scan(sel, s_wbuf, &tot);
-                if (sel && pos >= p_lo && pos < p_hi) s_prow[pos - p_lo] = crow + e;
-            } else {
-                // radix select over 4 digits of 8 bits, most significant first: the threshold
-                // key theta and `pneed` = how many keys equal to theta are taken (the
-                // lowest-index ones), so that exactly r_part tokens are selected.
-                uint32_t prefix = 0, mask = 0;
-                int32_t pneed = r_part;
-                for (int pass = 0; pass < 4; ++pass) {
-                    const int shift = 24 - 8 * pass;
-                    s_hist[tid] = 0;
-                    __syncthreads();
-                    for (int i = tid; i < csz; i += kNT) {
-                        const uint32_t k = key_at(i);
-                        if ((k & mask) == prefix) atomicAdd(&s_hist[(k >> shift) & 255u], 1);
-                    }
-                    __syncthreads();
-                    if (warp == 0) radix_pick_bin(s_hist, pneed, false, s_wbuf + 32);
-                    __syncthreads();
-                    pneed -= s_wbuf[33];
-                    prefix |= (uint32_t)s_wbuf[32] << shift;
-                    mask |= 255u << shift;
-                }
-                const uint32_t theta = prefix;
-                int32_t eq_run = 0, sel_run = 0;
-                for (int bse = 0; bse < csz; bse += kNT) {
-                    const int i = bse + tid;
-                    const uint32_t k = i < csz ? key_at(i) : 0u;
-                    const int32_t eq = (i < csz && k == theta) ? 1 : 0;
-                    int32_t eq_tot;
-                    const int32_t eq_before = eq_run + block_excl_scan(eq, s_wbuf, &eq_tot);
-                    const int32_t sel = (i < csz) && (k > theta || (eq && eq_before < pneed));
-                    int32_t sel_tot;
-                    const int32_t pos = sel_run + block_excl_scan(sel, s_wbuf, &sel_tot);
-                    if (sel && pos >= p_lo && pos < p_hi) s_prow[pos - p_lo] = crow + i;
-                    eq_run += eq_tot;
-                    sel_run += sel_tot;
-                }
-            }
-            __syncthreads();
-        }
-        if (n_chunks > 0) issue(0);
-        if (n_chunks > 1) issue(1);
-        for (int ch = 0; ch < n_chunks; ++ch) {
-            if (ch + 1 < n_chunks) cp_async_wait<1>(); else cp_async_wait<0>();
+            if (next > ch + 1) cp_async_wait<1>(); else cp_async_wait<0>();
             __syncthreads();
             const int32_t c0 = lo + ch * chunk;
-            const int n = (hi - c0) < chunk ? (hi - c0) : chunk;
-            const int pb0 = n_chunks == 1 ? 0 : (ch & 1) * chunk;
+            n = (hi - c0) < chunk ? (hi - c0) : chunk;
+            pb0 = n_chunks == 1 ? 0 : (ch & 1) * chunk;
             if (kMixed) {
                 convert_far(pb0, n);
                 __syncthreads();
             }
-            if (s_wbuf[kWBad] == 0) attend(pb0, n, nullptr, true);
-            if (ch + 2 < n_chunks) {
-                __syncthreads();  // every warp is done with this slot
-                issue(ch + 2);
-            }
         }
+        if (s_wbuf[kWBad] == 0) attend(pb0, n, resident ? s_prow : nullptr, !resident);
     }
 
     // ---------------------------------------------------------------- phase 5: combine
@@ -1287,9 +1410,11 @@ int ring_rows(int S, int budget) {
 }
 
 // One launch plan per (device, units, C, budget), found once. The cluster size S is the
-// largest power of two <= 16 (and <= 64 / G, which bounds CTA 0's combine buffer) with all
-// U * S CTAs on distinct SMs; with more units than SMs, S = 1. The ring takes one CTA's share
-// of the budget, reduced in steps of 16 rows while the launch does not fit.
+// largest power of two <= 16 (and <= 64 / G, which bounds CTA 0's combine buffer) whose
+// U * S CTAs take at most half of the SMs when the units are few (U * 16 <= SMs), so that the
+// next launch's CTAs, started early by programmatic dependent launch, find SMs of their own;
+// with more units, at most all of the SMs; with more units than SMs, S = 1. The ring takes one
+// CTA's share of the budget, reduced in steps of 16 rows while the launch does not fit.
 template <int G, bool kPerHead, bool kMixed>
 int plan_for(const DecodeArgs& a, int num_sms, Plan* out) {
     static std::mutex mtx;
@@ -1311,8 +1436,9 @@ int plan_for(const DecodeArgs& a, int num_sms, Plan* out) {
     }
     auto kern = select_attend_kernel<G, kPerHead, kMixed>;
     Plan best{};
+    const int64_t sm_cap = (int64_t)U * 16 <= num_sms ? num_sms / 2 : num_sms;
     for (int S = 16; S >= 1 && best.p.S == 0; S /= 2) {
-        if (S > 1 && (S * G > 64 || (int64_t)U * S > num_sms)) continue;
+        if (S > 1 && (S * G > 64 || (int64_t)U * S > sm_cap)) continue;
         for (int RB = ring_rows(S, a.budget); RB >= 64 && best.p.S == 0; RB -= 16) {
             const int pc = prow_capacity(a.budget, S);
             const Layout L = make_layout(G, S, a.C, RB, pc);
@@ -1346,15 +1472,17 @@ int launch_g(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     cfg.blockDim = dim3(kNT);
     cfg.dynamicSmemBytes = plan.smem;
     cfg.stream = s;
-    cudaLaunchAttribute attrs[2];
+    cudaLaunchAttribute attrs[3];
     attrs[0].id = cudaLaunchAttributeClusterDimension;
     attrs[0].val.clusterDim.x = (unsigned)S;
     attrs[0].val.clusterDim.y = 1;
     attrs[0].val.clusterDim.z = 1;
     attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attrs[1].val.programmaticStreamSerializationAllowed = 1;
+    attrs[2].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;  // one CTA per SM
+    attrs[2].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicySpread;
     cfg.attrs = attrs;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = 3;
     cudaError_t e = cudaLaunchKernelEx(&cfg, select_attend_kernel<G, kPerHead, kMixed>, a, plan.p);
     if (e != cudaSuccess) return cuda_fail(e, "select_attend: launch");
     return CKV_OK;
