@@ -35,12 +35,15 @@
 //      block scan of their sizes;
 //   3. the selected rows form one index space: sinks, pending (in append order, from the
 //      two-window pending ring), whole clusters by index, then the partial tokens of the cut
-//      cluster in store order. With a partial fill and S > 1, CTA S-1 takes exactly the
-//      partial tokens: it bulk-copies the cut cluster's K and V rows (started during the
-//      selection when the histogram isolates the cut), ranks the tokens by qbar . k there and
-//      attends the top ones in place. The other CTAs split the rest evenly;
-//   4. rows reach a shared-memory ring through cp.async (16 bytes per thread, coalesced
-//      rows, XOR-swizzled 16-byte chunks). Each warp runs flash-decode on 16-row tiles with
+//      cluster in store order. With a partial fill and S > 1, CTA S-1 takes the partial
+//      tokens: it bulk-copies the cut cluster's K and V rows (started during the selection
+//      when the histogram isolates the cut), ranks the tokens by qbar . k there and attends
+//      the top ones in place; it also takes the last whole rows, up to an even share of the
+//      work less the cut cluster it loaded. The other CTAs split the rest evenly;
+//   4. rows reach a shared-memory ring by one bulk copy (cp.async.bulk) per K or V row,
+//      issued by the thread that resolves the row's source, and complete on the chunk's
+//      mbarrier. Ring rows are 272 bytes apart, so the 8 rows of a matrix load fall on
+//      distinct banks. Each warp runs flash-decode on 16-row tiles with
 //      tensor-core MMAs (mma.sync m16n8k16, bf16 in, fp32 accumulate): S^T = K Q^T with the
 //      rows as M and the G query heads as N, an online softmax per head, then O^T += V^T P
 //      with P split into bf16 high and low parts;
@@ -54,7 +57,7 @@
 // (sequence, query head) units). Another instantiates the mixed-precision decode of the
 // explainer's outlook (section 7, lower precision for far clusters): the selection is the
 // same, but the rows of clusters at walk rank >= n_near arrive as fp8 e4m3 codes with one fp32
-// scale per row. Their codes are staged in the upper half of their ring row, converted
+// scale per row. Their codes are bulk-copied into the upper half of their ring row, converted
 // exactly to bf16 (e4m3 values are bf16 values) by one warp per row, and the row's scales
 // multiply its scores (K) and its softmax weights in the P V product (V).
 #include <cuda_fp8.h>
@@ -74,13 +77,17 @@ constexpr int kNT = 256;          // threads per CTA
 constexpr int kWarps = kNT / 32;
 constexpr int kPartCap = 4096;    // cut-cluster tokens ranked in shared memory (outside the ring path)
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kRowBytes = 2 * kD * 2;  // one K row and one V row, bf16
+// Ring row pitch: a 256-byte bf16 row plus 16 bytes, so that the 8 rows a matrix load reads at
+// one 16-byte column fall on 8 distinct groups of 4 banks.
+constexpr int kPitch = 2 * kD + 16;
+constexpr int kRowBytes = 2 * kPitch;  // one K row and one V row
 constexpr int kCombStride = 130;       // accumulator[128], max, sum
 
 // wbuf slots
 constexpr int kWCnt = 40;     // candidates found in the cut's bucket
 constexpr int kWCut = 41;     // the cut cluster
 constexpr int kWPre = 42;     // tokens of bucket b* ranked before the cut
+constexpr int kWCopyC = 43;   // the cluster whose rows the early cut copies fetch
 constexpr int kWCopy = 45;    // the cut cluster's bulk copies were issued
 constexpr int kWBad = 46;     // a bounded wait of this CTA gave up
 constexpr int kWCnt2 = 47;    // candidates found in the bucket of walk rank n_near - 1
@@ -100,17 +107,14 @@ CKV_DEV uint64_t walk_key(float score, int c) {
     return ((uint64_t)orderable(score) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)c);
 }
 
-// 16-byte chunk j of ring row p, XOR-swizzled by the row's low 3 bits.
-CKV_DEV uint32_t swz_addr(uint32_t base, int p, int j) {
-    return base + (uint32_t)p * 256u + ((uint32_t)(j ^ (p & 7)) << 4);
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) into this CTA's
+// shared memory, completing on the mbarrier at shared address `bar`.
+CKV_DEV void bulk_row(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
 }
-CKV_DEV void cp_async16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-CKV_DEV void cp_async4(uint32_t dst, const void* src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-CKV_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 CKV_DEV void sts_v4(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
                  "r"(v.w)
@@ -141,10 +145,6 @@ CKV_DEV uint2 fp8_row_values(uint2 w, float* scale_out) {
     const __nv_fp8x2_storage_t c23 = __nv_cvt_float2_to_fp8x2(
         make_float2(__fdiv_rn(x2, scale), __fdiv_rn(x3, scale)), __NV_SATFINITE, __NV_E4M3);
     return make_uint2(e4m3x2_to_bf16x2(c01), e4m3x2_to_bf16x2(c23));
-}
-template <int N>
-CKV_DEV void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 CKV_DEV void ldsm_x4(uint32_t a, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -180,27 +180,35 @@ CKV_DEV uint4 lds_v4(uint32_t addr) {
     return v;
 }
 
-// qbar . k over one half (64 dims) of a 256-byte key row in global memory: 8 independent
-// 16-byte loads, then fp32 FMAs in dimension order.
-CKV_DEV float half_row_dot(const uint16_t* row, int half, const float* qbar) {
-    uint4 w[8];
+// qbar . k over one 64-dimension half (`half`) of two K rows, with all 16 loads in flight; a
+// negative row index gives 0. Dimensions in ascending order, one fmaf chain per row.
+CKV_DEV void half_row_dot2(const uint16_t* kp, int32_t ia, int32_t ib, int half, const float* qbar,
+                           float* sa, float* sb) {
+    uint4 w[2][8];
 #pragma unroll
-    for (int t = 0; t < 8; ++t) w[t] = ldg_nc_v4(row + 64 * half + 8 * t);
+    for (int t = 0; t < 8; ++t) {
+        w[0][t] = ia >= 0 ? ldg_nc_v4(kp + (int64_t)ia * kD + 64 * half + 8 * t) : make_uint4(0u, 0u, 0u, 0u);
+        w[1][t] = ib >= 0 ? ldg_nc_v4(kp + (int64_t)ib * kD + 64 * half + 8 * t) : make_uint4(0u, 0u, 0u, 0u);
+    }
     const float4* q4 = reinterpret_cast<const float4*>(qbar + 64 * half);
-    float s = 0.f;
+    float s[2] = {0.f, 0.f};
 #pragma unroll
     for (int t = 0; t < 8; ++t) {
         const float4 qa = q4[2 * t], qb = q4[2 * t + 1];
-        s = fmaf(qa.x, bf16_lo(w[t].x), s);
-        s = fmaf(qa.y, bf16_hi(w[t].x), s);
-        s = fmaf(qa.z, bf16_lo(w[t].y), s);
-        s = fmaf(qa.w, bf16_hi(w[t].y), s);
-        s = fmaf(qb.x, bf16_lo(w[t].z), s);
-        s = fmaf(qb.y, bf16_hi(w[t].z), s);
-        s = fmaf(qb.z, bf16_lo(w[t].w), s);
-        s = fmaf(qb.w, bf16_hi(w[t].w), s);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            s[r] = fmaf(qa.x, bf16_lo(w[r][t].x), s[r]);
+            s[r] = fmaf(qa.y, bf16_hi(w[r][t].x), s[r]);
+            s[r] = fmaf(qa.z, bf16_lo(w[r][t].y), s[r]);
+            s[r] = fmaf(qa.w, bf16_hi(w[r][t].y), s[r]);
+            s[r] = fmaf(qb.x, bf16_lo(w[r][t].z), s[r]);
+            s[r] = fmaf(qb.y, bf16_hi(w[r][t].z), s[r]);
+            s[r] = fmaf(qb.z, bf16_lo(w[r][t].w), s[r]);
+            s[r] = fmaf(qb.w, bf16_hi(w[r][t].w), s[r]);
+        }
     }
-    return s;
+    *sa = s[0];
+    *sb = s[1];
 }
 
 // Exclusive block scan of one int per thread: x = this thread's exclusive prefix, y = the
@@ -343,15 +351,11 @@ CKV_DEV int cut_bucket_warp(const int32_t* hist, int32_t need, int32_t* above_ou
     return __shfl_sync(0xffffffffu, bin, src);
 }
 
-// Partial tokens of a cut cluster that is not held in shared memory (a large cluster, or a
-// CTA that is not the dedicated one): this CTA's share [p_lo, p_hi) of the cut's top r_part
-// tokens by qbar . k (ties: lower index, i.e. store order), as store rows in prow. The keys
-// are scored from global memory, into shared memory, or, above kPartCap tokens, into a
-// global scratch written once, split across the cluster's CTAs (every CTA of the cluster
-// calls this function then, for the cluster barrier). Not inlined: a cold path.
+// Arguments of partial_rows (below), the partial tokens of a cut cluster that is not held in
+// the ring (a large cluster, or a CTA that is not the dedicated one). Not inlined: a cold path.
 struct PartialArgs {
     const uint16_t* kp;  // the cut cluster's first K row
-    uint32_t* gkeys;     // global key scratch of the unit (above kPartCap tokens)
+    uint32_t* gkeys;     // global key scratch of the unit (cuts of more than kNT tokens)
     const float* qbar;   // shared [128]
     uint32_t* pkey;      // shared [kPartCap + 4]
     int32_t* hist;       // shared [256]
@@ -360,21 +364,31 @@ struct PartialArgs {
     int32_t crow, csz, r_part, p_lo, p_hi;
     int32_t rank, S;
 };
+// The cut cluster's partial rows of this CTA: the top r_part tokens by qbar . k (ties: lower
+// index), listed at selection positions [p_lo, p_hi) of the partial fill. A cut of more than
+// kNT tokens is scored by every CTA of the cluster (an even share each) into the unit's global
+// key scratch, then read back after a cluster barrier (into shared memory when it fits);
+// every CTA of the cluster must call this then.
 __device__ __noinline__ void partial_rows(const PartialArgs& P) {
     const int tid = threadIdx.x, warp = tid >> 5;
-    const bool big_cut = P.csz > kPartCap;
+    const bool coop = P.csz > kNT;
+    const bool in_smem = P.csz <= kPartCap;
     auto score_keys = [&](int32_t k0, int32_t k1, uint32_t* dst) {
-        // two threads per row, one memory round trip per pass
-        for (int32_t i0 = k0; i0 < k1; i0 += kNT / 2) {  // CTA-uniform trip count
-            const int32_t i = i0 + (tid >> 1);
+        // two threads per row, two rows per thread pair: one memory round trip per 256 rows
+        for (int32_t i0 = k0; i0 < k1; i0 += kNT) {  // CTA-uniform trip count
+            const int32_t ia = i0 + (tid >> 1), ib = ia + kNT / 2;
             const int half = tid & 1;
-            float sc = 0.f;
-            if (i < k1) sc = half_row_dot(P.kp + (int64_t)i * kD, half, P.qbar);
-            sc += __shfl_xor_sync(0xffffffffu, sc, 1);
-            if (i < k1 && half == 0) dst[i] = orderable(sc);
+            float sa, sb;
+            half_row_dot2(P.kp, ia < k1 ? ia : -1, ib < k1 ? ib : -1, half, P.qbar, &sa, &sb);
+            sa += __shfl_xor_sync(0xffffffffu, sa, 1);
+            sb += __shfl_xor_sync(0xffffffffu, sb, 1);
+            if (half == 0) {
+                if (ia < k1) dst[ia] = orderable(sa);
+                if (ib < k1) dst[ib] = orderable(sb);
+            }
         }
     };
-    if (big_cut) {
+    if (coop) {
         const int32_t k0 = (int32_t)((int64_t)P.csz * P.rank / P.S);
         const int32_t k1 = (int32_t)((int64_t)P.csz * (P.rank + 1) / P.S);
         score_keys(k0, k1, P.gkeys);
@@ -382,13 +396,15 @@ __device__ __noinline__ void partial_rows(const PartialArgs& P) {
         cluster_wait_acquire();
     }
     if (P.p_hi <= P.p_lo) return;
-    auto key_at = [&](int i) -> uint32_t { return big_cut ? __ldcg(P.gkeys + i) : P.pkey[i]; };
-    if (!big_cut) {
+    if (coop && in_smem) {
+        for (int i = tid; i < P.csz; i += kNT) P.pkey[i] = __ldcg(P.gkeys + i);
+    } else if (!coop) {
         score_keys(0, P.csz, P.pkey);
-        if (tid < 4) P.pkey[P.csz + tid] = 0u;  // pad: never outranks a key
     }
+    if (in_smem && tid < 4) P.pkey[P.csz + tid] = 0u;  // pad: never outranks a key
+    auto key_at = [&](int i) -> uint32_t { return in_smem ? P.pkey[i] : __ldcg(P.gkeys + i); };
     __syncthreads();
-    if (!big_cut && P.csz <= kNT) {
+    if (P.csz <= kNT) {
         // comparison rank (ties: lower index), tpe threads per token, 4 keys per load
         const int tpe = P.csz <= 32 ? 8 : (P.csz <= 64 ? 4 : (P.csz <= 128 ? 2 : 1));
         const int e = tid / tpe, sub = tid % tpe;
@@ -436,18 +452,37 @@ __device__ __noinline__ void partial_rows(const PartialArgs& P) {
             mask |= 255u << shift;
         }
         const uint32_t theta = prefix;
-        int32_t eq_run = 0, sel_run = 0;
-        for (int bse = 0; bse < P.csz; bse += kNT) {  // CTA-uniform trip count
-            const int i = bse + tid;
-            const uint32_t k = i < P.csz ? key_at(i) : 0u;
-            const int32_t eq = (i < P.csz && k == theta) ? 1 : 0;
-            const int2 e2 = block_excl_scan(eq, P.wbuf);
-            const int32_t sel = (i < P.csz) && (k > theta || (eq && eq_run + e2.x < pneed));
-            const int2 s2 = block_excl_scan(sel, P.wbuf);
-            const int32_t pos = sel_run + s2.x;
-            if (sel && pos >= P.p_lo && pos < P.p_hi) P.prow[pos - P.p_lo] = P.crow + i;
-            eq_run += e2.y;
-            sel_run += s2.y;
+        // a contiguous run of keys per thread, in index order: the keys equal to theta before
+        // the run (one scan), then the selected keys before the run (another scan)
+        const int per = (P.csz + kNT - 1) / kNT;
+        const int i0 = tid * per;
+        const int i1 = i0 + per < P.csz ? i0 + per : P.csz;
+        int32_t neq = 0;
+        for (int i = i0; i < i1; ++i) neq += key_at(i) == theta ? 1 : 0;
+        const int32_t eq0 = block_excl_scan(neq, P.wbuf).x;
+        int32_t nsel = 0, eq = eq0;
+        for (int i = i0; i < i1; ++i) {
+            const uint32_t k = key_at(i);
+            if (k > theta) {
+                ++nsel;
+            } else if (k == theta) {
+                nsel += eq < pneed ? 1 : 0;
+                ++eq;
+            }
+        }
+        int32_t pos = block_excl_scan(nsel, P.wbuf).x;
+        eq = eq0;
+        for (int i = i0; i < i1; ++i) {
+            const uint32_t k = key_at(i);
+            bool sel = k > theta;
+            if (k == theta) {
+                sel = eq < pneed;
+                ++eq;
+            }
+            if (sel) {
+                if (pos >= P.p_lo && pos < P.p_hi) P.prow[pos - P.p_lo] = P.crow + i;
+                ++pos;
+            }
         }
     }
     __syncthreads();
@@ -496,7 +531,7 @@ __host__ __device__ inline Layout make_layout(int G, int S, int C, int RB, int p
     L.scl = take(4u * ((kWarps + S) * G + 2 * G));
     L.ccomb = take(4u * S * G * kCombStride);
     L.pbuf = take(2u * kWarps * 256);
-    L.bars = take(8u * 2);
+    L.bars = take(8u * 4);
     L.total = p;
     return L;
 }
@@ -545,12 +580,13 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     float* const s_ccomb = (float*)(base + Ly.ccomb);
     uint16_t* const s_pbuf = (uint16_t*)(base + Ly.pbuf);
     uint64_t* const cbar = (uint64_t*)(base + Ly.bars);      // centroid slice
-    uint64_t* const fbar = cbar + 1;                         // cut cluster rows
+    uint64_t* const fbar = cbar + 1;                         // cut cluster rows (kNT arrivals)
+    uint64_t* const rbar = cbar + 2;                         // [2] ring chunk slots (kNT arrivals)
     float* const s_cent = (float*)(base + Ly.ring);          // centroid slice (aliases the ring)
     float* const s_wcomb = (float*)(base + Ly.ring);         // warp partials (after the rows)
     uint32_t* const s_pkey = (uint32_t*)(base + Ly.ring);    // cut keys (before the rows)
     const uint32_t ringK = smem_u32(base + Ly.ring);
-    const uint32_t ringV = ringK + (uint32_t)RB * 256u;
+    const uint32_t ringV = ringK + (uint32_t)RB * kPitch;
 
     const int64_t kp_base = (int64_t)su * a.kp_ustride;
     const int64_t sp_base = (int64_t)su * a.sp_ustride;
@@ -566,7 +602,9 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     pdl_launch_dependents();
     if (tid == 0) {
         mbar_init(cbar, 1);
-        mbar_init(fbar, 1);
+        mbar_init(fbar, kNT);
+        mbar_init(rbar, kNT);
+        mbar_init(rbar + 1, kNT);
         fence_mbar_init();
         s_wbuf[kWCnt] = 0;
         s_wbuf[kWCopy] = 0;
@@ -612,6 +650,20 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     __syncthreads();
     bool ok = true;
     auto size_of = [&](int c) { return s_off[c + 1] - s_off[c]; };
+    // The cut cluster's rows [row0, row0 + w), w <= kNT, into ring rows 0.. (every thread
+    // arrives on fbar once; thread t copies row t). The fence orders this CTA's earlier
+    // shared-memory accesses of the ring before the copies' writes.
+    auto copy_cut_rows = [&](int32_t row0, int32_t w) {
+        fence_proxy_async();
+        if (tid < w) {
+            mbar_arrive_expect_tx(fbar, 2u * kD * 2u);
+            const int64_t row = kp_base + row0 + tid;
+            bulk_row(ringK + (uint32_t)tid * kPitch, a.kp + row * kD, kD * 2, smem_u32(fbar));
+            bulk_row(ringV + (uint32_t)tid * kPitch, a.vp + row * kD, kD * 2, smem_u32(fbar));
+        } else {
+            mbar_arrive(fbar);
+        }
+    };
     // The slice's scores go to this CTA's own shared memory, with the slice's smallest and
     // largest order keys (over the clusters with tokens; over every cluster in the mixed-
     // precision instantiation, whose rank counts empty clusters too). After one cluster
@@ -738,17 +790,13 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         // every warp finds the cut's bucket itself (no extra block barrier)
         bstar = cut_bucket_warp(s_hist, R, &w_above);
         // When b* holds a single cluster with tokens, that cluster is the cut: CTA S-1, which
-        // fills the partial tokens, starts copying its K and V rows now.
+        // fills the partial tokens, starts copying its K and V rows once the candidates below
+        // are listed.
         if ((int)rank == S - 1 && S > 1 && s_hcnt[bstar] == 1) {
             for (int c = tid; c < C; c += kNT) {
                 const int32_t w = size_of(c);
                 if (w > 0 && w <= RB && w <= kNT && s_bkt[c] == bstar) {
-                    fence_proxy_async();  // the ring's centroid reads come before the copies
-                    const int64_t row = kp_base + s_off[c];
-                    const uint32_t bytes = (uint32_t)w * kD * 2;
-                    mbar_arrive_expect_tx(fbar, 2 * bytes);
-                    bulk_load(base + Ly.ring, a.kp + row * kD, bytes, fbar);
-                    bulk_load(base + Ly.ring + (size_t)RB * 256, a.vp + row * kD, bytes, fbar);
+                    s_wbuf[kWCopyC] = c;
                     s_wbuf[kWCopy] = 1;
                 }
             }
@@ -764,6 +812,10 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
             if (in_b) s_cand[pos0 + __popc(bal & ((1u << lane) - 1u))] = c;
         }
         __syncthreads();
+        if (s_wbuf[kWCopy] != 0) {
+            const int c = s_wbuf[kWCopyC];
+            copy_cut_rows(s_off[c], size_of(c));
+        }
         const int32_t n_b = s_wbuf[kWCnt];
         // exact rank of each candidate among them: 8 threads per candidate
         for (int i0 = 0; i0 < n_b; i0 += kNT / 8) {
@@ -883,16 +935,20 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     const int32_t base_p = base_w + W;
     const int32_t T = base_p + r_part;
     // Work split of the selection index space [0, T). With a partial fill, CTA S-1 takes
-    // exactly the partial tokens (it also ranks them) and the other CTAs split the rest.
+    // the partial tokens (it also loads and ranks the cut cluster) and the last x whole
+    // positions, x = an even share T / S less the cut cluster's rows and a fixed allowance
+    // for the ranking (64 rows), at least 0; the other CTAs split the rest.
     const bool dedicated = r_part > 0 && S > 1 && r_part <= P.prow_cap;
     int32_t lo, hi;
     if (dedicated) {
+        int32_t x = T / S - csz - 64;
+        x = x < 0 ? 0 : (x > base_p ? base_p : x);
         if ((int)rank == S - 1) {
-            lo = base_p;
+            lo = base_p - x;
             hi = T;
         } else {
-            lo = split_point(base_p, rank, S - 1);
-            hi = split_point(base_p, rank + 1, S - 1);
+            lo = split_point(base_p - x, rank, S - 1);
+            hi = split_point(base_p - x, rank + 1, S - 1);
         }
     } else {
         lo = split_point(T, rank, S);
@@ -900,40 +956,16 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     }
     const int32_t p_lo = lo > base_p ? lo - base_p : 0;
     const int32_t p_hi = hi > base_p ? hi - base_p : 0;
-    const bool big_cut = csz > kPartCap;
+    const bool coop_cut = csz > kNT;  // scored by every CTA of the cluster (see partial_rows)
     const bool resident = dedicated && (int)rank == S - 1 && csz <= RB && csz <= kNT;
     const bool cut_far = kMixed && has_cut && is_far(cut_c);
     int32_t* sel_out = a.sel_idx ? a.sel_idx + (int64_t)unit * a.budget : nullptr;
     const int32_t* ids = a.ids + kp_base;
 
     // ---------------------------------------------------------------- phase 3/4: rows
-    // rsrc[p] names the source of ring row p: a store row (>= 0) or a sink / pending row
-    // (-1 - index).
-    // parts: 1 = K rows, 2 = V rows, 3 = both (one commit group)
-    // A far row (kMixed) arrives as its 128 fp8 codes, staged unswizzled in the upper half of
-    // its ring row, plus its two scales; convert_far turns the codes into the bf16 row.
-    auto copy_rows = [&](int p0, int n, int parts) {
-        const int per_row = parts == 3 ? 32 : 16;
-        for (int i = tid; i < n * per_row; i += kNT) {
-            const int p = p0 + i / per_row, j = i & 15;
-            const int part = parts == 3 ? (i >> 4) & 1 : parts - 1;
-            const int32_t r = s_rsrc[p];
-            if (kMixed && r >= 0 && (r & kFarBit) != 0) {
-                const int64_t row = kp_base + (r & ~kFarBit);
-                if (j < 8)
-                    cp_async16((part ? ringV : ringK) + (uint32_t)p * 256u + 128u + (uint32_t)j * 16u,
-                               (part ? a.vp8 : a.kp8) + row * kD + j * 16);
-                else if (j == 8)
-                    cp_async4(smem_u32(part ? &s_rvs[p] : &s_rks[p]), (part ? a.vs8 : a.ks8) + row);
-                continue;
-            }
-            const uint16_t* src = r >= 0 ? (part ? a.vp : a.kp) + (kp_base + r) * kD
-                                         : (part ? a.spv : a.spk) + (sp_base + (-1 - r)) * kD;
-            cp_async16(swz_addr(part ? ringV : ringK, p, j), src + j * 8);
-            if (kMixed && j == 0) (part ? s_rvs : s_rks)[p] = 1.f;
-        }
-        cp_async_commit();
-    };
+    // A far row (kMixed) arrives as its 128 fp8 codes in the upper half of its ring row, its
+    // two scales in rks / rvs; convert_far turns the codes into the bf16 row. rsrc[p] names
+    // the source of ring row p (kMixed only): a store row (kFarBit when far) or -1.
     // Far rows of ring rows [p0, p0 + n): one warp per row; lanes 0-7 hold the K code chunks,
     // lanes 8-15 the V code chunks (16 codes each), all read before any bf16 chunk is written.
     auto convert_far = [&](int p0, int n) {
@@ -941,7 +973,7 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
             const int32_t r = s_rsrc[p];
             if (r < 0 || (r & kFarBit) == 0) continue;  // uniform across the warp
             const int jj = lane & 7;
-            const uint32_t rb = (lane < 8 ? ringK : ringV) + (uint32_t)p * 256u;
+            const uint32_t rb = (lane < 8 ? ringK : ringV) + (uint32_t)p * kPitch;
             uint4 c = make_uint4(0u, 0u, 0u, 0u);
             if (lane < 16) c = lds_v4(rb + 128u + (uint32_t)jj * 16u);
             __syncwarp();
@@ -950,62 +982,80 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
                                             e4m3x2_to_bf16x2(c.y & 0xFFFFu), e4m3x2_to_bf16x2(c.y >> 16));
                 const uint4 hi = make_uint4(e4m3x2_to_bf16x2(c.z & 0xFFFFu), e4m3x2_to_bf16x2(c.z >> 16),
                                             e4m3x2_to_bf16x2(c.w & 0xFFFFu), e4m3x2_to_bf16x2(c.w >> 16));
-                sts_v4(swz_addr(rb - (uint32_t)p * 256u, p, 2 * jj), lo);
-                sts_v4(swz_addr(rb - (uint32_t)p * 256u, p, 2 * jj + 1), hi);
+                sts_v4(rb + (uint32_t)(2 * jj) * 16u, lo);
+                sts_v4(rb + (uint32_t)(2 * jj + 1) * 16u, hi);
             }
             __syncwarp();
         }
     };
-    // Sources (and, when asked for, original token ids) of the selection positions [c0, c1),
-    // written to ring rows p0 ...
-    auto fill_rsrc = [&](int32_t c0, int32_t c1, int p0) {
-        for (int32_t idx = c0 + tid; idx < c1; idx += kNT) {
-            int32_t r;
-            if (idx < base_w) {  // a sink, or pending token idx - n_sink of the ring
-                r = -1 - (idx < a.n_sink ? idx : a.n_sink + (a.pstart + idx - a.n_sink) % a.pring);
-            } else if (idx < base_p) {
-                const int32_t x = idx - base_w;
-                int k0 = 0, khi = n_whole - 1;  // the whole cluster holding x: last wl_pre <= x
-                while (k0 < khi) {
-                    const int mid = (k0 + khi + 1) >> 1;
-                    if (wl_pre[mid] <= x) k0 = mid; else khi = mid - 1;
-                }
-                const int32_t o = wl_off[k0];
-                r = (o & ~kFarBit) + (x - wl_pre[k0]);
-                if (kMixed && (o & kFarBit)) r |= kFarBit;
-            } else {
-                r = s_prow[idx - base_p - p_lo];
-                if (kMixed && cut_far) r |= kFarBit;
-            }
-            s_rsrc[p0 + (idx - c0)] = r;
-            if (sel_out)
-                sel_out[idx] = r >= 0 ? ids[r & ~kFarBit] : (idx < a.n_sink ? idx : (int32_t)(a.m + idx));
-        }
-    };
 
     if (!ok) s_wbuf[kWBad] = 1;
-    const int32_t n_rows = resident ? csz : hi - lo;
-    const int chunk = (resident || n_rows <= RB) ? RB : RB / 2;
-    const int n_chunks = resident ? 1 : (n_rows + chunk - 1) / chunk;
+    // Streamed positions [lo, s_hi): the resident cut cluster's partial tokens are attended
+    // from the rows already in the ring, before the stream reuses it.
+    const int32_t s_hi = resident ? (hi < base_p ? hi : base_p) : hi;
+    const int32_t n_rows = s_hi - lo;
+    const int chunk = n_rows <= RB ? RB : RB / 2;  // <= RB <= kNT: one position per thread
+    const int n_chunks = (n_rows + chunk - 1) / chunk;
+    // Chunk ch: selection positions [lo + ch * chunk, ...) into ring slot ch & 1. Thread t
+    // resolves position c0 + t (a sink or pending row, a whole cluster's row found by binary
+    // search over the compact list, or a partial row), arrives on the slot's mbarrier with the
+    // bytes it copies, then issues its K and V row copies.
     auto issue = [&](int ch) {  // every thread
         const int32_t c0 = lo + ch * chunk;
-        const int32_t c1 = (c0 + chunk < hi) ? c0 + chunk : hi;
-        const int p0 = n_chunks == 1 ? 0 : (ch & 1) * chunk;
-        fill_rsrc(c0, c1, p0);
-        __syncthreads();
-        copy_rows(p0, c1 - c0, 3);
+        const int32_t c1 = (c0 + chunk < s_hi) ? c0 + chunk : s_hi;
+        const int p = (n_chunks == 1 ? 0 : (ch & 1) * chunk) + tid;
+        const uint32_t bar = smem_u32(rbar + (ch & 1));
+        const int32_t idx = c0 + tid;
+        fence_proxy_async();  // this CTA's earlier accesses of the ring come before the copies
+        if (idx >= c1) {
+            mbar_arrive(rbar + (ch & 1));
+            return;
+        }
+        int32_t r;
+        if (idx < base_w) {  // a sink, or pending token idx - n_sink of the ring
+            r = -1 - (idx < a.n_sink ? idx : a.n_sink + (a.pstart + idx - a.n_sink) % a.pring);
+        } else if (idx < base_p) {
+            const int32_t x = idx - base_w;
+            int k0 = 0, khi = n_whole - 1;  // the whole cluster holding x: last wl_pre <= x
+            while (k0 < khi) {
+                const int mid = (k0 + khi + 1) >> 1;
+                if (wl_pre[mid] <= x) k0 = mid; else khi = mid - 1;
+            }
+            const int32_t o = wl_off[k0];
+            r = (o & ~kFarBit) + (x - wl_pre[k0]);
+            if (kMixed && (o & kFarBit)) r |= kFarBit;
+        } else {
+            r = s_prow[idx - base_p - p_lo];
+            if (kMixed && cut_far) r |= kFarBit;
+        }
+        const uint32_t dk = ringK + (uint32_t)p * kPitch, dv = ringV + (uint32_t)p * kPitch;
+        if (kMixed && r >= 0 && (r & kFarBit) != 0) {
+            const int64_t row = kp_base + (r & ~kFarBit);
+            mbar_arrive_expect_tx(rbar + (ch & 1), 2u * kD);
+            bulk_row(dk + 128u, a.kp8 + row * kD, kD, bar);
+            bulk_row(dv + 128u, a.vp8 + row * kD, kD, bar);
+            s_rks[p] = a.ks8[row];
+            s_rvs[p] = a.vs8[row];
+        } else {
+            const uint16_t* sk = r >= 0 ? a.kp + (kp_base + r) * kD : a.spk + (sp_base + (-1 - r)) * kD;
+            const uint16_t* sv = r >= 0 ? a.vp + (kp_base + r) * kD : a.spv + (sp_base + (-1 - r)) * kD;
+            mbar_arrive_expect_tx(rbar + (ch & 1), 2u * kD * 2u);
+            bulk_row(dk, sk, kD * 2, bar);
+            bulk_row(dv, sv, kD * 2, bar);
+            if (kMixed) {
+                s_rks[p] = 1.f;
+                s_rvs[p] = 1.f;
+            }
+        }
+        if (kMixed) s_rsrc[p] = r;
+        if (sel_out)
+            sel_out[idx] = r >= 0 ? ids[r & ~kFarBit] : (idx < a.n_sink ? idx : (int32_t)(a.m + idx));
     };
 
     if (resident) {
-        // ---- the cut cluster in shared memory (plain 256-byte rows): two bulk copies, issued
-        // during the selection when the histogram isolated the cut, else now
-        if (tid == 0 && s_wbuf[kWCopy] == 0) {
-            fence_proxy_async();  // the ring's centroid reads come before the copies
-            const uint32_t bytes = (uint32_t)csz * kD * 2;
-            mbar_arrive_expect_tx(fbar, 2 * bytes);
-            bulk_load(base + Ly.ring, a.kp + (kp_base + crow) * kD, bytes, fbar);
-            bulk_load(base + Ly.ring + (size_t)RB * 256, a.vp + (kp_base + crow) * kD, bytes, fbar);
-        }
+        // ---- the cut cluster in shared memory (ring rows 0..csz-1): one bulk copy per row,
+        // issued during the selection when the histogram isolated the cut, else now
+        if (s_wbuf[kWCopy] == 0) copy_cut_rows(crow, csz);
         const bool got = __syncthreads_and(mbar_wait(fbar, 0, a.err) ? 1 : 0) != 0;
         if (!got) s_wbuf[kWBad] = 1;
         // qbar . k, a half-warp per row (16-byte reads covering one 256-byte row), 8 rows
@@ -1020,7 +1070,7 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
                 const int e = r0 + hw + k * (kNT / 16);
                 sk[k] = 0.f;
                 if (got && e < csz) {
-                    const uint4 w = lds_v4(ringK + (uint32_t)e * 256u + l16 * 16);
+                    const uint4 w = lds_v4(ringK + (uint32_t)e * kPitch + l16 * 16);
                     float t = qa.x * bf16_lo(w.x);
                     t = fmaf(qa.y, bf16_hi(w.x), t);
                     t = fmaf(qa.z, bf16_lo(w.y), t);
@@ -1081,8 +1131,8 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
                 if (cut_far) {
 #pragma unroll
                     for (int part = 0; part < 2; ++part) {
-                        uint2* row = reinterpret_cast<uint2*>(base + Ly.ring + (size_t)part * RB * 256 +
-                                                              (size_t)er * 256);
+                        uint2* row = reinterpret_cast<uint2*>(base + Ly.ring + (size_t)part * RB * kPitch +
+                                                              (size_t)er * kPitch);
                         float sc;
                         const uint2 v = fp8_row_values(row[lane], &sc);
                         __syncwarp();
@@ -1106,7 +1156,7 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         }
         // partial tokens of this CTA's share outside the ring path: rows into prow (every CTA
         // of the cluster takes part when the keys go through the global scratch)
-        if (r_part > 0 && (big_cut || p_hi > p_lo)) {
+        if (r_part > 0 && (coop_cut || p_hi > p_lo)) {
             PartialArgs pa;
             pa.kp = a.kp + (kp_base + crow) * kD;
             pa.gkeys = a.part_scratch ? reinterpret_cast<uint32_t*>(a.part_scratch) +
@@ -1144,12 +1194,9 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     float m2[2] = {-INFINITY, -INFINITY}, l2[2] = {0.f, 0.f};  // heads 2 t4, 2 t4 + 1
     uint16_t* pw = s_pbuf + warp * 256;  // [2][8 heads][16 rows] bf16 (high, low)
     const float qscale = kLog2e * rsqrtf((float)kD);
-    // rows: ring row of tile row t is pos[t] (pos != nullptr) or p0 + t;
-    // swz: rows XOR-swizzled (cp.async ring) or plain (bulk copies of the cut cluster)
-    auto attend = [&](int p0, int n, const int32_t* pos, bool swz) {
-        auto addr = [&](uint32_t rbase, int p, int j) {
-            return rbase + (uint32_t)p * 256u + ((uint32_t)(j ^ (swz ? (p & 7) : 0)) << 4);
-        };
+    // rows: ring row of tile row t is pos[t] (pos != nullptr) or p0 + t
+    auto attend = [&](int p0, int n, const int32_t* pos) {
+        auto addr = [&](uint32_t rbase, int p, int j) { return rbase + (uint32_t)p * kPitch + ((uint32_t)j << 4); };
         const int n_tiles = (n + 15) >> 4;
         for (int tile = warp; tile < n_tiles; tile += kWarps) {
             const int r0 = tile * 16;
@@ -1225,29 +1272,32 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         }
     };
 
-    // ---- attention, chunk by chunk: the resident cut cluster is one chunk (its selected rows
-    // listed in prow, plain rows); otherwise the rows stream through the ring, two chunks in
-    // flight. One call site for each of issue and attend keeps the code small.
+    // ---- attention, chunk by chunk: the resident cut cluster first (its selected rows listed
+    // in prow), as chunk -1; then the streamed rows through the ring, two chunks in flight.
+    // One call site for each of issue and attend keeps the code small.
     int next = 0;  // chunks issued
-    for (int ch = 0; ch < n_chunks; ++ch) {  // CTA-uniform trip count
+    for (int ch = resident ? -1 : 0; ch < n_chunks; ++ch) {  // CTA-uniform trip count
         int pb0 = 0, n = r_part;
-        if (!resident) {
+        const int32_t* pos = s_prow;
+        if (ch >= 0) {
             while (next < n_chunks && next <= ch + 1) {
-                if (next >= 2) __syncthreads();  // every warp is done with this slot
+                // the slot (or, after the resident chunk, the ring) is no longer read
+                if (next >= 2 || (resident && next == 0)) __syncthreads();
                 issue(next);
                 ++next;
             }
-            if (next > ch + 1) cp_async_wait<1>(); else cp_async_wait<0>();
-            __syncthreads();
+            if (!mbar_wait(rbar + (ch & 1), (uint32_t)(ch >> 1) & 1u, a.err)) s_wbuf[kWBad] = 1;
             const int32_t c0 = lo + ch * chunk;
-            n = (hi - c0) < chunk ? (hi - c0) : chunk;
+            n = (s_hi - c0) < chunk ? (s_hi - c0) : chunk;
             pb0 = n_chunks == 1 ? 0 : (ch & 1) * chunk;
+            pos = nullptr;
             if (kMixed) {
+                __syncthreads();  // rsrc and the scales of the chunk
                 convert_far(pb0, n);
                 __syncthreads();
             }
         }
-        if (s_wbuf[kWBad] == 0) attend(pb0, n, resident ? s_prow : nullptr, !resident);
+        if (s_wbuf[kWBad] == 0) attend(pb0, n, pos);
     }
 
     // ---------------------------------------------------------------- phase 5: combine
