@@ -369,7 +369,7 @@ int ckv_create(const ckv_config* cfg, ckv_ctx** out) {
     rc = rc ? rc : dev_alloc(&c->ws.assign, (size_t)(U * c->cap_c), c);
     rc = rc ? rc : dev_alloc(&c->ws.best, (size_t)(U * c->cap_c), c);
     rc = rc ? rc : dev_alloc(&c->ws.perm, (size_t)(U * c->cap_c), c);
-    rc = rc ? rc : dev_alloc(&c->ws.chunk, (size_t)(U * n_chunks(c->cap_c) * cmax), c);
+    rc = rc ? rc : dev_alloc(&c->ws.chunk, (size_t)(2 * U * n_chunks(c->cap_c) * cmax), c);  // two count buffers
     rc = rc ? rc : dev_alloc(&c->ws.part, (size_t)(U * c->group * c->cap_c), c);  // per query head
     rc = rc ? rc : dev_alloc(&c->err, 4, c);
     if (rc == CKV_OK) {
@@ -441,17 +441,25 @@ int cluster_prefill(ckv_ctx* ctx, int32_t layer, const void* K, const void* V, i
     rl.ids = c->ids + c->rows_kp(layer, 0);
     rl.ustride_rows = c->cap_c;
     rl.id_base = ns;
-    AssignPlan plan;
-    rc = prepare_kmeans_assign(kv, c->ws.mu_hat, cmax, C, c->ws.assign, c->cap_c, c->ws.best,
-                               c->cap_c, c->err, &plan);
+    // The assignment launch counts each key into its chunk's histogram. Iterations alternate
+    // between two count buffers: the scatter of iteration i zeroes the one iteration i + 1
+    // counts into (the first is zeroed here).
+    const size_t cnt_elems = (size_t)U * (size_t)n_chunks(n - ns) * (size_t)C;
+    int32_t* cnt[2] = {c->ws.chunk, c->ws.chunk + (size_t)U * n_chunks(c->cap_c) * cmax};
+    cudaError_t ze = cudaMemsetAsync(cnt[0], 0, cnt_elems * sizeof(int32_t), s);
+    if (ze != cudaSuccess) return cuda_fail(ze, "prefill: zero counts");
+    AssignPlan plan[2];
+    for (int b = 0; b < 2 && !rc; ++b)
+        rc = prepare_kmeans_assign(kv, c->ws.mu_hat, cmax, C, c->ws.assign, c->cap_c, c->ws.best,
+                                   c->cap_c, c->err, &plan[b], cnt[b]);
     if (rc) return rc;
     for (int it = 0; it < c->cfg.iters; ++it) {
-        rc = run_kmeans_assign(plan, s);
+        rc = run_kmeans_assign(plan[it & 1], s);
         if (rc) return rc;
         const bool last = it + 1 == c->cfg.iters;
         rc = launch_kmeans_update(kv, c->ws.assign, c->cap_c, C, mu, cmax, c->ws.mu_hat, cmax,
-                                  offs, cmax + 1, c->ws.perm, c->cap_c, c->ws.chunk,
-                                  last ? &rl : nullptr, c->err, s);
+                                  offs, cmax + 1, c->ws.perm, c->cap_c, cnt[it & 1],
+                                  last ? &rl : nullptr, c->err, s, true, last ? nullptr : cnt[(it + 1) & 1]);
         if (rc) return rc;
     }
     if (ns > 0) {

@@ -41,7 +41,7 @@ struct Workspace {
     int32_t* assign = nullptr;   // [U][cap_c]
     float* best = nullptr;       // [U][cap_c]
     int32_t* perm = nullptr;     // [U][cap_c]
-    int32_t* chunk = nullptr;    // [U][n_chunks(cap_c)][Cmax]
+    int32_t* chunk = nullptr;    // 2 x [U][n_chunks(cap_c)][Cmax] (two count buffers)
     float* part = nullptr;       // decode partial-cut scratch [U][cap_c] (keys of the cut cluster)
     int32_t U = 0;
     int64_t cap = 0;
@@ -136,9 +136,12 @@ struct AssignPlanImpl;
 struct AssignPlan {
     std::shared_ptr<AssignPlanImpl> impl;
 };
+// counts (optional): [U][n_chunks(m)][C] integer counts, zero on entry; the launch adds one
+// for every key to (its chunk, its cluster), which is what the update's count kernel computes.
 int prepare_kmeans_assign(const KeysView& k, const uint16_t* mu_hat, int64_t muhat_ustride,
                           int32_t C, int32_t* assign, int64_t assign_ustride, float* best,
-                          int64_t best_ustride, uint32_t* err, AssignPlan* out);
+                          int64_t best_ustride, uint32_t* err, AssignPlan* out,
+                          int32_t* counts = nullptr);
 int run_kmeans_assign(const AssignPlan& plan, cudaStream_t s);
 
 struct Relayout {  // final-iteration relayout of K and V into the cluster-major store
@@ -150,11 +153,16 @@ struct Relayout {  // final-iteration relayout of K and V into the cluster-major
     int32_t id_base = 0;       // original id of local key 0
 };
 
+// chunk_ws: [U][n_chunks(m)][C] ints. counted: chunk_ws already holds the per-chunk counts of
+// `assign` (from the assignment launch), so the count kernel is skipped. zero_next (optional):
+// another [U][n_chunks(m)][C] buffer that the scatter sets to zero, ready for the next
+// assignment launch to count into.
 int launch_kmeans_update(const KeysView& k, const int32_t* assign, int64_t assign_ustride,
                          int32_t C, float* mu, int64_t mu_ustride, uint16_t* mu_hat,
                          int64_t muhat_ustride, int32_t* offsets, int64_t off_ustride,
                          int32_t* perm, int64_t perm_ustride, int32_t* chunk_ws,
-                         const Relayout* relayout, uint32_t* err, cudaStream_t s);
+                         const Relayout* relayout, uint32_t* err, cudaStream_t s,
+                         bool counted = false, int32_t* zero_next = nullptr);
 
 int launch_copy_sinks(const uint16_t* K, const uint16_t* V, int64_t n, int32_t U, int32_t n_sink,
                       uint16_t* spk, uint16_t* spv, int64_t sp_ustride_rows, cudaStream_t s);

@@ -18,7 +18,9 @@
 //   warps 0..15 epilogue: warp w reads TMEM lanes 32*(w%4).. (its rows) and column quarter
 //               w/4 of each slot with tcgen05.ld, frees the slot, takes the maximum of each
 //               32 columns with three-input max instructions and the first column holding
-//               it, and merges the four quarters through shared memory.
+//               it, and merges the four quarters through shared memory. When asked, each
+//               key's final cluster is also counted into its 1024-key chunk's histogram
+//               (integer atomics), the counting sort's first pass.
 // For C > 512 the host launches once per 512-centroid chunk. Each later launch merges into
 // the running (best value, index) of the earlier ones, so ties still go to the lower c.
 #include "ckv_common.cuh"
@@ -51,6 +53,9 @@ struct AssignParams {
     int64_t assign_ustride;
     float* best;
     int64_t best_ustride;
+    int32_t* counts;       // [U][nch][C_all] chunk counts to add to (last launch only), or null
+    int32_t nch;
+    int32_t C_all;
     uint32_t* err;
 };
 
@@ -326,6 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     p.assign[(int64_t)u * p.assign_ustride + r] = bidx;
                     if (p.store_best) p.best[(int64_t)u * p.best_ustride + r] = best;
+                    else if (p.counts)
+                        atomicAdd(p.counts + ((int64_t)u * p.nch + r / kChunk) * p.C_all + bidx, 1);
                 }
             }
         }
@@ -349,7 +356,7 @@ struct AssignPlanImpl {
 
 int prepare_kmeans_assign(const KeysView& k, const uint16_t* mu_hat, int64_t muhat_ustride,
                           int32_t C, int32_t* assign, int64_t assign_ustride, float* best,
-                          int64_t best_ustride, uint32_t* err, AssignPlan* out) {
+                          int64_t best_ustride, uint32_t* err, AssignPlan* out, int32_t* counts) {
     auto impl = std::make_shared<AssignPlanImpl>();
     out->impl = impl;
     if (k.m <= 0 || k.U <= 0) return CKV_OK;
@@ -365,6 +372,9 @@ int prepare_kmeans_assign(const KeysView& k, const uint16_t* mu_hat, int64_t muh
     p.assign_ustride = assign_ustride;
     p.best = best;
     p.best_ustride = best_ustride;
+    p.counts = counts;
+    p.nch = (int32_t)n_chunks(k.m);
+    p.C_all = C;
     p.err = err;
     const int nchunks = (C + 2 * kSlotCols - 1) / (2 * kSlotCols);
     const int sms = num_sms_of_current_device();

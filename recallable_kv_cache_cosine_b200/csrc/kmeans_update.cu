@@ -227,7 +227,7 @@ constexpr int kScatterKeysPerWarp = kChunk / kScatterWarps;  // 128
 __global__ void __launch_bounds__(kScatterWarps * 32) kmeans_scatter_kernel(
     const int32_t* assign, int64_t a_ustride, int64_t m, int32_t C, int32_t nch,
     const int32_t* chunk, const int32_t* offsets, int64_t off_ustride, int32_t* perm,
-    int64_t perm_ustride) {
+    int64_t perm_ustride, int32_t* zero_next) {
     pdl_launch_dependents();  // let the next kernel in the stream be scheduled early
     pdl_wait();               // the previous kernel's writes are visible from here on
     extern __shared__ int32_t cntw[];  // [kScatterWarps][C] counts, then first positions
@@ -244,6 +244,10 @@ __global__ void __launch_bounds__(kScatterWarps * 32) kmeans_scatter_kernel(
         sa[i] = c;
     }
     for (int i = tid; i < kScatterWarps * C; i += kScatterWarps * 32) cntw[i] = 0;
+    if (zero_next) {  // this chunk's row of the next iteration's count buffer
+        int32_t* z = zero_next + ((int64_t)u * nch + ch) * C;
+        for (int c = tid; c < C; c += kScatterWarps * 32) z[c] = 0;
+    }
     __syncthreads();
     int32_t* mine = cntw + warp * C;
     const uint32_t lt = (1u << lane) - 1u;
@@ -410,7 +414,8 @@ int launch_kmeans_update(const KeysView& k, const int32_t* assign, int64_t assig
                          int32_t C, float* mu, int64_t mu_ustride, uint16_t* mu_hat,
                          int64_t muhat_ustride, int32_t* offsets, int64_t off_ustride,
                          int32_t* perm, int64_t perm_ustride, int32_t* chunk_ws,
-                         const Relayout* relayout, uint32_t* err, cudaStream_t s) {
+                         const Relayout* relayout, uint32_t* err, cudaStream_t s, bool counted,
+                         int32_t* zero_next) {
     const int32_t nch = (int32_t)n_chunks(k.m);
     cudaError_t e;
     const size_t hsmem = (size_t)C * sizeof(int32_t);
@@ -420,7 +425,7 @@ int launch_kmeans_update(const KeysView& k, const int32_t* assign, int64_t assig
     if (rc == CKV_OK) rc = ensure_smem((const void*)kmeans_scatter_kernel, scsmem, "scatter: set smem");
     if (rc == CKV_OK) rc = ensure_smem((const void*)kmeans_scan_kernel, ssmem, "scan: set smem");
     if (rc != CKV_OK) return rc;
-    if (nch > 0) {
+    if (nch > 0 && !counted) {
         e = launch_pdl(kmeans_count_kernel, dim3(nch, k.U), dim3(256), hsmem, s, assign,
                        assign_ustride, k.m, C, nch, chunk_ws, err);
         if (e != cudaSuccess) return cuda_fail(e, "update: count launch");
@@ -431,7 +436,7 @@ int launch_kmeans_update(const KeysView& k, const int32_t* assign, int64_t assig
     if (nch > 0) {
         e = launch_pdl(kmeans_scatter_kernel, dim3(nch, k.U), dim3(kScatterWarps * 32), scsmem, s, assign,
                        assign_ustride, k.m, C, nch, chunk_ws, offsets, off_ustride, perm,
-                       perm_ustride);
+                       perm_ustride, zero_next);
         if (e != cudaSuccess) return cuda_fail(e, "update: scatter launch");
     }
     Relayout rl{};
