@@ -52,7 +52,7 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 
 # DRAM bytes per select+attend launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum)
 # for the current kernel, or None when the kernel changed after the counters were taken.
-SELECT_ATTEND_TRAFFIC = 6.137e6  # ncu --set full, two launches of the 32k / budget-1k layer, cold L2
+SELECT_ATTEND_TRAFFIC = None  # the kernel changed after the last ncu capture
 
 
 def peaks():
@@ -448,8 +448,10 @@ def split_pass(ckv, ctx, q, s, L, dev, hbm_gbs):
 
 
 def launches_per_prefill(C, iters):
+    # init; per Lloyd iteration the assignment launches (one per 512 centroids, the last one
+    # also counting the chunk histograms), scan, scatter and mean; the sink copy
     assign_launches = (C + 511) // 512
-    return 1 + iters * (assign_launches + 4) + 1
+    return 1 + iters * (assign_launches + 3) + 1
 
 
 def run_gpu(args, world, rank, local):
@@ -659,6 +661,30 @@ def run_gpu(args, world, rank, local):
     ctx.close()
 
 
+# Decode shapes that `--shape` runs alone (small, self-contained cases for profilers).
+SHAPES = {
+    "headline": dict(B=1, budget=BUDGET, n=N_CTX, C=C_CLUSTERS),
+    "batch8_budget2k": dict(B=8, budget=2048, n=N_CTX, C=C_CLUSTERS),
+    "batch4_budget1k": dict(B=4, budget=1024, n=N_CTX, C=C_CLUSTERS),
+    "long_128k": dict(B=1, budget=2048, n=131072, C=1600),
+}
+
+
+def run_shape(args):
+    """One decode shape only: --layers layer stores, --decode-steps steps, one JSON line."""
+    import recallable_kv_cache_cosine_b200 as ckv
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    hbm_gbs, _, peak_kind = peaks()
+    sh = SHAPES[args.shape]
+    s = torch.cuda.Stream(device=dev)
+    r = decode_shape(ckv, s, dev, hbm_gbs, L=args.layers, D=args.decode_steps,
+                     what=f"{args.shape}: batch {sh['B']} x 8 KV heads, n={sh['n']}, C={sh['C']}, "
+                          f"budget {sh['budget']}, {args.layers} layer stores", **sh)
+    r.update({"shape": args.shape, "peak_kind": peak_kind})
+    print(json.dumps(r), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -669,10 +695,16 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=64)
     ap.add_argument("--cpu-layer-steps", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shape", choices=sorted(SHAPES), default=None,
+                    help="time one decode shape alone (1 GPU) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_env()
+    if args.shape and args.impl == "ours":
+        if rank == 0:
+            run_shape(args)
+        return
     if args.impl == "reference":
         run_reference(args, world, rank)
         return

@@ -580,8 +580,8 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     float* const s_ccomb = (float*)(base + Ly.ccomb);
     uint16_t* const s_pbuf = (uint16_t*)(base + Ly.pbuf);
     uint64_t* const cbar = (uint64_t*)(base + Ly.bars);      // centroid slice
-    uint64_t* const fbar = cbar + 1;                         // cut cluster rows (kNT arrivals)
-    uint64_t* const rbar = cbar + 2;                         // [2] ring chunk slots (kNT arrivals)
+    uint64_t* const fbar = cbar + 1;                         // cut cluster rows (a warp's arrival each)
+    uint64_t* const rbar = cbar + 2;                         // [2] ring chunk slots (a warp's arrival each)
     float* const s_cent = (float*)(base + Ly.ring);          // centroid slice (aliases the ring)
     float* const s_wcomb = (float*)(base + Ly.ring);         // warp partials (after the rows)
     uint32_t* const s_pkey = (uint32_t*)(base + Ly.ring);    // cut keys (before the rows)
@@ -602,9 +602,9 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     pdl_launch_dependents();
     if (tid == 0) {
         mbar_init(cbar, 1);
-        mbar_init(fbar, kNT);
-        mbar_init(rbar, kNT);
-        mbar_init(rbar + 1, kNT);
+        mbar_init(fbar, kWarps);
+        mbar_init(rbar, kWarps);
+        mbar_init(rbar + 1, kWarps);
         fence_mbar_init();
         s_wbuf[kWCnt] = 0;
         s_wbuf[kWCopy] = 0;
@@ -650,18 +650,26 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     __syncthreads();
     bool ok = true;
     auto size_of = [&](int c) { return s_off[c + 1] - s_off[c]; };
-    // The cut cluster's rows [row0, row0 + w), w <= kNT, into ring rows 0.. (every thread
-    // arrives on fbar once; thread t copies row t). The fence orders this CTA's earlier
-    // shared-memory accesses of the ring before the copies' writes.
+    // One arrival per warp on a chunk mbarrier, announcing the bytes its lanes copy (before
+    // any of those copies is issued, so the transaction count never goes below zero).
+    auto warp_arrive = [&](uint64_t* bar, uint32_t bytes) {
+        const uint32_t total = __reduce_add_sync(0xffffffffu, bytes);
+        if (lane == 0) {
+            if (total) mbar_arrive_expect_tx(bar, total);
+            else mbar_arrive(bar);
+        }
+        __syncwarp();
+    };
+    // The cut cluster's rows [row0, row0 + w), w <= kNT, into ring rows 0.. (thread t copies
+    // row t). The fence orders this CTA's earlier shared-memory accesses of the ring before
+    // the copies' writes.
     auto copy_cut_rows = [&](int32_t row0, int32_t w) {
         fence_proxy_async();
+        warp_arrive(fbar, tid < w ? 2u * kD * 2u : 0u);
         if (tid < w) {
-            mbar_arrive_expect_tx(fbar, 2u * kD * 2u);
             const int64_t row = kp_base + row0 + tid;
             bulk_row(ringK + (uint32_t)tid * kPitch, a.kp + row * kD, kD * 2, smem_u32(fbar));
             bulk_row(ringV + (uint32_t)tid * kPitch, a.vp + row * kD, kD * 2, smem_u32(fbar));
-        } else {
-            mbar_arrive(fbar);
         }
     };
     // The slice's scores go to this CTA's own shared memory, with the slice's smallest and
@@ -998,8 +1006,8 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     const int n_chunks = (n_rows + chunk - 1) / chunk;
     // Chunk ch: selection positions [lo + ch * chunk, ...) into ring slot ch & 1. Thread t
     // resolves position c0 + t (a sink or pending row, a whole cluster's row found by binary
-    // search over the compact list, or a partial row), arrives on the slot's mbarrier with the
-    // bytes it copies, then issues its K and V row copies.
+    // search over the compact list, or a partial row); each warp announces its lanes' bytes on
+    // the slot's mbarrier, then every lane issues its K and V row copies.
     auto issue = [&](int ch) {  // every thread
         const int32_t c0 = lo + ch * chunk;
         const int32_t c1 = (c0 + chunk < s_hi) ? c0 + chunk : s_hi;
@@ -1007,12 +1015,10 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         const uint32_t bar = smem_u32(rbar + (ch & 1));
         const int32_t idx = c0 + tid;
         fence_proxy_async();  // this CTA's earlier accesses of the ring come before the copies
+        int32_t r = 0;
         if (idx >= c1) {
-            mbar_arrive(rbar + (ch & 1));
-            return;
-        }
-        int32_t r;
-        if (idx < base_w) {  // a sink, or pending token idx - n_sink of the ring
+            // no row
+        } else if (idx < base_w) {  // a sink, or pending token idx - n_sink of the ring
             r = -1 - (idx < a.n_sink ? idx : a.n_sink + (a.pstart + idx - a.n_sink) % a.pring);
         } else if (idx < base_p) {
             const int32_t x = idx - base_w;
@@ -1028,10 +1034,12 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
             r = s_prow[idx - base_p - p_lo];
             if (kMixed && cut_far) r |= kFarBit;
         }
+        const bool far = kMixed && r >= 0 && (r & kFarBit) != 0;
+        warp_arrive(rbar + (ch & 1), idx >= c1 ? 0u : (far ? 2u * kD : 2u * kD * 2u));
+        if (idx >= c1) return;
         const uint32_t dk = ringK + (uint32_t)p * kPitch, dv = ringV + (uint32_t)p * kPitch;
-        if (kMixed && r >= 0 && (r & kFarBit) != 0) {
+        if (far) {
             const int64_t row = kp_base + (r & ~kFarBit);
-            mbar_arrive_expect_tx(rbar + (ch & 1), 2u * kD);
             bulk_row(dk + 128u, a.kp8 + row * kD, kD, bar);
             bulk_row(dv + 128u, a.vp8 + row * kD, kD, bar);
             s_rks[p] = a.ks8[row];
@@ -1039,7 +1047,6 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         } else {
             const uint16_t* sk = r >= 0 ? a.kp + (kp_base + r) * kD : a.spk + (sp_base + (-1 - r)) * kD;
             const uint16_t* sv = r >= 0 ? a.vp + (kp_base + r) * kD : a.spv + (sp_base + (-1 - r)) * kD;
-            mbar_arrive_expect_tx(rbar + (ch & 1), 2u * kD * 2u);
             bulk_row(dk, sk, kD * 2, bar);
             bulk_row(dv, sv, kD * 2, bar);
             if (kMixed) {
