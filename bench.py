@@ -235,8 +235,12 @@ def decode_shape(ckv, s, dev, hbm_gbs, B, L, D, budget, n, C, what, mixed_n_near
                     K[b, h], V[b, h] = si.keys_values_torch(SEED + 7, si.unit_id(l, b, h, B, HKV), n,
                                                             C, dev)
                 qs[:, l, b] = si.queries_torch(SEED + 7, l, b, D, HQ, dev)
+            # the prefill on s reads K / V after they are written; the next layer's K / V
+            # are written after it ends
+            s.wait_stream(torch.cuda.current_stream())
             with torch.cuda.stream(s):
                 cx.cluster_prefill(l, K, V, C, stream=s)
+            torch.cuda.current_stream().wait_stream(s)
         if mixed_n_near is not None:
             cx.enable_fp8(stream=s)
         s.synchronize()
@@ -334,6 +338,7 @@ def extra_measurements(ckv, ctx, q, out, s, L, dev, hbm_gbs, bf16_tflops):
             Ks[0, h], Vs[0, h] = si.keys_values_torch(SEED + 11, h, n_s, c_s, dev)
         cs = ckv.ClusterKV(n_layers=1, batch=1, n_kv_heads=HKV, n_q_heads=HQ, capacity=n_s,
                            max_clusters=c_s, seed=SEED)
+        s.wait_stream(torch.cuda.current_stream())  # the inputs are written
         with torch.cuda.stream(s):
             cs.cluster_prefill(0, Ks, Vs, c_s, stream=s)
         s.synchronize()
@@ -415,6 +420,7 @@ def split_pass(ckv, ctx, q, s, L, dev, hbm_gbs):
                        max_clusters=cmax, seed=SEED)
     drift = torch.empty(HKV, C_CLUSTERS, dtype=torch.float32, device=dev)
     cnt = torch.empty(HKV, dtype=torch.int32, device=dev)
+    s.wait_stream(torch.cuda.current_stream())  # the inputs are written
     res = {}
     try:
         for label, tau, mx in (("detect_only", float("inf"), 0), ("median", None, cmax - C_CLUSTERS)):
@@ -506,6 +512,7 @@ def run_gpu(args, world, rank, local):
     launches["C"] = 2 * W + 1
 
     # ------------------------------------------------------------ capture B and C
+    s.wait_stream(torch.cuda.current_stream())  # the inputs are written
     with torch.cuda.stream(s):
         section_a()
     s.synchronize()
