@@ -52,7 +52,7 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 
 # DRAM bytes per select+attend launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum)
 # for the current kernel, or None when the kernel changed after the counters were taken.
-SELECT_ATTEND_TRAFFIC = None  # the kernel changed after the last ncu capture
+SELECT_ATTEND_TRAFFIC = 6.092e6  # dram read + write per launch, ncu --set full of the headline layer (cold L2)
 
 
 def peaks():
@@ -607,7 +607,7 @@ def run_gpu(args, world, rank, local):
 
     # ------------------------------------------------------------ more shapes (rank 0)
     extra = {}
-    if rank == 0:
+    if rank == 0 and not args.no_extras:
         extra = extra_measurements(ckv, ctx, q, out, s, L, dev, hbm_gbs, bf16_tflops)
 
     # ------------------------------------------------------------ CPU baseline (rank 0, N = 1)
@@ -702,6 +702,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=64)
     ap.add_argument("--cpu-layer-steps", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other shapes, the sweep, per-head and split timings")
     ap.add_argument("--shape", choices=sorted(SHAPES), default=None,
                     help="time one decode shape alone (1 GPU) and exit")
     args = ap.parse_args()
