@@ -1470,8 +1470,9 @@ int ring_rows(int S, int budget) {
 // largest power of two <= 16 (and <= 64 / G, which bounds CTA 0's combine buffer) whose
 // U * S CTAs take at most half of the SMs when the units are few (U * 16 <= SMs), so that the
 // next launch's CTAs, started early by programmatic dependent launch, find SMs of their own;
-// with more units, at most all of the SMs; with more units than SMs, S = 1. The ring takes one
-// CTA's share of the budget, reduced in steps of 16 rows while the launch does not fit.
+// with more units, at most two CTAs per SM (then the layout must fit two per SM); with more
+// units than that, S = 1. The ring takes one CTA's share of the budget, reduced in steps of
+// 16 rows while the launch does not fit.
 template <int G, bool kPerHead, bool kMixed>
 int plan_for(const DecodeArgs& a, int num_sms, Plan* out) {
     static std::mutex mtx;
@@ -1493,13 +1494,16 @@ int plan_for(const DecodeArgs& a, int num_sms, Plan* out) {
     }
     auto kern = select_attend_kernel<G, kPerHead, kMixed>;
     Plan best{};
-    const int64_t sm_cap = (int64_t)U * 16 <= num_sms ? num_sms / 2 : num_sms;
+    const int64_t sm_cap = (int64_t)U * 16 <= num_sms ? num_sms / 2 : 2 * (int64_t)num_sms;
+    constexpr uint32_t kTwoPerSm = 113 * 1024;  // two CTAs share one SM's 228 KB
     for (int S = 16; S >= 1 && best.p.S == 0; S /= 2) {
         if (S > 1 && (S * G > 64 || (int64_t)U * S > sm_cap)) continue;
         for (int RB = ring_rows(S, a.budget); RB >= 64 && best.p.S == 0; RB -= 16) {
             const int pc = prow_capacity(a.budget, S);
             const Layout L = make_layout(G, S, a.C, RB, pc);
             if (L.total > 227 * 1024) continue;
+            // more CTAs than SMs: the launch is one wave only with two CTAs per SM
+            if (S > 1 && (int64_t)U * S > num_sms && L.total > kTwoPerSm) continue;
             int nclusters = 0;
             const int rc = max_active_clusters(kern, S, L.total, &smem_set, &nonportable_set, &nclusters);
             if (rc != CKV_OK) return rc;
