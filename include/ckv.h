@@ -111,8 +111,10 @@ CKV_API int cluster_prefill(ckv_ctx* ctx, int32_t layer, const void* K, const vo
  *   out       : device fp32 [batch, n_q_heads, 128].
  *   sel_idx   : optional device int32 [batch, n_kv_heads, budget]. Original token ids of
  *               the selected rows in the kernel's order: sinks, pending, the whole clusters
- *               in cluster-index order (each in store order), then the partial tokens (in
- *               store order). Entries past the count are -1.
+ *               in walk order (descending centroid score, ties to the lower cluster index;
+ *               each in store order), then the partial tokens (in store order). Entries past
+ *               the count are -1. Without a cut (every token fits) the whole clusters come
+ *               in cluster-index order.
  *   sel_count : optional device int32 [batch, n_kv_heads] = min(budget, n_total).
  * Reads the store only, so it can be captured in a CUDA graph. The token counts are read
  * at call time and baked into a captured launch. The kernel uses programmatic dependent

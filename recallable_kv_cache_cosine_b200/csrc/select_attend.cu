@@ -22,19 +22,17 @@
 //      store. The queries, the sink / pending rows and every output are touched only after
 //      the wait;
 //   1. qbar = sum of the group's queries; each CTA scores its slice (a warp per centroid,
-//      four in flight) and writes the scores into every CTA of the cluster through
-//      distributed shared memory;
+//      four in flight) into its own shared memory; after one cluster barrier every CTA reads
+//      the other slices through distributed shared memory;
 //   2. every CTA computes the same selection on its own. The walk in descending
 //      (score, -index) order stops at the first cluster whose inclusive token count exceeds
 //      the remaining budget R: the cut, a size-weighted quantile of the scores. The scores are
 //      mapped monotonically onto 256 linear buckets between the smallest and the largest;
-//      a size-weighted histogram gives the cut's bucket b*. Every cluster of a higher bucket
-//      is taken whole; only the few clusters of bucket b* are ranked exactly, which gives the
-//      cut and the whole clusters of b* (those ranked before the cut). Whole clusters are laid
-//      out in cluster-index order (attention over a set does not depend on row order), by one
-//      block scan of their sizes;
+//      a size-weighted histogram gives the cut's bucket b*. The clusters of b* and above (a
+//      dozen or two) are compacted and ranked exactly among themselves in one pass, which
+//      gives each one's walk rank and prefix: the whole clusters in walk order, and the cut;
 //   3. the selected rows form one index space: sinks, pending (in append order, from the
-//      two-window pending ring), whole clusters by index, then the partial tokens of the cut
+//      two-window pending ring), whole clusters in walk order, then the partial tokens of the cut
 //      cluster in store order. With a partial fill and S > 1, CTA S-1 takes the partial
 //      tokens: it bulk-copies the cut cluster's K and V rows (started during the selection
 //      when the histogram isolates the cut), ranks the tokens by qbar . k there and attends
@@ -84,14 +82,14 @@ constexpr int kRowBytes = 2 * kPitch;  // one K row and one V row
 constexpr int kCombStride = 130;       // accumulator[128], max, sum
 
 // wbuf slots
-constexpr int kWCnt = 40;     // candidates found in the cut's bucket
+constexpr int kWRank = 43;    // the cut's walk rank (the number of whole clusters)
 constexpr int kWCut = 41;     // the cut cluster
 constexpr int kWPre = 42;     // tokens of bucket b* ranked before the cut
-constexpr int kWCopyC = 43;   // the cluster whose rows the early cut copies fetch
 constexpr int kWCopy = 45;    // the cut cluster's bulk copies were issued
 constexpr int kWBad = 46;     // a bounded wait of this CTA gave up
 constexpr int kWCnt2 = 47;    // candidates found in the bucket of walk rank n_near - 1
 constexpr int kWNear = 64;    // [2] the walk key of rank n_near - 1 (two halves)
+constexpr int kWList = 66;    // [8] candidates compacted by each warp
 constexpr int32_t kFarBit = 0x40000000;  // rsrc flag: a store row read from the fp8 copy
 
 CKV_DEV uint32_t orderable(float f) {
@@ -490,8 +488,8 @@ __device__ __noinline__ void partial_rows(const PartialArgs& P) {
 
 // Shared-memory layout, computed identically on the host (launch size) and the device.
 struct Layout {
-    uint32_t ring, qbar, qh, score, off, spre, cand, bkt, hist, hcnt, hnear, rkey, prow, rsrc, rks,
-        rvs, wbuf, scl, ccomb, pbuf, bars, total;
+    uint32_t ring, qbar, qh, score, off, spre, cand, clist, bkt, hist, hcnt, hnear, rkey, prow,
+        rsrc, rks, rvs, wbuf, scl, ccomb, pbuf, bars, total;
 };
 // The ring also holds, before any row arrives, the centroid slice (up to ring / 512 rows of
 // fp32 centroids per chunk) and the cut cluster's keys; after the last row, the warp partials.
@@ -531,6 +529,10 @@ __host__ __device__ inline Layout make_layout(int G, int S, int C, int RB, int p
     L.scl = take(4u * ((kWarps + S) * G + 2 * G));
     L.ccomb = take(4u * S * G * kCombStride);
     L.pbuf = take(2u * kWarps * 256);
+    // the warps' candidate lists (walk keys) live in pbuf, which only the attention uses, when
+    // they fit (C <= 512)
+    const uint32_t nlist = 256u * (uint32_t)((C + 255) / 256);
+    L.clist = 8u * nlist <= 2u * kWarps * 256 ? L.pbuf : take(8u * nlist);
     L.bars = take(8u * 4);
     L.total = p;
     return L;
@@ -566,6 +568,7 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     int32_t* const s_off = (int32_t*)(base + Ly.off);
     int32_t* const s_spre = (int32_t*)(base + Ly.spre);
     int32_t* const s_cand = (int32_t*)(base + Ly.cand);
+    uint64_t* const s_clist = (uint64_t*)(base + Ly.clist);  // candidates' walk keys (warp lists)
     uint8_t* const s_bkt = base + Ly.bkt;  // every cluster's score bucket
     int32_t* const s_hist = (int32_t*)(base + Ly.hist);
     int32_t* const s_hcnt = (int32_t*)(base + Ly.hcnt);
@@ -602,11 +605,10 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     pdl_launch_dependents();
     if (tid == 0) {
         mbar_init(cbar, 1);
-        mbar_init(fbar, kWarps);
+        mbar_init(fbar, 1);
         mbar_init(rbar, kWarps);
         mbar_init(rbar + 1, kWarps);
         fence_mbar_init();
-        s_wbuf[kWCnt] = 0;
         s_wbuf[kWCopy] = 0;
         s_wbuf[kWBad] = 0;
     }
@@ -659,18 +661,6 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
             else mbar_arrive(bar);
         }
         __syncwarp();
-    };
-    // The cut cluster's rows [row0, row0 + w), w <= kNT, into ring rows 0.. (thread t copies
-    // row t). The fence orders this CTA's earlier shared-memory accesses of the ring before
-    // the copies' writes.
-    auto copy_cut_rows = [&](int32_t row0, int32_t w) {
-        fence_proxy_async();
-        warp_arrive(fbar, tid < w ? 2u * kD * 2u : 0u);
-        if (tid < w) {
-            const int64_t row = kp_base + row0 + tid;
-            bulk_row(ringK + (uint32_t)tid * kPitch, a.kp + row * kD, kD * 2, smem_u32(fbar));
-            bulk_row(ringV + (uint32_t)tid * kPitch, a.vp + row * kD, kD * 2, smem_u32(fbar));
-        }
     };
     // The slice's scores go to this CTA's own shared memory, with the slice's smallest and
     // largest order keys (over the clusters with tokens; over every cluster in the mixed-
@@ -768,8 +758,6 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         const float t = (sc + 0.0f - smin) * inv;
         return (int)fminf(fmaxf(t, 0.f), 255.f);
     };
-    int32_t cut_c = -1, w_cut = 0;  // w_cut: tokens of bucket b* ranked before the cut
-    uint64_t kcut = 0;
     // mixed precision: the walk key of rank n_near - 1 separates near from far clusters
     const bool mid_near = kMixed && a.n_near > 0 && a.n_near < C;
     if (has_cut || mid_near) {
@@ -798,57 +786,22 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         // every warp finds the cut's bucket itself (no extra block barrier)
         bstar = cut_bucket_warp(s_hist, R, &w_above);
         // When b* holds a single cluster with tokens, that cluster is the cut: CTA S-1, which
-        // fills the partial tokens, starts copying its K and V rows once the candidates below
-        // are listed.
+        // fills the partial tokens, starts the bulk copies of its K and V rows (plain 256-byte
+        // rows) now, while the whole clusters are still being ranked.
         if ((int)rank == S - 1 && S > 1 && s_hcnt[bstar] == 1) {
             for (int c = tid; c < C; c += kNT) {
                 const int32_t w = size_of(c);
                 if (w > 0 && w <= RB && w <= kNT && s_bkt[c] == bstar) {
-                    s_wbuf[kWCopyC] = c;
+                    fence_proxy_async();  // the ring's centroid reads come before the copies
+                    const int64_t row = kp_base + s_off[c];
+                    const uint32_t bytes = (uint32_t)w * kD * 2;
+                    mbar_arrive_expect_tx(fbar, 2 * bytes);
+                    bulk_load(base + Ly.ring, a.kp + row * kD, bytes, fbar);
+                    bulk_load(base + Ly.ring + (size_t)RB * kPitch, a.vp + row * kD, bytes, fbar);
                     s_wbuf[kWCopy] = 1;
                 }
             }
         }
-        // the clusters of bucket b* (any order)
-        for (int c0 = 0; c0 < C; c0 += kNT) {
-            const int c = c0 + tid;
-            const bool in_b = c < C && size_of(c) > 0 && s_bkt[c] == bstar;
-            const uint32_t bal = __ballot_sync(0xffffffffu, in_b);
-            int32_t pos0 = 0;
-            if (lane == 0 && bal) pos0 = atomicAdd(&s_wbuf[kWCnt], __popc(bal));
-            pos0 = __shfl_sync(0xffffffffu, pos0, 0);
-            if (in_b) s_cand[pos0 + __popc(bal & ((1u << lane) - 1u))] = c;
-        }
-        __syncthreads();
-        if (s_wbuf[kWCopy] != 0) {
-            const int c = s_wbuf[kWCopyC];
-            copy_cut_rows(s_off[c], size_of(c));
-        }
-        const int32_t n_b = s_wbuf[kWCnt];
-        // exact rank of each candidate among them: 8 threads per candidate
-        for (int i0 = 0; i0 < n_b; i0 += kNT / 8) {
-            const int i = i0 + (tid >> 3), sub = tid & 7;
-            const int ci = i < n_b ? s_cand[i] : 0;
-            const uint64_t ki = i < n_b ? walk_key(s_score[ci], ci) : ~0ull;
-            int32_t pre = 0;
-            for (int j = sub; j < n_b; j += 8) {
-                const int cj = s_cand[j];
-                if (walk_key(s_score[cj], cj) > ki) pre += size_of(cj);
-            }
-#pragma unroll
-            for (int o = 4; o > 0; o >>= 1) pre += __shfl_xor_sync(0xffffffffu, pre, o);
-            if (i < n_b && sub == 0) {
-                const int32_t before = w_above + pre;
-                if (before <= R && R < before + size_of(ci)) {  // the cut (exactly one)
-                    s_wbuf[kWCut] = ci;
-                    s_wbuf[kWPre] = pre;
-                }
-            }
-        }
-        __syncthreads();
-        cut_c = s_wbuf[kWCut];
-        w_cut = s_wbuf[kWPre];
-        kcut = walk_key(s_score[cut_c], cut_c);
     }
     // near(c): walk rank < n_near, i.e. walk key >= the key of rank n_near - 1. The count
     // histogram over the same buckets gives the bucket of that rank; its clusters are ranked
@@ -892,27 +845,84 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         if (a.n_near <= 0) return true;
         return walk_key(s_score[c], c) < k_near;
     };
-    // whole clusters: every cluster without a cut; else buckets above b*, and the clusters of
-    // b* ranked before the cut. Their rows are laid out in cluster-index order. One block scan
-    // (a contiguous run of clusters per thread) of their sizes and counts gives the compact
-    // list of the whole clusters: wl_pre[k] = the selection position of the k-th one's first
-    // row, wl_off[k] = its first store row (kFarBit set when it is attended from the fp8 copy).
-    auto whole_size = [&](int c) -> int32_t {
-        const int32_t w = size_of(c);
-        if (w == 0 || !has_cut) return w;
-        const int bk = s_bkt[c];
-        return (bk > bstar || (bk == bstar && walk_key(s_score[c], c) > kcut)) ? w : 0;
-    };
+    // Whole clusters, laid out in walk order. With a cut, the candidates are the clusters with
+    // tokens in buckets >= b* (a dozen or two): each warp compacts the ones it visits into its
+    // own list, and 8 threads per candidate count the candidates before it in walk order and
+    // their tokens. A candidate whose prefix plus size fits R is whole at that rank; the one
+    // whose prefix fits and whose prefix plus size does not is the cut (its rank is the number
+    // of whole clusters). Without a cut every cluster with tokens is whole; they are listed in
+    // cluster-index order by one block scan. wl_pre[k] = the selection position (past the
+    // sinks and pending rows) of the k-th whole cluster's first row, wl_off[k] = its first
+    // store row (kFarBit set when it is attended from the fp8 copy).
     int32_t* const wl_pre = s_spre;  // [n_whole + 1]
     int32_t* const wl_off = s_cand;  // [n_whole]
     int32_t n_whole;
-    {
+    int32_t cut_c = -1, W_cut = 0;
+    if (has_cut) {
+        const int cap = 32 * ((C + kNT - 1) / kNT);  // one list of cap entries per warp
+        int32_t n_mine = 0;
+        for (int c0 = 0; c0 < C; c0 += kNT) {  // CTA-uniform trip count
+            const int c = c0 + tid;
+            const bool cand = c < C && size_of(c) > 0 && s_bkt[c] >= bstar;
+            const uint32_t bal = __ballot_sync(0xffffffffu, cand);
+            if (cand) s_clist[warp * cap + n_mine + __popc(bal & ((1u << lane) - 1u))] = walk_key(s_score[c], c);
+            n_mine += __popc(bal);
+        }
+        if (lane == 0) s_wbuf[kWList + warp] = n_mine;
+        __syncthreads();
+        int32_t pref[kWarps + 1];  // list starts in the flat candidate order
+        pref[0] = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) pref[w + 1] = pref[w] + s_wbuf[kWList + w];
+        const int32_t n_cand = pref[kWarps];
+        auto slot_of = [&](int f) {  // flat candidate index -> slot in the warp lists
+            int slot = f;
+#pragma unroll
+            for (int v = 1; v < kWarps; ++v)
+                if (f >= pref[v]) slot = f - pref[v] + v * cap;
+            return slot;
+        };
+        for (int i0 = 0; i0 < n_cand; i0 += kNT / 8) {  // CTA-uniform trip count
+            const int i = i0 + (tid >> 3), sub = tid & 7;
+            const uint64_t ki = i < n_cand ? s_clist[slot_of(i)] : ~0ull;
+            const int ci = (int)(0xFFFFFFFFu - (uint32_t)(ki & 0xFFFFFFFFull));
+            int32_t rk = 0, pre = 0;
+            for (int j = sub; j < n_cand; j += 8) {
+                const uint64_t kj = s_clist[slot_of(j)];
+                if (kj > ki) {
+                    ++rk;
+                    pre += size_of((int)(0xFFFFFFFFu - (uint32_t)(kj & 0xFFFFFFFFull)));
+                }
+            }
+#pragma unroll
+            for (int o = 4; o > 0; o >>= 1) {
+                rk += __shfl_xor_sync(0xffffffffu, rk, o);
+                pre += __shfl_xor_sync(0xffffffffu, pre, o);
+            }
+            if (i < n_cand && sub == 0) {
+                const int c = ci;
+                if (pre + size_of(c) <= R) {  // whole
+                    wl_pre[rk] = pre;
+                    wl_off[rk] = s_off[c] | ((kMixed && is_far(c)) ? kFarBit : 0);
+                } else if (pre <= R) {  // the cut
+                    s_wbuf[kWCut] = c;
+                    s_wbuf[kWPre] = pre;
+                    s_wbuf[kWRank] = rk;
+                }
+            }
+        }
+        __syncthreads();
+        cut_c = s_wbuf[kWCut];
+        W_cut = s_wbuf[kWPre];
+        n_whole = s_wbuf[kWRank];
+        if (tid == 0) wl_pre[n_whole] = W_cut;
+    } else {
         const int per = (C + kNT - 1) / kNT;
         const int c0 = tid * per;
         int32_t lsz = 0, lcnt = 0;
         for (int j = 0; j < per; ++j)
             if (c0 + j < C) {
-                const int32_t w = whole_size(c0 + j);
+                const int32_t w = size_of(c0 + j);
                 lsz += w;
                 lcnt += w > 0 ? 1 : 0;
             }
@@ -921,7 +931,7 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         for (int j = 0; j < per; ++j)
             if (c0 + j < C) {
                 const int c = c0 + j;
-                const int32_t w = whole_size(c);
+                const int32_t w = size_of(c);
                 if (w > 0) {
                     wl_pre[k] = run;
                     wl_off[k] = s_off[c] | ((kMixed && is_far(c)) ? kFarBit : 0);
@@ -935,7 +945,7 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     __syncthreads();
 
     // Index-space quantities are below the budget (int32).
-    const int32_t W = has_cut ? w_above + w_cut : m_tot;  // tokens in whole clusters
+    const int32_t W = has_cut ? W_cut : m_tot;  // tokens in whole clusters
     const int32_t r_part = has_cut ? R - W : 0;
     const int32_t csz = has_cut ? size_of(cut_c) : 0;
     const int32_t crow = has_cut ? s_off[cut_c] : 0;
@@ -1060,9 +1070,16 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     };
 
     if (resident) {
-        // ---- the cut cluster in shared memory (ring rows 0..csz-1): one bulk copy per row,
-        // issued during the selection when the histogram isolated the cut, else now
-        if (s_wbuf[kWCopy] == 0) copy_cut_rows(crow, csz);
+        // ---- the cut cluster in shared memory as plain 256-byte rows (K at the ring's start,
+        // V at the V half): two bulk copies, issued during the selection when the histogram
+        // isolated the cut, else now
+        if (tid == 0 && s_wbuf[kWCopy] == 0) {
+            fence_proxy_async();  // the ring's earlier shared-memory reads come before the copies
+            const uint32_t bytes = (uint32_t)csz * kD * 2;
+            mbar_arrive_expect_tx(fbar, 2 * bytes);
+            bulk_load(base + Ly.ring, a.kp + (kp_base + crow) * kD, bytes, fbar);
+            bulk_load(base + Ly.ring + (size_t)RB * kPitch, a.vp + (kp_base + crow) * kD, bytes, fbar);
+        }
         const bool got = __syncthreads_and(mbar_wait(fbar, 0, a.err) ? 1 : 0) != 0;
         if (!got) s_wbuf[kWBad] = 1;
         // qbar . k, a half-warp per row (16-byte reads covering one 256-byte row), 8 rows
@@ -1077,7 +1094,7 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
                 const int e = r0 + hw + k * (kNT / 16);
                 sk[k] = 0.f;
                 if (got && e < csz) {
-                    const uint4 w = lds_v4(ringK + (uint32_t)e * kPitch + l16 * 16);
+                    const uint4 w = lds_v4(ringK + (uint32_t)e * 256u + l16 * 16);
                     float t = qa.x * bf16_lo(w.x);
                     t = fmaf(qa.y, bf16_hi(w.x), t);
                     t = fmaf(qa.z, bf16_lo(w.y), t);
@@ -1139,7 +1156,7 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
 #pragma unroll
                     for (int part = 0; part < 2; ++part) {
                         uint2* row = reinterpret_cast<uint2*>(base + Ly.ring + (size_t)part * RB * kPitch +
-                                                              (size_t)er * kPitch);
+                                                              (size_t)er * 256);
                         float sc;
                         const uint2 v = fp8_row_values(row[lane], &sc);
                         __syncwarp();
@@ -1203,7 +1220,9 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     const float qscale = kLog2e * rsqrtf((float)kD);
     // rows: ring row of tile row t is pos[t] (pos != nullptr) or p0 + t
     auto attend = [&](int p0, int n, const int32_t* pos) {
-        auto addr = [&](uint32_t rbase, int p, int j) { return rbase + (uint32_t)p * kPitch + ((uint32_t)j << 4); };
+        // the resident cut cluster (pos != nullptr) sits in plain 256-byte rows
+        const uint32_t pitch = pos != nullptr ? 256u : (uint32_t)kPitch;
+        auto addr = [&](uint32_t rbase, int p, int j) { return rbase + (uint32_t)p * pitch + ((uint32_t)j << 4); };
         const int n_tiles = (n + 15) >> 4;
         for (int tile = warp; tile < n_tiles; tile += kWarps) {
             const int r0 = tile * 16;

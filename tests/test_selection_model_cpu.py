@@ -2,20 +2,20 @@
 Python, agrees with the oracle's sorted walk (ClusterKV explainer, section 3.3) on
 adversarial cases.
 
-The kernel does not sort the clusters. Each CTA:
+The kernel does not sort all the clusters. Each CTA:
 1. maps the fp32 scores monotonically onto 256 linear buckets between the smallest and the
    largest score of the clusters with tokens;
 2. builds a histogram of cluster sizes per bucket and finds the bucket b* holding the cut
    (the first cluster, in descending (score, -index) order, whose inclusive size exceeds the
-   remaining budget) and the tokens in the buckets above it;
-3. ranks exactly, by the key (orderable score, -index), only the clusters of bucket b*; the
-   orderable score maps -0 and +0 to one key, so they tie like equal doubles. The cut is the
-   one whose prefix (tokens above b* plus the b* clusters before it) fits while its size
-   does not; the whole clusters are every cluster of a higher bucket and the b* clusters
-   ranked before the cut;
-4. lays the whole clusters out in cluster-index order: spre is the exclusive prefix of the
-   whole sizes, and selection position x maps to the last cluster c with spre[c] <= x, row
-   offsets[c] + x - spre[c] (a binary search).
+   remaining budget);
+3. compacts the clusters with tokens in buckets >= b* (the candidates) and ranks each one
+   among them by the key (orderable score, -index), with the tokens of the candidates before
+   it (its prefix); the orderable score maps -0 and +0 to one key, so they tie like equal
+   doubles. A candidate whose prefix plus size fits is whole at its rank; the one whose
+   prefix fits and whose prefix plus size does not is the cut;
+4. lays the whole clusters out in that rank (walk) order: selection position x maps to the
+   whole cluster k with the largest prefix <= x, row offsets[c_k] + x - prefix_k (a binary
+   search).
 
 This model is checked against the oracle's `select` on stores whose scores are exactly the
 chosen fp32 values (centroid c = s_c * e_0, query e_0): many ties, all-equal scores, a tiny
@@ -36,7 +36,8 @@ def _orderable(x: np.float32) -> int:
 
 
 def bucket_cut(sc: np.ndarray, sz: np.ndarray, R: int):
-    """Whole clusters (set), cut cluster and W (tokens in whole clusters), or None if all fit."""
+    """Whole clusters in walk order (list of (cluster, prefix)), the cut cluster and W (tokens
+    in whole clusters), or None if all fit."""
     sc = sc.astype(np.float32)
     if sz.sum() <= R:
         return None
@@ -55,37 +56,37 @@ def bucket_cut(sc: np.ndarray, sz: np.ndarray, R: int):
             bstar = d
             break
         above += hist[d]
-    cand = [c for c in range(len(sc)) if sz[c] > 0 and b[c] == bstar]
+    cand = [c for c in range(len(sc)) if sz[c] > 0 and b[c] >= bstar]
     key = {c: (_orderable(sc[c]) << 32) | (0xFFFFFFFF - c) for c in range(len(sc))}
-    cuts = []
+    whole, cuts = {}, []
     for c in cand:
-        pre = sum(int(sz[j]) for j in cand if key[j] > key[c])
-        if above + pre <= R < above + pre + sz[c]:
-            cuts.append((c, pre))
+        before = [j for j in cand if key[j] > key[c]]
+        rank, pre = len(before), sum(int(sz[j]) for j in before)
+        if pre + sz[c] <= R:
+            whole[rank] = (c, pre)
+        elif pre <= R:
+            cuts.append((c, pre, rank))
     assert len(cuts) == 1
-    cut, pre_cut = cuts[0]
-    whole = {c for c in range(len(sc))
-             if sz[c] > 0 and (b[c] > bstar or (b[c] == bstar and key[c] > key[cut]))}
-    return whole, cut, above + pre_cut
+    cut, pre_cut, rank_cut = cuts[0]
+    assert sorted(whole) == list(range(rank_cut))  # the whole clusters take ranks 0 .. cut - 1
+    return [whole[k] for k in range(rank_cut)], cut, pre_cut
 
 
-def layout_rows(offs: np.ndarray, whole: set, W: int) -> list:
-    """Store rows of selection positions 0..W-1 of the whole clusters (cluster-index order)."""
-    C = len(offs) - 1
-    wsz = [int(offs[c + 1] - offs[c]) if c in whole else 0 for c in range(C)]
-    spre = np.concatenate([[0], np.cumsum(wsz)]).astype(np.int64)
-    assert spre[C] == W
+def layout_rows(offs: np.ndarray, whole: list, W: int) -> list:
+    """Store rows of selection positions 0..W-1 of the whole clusters (walk order)."""
+    pre = [p for _, p in whole] + [W]
     rows = []
     for x in range(W):
-        k0, khi = 0, C - 1  # last cluster with spre[k] <= x
+        k0, khi = 0, len(whole) - 1  # the last whole cluster with prefix <= x
         while k0 < khi:
             mid = (k0 + khi + 1) >> 1
-            if spre[mid] <= x:
+            if pre[mid] <= x:
                 k0 = mid
             else:
                 khi = mid - 1
-        assert k0 in whole and spre[k0] <= x < spre[k0] + wsz[k0]
-        rows.append(int(offs[k0] + x - spre[k0]))
+        c = whole[k0][0]
+        assert pre[k0] <= x < pre[k0 + 1] and pre[k0 + 1] - pre[k0] == offs[c + 1] - offs[c]
+        rows.append(int(offs[c] + x - pre[k0]))
     return rows
 
 
@@ -130,8 +131,8 @@ def test_bucket_histogram_cut_equals_the_sorted_walk():
         assert cut == sel.cut, (trial, cut, sel.cut)
         assert R - W == sel.r, (trial, R - W, sel.r)
         taken = {int(c) for c in np.searchsorted(st.offsets, sel.rows[sel.rows >= 0], side="right") - 1}
-        assert whole == taken - {cut}, trial
-        # the whole clusters' rows, laid out by cluster index, are the oracle's whole rows
+        assert {c for c, _ in whole} == taken - {cut}, trial
+        # the whole clusters' rows, laid out in walk order, are the oracle's whole rows
         rows = layout_rows(st.offsets, whole, W)
         assert len(set(rows)) == W
         want = {int(r) for r in sel.rows[sel.rows >= 0]
