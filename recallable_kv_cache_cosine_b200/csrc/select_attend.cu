@@ -113,6 +113,14 @@ CKV_DEV void bulk_row(uint32_t dst, const void* src, uint32_t bytes, uint32_t ba
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
+CKV_DEV void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// Arrives on the mbarrier once every cp.async this thread issued so far has completed (the
+// barrier's expected count includes this arrival).
+CKV_DEV void cp_async_mbar_arrive(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 CKV_DEV void sts_v4(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
                  "r"(v.w)
@@ -606,8 +614,8 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     if (tid == 0) {
         mbar_init(cbar, 1);
         mbar_init(fbar, 1);
-        mbar_init(rbar, kWarps);
-        mbar_init(rbar + 1, kWarps);
+        mbar_init(rbar, kWarps + kNT);  // a byte-count arrival per warp, a cp.async one per thread
+        mbar_init(rbar + 1, kWarps + kNT);
         fence_mbar_init();
         s_wbuf[kWCopy] = 0;
         s_wbuf[kWBad] = 0;
@@ -1045,10 +1053,13 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
             if (kMixed && cut_far) r |= kFarBit;
         }
         const bool far = kMixed && r >= 0 && (r & kFarBit) != 0;
-        warp_arrive(rbar + (ch & 1), idx >= c1 ? 0u : (far ? 2u * kD : 2u * kD * 2u));
-        if (idx >= c1) return;
+        // bulk-copied bytes: the K row (bf16) or both rows' codes (fp8); a bf16 V row comes by
+        // cp.async, tracked by this thread's cp.async arrival below
+        warp_arrive(rbar + (ch & 1), idx >= c1 ? 0u : (far ? 2u * kD : kD * 2u));
         const uint32_t dk = ringK + (uint32_t)p * kPitch, dv = ringV + (uint32_t)p * kPitch;
-        if (far) {
+        if (idx >= c1) {
+            // no row
+        } else if (far) {
             const int64_t row = kp_base + (r & ~kFarBit);
             bulk_row(dk + 128u, a.kp8 + row * kD, kD, bar);
             bulk_row(dv + 128u, a.vp8 + row * kD, kD, bar);
@@ -1057,13 +1068,18 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         } else {
             const uint16_t* sk = r >= 0 ? a.kp + (kp_base + r) * kD : a.spk + (sp_base + (-1 - r)) * kD;
             const uint16_t* sv = r >= 0 ? a.vp + (kp_base + r) * kD : a.spv + (sp_base + (-1 - r)) * kD;
+            // two copy engines in parallel: the K row by the bulk-copy unit, the V row by
+            // cp.async through the load/store path
             bulk_row(dk, sk, kD * 2, bar);
-            bulk_row(dv, sv, kD * 2, bar);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) cp_async16(dv + (uint32_t)j * 16u, sv + j * 8);
             if (kMixed) {
                 s_rks[p] = 1.f;
                 s_rvs[p] = 1.f;
             }
         }
+        cp_async_mbar_arrive(rbar + (ch & 1));  // every thread, once per chunk
+        if (idx >= c1) return;
         if (kMixed) s_rsrc[p] = r;
         if (sel_out)
             sel_out[idx] = r >= 0 ? ids[r & ~kFarBit] : (idx < a.n_sink ? idx : (int32_t)(a.m + idx));
