@@ -1057,6 +1057,7 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         // cp.async, tracked by this thread's cp.async arrival below
         warp_arrive(rbar + (ch & 1), idx >= c1 ? 0u : (far ? 2u * kD : kD * 2u));
         const uint32_t dk = ringK + (uint32_t)p * kPitch, dv = ringV + (uint32_t)p * kPitch;
+        const uint16_t* sv = nullptr;  // a bf16 V row this thread's position needs
         if (idx >= c1) {
             // no row
         } else if (far) {
@@ -1067,16 +1068,22 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
             s_rvs[p] = a.vs8[row];
         } else {
             const uint16_t* sk = r >= 0 ? a.kp + (kp_base + r) * kD : a.spk + (sp_base + (-1 - r)) * kD;
-            const uint16_t* sv = r >= 0 ? a.vp + (kp_base + r) * kD : a.spv + (sp_base + (-1 - r)) * kD;
-            // two copy engines in parallel: the K row by the bulk-copy unit, the V row by
-            // cp.async through the load/store path
-            bulk_row(dk, sk, kD * 2, bar);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) cp_async16(dv + (uint32_t)j * 16u, sv + j * 8);
+            sv = r >= 0 ? a.vp + (kp_base + r) * kD : a.spv + (sp_base + (-1 - r)) * kD;
+            bulk_row(dk, sk, kD * 2, bar);  // the K row by the bulk-copy unit
             if (kMixed) {
                 s_rks[p] = 1.f;
                 s_rvs[p] = 1.f;
             }
+        }
+        // the warp's V rows by cp.async through the load/store path, in parallel with the bulk
+        // copies: two rows per instruction (lanes 0-15 and 16-31, 16 bytes each, coalesced)
+#pragma unroll 4
+        for (int i = 0; i < 32; i += 2) {  // warp-uniform trip count
+            const int src_lane = i + (lane >> 4);
+            const uint16_t* v = (const uint16_t*)__shfl_sync(0xffffffffu, (unsigned long long)sv, src_lane);
+            const int j = lane & 15;
+            if (v != nullptr)
+                cp_async16(ringV + (uint32_t)(p - lane + src_lane) * kPitch + (uint32_t)j * 16u, v + j * 8);
         }
         cp_async_mbar_arrive(rbar + (ch & 1));  // every thread, once per chunk
         if (idx >= c1) return;
