@@ -16,9 +16,10 @@
 //               C <= 256, consecutive tiles alternate slots (double buffering). With
 //               256 < C <= 512, every tile uses both slots.
 //   warps 0..15 epilogue: warp w reads TMEM lanes 32*(w%4).. (its rows) and column quarter
-//               w/4 of each slot with tcgen05.ld, frees the slot, takes the maximum of each
-//               32 columns with three-input max instructions and the first column holding
-//               it, and merges the four quarters through shared memory. When asked, each
+//               w/4 of each slot with tcgen05.ld, frees the slot, takes each 32-column
+//               block's maximum with three-input max instructions, then the first column
+//               holding the slot's maximum (one search per slot), and merges the four
+//               quarters through shared memory. When asked, each
 //               key's final cluster is also counted into its 1024-key chunk's histogram
 //               (integer atomics), the counting sort's first pass.
 // For C > 512 the host launches once per 512-centroid chunk. Each later launch merges into
@@ -285,6 +286,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->t_empty[h]);
                 const int cbase = p.c_lo + hb * kSlotCols + col0;
+                // the maximum of each 32-column block, then one first-index search in the
+                // first block that holds the slot's maximum (if it beats the running best)
+                float mxb[2] = {-INFINITY, -INFINITY};
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     const int c0 = col0 + cc * 32;
@@ -294,11 +298,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int j = 0; j < 32; ++j)
                             if (c0 + j >= valid) v[cc][j] = -INFINITY;
                     }
-                    const float mx = max32(v[cc]);
-                    if (mx > best) {  // ascending column order: ties keep the lower index
-                        best = mx;
-                        bidx = cbase + cc * 32 + first_index(v[cc], mx);
-                    }
+                    mxb[cc] = max32(v[cc]);
+                }
+                const float mx = fmaxf(mxb[0], mxb[1]);
+                if (mx > best) {  // ascending column order: ties keep the lower index
+                    const bool in1 = !(mxb[0] == mx);
+                    float t[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) t[j] = in1 ? v[1][j] : v[0][j];
+                    best = mx;
+                    bidx = cbase + (in1 ? 32 : 0) + first_index(t, mx);
                 }
             }
             const int buf = (int)(i & 1);
