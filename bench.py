@@ -354,9 +354,9 @@ def extra_measurements(ckv, ctx, q, out, s, L, dev, hbm_gbs, bf16_tflops):
         cs.check_device_error(stream=s)
         t = statistics.median(ts)
         kps = HKV * (n_s - N_SINK) / t
-        roof = min(bf16_tflops * 1e12 / (2 * c_s * 128), hbm_gbs * 1e9 / 512) / ITERS
+        roof, bound = kmeans_roofline(c_s, hbm_gbs, bf16_tflops)
         sweep.append({"n": n_s, "C": c_s, "ms_per_layer": t * 1e3, "keys_per_s": kps,
-                      "roofline_keys_per_s": roof, "frac": kps / roof})
+                      "roofline_keys_per_s": roof, "frac": kps / roof, "bound": bound})
         cs.close()
         del Ks, Vs
     res["prefill_sweep"] = sweep
@@ -451,6 +451,14 @@ def split_pass(ckv, ctx, q, s, L, dev, hbm_gbs):
     res["what"] = ("one layer, 8 KV heads x 32752 keys, C=400; CUDA events around the call; "
                    "the call reads nothing back and can be captured in a CUDA graph")
     return res
+
+
+def kmeans_roofline(C, hbm_gbs, bf16_tflops):
+    """Keys/s bound of cluster_prefill: per key and Lloyd iteration 2*C*128 flops on the tensor
+    cores and two 256-byte key reads (assignment, mean); the smaller rate binds."""
+    tensor = bf16_tflops * 1e12 / (2 * C * 128)
+    hbm = hbm_gbs * 1e9 / 512
+    return min(tensor, hbm) / ITERS, ("tensor" if tensor < hbm else "hbm")
 
 
 def launches_per_prefill(C, iters):
@@ -565,7 +573,7 @@ def run_gpu(args, world, rank, local):
     value = tB / layer_steps * 1e6
     keys = K_steps * L * units * (N_CTX - N_SINK) * world
     keys_per_s = keys / tA
-    keys_roof = min(bf16_tflops * 1e12 / (2 * C_CLUSTERS * 128), hbm_gbs * 1e9 / 512) / ITERS
+    keys_roof, keys_bound = kmeans_roofline(C_CLUSTERS, hbm_gbs, bf16_tflops)
     launch_us = tB / (K_steps * D * L) * 1e6
     m = N_CTX - N_SINK
     bytes_launch = select_attend_bytes(units, BUDGET, C_CLUSTERS, m, G)
@@ -646,7 +654,8 @@ def run_gpu(args, world, rank, local):
                          "us_per_launch": launch_us, "peak_kind": peak_kind},
             "kmeans": {"keys_per_s": keys_per_s, "roofline_keys_per_s": keys_roof,
                        "frac": keys_per_s / keys_roof, "prefill_ms_per_layer": tA / (K_steps * L) * 1e3,
-                       "bound": "min(tensor at 2*C*128 flop/key, HBM at 2 key reads)/iters"},
+                       "bound": keys_bound,
+                       "roofline": "min(tensor at 2*C*128 flop/key, HBM at 2 key reads)/iters"},
             "incremental": {"us_per_token_layer": inc_us,
                             "what": "append_kv + select_and_attend per token, recluster every 320"},
             "sections_ms_per_step": {"prefill": tA / K_steps * 1e3, "decode": tB / K_steps * 1e3,
