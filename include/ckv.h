@@ -85,8 +85,15 @@ CKV_API int ckv_destroy(ckv_ctx* ctx);
 CKV_API const char* ckv_strerror(int code);
 CKV_API const char* ckv_last_error(void);
 
-/* Device bytes held by the context (stores + workspace). */
+/* Device bytes held by the context (stores + workspace + canaries). */
 CKV_API int64_t ckv_device_bytes(const ckv_ctx* ctx);
+
+/* Out-of-bounds write check (a debugging aid, compute-sanitizer being unavailable). Every
+ * device allocation of the context is followed by 256 canary bytes of 0xA5, written when it
+ * is allocated. Waits for the device, copies every canary to the host and sets *n_damaged
+ * to the number of allocations whose canary changed (0 when no kernel wrote past the end of
+ * a buffer). Host-synchronizing. Errors: CKV_EINVAL (null ctx or n_damaged), CKV_ECUDA. */
+CKV_API int ckv_check_canaries(ckv_ctx* ctx, int32_t* n_damaged);
 
 /* Prefill clustering of one layer ([EXPL] 3.2; steps: sinks, seeded init, `iters` Lloyd
  * iterations of cosine assignment on tensor cores and mean update, then the relayout of

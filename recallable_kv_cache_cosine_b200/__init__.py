@@ -54,6 +54,7 @@ SIGNATURES = {
     "ckv_strerror": (C.c_char_p, [C.c_int]),
     "ckv_last_error": (C.c_char_p, []),
     "ckv_device_bytes": (C.c_int64, [P]),
+    "ckv_check_canaries": (C.c_int, [P, P]),
     "cluster_prefill": (C.c_int, [P, I32, P, P, I64, I32, P]),
     "select_and_attend": (C.c_int, [P, I32, P, I32, P, P, P, P]),
     "select_and_attend_per_head": (C.c_int, [P, I32, P, I32, P, P, P, P]),
@@ -258,6 +259,13 @@ class ClusterKV:
 
     def check_device_error(self, stream=None):
         _check(lib().ckv_check_device_error(self._ctx, _stream(stream)), "ckv_check_device_error")
+
+    def damaged_canaries(self) -> int:
+        """Number of device allocations whose trailing canary bytes changed (waits for the
+        device)."""
+        n = C.c_int32(0)
+        _check(lib().ckv_check_canaries(self._ctx, C.byref(n)), "ckv_check_canaries")
+        return int(n.value)
 
     def enable_fp8(self, stream=None):
         """Keep an fp8 (e4m3, per-row scale) copy of every layer's clustered rows."""

@@ -122,13 +122,22 @@ int dev_alloc(T** p, size_t count, Ctx* c) {
         *p = nullptr;
         return CKV_OK;
     }
-    cudaError_t e = cudaMalloc((void**)p, bytes);
+    // the allocation carries kCanaryBytes of a fixed pattern right after its end
+    cudaError_t e = cudaMalloc((void**)p, bytes + kCanaryBytes);
     if (e != cudaSuccess) {
         (void)cudaGetLastError();
         set_error("cudaMalloc of " + std::to_string(bytes) + " bytes failed");
         return CKV_ENOMEM;
     }
-    c->bytes += (int64_t)bytes;
+    uint8_t* canary = reinterpret_cast<uint8_t*>(*p) + bytes;
+    e = cudaMemset(canary, kCanaryByte, kCanaryBytes);
+    if (e != cudaSuccess) {
+        cudaFree(*p);
+        *p = nullptr;
+        return cuda_fail(e, "canary memset");
+    }
+    c->canaries.emplace_back((void*)*p, canary);
+    c->bytes += (int64_t)(bytes + kCanaryBytes);
     return CKV_OK;
 }
 
@@ -406,6 +415,28 @@ int ckv_destroy(ckv_ctx* ctx) {
 }
 
 int64_t ckv_device_bytes(const ckv_ctx* ctx) { return ctx ? C_(ctx)->bytes : 0; }
+
+int ckv_check_canaries(ckv_ctx* ctx, int32_t* n_damaged) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    if (!n_damaged) return einval("null n_damaged");
+    Ctx* c = C_(ctx);
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "check canaries: synchronize");
+    std::vector<uint8_t> host(kCanaryBytes);
+    int32_t bad = 0;
+    for (const auto& pc : c->canaries) {
+        e = cudaMemcpy(host.data(), pc.second, kCanaryBytes, cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return cuda_fail(e, "check canaries: copy");
+        for (size_t i = 0; i < kCanaryBytes; ++i)
+            if (host[i] != kCanaryByte) {
+                ++bad;
+                break;
+            }
+    }
+    *n_damaged = bad;
+    return CKV_OK;
+}
 
 int cluster_prefill(ckv_ctx* ctx, int32_t layer, const void* K, const void* V, int64_t n,
                     int32_t C, void* stream) {
@@ -814,7 +845,14 @@ int ckv_enable_fp8(ckv_ctx* ctx, void* stream) {
         if (!rc) rc = dev_alloc(&vs, rows, c);
         if (rc) {
             for (void* p : {(void*)k8, (void*)v8, (void*)ks, (void*)vs})
-                if (p) cudaFree(p);
+                if (p) {
+                    for (size_t i = 0; i < c->canaries.size(); ++i)
+                        if (c->canaries[i].first == p) {
+                            c->canaries.erase(c->canaries.begin() + (ptrdiff_t)i);
+                            break;
+                        }
+                    cudaFree(p);
+                }
             return rc;
         }
         c->kp8 = k8;

@@ -92,6 +92,9 @@ struct Ctx {
     uint32_t* err = nullptr;  // device error word
     std::vector<LayerState> layers;
     int64_t bytes = 0;
+    // Canary bytes right after the end of every device allocation (kCanaryBytes of
+    // kCanaryByte), checked by ckv_check_canaries: (allocation, canary start).
+    std::vector<std::pair<void*, uint8_t*>> canaries;
 
     int64_t rows_kp(int layer, int u) const { return ((int64_t)layer * units + u) * cap_c; }
     int64_t rows_sp(int layer, int u) const { return ((int64_t)layer * units + u) * sp_rows; }
@@ -107,6 +110,8 @@ void set_error(const std::string& msg);
 int cuda_fail(cudaError_t e, const char* what);
 
 constexpr int kD = 128;       // head dim
+constexpr size_t kCanaryBytes = 256;
+constexpr unsigned char kCanaryByte = 0xA5;
 constexpr int kChunk = 1024;  // keys per counting-sort chunk
 inline int64_t n_chunks(int64_t m) { return (m + kChunk - 1) / kChunk; }
 
