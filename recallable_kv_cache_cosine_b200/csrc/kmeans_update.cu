@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(256) kmeans_count_kernel(const int32_t* assign
 // the keys counted (m, unless the count kernel skipped out-of-range assignments; the mean
 // kernel then never reaches perm entries that the scatter did not write);
 // chunk[u][ch][c] becomes the number of keys of cluster c in chunks before ch.
-__global__ void __launch_bounds__(1024) kmeans_scan_kernel(int32_t* chunk, int32_t nch, int32_t C,
+__global__ void __launch_bounds__(512) kmeans_scan_kernel(int32_t* chunk, int32_t nch, int32_t C,
                                                            int64_t m, int32_t* offsets,
                                                            int64_t off_ustride) {
     pdl_launch_dependents();  // let the next kernel in the stream be scheduled early
@@ -430,7 +430,7 @@ int launch_kmeans_update(const KeysView& k, const int32_t* assign, int64_t assig
                        assign_ustride, k.m, C, nch, chunk_ws, err);
         if (e != cudaSuccess) return cuda_fail(e, "update: count launch");
     }
-    e = launch_pdl(kmeans_scan_kernel, dim3(k.U), dim3(1024), ssmem, s, chunk_ws, nch, C, k.m,
+    e = launch_pdl(kmeans_scan_kernel, dim3(k.U), dim3(512), ssmem, s, chunk_ws, nch, C, k.m,
                    offsets, off_ustride);
     if (e != cudaSuccess) return cuda_fail(e, "update: scan launch");
     if (nch > 0) {
