@@ -621,6 +621,7 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         s_wbuf[kWBad] = 0;
     }
     __syncthreads();
+    cluster_arrive_relaxed();  // this CTA runs: the others may write its shared memory (phase 1)
     if (tid == 0 && nc > 0) {  // the slice's first chunk
         const uint32_t bytes = (uint32_t)min(nc, cch) * kD * 4;
         mbar_arrive_expect_tx(cbar, bytes);
@@ -670,11 +671,13 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         }
         __syncwarp();
     };
-    // The slice's scores go to this CTA's own shared memory, with the slice's smallest and
-    // largest order keys (over the clusters with tokens; over every cluster in the mixed-
-    // precision instantiation, whose rank counts empty clusters too). After one cluster
-    // barrier every CTA reads the other slices from the other CTAs.
+    // The slice's scores are stored into every CTA's shared memory, and so are the slice's
+    // smallest and largest order keys (over the clusters with tokens; over every cluster in
+    // the mixed-precision instantiation, whose rank counts empty clusters too). After one
+    // cluster barrier every CTA holds all C scores. The remote stores wait for the arrival
+    // that every CTA made once it started.
     uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
+    cluster_wait_acquire();
     {
         const float4 qv = reinterpret_cast<const float4*>(s_qbar)[lane];
         // The slice in chunks of at most cch centroids (one chunk unless C / S exceeds the
@@ -701,11 +704,19 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
                     s2 += __shfl_xor_sync(0xffffffffu, s2, o);
                     s3 += __shfl_xor_sync(0xffffffffu, s3, o);
                 }
-                const int j = j0 + lane * kWarps;  // lanes 0..3 store one score each
+                // every lane holds the four sums: lane (k, r) pushes score k into CTA r
+                for (int t = lane; t < 4 * S; t += 32) {  // S <= 16: at most two per lane
+                    const int kk = t / S, r = t % S;
+                    const int jk = j0 + kk * kWarps;
+                    if (jk < n1) {
+                        const float v = kk == 0 ? s0 : (kk == 1 ? s1 : (kk == 2 ? s2 : s3));
+                        st_cluster_f32(map_shared_rank(smem_u32(&s_score[c_begin + done + jk]), (uint32_t)r), v);
+                    }
+                }
+                const int j = j0 + lane * kWarps;  // lanes 0..3 fold one score each into the keys
                 if (lane < 4 && j < n1) {
                     const float v = lane == 0 ? s0 : (lane == 1 ? s1 : (lane == 2 ? s2 : s3));
                     const int c = c_begin + done + j;
-                    s_score[c] = v;
                     if (kMixed || size_of(c) > 0) {
                         const uint32_t key = orderable(v);
                         kmn = min(kmn, key);
@@ -743,18 +754,14 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
             s_wbuf[80] = (int32_t)kmn;  // this CTA's slice
             s_wbuf[81] = (int32_t)kmx;
         }
+        __syncthreads();
+        if (tid < S) {  // this slice's smallest and largest keys into every CTA
+            st_cluster_u32(map_shared_rank(smem_u32(&s_wbuf[96 + rank]), (uint32_t)tid), (uint32_t)s_wbuf[80]);
+            st_cluster_u32(map_shared_rank(smem_u32(&s_wbuf[112 + rank]), (uint32_t)tid), (uint32_t)s_wbuf[81]);
+        }
     }
     cluster_arrive_release();
-    cluster_wait_acquire();  // every slice is written, in every CTA
-    for (int c = tid; c < C; c += kNT) {
-        const int r = (S * (c + 1) - 1) / C;  // the CTA whose slice holds c
-        if (r != (int)rank) s_score[c] = ld_cluster_f32(map_shared_rank(smem_u32(&s_score[c]), (uint32_t)r));
-    }
-    if (tid < S) {
-        s_wbuf[96 + tid] = (int32_t)ld_cluster_u32(map_shared_rank(smem_u32(&s_wbuf[80]), (uint32_t)tid));
-        s_wbuf[112 + tid] = (int32_t)ld_cluster_u32(map_shared_rank(smem_u32(&s_wbuf[81]), (uint32_t)tid));
-    }
-    __syncthreads();
+    cluster_wait_acquire();  // every slice's scores and keys are in every CTA
 
     // ---------------------------------------------------------------- phase 2: selection
     const int32_t m_tot = s_off[C] - s_off[0];
