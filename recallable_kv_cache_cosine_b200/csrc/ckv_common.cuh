@@ -71,6 +71,28 @@ CKV_DEV bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint32_t* err, uint64
 CKV_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
     return mbar_wait_for(bar, parity, err, kWaitNs);
 }
+// The same wait with acquire at cluster scope: for phases completed by other CTAs' st.async.
+CKV_DEV bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+CKV_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t* err) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if ((it & 255u) == 255u && globaltimer() - t0 > kWaitNs) {
+            if (err) atomicOr(err, kErrTimeout);
+            return false;
+        }
+    }
+}
 
 // ------------------------------------------------------------------ TMA
 CKV_DEV void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int32_t x,
@@ -183,26 +205,32 @@ CKV_DEV void cluster_arrive_relaxed() {
 CKV_DEV void cluster_wait_acquire() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-CKV_DEV void cluster_sync() {
-    cluster_arrive_release();
-    cluster_wait_acquire();
-}
 // Address of the same shared variable in CTA `rank` of this cluster.
 CKV_DEV uint32_t map_shared_rank(uint32_t local_addr, uint32_t rank) {
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
     return r;
 }
-CKV_DEV void st_cluster_f32(uint32_t addr, float v) {
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-CKV_DEV void st_cluster_u32(uint32_t addr, uint32_t v) {
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-CKV_DEV void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b),
-                 "r"(c), "r"(d)
+// Asynchronous stores into the shared memory of a CTA of this cluster (cluster addresses from
+// map_shared_rank): each performs complete-tx of its bytes on `mbar`, an mbarrier in that same
+// CTA, whose waiter (mbar_wait_cluster) then sees the stored values.
+CKV_DEV void st_async_f32(uint32_t addr, float v, uint32_t mbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];" ::"r"(addr),
+                 "f"(v), "r"(mbar)
                  : "memory");
+}
+CKV_DEV void st_async_v2_u32(uint32_t addr, uint32_t a, uint32_t b, uint32_t mbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1, %2}, [%3];" ::"r"(
+                     addr),
+                 "r"(a), "r"(b), "r"(mbar)
+                 : "memory");
+}
+CKV_DEV void st_async_v4_u32(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t mbar) {
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+            addr),
+        "r"(a), "r"(b), "r"(c), "r"(d), "r"(mbar)
+        : "memory");
 }
 CKV_DEV void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

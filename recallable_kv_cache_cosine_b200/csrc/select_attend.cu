@@ -79,7 +79,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 // one 16-byte column fall on 8 distinct groups of 4 banks.
 constexpr int kPitch = 2 * kD + 16;
 constexpr int kRowBytes = 2 * kPitch;  // one K row and one V row
-constexpr int kCombStride = 130;       // accumulator[128], max, sum
+constexpr int kCombStride = 132;       // accumulator[128], max, sum, 2 pad (16-byte rows)
 
 // wbuf slots
 constexpr int kWRank = 43;    // the cut's walk rank (the number of whole clusters)
@@ -275,16 +275,6 @@ __device__ __noinline__ int4 block_excl_scan2(int32_t a, int32_t b, int32_t* wsc
     return make_int4(ba + ia - a, bb + ib - b, ta, tb);
 }
 
-CKV_DEV float ld_cluster_f32(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-    return v;
-}
-CKV_DEV uint32_t ld_cluster_u32(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
-}
 
 // Warp 0 of a radix pass: bins hold weights in descending digit order; find the digit whose
 // bin contains the position `need` (0-based, counting weight from the top), i.e. the first
@@ -509,7 +499,7 @@ __host__ __device__ inline uint32_t ring_bytes(int G, int RB) {
     if (k > r) r = k;
     return r;
 }
-__host__ __device__ inline Layout make_layout(int G, int S, int C, int RB, int prow_cap) {
+__host__ __device__ inline Layout make_layout(int G, int S, int C, int RB, int prow_cap, bool mixed) {
     Layout L{};
     uint32_t p = 0;
     auto take = [&](uint32_t bytes) {
@@ -530,9 +520,9 @@ __host__ __device__ inline Layout make_layout(int G, int S, int C, int RB, int p
     L.hnear = take(4u * 256);
     L.rkey = take(4u * (RB + 4));
     L.prow = take(4u * prow_cap);
-    L.rsrc = take(4u * RB);
-    L.rks = take(4u * RB);
-    L.rvs = take(4u * RB);
+    L.rsrc = take(mixed ? 4u * RB : 0u);  // far-row sources and scales: mixed precision only
+    L.rks = take(mixed ? 4u * RB : 0u);
+    L.rvs = take(mixed ? 4u * RB : 0u);
     L.wbuf = take(4u * 128);
     L.scl = take(4u * ((kWarps + S) * G + 2 * G));
     L.ccomb = take(4u * S * G * kCombStride);
@@ -541,7 +531,7 @@ __host__ __device__ inline Layout make_layout(int G, int S, int C, int RB, int p
     // they fit (C <= 512)
     const uint32_t nlist = 256u * (uint32_t)((C + 255) / 256);
     L.clist = 8u * nlist <= 2u * kWarps * 256 ? L.pbuf : take(8u * nlist);
-    L.bars = take(8u * 4);
+    L.bars = take(8u * 6);
     L.total = p;
     return L;
 }
@@ -550,6 +540,7 @@ struct Params {
     int32_t S;         // CTAs per unit (thread-block cluster size)
     int32_t RB;        // ring rows
     int32_t prow_cap;  // partial rows one CTA may own
+    int32_t hold;      // 1: the CTAs of a cluster leave together, when CTA 0 is done
 };
 
 // kPerHead: one selection per query head. The kernel then runs with G = 1 over virtual
@@ -567,7 +558,7 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     const int b = unit / a.Hkv, h = unit % a.Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    const Layout Ly = make_layout(G, S, C, RB, P.prow_cap);
+    const Layout Ly = make_layout(G, S, C, RB, P.prow_cap, kMixed);
     const int cch = (int)(ring_bytes(G, RB) / (kD * 4));  // centroid rows per slice chunk
     uint8_t* const base = smem_raw;
     float* const s_qbar = (float*)(base + Ly.qbar);
@@ -593,6 +584,8 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     uint64_t* const cbar = (uint64_t*)(base + Ly.bars);      // centroid slice
     uint64_t* const fbar = cbar + 1;                         // cut cluster rows (a warp's arrival each)
     uint64_t* const rbar = cbar + 2;                         // [2] ring chunk slots (a warp's arrival each)
+    uint64_t* const xbar = cbar + 4;                         // the other slices' scores and keys
+    uint64_t* const obar = cbar + 5;                         // the other CTAs' partials (CTA 0)
     float* const s_cent = (float*)(base + Ly.ring);          // centroid slice (aliases the ring)
     float* const s_wcomb = (float*)(base + Ly.ring);         // warp partials (after the rows)
     uint32_t* const s_pkey = (uint32_t*)(base + Ly.ring);    // cut keys (before the rows)
@@ -616,12 +609,22 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         mbar_init(fbar, 1);
         mbar_init(rbar, kWarps + kNT);  // a byte-count arrival per warp, a cp.async one per thread
         mbar_init(rbar + 1, kWarps + kNT);
+        mbar_init(xbar, 1);
+        mbar_init(obar, 1);
         fence_mbar_init();
+        // bytes the other CTAs store here: their slices' scores and two keys each; into CTA 0,
+        // their partials
+        const uint32_t bx = 4u * (uint32_t)(C - nc) + 8u * (uint32_t)(S - 1);
+        if (bx) mbar_arrive_expect_tx(xbar, bx);
+        else mbar_arrive(xbar);
+        const uint32_t bo = rank == 0 ? 4u * (uint32_t)((S - 1) * G * kCombStride) : 0u;
+        if (bo) mbar_arrive_expect_tx(obar, bo);
+        else mbar_arrive(obar);
         s_wbuf[kWCopy] = 0;
         s_wbuf[kWBad] = 0;
     }
     __syncthreads();
-    cluster_arrive_relaxed();  // this CTA runs: the others may write its shared memory (phase 1)
+    cluster_arrive_relaxed();  // this CTA runs and its mbarriers are set: others may store here
     if (tid == 0 && nc > 0) {  // the slice's first chunk
         const uint32_t bytes = (uint32_t)min(nc, cch) * kD * 4;
         mbar_arrive_expect_tx(cbar, bytes);
@@ -673,9 +676,10 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     };
     // The slice's scores are stored into every CTA's shared memory, and so are the slice's
     // smallest and largest order keys (over the clusters with tokens; over every cluster in
-    // the mixed-precision instantiation, whose rank counts empty clusters too). After one
-    // cluster barrier every CTA holds all C scores. The remote stores wait for the arrival
-    // that every CTA made once it started.
+    // the mixed-precision instantiation, whose rank counts empty clusters too): asynchronous
+    // stores that count their bytes on the receiver's mbarrier xbar, so that each CTA goes on
+    // once its own copy is complete. The remote stores wait for the arrival every CTA made
+    // once it started.
     uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
     cluster_wait_acquire();
     {
@@ -704,19 +708,11 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
                     s2 += __shfl_xor_sync(0xffffffffu, s2, o);
                     s3 += __shfl_xor_sync(0xffffffffu, s3, o);
                 }
-                // every lane holds the four sums: lane (k, r) pushes score k into CTA r
-                for (int t = lane; t < 4 * S; t += 32) {  // S <= 16: at most two per lane
-                    const int kk = t / S, r = t % S;
-                    const int jk = j0 + kk * kWarps;
-                    if (jk < n1) {
-                        const float v = kk == 0 ? s0 : (kk == 1 ? s1 : (kk == 2 ? s2 : s3));
-                        st_cluster_f32(map_shared_rank(smem_u32(&s_score[c_begin + done + jk]), (uint32_t)r), v);
-                    }
-                }
-                const int j = j0 + lane * kWarps;  // lanes 0..3 fold one score each into the keys
+                const int j = j0 + lane * kWarps;  // lanes 0..3 store one score each
                 if (lane < 4 && j < n1) {
                     const float v = lane == 0 ? s0 : (lane == 1 ? s1 : (lane == 2 ? s2 : s3));
                     const int c = c_begin + done + j;
+                    s_score[c] = v;
                     if (kMixed || size_of(c) > 0) {
                         const uint32_t key = orderable(v);
                         kmn = min(kmn, key);
@@ -756,12 +752,40 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         }
         __syncthreads();
         if (tid < S) {  // this slice's smallest and largest keys into every CTA
-            st_cluster_u32(map_shared_rank(smem_u32(&s_wbuf[96 + rank]), (uint32_t)tid), (uint32_t)s_wbuf[80]);
-            st_cluster_u32(map_shared_rank(smem_u32(&s_wbuf[112 + rank]), (uint32_t)tid), (uint32_t)s_wbuf[81]);
+            int32_t* dst = &s_wbuf[96 + 2 * rank];
+            if (tid == (int)rank) {
+                dst[0] = s_wbuf[80];
+                dst[1] = s_wbuf[81];
+            } else {
+                st_async_v2_u32(map_shared_rank(smem_u32(dst), (uint32_t)tid), (uint32_t)s_wbuf[80],
+                                (uint32_t)s_wbuf[81], map_shared_rank(smem_u32(xbar), (uint32_t)tid));
+            }
+        }
+        // the slice's scores into every other CTA: 16-byte pieces over the 16-byte aligned
+        // interior [a0, a1), single floats at the two ends
+        const int a0 = min((c_begin + 3) & ~3, c_end), a1 = max(c_end & ~3, a0);
+        const int nv = (a1 - a0) >> 2, nhead = a0 - c_begin, per = nv + nhead + (c_end - a1);
+        for (int t = tid; t < (S - 1) * per; t += kNT) {
+            const int k = t / per, i = t - k * per;
+            const uint32_t r = (uint32_t)(k < (int)rank ? k : k + 1);  // every CTA but this one
+            const uint32_t bar = map_shared_rank(smem_u32(xbar), r);
+            if (i < nv) {
+                const int c = a0 + 4 * i;
+                const uint4 v = *reinterpret_cast<const uint4*>(&s_score[c]);
+                st_async_v4_u32(map_shared_rank(smem_u32(&s_score[c]), r), v.x, v.y, v.z, v.w, bar);
+            } else {
+                const int e = i - nv;
+                const int c = e < nhead ? c_begin + e : a1 + (e - nhead);
+                st_async_f32(map_shared_rank(smem_u32(&s_score[c]), r), s_score[c], bar);
+            }
         }
     }
-    cluster_arrive_release();
-    cluster_wait_acquire();  // every slice's scores and keys are in every CTA
+    // every slice's scores and keys are here: warp 0 waits (the others sleep at the block
+    // barrier, leaving the issue slots to a co-resident CTA), then each thread acquires the
+    // completed phase itself
+    if (warp == 0) ok = mbar_wait_cluster(xbar, 0, a.err) && ok;
+    __syncthreads();
+    if (warp != 0) ok = mbar_try_wait_cluster(xbar, 0) && ok;
 
     // ---------------------------------------------------------------- phase 2: selection
     const int32_t m_tot = s_off[C] - s_off[0];
@@ -779,8 +803,8 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         // the smallest and largest score over the slices, then every cluster's bucket
         uint32_t gmn = 0xFFFFFFFFu, gmx = 0u;
         for (int r = 0; r < S; ++r) {
-            gmn = min(gmn, (uint32_t)s_wbuf[96 + r]);
-            gmx = max(gmx, (uint32_t)s_wbuf[112 + r]);
+            gmn = min(gmn, (uint32_t)s_wbuf[96 + 2 * r]);
+            gmx = max(gmx, (uint32_t)s_wbuf[97 + 2 * r]);
         }
         const float mn = from_orderable(gmn), mx = from_orderable(gmx);
         const float range = mx - mn;
@@ -1408,28 +1432,45 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         }
     }
     __syncthreads();
-    // warps -> CTA partial, written into CTA 0's combine buffer
+    // warps -> CTA partial: CTA 0 keeps its own, the others store theirs into CTA 0's combine
+    // buffer (16 bytes per asynchronous store, counted on CTA 0's mbarrier obar)
     {
         const uint32_t dst0 = map_shared_rank(smem_u32(s_ccomb), 0);
-        for (int t = tid; t < G * kCombStride; t += kNT) {
-            const int g = t / kCombStride, e = t % kCombStride;
-            float v;
-            if (e == 128) {
-                v = sums[g];
-            } else if (e == 129) {
-                v = sums[G + g];
-            } else {
-                v = 0.f;
+        const uint32_t bar0 = map_shared_rank(smem_u32(obar), 0);
+        static_assert(kCombStride % 4 == 0, "partials move in 16-byte pieces");
+        for (int t = tid; t < G * (kCombStride / 4); t += kNT) {
+            const int g = t / (kCombStride / 4), e0 = 4 * (t % (kCombStride / 4));
+            float v[4];
 #pragma unroll
-                for (int w = 0; w < kWarps; ++w)
-                    v = fmaf(s_wcomb[(w * G + g) * kCombStride + e], wsc[w * G + g], v);
+            for (int q = 0; q < 4; ++q) {
+                const int e = e0 + q;
+                if (e == 128) {
+                    v[q] = sums[g];
+                } else if (e == 129) {
+                    v[q] = sums[G + g];
+                } else if (e > 129) {
+                    v[q] = 0.f;
+                } else {
+                    float x = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kWarps; ++w)
+                        x = fmaf(s_wcomb[(w * G + g) * kCombStride + e], wsc[w * G + g], x);
+                    v[q] = x;
+                }
             }
-            st_cluster_f32(dst0 + (uint32_t)(((rank * G + g) * kCombStride + e) * 4), v);
+            const int off = (g * kCombStride + e0);  // rank 0's rows come first
+            if (rank == 0)
+                *reinterpret_cast<float4*>(s_ccomb + off) = make_float4(v[0], v[1], v[2], v[3]);
+            else
+                st_async_v4_u32(dst0 + (uint32_t)((rank * G * kCombStride + off) * 4), __float_as_uint(v[0]),
+                                __float_as_uint(v[1]), __float_as_uint(v[2]), __float_as_uint(v[3]), bar0);
         }
     }
-    cluster_arrive_release();
-    cluster_wait_acquire();
     if (rank == 0) {
+        // the others' partials (warp 0 waits, as for the scores); CTA 0's own
+        if (warp == 0) (void)mbar_wait_cluster(obar, 0, a.err);
+        __syncthreads();
+        if (warp != 0) (void)mbar_try_wait_cluster(obar, 0);
         // thread (g, r) in groups of S lanes (S is a power of two <= 16)
         if (tid < S * G) {
             const int active = min(32, S * G - 32 * warp);
@@ -1458,6 +1499,10 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     }
     if (sel_out && rank == (uint32_t)(S - 1)) {
         for (int32_t i = T + tid; i < a.budget; i += kNT) sel_out[i] = -1;
+    }
+    if (P.hold) {  // the cluster's CTAs leave together
+        cluster_arrive_relaxed();
+        cluster_wait_acquire();
     }
 }
 
@@ -1549,7 +1594,7 @@ int plan_for(const DecodeArgs& a, int num_sms, Plan* out) {
         if (S > 1 && (S * G > 64 || (int64_t)U * S > sm_cap)) continue;
         for (int RB = ring_rows(S, a.budget); RB >= 64 && best.p.S == 0; RB -= 16) {
             const int pc = prow_capacity(a.budget, S);
-            const Layout L = make_layout(G, S, a.C, RB, pc);
+            const Layout L = make_layout(G, S, a.C, RB, pc, kMixed);
             if (L.total > 227 * 1024) continue;
             // more CTAs than SMs: the launch is one wave only with two CTAs per SM
             if (S > 1 && (int64_t)U * S > num_sms && L.total > kTwoPerSm) continue;
@@ -1557,7 +1602,12 @@ int plan_for(const DecodeArgs& a, int num_sms, Plan* out) {
             const int rc = max_active_clusters(kern, S, L.total, &smem_set, &nonportable_set, &nclusters);
             if (rc != CKV_OK) return rc;
             if (nclusters <= 0) continue;
-            best.p = Params{S, RB, pc};
+            // Two CTAs per SM: when CTAs leave ahead of their cluster's CTA 0, the next launch
+            // places clusters into the gaps piecemeal, and then one of its clusters can wait for
+            // room until a whole cluster of that launch ends (measured: 18 -> 26 us per launch
+            // at 32 units, back to back). There the CTAs of a cluster leave together.
+            const int32_t hold = (S > 1 && (int64_t)U * S > num_sms) ? 1 : 0;
+            best.p = Params{S, RB, pc, hold};
             best.smem = L.total;
         }
     }
