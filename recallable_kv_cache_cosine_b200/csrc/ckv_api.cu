@@ -714,21 +714,44 @@ int ckv_export_unit(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h,
         {dst->mu, c->mu + c->mu_rows(layer, u) * kD, sizeof(float) * (size_t)L.C * kD},
         {dst->offsets, c->offsets + c->off_base(layer, u), sizeof(int32_t) * (size_t)(L.C + 1)},
         {dst->ids, c->ids + c->rows_kp(layer, u), sizeof(int32_t) * (size_t)L.m},
-        {dst->kp, c->kp + c->rows_kp(layer, u) * kD, (size_t)(2 * L.m * kD)},
-        {dst->vp, c->vp + c->rows_kp(layer, u) * kD, (size_t)(2 * L.m * kD)},
-        {dk, spk_u, (size_t)(2 * ns * kD)},
-        {dv, spv_u, (size_t)(2 * ns * kD)},
-        {dk ? dk + ns * kD : nullptr, spk_u + (ns + L.pstart) * kD, (size_t)(2 * run1 * kD)},
-        {dv ? dv + ns * kD : nullptr, spv_u + (ns + L.pstart) * kD, (size_t)(2 * run1 * kD)},
-        {dk ? dk + (ns + run1) * kD : nullptr, spk_u + ns * kD, (size_t)(2 * run2 * kD)},
-        {dv ? dv + (ns + run1) * kD : nullptr, spv_u + ns * kD, (size_t)(2 * run2 * kD)},
     };
     for (auto& it : items) {
         if (!it.d || it.n == 0) continue;
         cudaError_t e = cudaMemcpyAsync(it.d, it.s, it.n, cudaMemcpyDefault, s);
         if (e != cudaSuccess) return cuda_fail(e, "export: copy");
     }
-    cudaError_t e = cudaStreamSynchronize(s);
+    // K / V rows: stored rows r0 .. r0 + rows - 1, copied to a scratch buffer, put back in
+    // logical chunk order there, then copied out
+    struct Rows { void* d; const uint16_t* s; int64_t rows, r0; } rows[] = {
+        {dst->kp, c->kp + c->rows_kp(layer, u) * kD, L.m, 0},
+        {dst->vp, c->vp + c->rows_kp(layer, u) * kD, L.m, 0},
+        {dk, spk_u, ns, 0},
+        {dv, spv_u, ns, 0},
+        {dk ? dk + ns * kD : nullptr, spk_u + (ns + L.pstart) * kD, run1, ns + L.pstart},
+        {dv ? dv + ns * kD : nullptr, spv_u + (ns + L.pstart) * kD, run1, ns + L.pstart},
+        {dk ? dk + (ns + run1) * kD : nullptr, spk_u + ns * kD, run2, ns},
+        {dv ? dv + (ns + run1) * kD : nullptr, spv_u + ns * kD, run2, ns},
+    };
+    int64_t total = 0;
+    for (auto& g : rows)
+        if (g.d && g.rows > 0) total += g.rows;
+    uint16_t* tmp = nullptr;
+    cudaError_t e = cudaSuccess;
+    if (total > 0) e = cudaMallocAsync((void**)&tmp, (size_t)total * kD * 2, s);
+    if (e != cudaSuccess) return cuda_fail(e, "export: scratch");
+    int64_t at = 0;
+    for (auto& g : rows) {
+        if (!g.d || g.rows <= 0 || rc) continue;
+        uint16_t* t = tmp + at * kD;
+        e = cudaMemcpyAsync(t, g.s, (size_t)g.rows * kD * 2, cudaMemcpyDeviceToDevice, s);
+        if (e == cudaSuccess) rc = launch_swizzle_rows(t, 16, g.r0, g.rows, s);
+        if (e == cudaSuccess && !rc) e = cudaMemcpyAsync(g.d, t, (size_t)g.rows * kD * 2, cudaMemcpyDefault, s);
+        if (e != cudaSuccess) rc = cuda_fail(e, "export: copy rows");
+        at += g.rows;
+    }
+    if (tmp) cudaFreeAsync(tmp, s);
+    e = cudaStreamSynchronize(s);
+    if (rc) return rc;
     return e == cudaSuccess ? CKV_OK : cuda_fail(e, "export: sync");
 }
 
@@ -789,6 +812,17 @@ int ckv_import_unit(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h, int64_t m
         e = cudaMemcpyAsync(it.d, it.s, it.n, cudaMemcpyDefault, s);
         if (e != cudaSuccess) return cuda_fail(e, "import: copy");
     }
+    // the copied K / V rows into stored chunk order, in place
+    const struct { uint16_t* p; int64_t rows, r0; } swz_rows[] = {
+        {c->kp + c->rows_kp(layer, u) * kD, m, 0},
+        {c->vp + c->rows_kp(layer, u) * kD, m, 0},
+        {spk_u, ns, 0},
+        {spv_u, ns, 0},
+        {spk_u + (ns + pstart) * kD, pending, ns + pstart},
+        {spv_u + (ns + pstart) * kD, pending, ns + pstart},
+    };
+    for (const auto& g : swz_rows)
+        if ((rc = launch_swizzle_rows(g.p, 16, g.r0, g.rows, s))) return rc;
     if (c->kp8 && m > 0) {  // the unit's fp8 copy
         const int64_t o = c->rows_kp(layer, u);
         rc = launch_quantize_rows(c->kp + o * kD, c->vp + o * kD, c->kp8 + o * kD, c->vp8 + o * kD,
@@ -886,14 +920,27 @@ int ckv_export_unit_fp8(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h, void*
     const int64_t o = c->rows_kp(layer, b * c->cfg.n_kv_heads + h);
     cudaStream_t s = (cudaStream_t)stream;
     struct Item { void* d; const void* s; size_t n; } items[] = {
-        {k8, c->kp8 + o * kD, (size_t)L.m * kD}, {v8, c->vp8 + o * kD, (size_t)L.m * kD},
         {ks, c->ks8 + o, sizeof(float) * (size_t)L.m}, {vs, c->vs8 + o, sizeof(float) * (size_t)L.m}};
     for (auto& it : items) {
         if (!it.d || it.n == 0) continue;
         cudaError_t e = cudaMemcpyAsync(it.d, it.s, it.n, cudaMemcpyDefault, s);
         if (e != cudaSuccess) return cuda_fail(e, "export fp8: copy");
     }
-    cudaError_t e = cudaStreamSynchronize(s);
+    // the code rows (stored in 8-byte units of swizzled chunk order) through a scratch buffer
+    uint8_t* tmp = nullptr;
+    cudaError_t e = L.m > 0 ? cudaMallocAsync((void**)&tmp, (size_t)L.m * kD, s) : cudaSuccess;
+    if (e != cudaSuccess) return cuda_fail(e, "export fp8: scratch");
+    const struct { void* d; const uint8_t* s; } rows[] = {{k8, c->kp8 + o * kD}, {v8, c->vp8 + o * kD}};
+    for (const auto& g : rows) {
+        if (!g.d || L.m <= 0 || rc) continue;
+        e = cudaMemcpyAsync(tmp, g.s, (size_t)L.m * kD, cudaMemcpyDeviceToDevice, s);
+        if (e == cudaSuccess) rc = launch_swizzle_rows(tmp, 8, 0, L.m, s);
+        if (e == cudaSuccess && !rc) e = cudaMemcpyAsync(g.d, tmp, (size_t)L.m * kD, cudaMemcpyDefault, s);
+        if (e != cudaSuccess) rc = cuda_fail(e, "export fp8: copy rows");
+    }
+    if (tmp) cudaFreeAsync(tmp, s);
+    e = cudaStreamSynchronize(s);
+    if (rc) return rc;
     return e == cudaSuccess ? CKV_OK : cuda_fail(e, "export fp8: sync");
 }
 

@@ -237,6 +237,16 @@ CKV_DEV void pdl_launch_dependents() {
 }
 CKV_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// ------------------------------------------------------------------ stored row layout
+// Every stored K/V row (the cluster store, its fp8 copy, the sink and pending rows) keeps its
+// 16-byte chunk c (8 bf16 values; 8-byte units of 8 codes in the fp8 copy) at chunk position
+// c ^ (r & 7), r = the row's index counted from its unit's first row. Any 8 consecutive rows
+// then hold one logical chunk in 8 different bank groups, so a run of rows copied into shared
+// memory as it is can be read by matrix loads without bank conflicts.
+CKV_DEV int swz(int64_t r, int c) { return c ^ (int)(r & 7); }
+// Element offset of logical element d (0..127) of bf16 row r inside the stored row.
+CKV_DEV int swz_elem(int64_t r, int d) { return (swz(r, d >> 3) << 3) | (d & 7); }
+
 // ------------------------------------------------------------------ misc
 CKV_DEV float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 CKV_DEV float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }

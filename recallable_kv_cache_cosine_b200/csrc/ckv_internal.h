@@ -232,6 +232,10 @@ int launch_quantize_rows(const uint16_t* kp, const uint16_t* vp, uint8_t* kp8, u
                          float* ks, float* vs, int64_t ustride, int64_t r0, int64_t nrows,
                          int32_t U, cudaStream_t s);
 
+// Rows [0, n) at `rows` are stored rows r0 .. r0 + n - 1 of a unit (16 units of unit_bytes
+// each: 16 for bf16 rows, 8 for fp8 rows): swaps their order between logical and stored.
+int launch_swizzle_rows(void* rows, int32_t unit_bytes, int64_t r0, int64_t n, cudaStream_t s);
+
 // One bounded mbarrier wait that nothing completes, with the given limit (test hook).
 int launch_expire_wait(uint32_t* err, uint64_t limit_ns, uint32_t* waited_ns, cudaStream_t s);
 

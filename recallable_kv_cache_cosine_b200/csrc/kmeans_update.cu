@@ -336,8 +336,8 @@ __global__ void __launch_bounds__(kMeanThreads) kmeans_mean_kernel(KeysView k, c
         if (relay) {  // V rows and token ids while the key rows arrive
             for (int i = tid; i < n * 16; i += kMeanThreads) {
                 const int r = i >> 4, ch = i & 15;
-                const int64_t dst = (int64_t)u * rl.ustride_rows + j0 + r;
-                reinterpret_cast<uint4*>(rl.vp + dst * kD)[ch] =
+                const int64_t dst = (int64_t)u * rl.ustride_rows + j0 + r;  // stored row j0 + r
+                reinterpret_cast<uint4*>(rl.vp + dst * kD)[swz(j0 + r, ch)] =
                     reinterpret_cast<const uint4*>(vals + (int64_t)sidx[r] * kD)[ch];
             }
             for (int r = tid; r < n; r += kMeanThreads)
@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(kMeanThreads) kmeans_mean_kernel(KeysView k, c
             for (int i = tid; i < n * 16; i += kMeanThreads) {
                 const int rr = i >> 4, ch = i & 15;
                 const int64_t dst = (int64_t)u * rl.ustride_rows + j0 + rr;
-                reinterpret_cast<uint4*>(rl.kp + dst * kD)[ch] =
+                reinterpret_cast<uint4*>(rl.kp + dst * kD)[swz(j0 + rr, ch)] =
                     reinterpret_cast<const uint4*>(srow + rr * kD)[ch];
             }
         }
@@ -389,9 +389,10 @@ __global__ void copy_sinks_kernel(const uint16_t* K, const uint16_t* V, int64_t 
     const uint4* vs = reinterpret_cast<const uint4*>(V + (int64_t)u * n * kD);
     uint4* kd = reinterpret_cast<uint4*>(spk + (int64_t)u * sp_ustride * kD);
     uint4* vd = reinterpret_cast<uint4*>(spv + (int64_t)u * sp_ustride * kD);
-    for (int64_t i = threadIdx.x; i < words; i += blockDim.x) {
-        kd[i] = ks[i];
-        vd[i] = vs[i];
+    for (int64_t i = threadIdx.x; i < words; i += blockDim.x) {  // stored row i / 16
+        const int64_t o = (i & ~15ll) | swz(i >> 4, (int)(i & 15));
+        kd[o] = ks[i];
+        vd[o] = vs[i];
     }
 }
 

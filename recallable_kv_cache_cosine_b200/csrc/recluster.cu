@@ -41,9 +41,10 @@ __global__ void __launch_bounds__(kRT) recluster_kernel(const ReclusterArgs a) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = kRT / 32;
     const uint16_t* wk = a.spk + ((int64_t)u * a.sp_ustride + a.win_row0) * kD;
     const uint16_t* wv = a.spv + ((int64_t)u * a.sp_ustride + a.win_row0) * kD;
-    // window keys into shared memory
+    // window keys into shared memory, in logical order (stored row win_row0 + i / 16)
     for (int i = tid; i < W * kD / 8; i += kRT)
-        reinterpret_cast<uint4*>(skey)[i] = reinterpret_cast<const uint4*>(wk)[i];
+        reinterpret_cast<uint4*>(skey)[i] =
+            reinterpret_cast<const uint4*>(wk)[(i & ~15) | swz(a.win_row0 + (i >> 4), i & 15)];
     for (int i = tid; i < W; i += kRT) sarr[i] = i;
     __syncthreads();
     if (tid == 0) {
@@ -145,13 +146,14 @@ __global__ void __launch_bounds__(kRT) recluster_kernel(const ReclusterArgs a) {
 
     // append to the store
     const int64_t row0 = (int64_t)u * a.kp_ustride + a.m_old;
-    for (int t = tid; t < W * (kD / 8); t += kRT) {
+    for (int t = tid; t < W * (kD / 8); t += kRT) {  // stored row m_old + j, logical chunk w
         const int j = t / (kD / 8), w = t % (kD / 8);
         const int src = sperm[j];
-        reinterpret_cast<uint4*>(a.kp + (row0 + j) * kD)[w] =
+        const int o = swz(a.m_old + j, w);
+        reinterpret_cast<uint4*>(a.kp + (row0 + j) * kD)[o] =
             reinterpret_cast<const uint4*>(skey + src * kD)[w];
-        reinterpret_cast<uint4*>(a.vp + (row0 + j) * kD)[w] =
-            reinterpret_cast<const uint4*>(wv + (int64_t)src * kD)[w];
+        reinterpret_cast<uint4*>(a.vp + (row0 + j) * kD)[o] =
+            reinterpret_cast<const uint4*>(wv + (int64_t)src * kD)[swz(a.win_row0 + src, w)];
     }
     for (int j = tid; j < W; j += kRT) a.ids[row0 + j] = (int32_t)(a.n_sink + a.m_old + sperm[j]);
     int32_t* off = a.offsets + (int64_t)u * a.off_ustride;
@@ -165,9 +167,9 @@ __global__ void append_kernel(const uint16_t* k, const uint16_t* v, uint16_t* sp
     pdl_launch_dependents();  // let the next kernel in the stream be scheduled early
     pdl_wait();               // the previous kernel's writes are visible from here on
     const int u = blockIdx.x, t = threadIdx.x;  // 16 threads x 16 bytes per row
-    const int64_t dst = ((int64_t)u * sp_ustride + row) * kD;
-    reinterpret_cast<uint4*>(spk + dst)[t] = reinterpret_cast<const uint4*>(k + (int64_t)u * kD)[t];
-    reinterpret_cast<uint4*>(spv + dst)[t] = reinterpret_cast<const uint4*>(v + (int64_t)u * kD)[t];
+    const int64_t dst = ((int64_t)u * sp_ustride + row) * kD;  // stored row `row`
+    reinterpret_cast<uint4*>(spk + dst)[swz(row, t)] = reinterpret_cast<const uint4*>(k + (int64_t)u * kD)[t];
+    reinterpret_cast<uint4*>(spv + dst)[swz(row, t)] = reinterpret_cast<const uint4*>(v + (int64_t)u * kD)[t];
 }
 
 }  // namespace

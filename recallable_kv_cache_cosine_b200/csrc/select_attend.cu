@@ -75,9 +75,11 @@ constexpr int kNT = 256;          // threads per CTA
 constexpr int kWarps = kNT / 32;
 constexpr int kPartCap = 4096;    // cut-cluster tokens ranked in shared memory (outside the ring path)
 constexpr float kLog2e = 1.4426950408889634f;
-// Ring row pitch: a 256-byte bf16 row plus 16 bytes, so that the 8 rows a matrix load reads at
-// one 16-byte column fall on 8 distinct groups of 4 banks.
-constexpr int kPitch = 2 * kD + 16;
+// Ring rows are stored rows copied as they are (256 bytes, chunks in stored order): a run of
+// consecutive store rows lands in consecutive ring rows by one bulk copy, and the chunk key of
+// each ring row (its store row & 7) spreads the 8 rows a matrix load reads at one logical
+// 16-byte column over 8 distinct groups of 4 banks.
+constexpr int kPitch = 2 * kD;
 constexpr int kRowBytes = 2 * kPitch;  // one K row and one V row
 constexpr int kCombStride = 132;       // accumulator[128], max, sum, 2 pad (16-byte rows)
 
@@ -113,14 +115,8 @@ CKV_DEV void bulk_row(uint32_t dst, const void* src, uint32_t bytes, uint32_t ba
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
-CKV_DEV void cp_async16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
 // Arrives on the mbarrier once every cp.async this thread issued so far has completed (the
 // barrier's expected count includes this arrival).
-CKV_DEV void cp_async_mbar_arrive(uint64_t* bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
 CKV_DEV void sts_v4(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
                  "r"(v.w)
@@ -188,13 +184,15 @@ CKV_DEV uint4 lds_v4(uint32_t addr) {
 
 // qbar . k over one 64-dimension half (`half`) of two K rows, with all 16 loads in flight; a
 // negative row index gives 0. Dimensions in ascending order, one fmaf chain per row.
-CKV_DEV void half_row_dot2(const uint16_t* kp, int32_t ia, int32_t ib, int half, const float* qbar,
-                           float* sa, float* sb) {
+CKV_DEV void half_row_dot2(const uint16_t* kp, int32_t row0, int32_t ia, int32_t ib, int half,
+                           const float* qbar, float* sa, float* sb) {
+    // kp[i] is store row row0 + i: logical chunk 8 half + t of it is stored at 8 half + (t ^ key)
     uint4 w[2][8];
+    const int ka = (row0 + ia) & 7, kb = (row0 + ib) & 7;
 #pragma unroll
     for (int t = 0; t < 8; ++t) {
-        w[0][t] = ia >= 0 ? ldg_nc_v4(kp + (int64_t)ia * kD + 64 * half + 8 * t) : make_uint4(0u, 0u, 0u, 0u);
-        w[1][t] = ib >= 0 ? ldg_nc_v4(kp + (int64_t)ib * kD + 64 * half + 8 * t) : make_uint4(0u, 0u, 0u, 0u);
+        w[0][t] = ia >= 0 ? ldg_nc_v4(kp + (int64_t)ia * kD + 64 * half + 8 * (t ^ ka)) : make_uint4(0u, 0u, 0u, 0u);
+        w[1][t] = ib >= 0 ? ldg_nc_v4(kp + (int64_t)ib * kD + 64 * half + 8 * (t ^ kb)) : make_uint4(0u, 0u, 0u, 0u);
     }
     const float4* q4 = reinterpret_cast<const float4*>(qbar + 64 * half);
     float s[2] = {0.f, 0.f};
@@ -375,7 +373,7 @@ __device__ __noinline__ void partial_rows(const PartialArgs& P) {
             const int32_t ia = i0 + (tid >> 1), ib = ia + kNT / 2;
             const int half = tid & 1;
             float sa, sb;
-            half_row_dot2(P.kp, ia < k1 ? ia : -1, ib < k1 ? ib : -1, half, P.qbar, &sa, &sb);
+            half_row_dot2(P.kp, P.crow, ia < k1 ? ia : -1, ib < k1 ? ib : -1, half, P.qbar, &sa, &sb);
             sa += __shfl_xor_sync(0xffffffffu, sa, 1);
             sb += __shfl_xor_sync(0xffffffffu, sb, 1);
             if (half == 0) {
@@ -487,7 +485,7 @@ __device__ __noinline__ void partial_rows(const PartialArgs& P) {
 // Shared-memory layout, computed identically on the host (launch size) and the device.
 struct Layout {
     uint32_t ring, qbar, qh, score, off, spre, cand, clist, bkt, hist, hcnt, hnear, rkey, prow,
-        rsrc, rks, rvs, wbuf, scl, ccomb, pbuf, bars, total;
+        rsrc, rks, rvs, key8, wbuf, scl, ccomb, pbuf, bars, total;
 };
 // The ring also holds, before any row arrives, the centroid slice (up to ring / 512 rows of
 // fp32 centroids per chunk) and the cut cluster's keys; after the last row, the warp partials.
@@ -523,6 +521,7 @@ __host__ __device__ inline Layout make_layout(int G, int S, int C, int RB, int p
     L.rsrc = take(mixed ? 4u * RB : 0u);  // far-row sources and scales: mixed precision only
     L.rks = take(mixed ? 4u * RB : 0u);
     L.rvs = take(mixed ? 4u * RB : 0u);
+    L.key8 = take((uint32_t)RB);  // per ring row: the chunk key of its store row
     L.wbuf = take(4u * 128);
     L.scl = take(4u * ((kWarps + S) * G + 2 * G));
     L.ccomb = take(4u * S * G * kCombStride);
@@ -577,6 +576,7 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     uint32_t* const s_rkey = (uint32_t*)(base + Ly.rkey);
     int32_t* const s_prow = (int32_t*)(base + Ly.prow);
     int32_t* const s_rsrc = (int32_t*)(base + Ly.rsrc);
+    uint8_t* const s_key8 = base + Ly.key8;
     int32_t* const s_wbuf = (int32_t*)(base + Ly.wbuf);
     float* const s_scl = (float*)(base + Ly.scl);
     float* const s_ccomb = (float*)(base + Ly.ccomb);
@@ -607,8 +607,8 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     if (tid == 0) {
         mbar_init(cbar, 1);
         mbar_init(fbar, 1);
-        mbar_init(rbar, kWarps + kNT);  // a byte-count arrival per warp, a cp.async one per thread
-        mbar_init(rbar + 1, kWarps + kNT);
+        mbar_init(rbar, kWarps);  // a byte-count arrival per warp
+        mbar_init(rbar + 1, kWarps);
         mbar_init(xbar, 1);
         mbar_init(obar, 1);
         fence_mbar_init();
@@ -1055,8 +1055,12 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     const int n_chunks = (n_rows + chunk - 1) / chunk;
     // Chunk ch: selection positions [lo + ch * chunk, ...) into ring slot ch & 1. Thread t
     // resolves position c0 + t (a sink or pending row, a whole cluster's row found by binary
-    // search over the compact list, or a partial row); each warp announces its lanes' bytes on
-    // the slot's mbarrier, then every lane issues its K and V row copies.
+    // search over the compact list, or a partial row) and records its ring row's chunk key.
+    // Rows come in runs that are consecutive in the store (the sinks, the pending rows up to the
+    // ring's end, the selected part of a whole cluster): the thread at a run's first position in
+    // the chunk copies the run's K rows and its V rows with one bulk copy each. A partial row,
+    // or a far row of the fp8 copy, is a run of its own. Each warp announces its lanes' bytes
+    // on the slot's mbarrier before any of them issues a copy.
     auto issue = [&](int ch) {  // every thread
         const int32_t c0 = lo + ch * chunk;
         const int32_t c1 = (c0 + chunk < s_hi) ? c0 + chunk : s_hi;
@@ -1064,11 +1068,20 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         const uint32_t bar = smem_u32(rbar + (ch & 1));
         const int32_t idx = c0 + tid;
         fence_proxy_async();  // this CTA's earlier accesses of the ring come before the copies
-        int32_t r = 0;
+        int32_t r = 0;               // >= 0: store row (| kFarBit when far); < 0: -1 - sink / pending row
+        bool starts = true;          // a run starts at idx
+        int32_t run_end = idx + 1;   // the end of that run in this chunk
         if (idx >= c1) {
-            // no row
-        } else if (idx < base_w) {  // a sink, or pending token idx - n_sink of the ring
-            r = -1 - (idx < a.n_sink ? idx : a.n_sink + (a.pstart + idx - a.n_sink) % a.pring);
+            starts = false;
+        } else if (idx < a.n_sink) {  // a sink
+            r = -1 - idx;
+            starts = idx == c0 || idx == 0;
+            run_end = min(c1, a.n_sink);
+        } else if (idx < base_w) {  // pending token i, at ring row q of the pending rows
+            const int32_t i = idx - a.n_sink, q = (a.pstart + i) % a.pring;
+            r = -1 - (a.n_sink + q);
+            starts = idx == c0 || i == 0 || q == 0;
+            run_end = min(min(c1, base_w), idx + (a.pring - q));
         } else if (idx < base_p) {
             const int32_t x = idx - base_w;
             int k0 = 0, khi = n_whole - 1;  // the whole cluster holding x: last wl_pre <= x
@@ -1079,46 +1092,40 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
             const int32_t o = wl_off[k0];
             r = (o & ~kFarBit) + (x - wl_pre[k0]);
             if (kMixed && (o & kFarBit)) r |= kFarBit;
+            starts = idx == c0 || x == wl_pre[k0];
+            run_end = min(c1, base_w + wl_pre[k0 + 1]);
         } else {
             r = s_prow[idx - base_p - p_lo];
             if (kMixed && cut_far) r |= kFarBit;
         }
         const bool far = kMixed && r >= 0 && (r & kFarBit) != 0;
-        // bulk-copied bytes: the K row (bf16) or both rows' codes (fp8); a bf16 V row comes by
-        // cp.async, tracked by this thread's cp.async arrival below
-        warp_arrive(rbar + (ch & 1), idx >= c1 ? 0u : (far ? 2u * kD : kD * 2u));
+        const bool issues = idx < c1 && (starts || far);
+        const int32_t len = far ? 1 : run_end - idx;
+        // bulk-copied bytes: the run's K and V rows (bf16), or the row's two code rows (fp8)
+        warp_arrive(rbar + (ch & 1), !issues ? 0u : (far ? 2u * kD : (uint32_t)len * kD * 4u));
         const uint32_t dk = ringK + (uint32_t)p * kPitch, dv = ringV + (uint32_t)p * kPitch;
-        const uint16_t* sv = nullptr;  // a bf16 V row this thread's position needs
-        if (idx >= c1) {
-            // no row
-        } else if (far) {
-            const int64_t row = kp_base + (r & ~kFarBit);
-            bulk_row(dk + 128u, a.kp8 + row * kD, kD, bar);
-            bulk_row(dv + 128u, a.vp8 + row * kD, kD, bar);
-            s_rks[p] = a.ks8[row];
-            s_rvs[p] = a.vs8[row];
-        } else {
-            const uint16_t* sk = r >= 0 ? a.kp + (kp_base + r) * kD : a.spk + (sp_base + (-1 - r)) * kD;
-            sv = r >= 0 ? a.vp + (kp_base + r) * kD : a.spv + (sp_base + (-1 - r)) * kD;
-            bulk_row(dk, sk, kD * 2, bar);  // the K row by the bulk-copy unit
-            if (kMixed) {
+        if (issues) {
+            if (far) {
+                const int64_t row = kp_base + (r & ~kFarBit);
+                bulk_row(dk + 128u, a.kp8 + row * kD, kD, bar);
+                bulk_row(dv + 128u, a.vp8 + row * kD, kD, bar);
+                s_rks[p] = a.ks8[row];
+                s_rvs[p] = a.vs8[row];
+            } else {
+                const int64_t rk = r >= 0 ? kp_base + r : sp_base + (-1 - r);
+                bulk_row(dk, (r >= 0 ? a.kp : a.spk) + rk * kD, (uint32_t)len * kD * 2u, bar);
+                bulk_row(dv, (r >= 0 ? a.vp : a.spv) + rk * kD, (uint32_t)len * kD * 2u, bar);
+            }
+        }
+        if (idx >= c1) return;
+        s_key8[p] = (uint8_t)((r >= 0 ? (r & ~kFarBit) : -1 - r) & 7);
+        if (kMixed) {
+            s_rsrc[p] = r;
+            if (!far) {
                 s_rks[p] = 1.f;
                 s_rvs[p] = 1.f;
             }
         }
-        // the warp's V rows by cp.async through the load/store path, in parallel with the bulk
-        // copies: two rows per instruction (lanes 0-15 and 16-31, 16 bytes each, coalesced)
-#pragma unroll 4
-        for (int i = 0; i < 32; i += 2) {  // warp-uniform trip count
-            const int src_lane = i + (lane >> 4);
-            const uint16_t* v = (const uint16_t*)__shfl_sync(0xffffffffu, (unsigned long long)sv, src_lane);
-            const int j = lane & 15;
-            if (v != nullptr)
-                cp_async16(ringV + (uint32_t)(p - lane + src_lane) * kPitch + (uint32_t)j * 16u, v + j * 8);
-        }
-        cp_async_mbar_arrive(rbar + (ch & 1));  // every thread, once per chunk
-        if (idx >= c1) return;
-        if (kMixed) s_rsrc[p] = r;
         if (sel_out)
             sel_out[idx] = r >= 0 ? ids[r & ~kFarBit] : (idx < a.n_sink ? idx : (int32_t)(a.m + idx));
     };
@@ -1134,10 +1141,11 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
             bulk_load(base + Ly.ring, a.kp + (kp_base + crow) * kD, bytes, fbar);
             bulk_load(base + Ly.ring + (size_t)RB * kPitch, a.vp + (kp_base + crow) * kD, bytes, fbar);
         }
+        for (int e = tid; e < csz; e += kNT) s_key8[e] = (uint8_t)((crow + e) & 7);
         const bool got = __syncthreads_and(mbar_wait(fbar, 0, a.err) ? 1 : 0) != 0;
         if (!got) s_wbuf[kWBad] = 1;
-        // qbar . k, a half-warp per row (16-byte reads covering one 256-byte row), 8 rows
-        // per half-warp in flight
+        // qbar . k, a half-warp per row (16-byte reads covering one 256-byte row; lane l16 reads
+        // the stored chunk that holds logical chunk l16), 8 rows per half-warp in flight
         const int hw = tid >> 4, l16 = tid & 15;
         const float4 qa = reinterpret_cast<const float4*>(s_qbar)[l16 * 2];
         const float4 qb4 = reinterpret_cast<const float4*>(s_qbar)[l16 * 2 + 1];
@@ -1148,7 +1156,7 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
                 const int e = r0 + hw + k * (kNT / 16);
                 sk[k] = 0.f;
                 if (got && e < csz) {
-                    const uint4 w = lds_v4(ringK + (uint32_t)e * 256u + l16 * 16);
+                    const uint4 w = lds_v4(ringK + (uint32_t)e * 256u + ((uint32_t)swz(crow + e, l16) << 4));
                     float t = qa.x * bf16_lo(w.x);
                     t = fmaf(qa.y, bf16_hi(w.x), t);
                     t = fmaf(qa.z, bf16_lo(w.y), t);
@@ -1275,8 +1283,10 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     // rows: ring row of tile row t is pos[t] (pos != nullptr) or p0 + t
     auto attend = [&](int p0, int n, const int32_t* pos) {
         // the resident cut cluster (pos != nullptr) sits in plain 256-byte rows
-        const uint32_t pitch = pos != nullptr ? 256u : (uint32_t)kPitch;
-        auto addr = [&](uint32_t rbase, int p, int j) { return rbase + (uint32_t)p * pitch + ((uint32_t)j << 4); };
+        // logical 16-byte chunk j of ring row p, whose chunk key is key
+        auto addr = [&](uint32_t rbase, int p, int key, int j) {
+            return rbase + (uint32_t)p * kPitch + ((uint32_t)(j ^ key) << 4);
+        };
         const int n_tiles = (n + 15) >> 4;
         for (int tile = warp; tile < n_tiles; tile += kWarps) {
             const int r0 = tile * 16;
@@ -1286,11 +1296,12 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
             if (tv >= n) tv = r0;
             const int pk = pos ? pos[tk] : p0 + tk;
             const int pv = pos ? pos[tv] : p0 + tv;
+            const int kk = s_key8[pk], kv = s_key8[pv];
             float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int s8 = 0; s8 < 8; ++s8) {
                 uint32_t a0, a1, a2, a3;
-                ldsm_x4(addr(ringK, pk, 2 * s8 + (mi >> 1)), a0, a1, a2, a3);
+                ldsm_x4(addr(ringK, pk, kk, 2 * s8 + (mi >> 1)), a0, a1, a2, a3);
                 mma_bf16_16816((s8 & 1) ? sb : sa, a0, a1, a2, a3, qb[s8][0], qb[s8][1]);
             }
             // S^T: [0], [1] = row g8, heads 2 t4, 2 t4 + 1; [2], [3] = row g8 + 8
@@ -1345,7 +1356,7 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
                 uint32_t a0, a1, a2, a3;
-                ldsm_x4_trans(addr(ringV, pv, 2 * mt + (mi & 1)), a0, a1, a2, a3);
+                ldsm_x4_trans(addr(ringV, pv, kv, 2 * mt + (mi & 1)), a0, a1, a2, a3);
                 mma_bf16_16816(oacc[mt], a0, a1, a2, a3, ph0, ph1);
                 mma_bf16_16816(oacc[mt], a0, a1, a2, a3, pl0, pl1);
             }

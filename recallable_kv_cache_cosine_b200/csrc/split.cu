@@ -67,14 +67,15 @@ __global__ void __launch_bounds__(kDriftWarps * 32) drift_kernel(const SplitArgs
     const float4 mu = reinterpret_cast<const float4*>(a.mu + ((int64_t)u * a.mu_ustride + c) * kD)[lane];
     const float mm = warp_sum(mu.x * mu.x + mu.y * mu.y + mu.z * mu.z + mu.w * mu.w);
     const float nm = __fsqrt_rn(mm);
-    const uint16_t* base = a.kp + (int64_t)u * a.kp_ustride * kD + lane * 4;
+    const uint16_t* base = a.kp + (int64_t)u * a.kp_ustride * kD;  // lane: dims 4 lane .. + 3
     float acc = 0.f;
     constexpr int kInFlight = 16;
     for (int32_t j = lo; j < hi; j += kInFlight) {  // warp-uniform trip count
         uint2 w[kInFlight];
 #pragma unroll
         for (int r = 0; r < kInFlight; ++r)
-            if (j + r < hi) w[r] = *reinterpret_cast<const uint2*>(base + (int64_t)(j + r) * kD);
+            if (j + r < hi)
+                w[r] = *reinterpret_cast<const uint2*>(base + (int64_t)(j + r) * kD + swz_elem(j + r, lane * 4));
 #pragma unroll
         for (int r = 0; r < kInFlight; ++r) {
             if (j + r >= hi) break;  // warp-uniform
@@ -156,10 +157,12 @@ __global__ void __launch_bounds__(kSplitThreads) split_kmeans_kernel(const Split
     const int64_t row0 = (int64_t)u * a.kp_ustride + lo;  // first row of the segment
     const uint16_t* gk = a.kp + row0 * kD;
     const bool staged = s <= kStageRows;
-    if (staged)
+    if (staged)  // in logical order (stored row lo + t / 16)
         for (int t = tid; t < s * (kD / 8); t += kSplitThreads)
-            reinterpret_cast<uint4*>(skey)[t] = reinterpret_cast<const uint4*>(gk)[t];
+            reinterpret_cast<uint4*>(skey)[t] = reinterpret_cast<const uint4*>(gk)[(t & ~15) | swz(lo + (t >> 4), t & 15)];
     const uint16_t* rows = staged ? skey : gk;
+    // offset of logical element d of segment row i in `rows`
+    auto col = [&](int64_t i, int d) { return staged ? d : swz_elem(lo + i, d); };
     int32_t* lab = staged ? slab : a.lab + row0;
     if (tid == 0) {
         // first two entries of a Fisher-Yates shuffle of 0..s-1 (SplitMix64 draws mapped by
@@ -175,7 +178,7 @@ __global__ void __launch_bounds__(kSplitThreads) split_kmeans_kernel(const Split
     __syncthreads();
     {
         const int ch = tid >> 7, d = tid & (kD - 1);
-        smu[ch * kD + d] = __uint_as_float((uint32_t)rows[(int64_t)sidx[ch] * kD + d] << 16);
+        smu[ch * kD + d] = __uint_as_float((uint32_t)rows[(int64_t)sidx[ch] * kD + col(sidx[ch], d)] << 16);
     }
     __syncthreads();
     for (int it = 0; it < a.iters; ++it) {
@@ -205,7 +208,7 @@ __global__ void __launch_bounds__(kSplitThreads) split_kmeans_kernel(const Split
                 const int i = i0 + r * kNW;
                 p0[r] = p1[r] = 0.f;
                 if (i < s) {
-                    const uint2 w = *reinterpret_cast<const uint2*>(rows + (int64_t)i * kD + lane * 4);
+                    const uint2 w = *reinterpret_cast<const uint2*>(rows + (int64_t)i * kD + col(i, lane * 4));
                     const float k0 = bf16_lo(w.x), k1 = bf16_hi(w.x), k2 = bf16_lo(w.y),
                                 k3 = bf16_hi(w.y);
                     p0[r] = fmaf(k3, h0.w, fmaf(k2, h0.z, fmaf(k1, h0.y, k0 * h0.x)));
@@ -239,7 +242,7 @@ __global__ void __launch_bounds__(kSplitThreads) split_kmeans_kernel(const Split
             const int part = tid >> 7, d = tid & (kD - 1);
             float a0 = 0.f, a1 = 0.f;
             for (int j = part; j < s; j += 2) {
-                const float v = __uint_as_float((uint32_t)rows[(int64_t)j * kD + d] << 16);
+                const float v = __uint_as_float((uint32_t)rows[(int64_t)j * kD + col(j, d)] << 16);
                 if (lab[j]) a1 += v;
                 else a0 += v;
             }
@@ -284,8 +287,10 @@ __global__ void __launch_bounds__(kSplitThreads) split_kmeans_kernel(const Split
     for (int i = tid; i < s; i += kSplitThreads) rid[i] = ids[i];
     __syncthreads();
     for (int t = tid; t < s * (kD / 8); t += kSplitThreads) {
+        // stored chunk w of row lo + i holds logical chunk w ^ key(lo + i): it moves to row
+        // lo + lab[i] at that logical chunk's position there
         const int i = t / (kD / 8), w = t % (kD / 8);
-        const int64_t dst = (int64_t)lab[i] * (kD / 8) + w;
+        const int64_t dst = (int64_t)lab[i] * (kD / 8) + swz(lo + lab[i], swz(lo + i, w));
         reinterpret_cast<uint4*>(kp)[dst] = reinterpret_cast<const uint4*>(rk)[t];
         reinterpret_cast<uint4*>(vp)[dst] = reinterpret_cast<const uint4*>(rv)[t];
     }
