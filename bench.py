@@ -52,7 +52,7 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 
 # DRAM bytes per select+attend launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum)
 # for the current kernel, or None when the kernel changed after the counters were taken.
-SELECT_ATTEND_TRAFFIC = 6.094e6  # dram read + write per launch, ncu --set full of the headline layer (cold L2)
+SELECT_ATTEND_TRAFFIC = 6.099e6  # dram read + write per launch, ncu --set full of the headline layer (cold L2)
 
 
 def peaks():
