@@ -686,31 +686,36 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
         const float4 qv = reinterpret_cast<const float4*>(s_qbar)[lane];
         // The slice in chunks of at most cch centroids (one chunk unless C / S exceeds the
         // ring); a warp per centroid (lane: dims 4 lane .. 4 lane + 3, a conflict-free 512-byte
-        // row), four centroids per warp in flight.
+        // row), eight centroids per warp in flight. The eight lane sums are reduced together:
+        // each exchange step halves the values a lane keeps (xor 16: four, xor 8: two, xor 4:
+        // one), then xor 2 and 1 finish the sum, so lane l ends with the full score of the
+        // warp's centroid number l >> 2 (9 shuffles for 8 scores).
         for (int done = 0, chunk_no = 0; done < nc; ++chunk_no) {
             const int n1 = min(nc - done, cch);
             ok = ok && mbar_wait(cbar, (uint32_t)(chunk_no & 1), a.err);
-            for (int j0 = warp; j0 < n1; j0 += 4 * kWarps) {
-                float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-                float* sk[4] = {&s0, &s1, &s2, &s3};
+            for (int j0 = warp; j0 < n1; j0 += 8 * kWarps) {
+                float p[8];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
+                for (int k = 0; k < 8; ++k) {
                     const int j = j0 + k * kWarps;
+                    p[k] = 0.f;
                     if (ok && j < n1) {
                         const float4 mv = reinterpret_cast<const float4*>(s_cent + (size_t)j * kD)[lane];
-                        *sk[k] = fmaf(qv.w, mv.w, fmaf(qv.z, mv.z, fmaf(qv.y, mv.y, qv.x * mv.x)));
+                        p[k] = fmaf(qv.w, mv.w, fmaf(qv.z, mv.z, fmaf(qv.y, mv.y, qv.x * mv.x)));
                     }
                 }
+                const bool hA = (lane & 16) != 0, hB = (lane & 8) != 0, hC = (lane & 4) != 0;
+                float q[4];
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    s0 += __shfl_xor_sync(0xffffffffu, s0, o);
-                    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-                    s2 += __shfl_xor_sync(0xffffffffu, s2, o);
-                    s3 += __shfl_xor_sync(0xffffffffu, s3, o);
-                }
-                const int j = j0 + lane * kWarps;  // lanes 0..3 store one score each
-                if (lane < 4 && j < n1) {
-                    const float v = lane == 0 ? s0 : (lane == 1 ? s1 : (lane == 2 ? s2 : s3));
+                for (int i = 0; i < 4; ++i)  // q[i]: centroid 4 hA + i
+                    q[i] = (hA ? p[4 + i] : p[i]) + __shfl_xor_sync(0xffffffffu, hA ? p[i] : p[4 + i], 16);
+                const float r0 = (hB ? q[2] : q[0]) + __shfl_xor_sync(0xffffffffu, hB ? q[0] : q[2], 8);
+                const float r1 = (hB ? q[3] : q[1]) + __shfl_xor_sync(0xffffffffu, hB ? q[1] : q[3], 8);
+                float v = (hC ? r1 : r0) + __shfl_xor_sync(0xffffffffu, hC ? r0 : r1, 4);
+                v += __shfl_xor_sync(0xffffffffu, v, 2);
+                v += __shfl_xor_sync(0xffffffffu, v, 1);
+                const int j = j0 + (lane >> 2) * kWarps;  // lanes 4 k store centroid k's score
+                if ((lane & 3) == 0 && j < n1) {
                     const int c = c_begin + done + j;
                     s_score[c] = v;
                     if (kMixed || size_of(c) > 0) {
