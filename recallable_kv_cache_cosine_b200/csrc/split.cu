@@ -76,17 +76,38 @@ __global__ void __launch_bounds__(kDriftWarps * 32) drift_kernel(const SplitArgs
         for (int r = 0; r < kInFlight; ++r)
             if (j + r < hi)
                 w[r] = *reinterpret_cast<const uint2*>(base + (int64_t)(j + r) * kD + swz_elem(j + r, lane * 4));
+        // the lane's partial k.mu (value 2 r) and k.k (value 2 r + 1) of the 16 rows, reduced
+        // together: each exchange halves the values a lane keeps (xor 16: 16 values, xor 8:
+        // 8, ... xor 1: one), so lane l ends with the full value l (31 shuffles for 32 sums)
+        float v[2 * kInFlight];
 #pragma unroll
         for (int r = 0; r < kInFlight; ++r) {
-            if (j + r >= hi) break;  // warp-uniform
-            const float k0 = bf16_lo(w[r].x), k1 = bf16_hi(w[r].x), k2 = bf16_lo(w[r].y),
-                        k3 = bf16_hi(w[r].y);
-            const float dot = warp_sum(k0 * mu.x + k1 * mu.y + k2 * mu.z + k3 * mu.w);
-            const float kk = warp_sum(k0 * k0 + k1 * k1 + k2 * k2 + k3 * k3);
+            v[2 * r] = v[2 * r + 1] = 0.f;
+            if (j + r < hi) {
+                const float k0 = bf16_lo(w[r].x), k1 = bf16_hi(w[r].x), k2 = bf16_lo(w[r].y),
+                            k3 = bf16_hi(w[r].y);
+                v[2 * r] = k0 * mu.x + k1 * mu.y + k2 * mu.z + k3 * mu.w;
+                v[2 * r + 1] = k0 * k0 + k1 * k1 + k2 * k2 + k3 * k3;
+            }
+        }
+#pragma unroll
+        for (int half = 16; half >= 1; half >>= 1) {
+            const bool hi_lane = (lane & half) != 0;
+#pragma unroll
+            for (int i = 0; i < half; ++i) {
+                const float keep = hi_lane ? v[half + i] : v[i];
+                const float give = hi_lane ? v[i] : v[half + i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, give, half);
+            }
+        }
+        const float kk = __shfl_xor_sync(0xffffffffu, v[0], 1);  // row lane >> 1's k.k, at even lanes
+        if ((lane & 1) == 0 && j + (lane >> 1) < hi) {
+            const float dot = v[0];
             const float cs = (kk > 0.f && mm > 0.f) ? __fdiv_rn(dot, __fmul_rn(__fsqrt_rn(kk), nm)) : 0.f;
             acc += 1.f - cs;
         }
     }
+    acc = warp_sum(acc);
     const float drift = hi > lo ? __fdiv_rn(acc, (float)(hi - lo)) : 0.f;
     if (lane == 0) {
         a.drift[(int64_t)u * a.Cmax + c] = drift;
