@@ -236,26 +236,39 @@ __global__ void __launch_bounds__(kSplitThreads) split_kmeans_kernel(const Split
                     p1[r] = fmaf(k3, h1.w, fmaf(k2, h1.z, fmaf(k1, h1.y, k0 * h1.x)));
                 }
             }
+            // the 8 lane sums (value 2 r: row r's dot with the first half, 2 r + 1: with the
+            // second) reduced together: xor 16 keeps four values per lane, xor 8 two, xor 4
+            // one, xor 2 and 1 finish; lane l ends with value l >> 2 (9 shuffles, not 40)
+            float v[8];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    p0[r] += __shfl_xor_sync(0xffffffffu, p0[r], o);
-                    p1[r] += __shfl_xor_sync(0xffffffffu, p1[r], o);
-                }
-            if (lane == 0) {
-                int ones = 0;
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int i = i0 + r * kNW;
-                    if (i < s) {
-                        const int l = p1[r] > p0[r] ? 1 : 0;
-                        lab[i] = l;
-                        ones += l;
-                    }
-                }
-                if (ones) atomicAdd(scnt, ones);
+            for (int r = 0; r < 4; ++r) {
+                v[2 * r] = p0[r];
+                v[2 * r + 1] = p1[r];
             }
+#pragma unroll
+            for (int half = 4; half >= 1; half >>= 1) {
+                const bool up = (lane & (4 * half)) != 0;  // lane bits 4, 3, 2
+#pragma unroll
+                for (int t = 0; t < half; ++t) {
+                    const float keep = up ? v[half + t] : v[t];
+                    const float give = up ? v[t] : v[half + t];
+                    v[t] = keep + __shfl_xor_sync(0xffffffffu, give, 4 * half);
+                }
+            }
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], 2);
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+            const float other = __shfl_xor_sync(0xffffffffu, v[0], 4);  // the row's other half
+            int ones = 0;
+            if ((lane & 7) == 0) {  // lane 8 r holds row r's first-half dot, lane 8 r + 4 its second
+                const int r = lane >> 3, i = i0 + r * kNW;
+                if (i < s) {
+                    const int l = other > v[0] ? 1 : 0;
+                    lab[i] = l;
+                    ones = l;
+                }
+            }
+            ones = __reduce_add_sync(0xffffffffu, ones);
+            if (lane == 0 && ones) atomicAdd(scnt, ones);
         }
         __syncthreads();
         {  // update: thread (part, d) sums dimension d of both halves over the rows of its
