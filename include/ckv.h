@@ -230,7 +230,10 @@ CKV_API int ckv_get_layer_info(const ckv_ctx* ctx, int32_t layer, ckv_layer_info
 /* Copy of one unit's store. Any NULL pointer is skipped. Buffers may be host or device
  * memory (cudaMemcpyDefault). The call synchronises `stream` before it returns.
  *   mu      fp32 [C, 128]          offsets int32 [C + 1]        ids int32 [m]
- *   kp, vp  bf16 [m, 128]          sp_k, sp_v bf16 [n_sink + pending, 128] */
+ *   kp, vp  bf16 [m, 128]          sp_k, sp_v bf16 [n_sink + pending, 128]
+ * Rows come out in plain element order. (Inside the context every stored row keeps its
+ * 16-byte chunk c at chunk c ^ (r & 7), r = its row index in the unit; the copy puts the rows
+ * back in order through a temporary device buffer, allocated on `stream`.) */
 typedef struct ckv_unit_buffers {
     float* mu;
     int32_t* offsets;
@@ -244,8 +247,8 @@ typedef struct ckv_unit_buffers {
 CKV_API int ckv_export_unit(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h,
                     const ckv_unit_buffers* dst, void* stream);
 
-/* Loads one unit's store from caller buffers (all seven non-NULL; layouts as above),
- * for decoding over stores built elsewhere. Synchronous, like ckv_export_unit. Sets the layer's counts to (m, C, pending),
+/* Loads one unit's store from caller buffers (all seven non-NULL; layouts as above, plain
+ * element order), for decoding over stores built elsewhere. Synchronous, like ckv_export_unit. Sets the layer's counts to (m, C, pending),
  * which must then agree across the layer's units. Offsets must be non-decreasing from 0
  * to m, ids must lie in [n_sink, n_total) and ascend inside each cluster (the decode's
  * lower-id tie rule relies on store order). */
@@ -285,8 +288,8 @@ CKV_API int select_and_attend_mixed(ckv_ctx* ctx, int32_t layer, const void* q, 
                                     int32_t n_near, float* out, int32_t* sel_idx,
                                     int32_t* sel_count, void* stream);
 
-/* Copy of one unit's fp8 rows (layouts: k8, v8 uint8 [m, 128]; ks, vs fp32 [m]); any NULL
- * pointer is skipped, host or device buffers. Synchronises `stream`. CKV_ESTATE without
+/* Copy of one unit's fp8 rows (layouts: k8, v8 uint8 [m, 128] in plain element order; ks, vs
+ * fp32 [m]); any NULL pointer is skipped, host or device buffers. Synchronises `stream`. CKV_ESTATE without
  * ckv_enable_fp8 or before the layer is clustered. */
 CKV_API int ckv_export_unit_fp8(ckv_ctx* ctx, int32_t layer, int32_t b, int32_t h, void* k8,
                                 float* ks, void* v8, float* vs, void* stream);
