@@ -88,18 +88,23 @@ __global__ void __launch_bounds__(kRT) recluster_kernel(const ReclusterArgs a) {
         }
         if (tid < Cn) scnt[tid] = 0;
         __syncthreads();
-        // assign (ties: lower c)
+        // assign (ties: lower c). Thread i walks its key row's 64 words starting at word
+        // (i mod 32), so the 32 lanes of a warp, each on its own row, read 32 different banks
+        // at every step (rows are 256 bytes apart: the same word of each would share a bank).
         for (int i = tid; i < W; i += kRT) {
-            const uint16_t* kr = skey + i * kD;
+            const uint32_t* kw = reinterpret_cast<const uint32_t*>(skey + i * kD);
+            const int rot = i & 31;
             float best = -INFINITY;
             int bi = 0;
             for (int c = 0; c < Cn; ++c) {
-                const float* mh = smh + c * kD;
+                const float2* m2 = reinterpret_cast<const float2*>(smh + c * kD);
                 float s = 0.f;
-                for (int d = 0; d < kD; d += 2) {
-                    const uint32_t w = *reinterpret_cast<const uint32_t*>(kr + d);
-                    s = fmaf(bf16_lo(w), mh[d], s);
-                    s = fmaf(bf16_hi(w), mh[d + 1], s);
+                for (int t = 0; t < kD / 2; ++t) {
+                    const int wi = (t + rot) & (kD / 2 - 1);
+                    const uint32_t w = kw[wi];
+                    const float2 mm = m2[wi];
+                    s = fmaf(bf16_lo(w), mm.x, s);
+                    s = fmaf(bf16_hi(w), mm.y, s);
                 }
                 if (s > best) {
                     best = s;
