@@ -115,8 +115,6 @@ CKV_DEV void bulk_row(uint32_t dst, const void* src, uint32_t bytes, uint32_t ba
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
-// Arrives on the mbarrier once every cp.async this thread issued so far has completed (the
-// barrier's expected count includes this arrival).
 CKV_DEV void sts_v4(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
                  "r"(v.w)
