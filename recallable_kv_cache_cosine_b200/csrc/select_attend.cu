@@ -22,8 +22,9 @@
 //      store. The queries, the sink / pending rows and every output are touched only after
 //      the wait;
 //   1. qbar = sum of the group's queries; each CTA scores its slice (a warp per centroid,
-//      four in flight) into its own shared memory; after one cluster barrier every CTA reads
-//      the other slices through distributed shared memory;
+//      eight in flight, their lane sums reduced together) and stores the scores into every
+//      CTA of the cluster by asynchronous remote stores (st.async) that count their bytes on
+//      the receiver's mbarrier; each CTA goes on once its own copy is complete;
 //   2. every CTA computes the same selection on its own. The walk in descending
 //      (score, -index) order stops at the first cluster whose inclusive token count exceeds
 //      the remaining budget R: the cut, a size-weighted quantile of the scores. The scores are
@@ -38,15 +39,17 @@
 //      when the histogram isolates the cut), ranks the tokens by qbar . k there and attends
 //      the top ones in place; it also takes the last whole rows, up to an even share of the
 //      work less the cut cluster it loaded. The other CTAs split the rest evenly;
-//   4. rows reach a shared-memory ring by one bulk copy (cp.async.bulk) per K or V row,
-//      issued by the thread that resolves the row's source, and complete on the chunk's
-//      mbarrier. Ring rows are 272 bytes apart, so the 8 rows of a matrix load fall on
-//      distinct banks. Each warp runs flash-decode on 16-row tiles with
+//   4. rows reach a shared-memory ring in runs: each run of consecutive store rows (the
+//      sinks, the pending rows, the selected part of a whole cluster) by one bulk copy
+//      (cp.async.bulk) for K and one for V, completing on the chunk's mbarrier. Ring rows are
+//      store rows as they are; the store keeps chunk c of row r at c ^ (r & 7), so the 8 rows
+//      of a matrix load fall on distinct banks. Each warp runs flash-decode on 16-row tiles with
 //      tensor-core MMAs (mma.sync m16n8k16, bf16 in, fp32 accumulate): S^T = K Q^T with the
 //      rows as M and the G query heads as N, an online softmax per head, then O^T += V^T P
 //      with P split into bf16 high and low parts;
-//   5. the warp partials (max, sum, accumulator) are merged per CTA, and the CTA partials in
-//      CTA 0 through distributed shared memory, which writes the fp32 output.
+//   5. the warp partials (max, sum, accumulator) are merged per CTA; the other CTAs store
+//      theirs into CTA 0 (st.async, counted on CTA 0's mbarrier), which merges them and
+//      writes the fp32 output.
 // Every loop that holds a warp-synchronous operation (shuffle, ballot, reduce) starts at a
 // warp- or CTA-uniform value and steps by a uniform stride, so all 32 lanes run every
 // iteration. Bounded waits that give up set the device error word; the CTA then skips its
@@ -1285,8 +1288,7 @@ __global__ void __launch_bounds__(kNT, 2) select_attend_kernel(const DecodeArgs 
     const float qscale = kLog2e * rsqrtf((float)kD);
     // rows: ring row of tile row t is pos[t] (pos != nullptr) or p0 + t
     auto attend = [&](int p0, int n, const int32_t* pos) {
-        // the resident cut cluster (pos != nullptr) sits in plain 256-byte rows
-        // logical 16-byte chunk j of ring row p, whose chunk key is key
+        // logical 16-byte chunk j of ring row p (a 256-byte store row), whose chunk key is key
         auto addr = [&](uint32_t rbase, int p, int key, int j) {
             return rbase + (uint32_t)p * kPitch + ((uint32_t)(j ^ key) << 4);
         };
