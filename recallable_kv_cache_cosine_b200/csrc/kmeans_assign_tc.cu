@@ -10,7 +10,7 @@
 //   warp 16     TMA producer: the unit's centroid block mu_hat (<= 512 rows, kept in shared
 //               memory while the unit lasts, each 256-row slot sized to its rows), then the
 //               128x128 bf16 key tiles through a ring of 3-6 stages (as many as shared
-//               memory allows). All loads use the 128-byte swizzle and no multicast.
+//               memory allows). All loads use the 128-byte swizzle; each CTA loads its own tiles.
 //   warp 17     allocates 512 TMEM columns. One thread issues tcgen05.mma (M=128, N<=256,
 //               K=16, bf16 x bf16 -> fp32) into two 256-column accumulator slots. With
 //               C <= 256, consecutive tiles alternate slots (double buffering). With
