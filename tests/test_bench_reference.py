@@ -32,3 +32,20 @@ def test_oracle_thread_setting_round_trips():
     assert prev >= 1
     assert oracle.set_threads(prev) == 1
     assert oracle.set_threads(0) == prev  # 0 reads the setting without changing it
+
+
+def test_kmeans_roofline_names_the_binding_term():
+    """min(tensor, HBM) keys/s per Lloyd iteration: with the fallback peaks (6.65 TB/s, 1.59
+    PFLOP/s) two 256-byte key reads bind at C = 100 and 400, the 2·C·128 flops at C = 1600."""
+    sys.path.insert(0, ROOT)
+    import bench
+    hbm, tflops = 6650.0, 1590.0
+    for C, term in ((100, "hbm"), (400, "hbm"), (1600, "tensor")):
+        roof, bound = bench.kmeans_roofline(C, hbm, tflops)
+        assert bound == term, C
+        want = min(tflops * 1e12 / (2 * C * 128), hbm * 1e9 / 512) / bench.ITERS
+        assert abs(roof - want) <= 1e-9 * want
+    # one init, per iteration one assignment launch per 512 centroids plus scan, scatter and
+    # mean, one sink copy
+    assert bench.launches_per_prefill(400, 10) == 1 + 10 * 4 + 1
+    assert bench.launches_per_prefill(1600, 10) == 1 + 10 * 7 + 1
